@@ -1,0 +1,427 @@
+#!/usr/bin/env python3
+"""Decode benchmark: greedy decode tok/s of the 7B-class Q4_0 model at batch 1
+(28 layers, hidden 3584, 28/4 heads, FFN 18944, vocab 152064, ctx 2000 + 512
+decode tokens), seeded synthetic random-init weights, on 1..N B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 7b] [--impl ours|reference]
+
+One step = one greedy decode token for the batch: embedding, 28 layers
+(fused RMSNorm+QKV GEMV, paged attention with RoPE + KV write, O GEMV +
+residual, fused RMSNorm+gate/up GEMV with SiLU gate, down GEMV + residual),
+final RMSNorm + LM-head GEMV + argmax.  The timed region replays CUDA graphs
+of decode steps whose last kernel feeds the next step on the device.  Every
+step streams ~4.1 GB of weights and KV (>> the 126 MB L2), so no L2 flush is
+needed between steps.  Multi-GPU: independent replicas (weak scaling), one
+process per GPU, time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode tok/s at batch 1 and 32; achieved HBM GB/s as % of 8 TB/s roofline"
+NOMINAL_HBM_GBS = 8000.0
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = max(mx, float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def step_bytes(cfg, model, avg_ctx):
+    """Algorithmic bytes of one decode step: every weight matrix streamed once
+    (4.5-bit blocks + fp32 norm gains), the KV read over the context, the new
+    K/V written (the embedding row is not counted)."""
+    kv_read = 2 * cfg.L * cfg.nkv * cfg.hd * 2 * avg_ctx * cfg.B
+    kv_write = 2 * cfg.L * cfg.nkv * cfg.hd * 2 * cfg.B
+    return model.weight_bytes_dense() + kv_read + kv_write
+
+
+def run_ours(args):
+    from token_decode_b200 import build, bw, runtime, synth
+    ws_, rank, local = dist_env()
+    if ws_ > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    build.build()
+    bw.lib()
+    cfg = synth.CONFIGS[args.config]
+    total = args.warmup + args.steps
+    # one generation = `cfg.steps` tokens from position ctx; longer runs start new generations
+    model = synth.make_model(cfg, "cuda", seed=rank)
+    kv = synth.make_kv(cfg, "cuda", seed=rank)
+    dm = runtime.DeviceModel(model, cfg.max_pages * synth.PAGE_TOKENS)
+    dkv = runtime.DeviceKV(kv)
+    dec = runtime.Decoder(dm, dkv, cfg.B)
+    toks = synth.start_tokens(cfg, rank)
+    stream = torch.cuda.Stream()
+
+    def reset():
+        dec.tokens_in.copy_(toks)
+        dec.pos.fill_(cfg.ctx)
+
+    G = 16  # steps per captured graph
+    graphs = {}
+
+    def graph_for(n):
+        if n not in graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.stream(stream):
+                dec.step(advance=True, stream=stream)   # warm the launch path outside capture
+                with torch.cuda.graph(g, stream=stream):
+                    for _ in range(n):
+                        dec.step(advance=True, stream=stream)
+            graphs[n] = g
+        return graphs[n]
+
+    def plan(nsteps, start):
+        """Replays of (graph size) covering nsteps, restarting generations at cfg.steps."""
+        out, done, p = [], 0, start
+        while done < nsteps:
+            left_gen = cfg.steps - p
+            if left_gen <= 0:
+                out.append("reset")
+                p = 0
+                continue
+            n = min(G, nsteps - done, left_gen)
+            out.append(n)
+            done += n
+            p += n
+        return out, p
+
+    def run(ops):
+        for op in ops:
+            if op == "reset":
+                with torch.cuda.stream(stream):
+                    reset()
+            else:
+                graph_for(op).replay()
+
+    torch.cuda.synchronize()
+    reset()
+    torch.cuda.synchronize()
+    warm_ops, p_after = plan(args.warmup, 0)
+    for op in warm_ops:
+        if op != "reset":
+            graph_for(op)
+    # graph capture ran extra steps: restart the generation before warm-up
+    with torch.cuda.stream(stream):
+        reset()
+    run(warm_ops)
+    timed_ops, _ = plan(args.steps, p_after)
+    for op in timed_ops:
+        if op != "reset":
+            graph_for(op)
+    # the captures above advanced the state; rebuild the exact start of the timed region
+    with torch.cuda.stream(stream):
+        reset()
+    run(warm_ops)
+    stream.synchronize()
+    if ws_ > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        run(timed_ops)
+        e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    err = bw.read_error(dec.ws, stream)
+    if ws_ > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    ms_step = ms / args.steps
+    tokens = args.steps * cfg.B * ws_
+    value = tokens / (ms / 1000.0)
+
+    # ---- end to end through the C ABI: host tokens in, host token out, every step
+    pin_in = torch.empty(cfg.B, dtype=torch.int32).pin_memory()
+    pin_out = torch.empty(cfg.B, dtype=torch.int32).pin_memory()
+    pin_in.copy_(toks)
+    n_e2e = min(args.steps, 64)
+    with torch.cuda.stream(stream):
+        reset()
+    stream.synchronize()
+    for _ in range(3):
+        with torch.cuda.stream(stream):
+            dec.tokens_in.copy_(pin_in, non_blocking=True)
+            dec.step(stream=stream)
+            dec.pos += 1
+            pin_out.copy_(dec.tokens_out, non_blocking=True)
+        stream.synchronize()
+        pin_in.copy_(pin_out)
+    t0 = time.perf_counter()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(n_e2e):
+        with torch.cuda.stream(stream):
+            dec.tokens_in.copy_(pin_in, non_blocking=True)
+            dec.step(stream=stream)
+            dec.pos += 1
+            pin_out.copy_(dec.tokens_out, non_blocking=True)
+        stream.synchronize()
+        pin_in.copy_(pin_out)
+    f1.record(stream)
+    f1.synchronize()
+    e2e_ms = f0.elapsed_time(f1)
+    e2e_value = n_e2e * cfg.B / (e2e_ms / 1000.0) * ws_
+
+    # ---- dominant kernel: the fused gate/up GEMV, every layer back to back
+    gu_bytes = sum(dm.layers[l].wgu.N * dm.layers[l].wgu.K * 9 // 16 for l in range(cfg.L))
+    gu_bytes += 0  # (9/16 byte per weight: 4-bit codes + a 2-byte scale per 32)
+    kws = bw.workspace(bw.gemv_workspace_bytes(2 * cfg.F, cfg.H, cfg.B, 0))
+    xin = torch.randn((cfg.B, cfg.H), device="cuda")
+    gam = torch.ones(cfg.H, device="cuda")
+    act = torch.empty((cfg.B, cfg.F), device="cuda")
+
+    def gu_all():
+        for l in range(cfg.L):
+            w = dm.layers[l].wgu
+            if cfg.fmt == synth.FMT_Q4_0:
+                bw.gemv_q4_0(w.q, w.s, w.N, w.K, xin, cfg.B, act, kws, gamma=gam,
+                             flags=bw.GEMV_RMSNORM | bw.GEMV_SILU_GATE, stream=stream)
+            else:
+                bw.gemv_nvfp4(w.q, w.s, w.ts, w.N, w.K, xin, cfg.B, act, kws, ts_up=w.ts_up,
+                              gamma=gam, flags=bw.GEMV_RMSNORM | bw.GEMV_SILU_GATE, stream=stream)
+    for _ in range(3):
+        gu_all()
+    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 5
+    k0.record(stream)
+    for _ in range(reps):
+        gu_all()
+    k1.record(stream)
+    k1.synchronize()
+    gu_ms = k0.elapsed_time(k1) / (reps * cfg.L)
+    gu_launch_bytes = gu_bytes / cfg.L
+    peak, peak_kind = _peaks()
+    achieved = gu_launch_bytes / (gu_ms / 1000.0) / 1e9
+
+    avg_ctx = cfg.ctx + (cfg.steps + 1) / 2
+    sb = step_bytes(cfg, model, avg_ctx)
+    step_gbs = sb / (ms_step / 1000.0) / 1e9
+    launches_per_step = 1 + 5 * cfg.L + 1
+    launches_per_step += (cfg.B - 1) // 4 * (4 * cfg.L + 1)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": "tok/s",
+        "n_gpus": ws_,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "q4_0 weights, fp32 accumulate, fp16 KV" if cfg.fmt == synth.FMT_Q4_0 else
+                 "nvfp4 weights, fp32 accumulate, fp16 KV",
+        "data": "synthetic (seeded random-init weights N(0,0.02) quantized; N(0,1) fp16 KV context)",
+        "config": {"workload": cfg.name, "batch": cfg.B, "context": cfg.ctx,
+                   "decode_tokens_per_generation": cfg.steps, "layers": cfg.L, "hidden": cfg.H,
+                   "heads": f"{cfg.nq}/{cfg.nkv}x{cfg.hd}", "ffn": cfg.F, "vocab": cfg.V,
+                   "parallelism": f"replicas x{ws_}",
+                   "l2": "inputs larger than L2 (each step streams ~%.2f GB)" % (sb / 1e9),
+                   "timing": "CUDA graphs of %d steps, on-device token/position advance" % G},
+        "hbm_gbs_step": round(step_gbs, 1),
+        "roofline_step_frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4),
+        "roofline_step_frac_of_measured": round(step_gbs / peak, 4),
+        "bytes_per_step": int(sb),
+        "roofline": {"bound": "hbm", "kernel": "gemv_kernel (fused RMSNorm + gate/up + SiLU gate)",
+                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "bytes_per_launch": int(gu_launch_bytes), "avg_launch_us": round(gu_ms * 1000, 3)},
+        "e2e": {"value": round(e2e_value, 3), "unit": "tok/s", "steps": n_e2e,
+                "h2d_bytes_per_step": 4 * cfg.B, "d2h_bytes_per_step": 4 * cfg.B,
+                "path": "bw_decode_step via the C ABI, pinned host token in/out, sync each step"},
+        "gpu_launches": launches_per_step * args.steps,
+        "device_error_word": err,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, model, kv, toks, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_ > 1:
+        import torch.distributed as dist
+        graphs.clear()
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _oracle_setup(cfg, model, kv):
+    import oracle
+    oracle.build()
+    return oracle, oracle.Model(model), oracle.KV(kv)
+
+
+def _oracle_token_seconds(oracle, om, okv, cfg, tok, n_layer_samples, t_budget):
+    """Seconds of one full oracle decode token, estimated from a bounded sample:
+    the head alone (embedding + final norm + LM head) and single layers."""
+    t = time.perf_counter()
+    oracle.decode_token(om, okv, 0, tok, cfg.ctx, layers=(0, 0))
+    t_head = time.perf_counter() - t
+    per_layer = []
+    for i in range(n_layer_samples):
+        l = (i * 7) % cfg.L
+        t = time.perf_counter()
+        oracle.decode_token(om, okv, 0, tok, cfg.ctx, layers=(l, l + 1))
+        per_layer.append(max(0.0, time.perf_counter() - t - t_head))
+        if sum(per_layer) > t_budget:
+            break
+    return t_head + cfg.L * statistics.mean(per_layer), t_head, per_layer
+
+
+def cpu_baseline(cfg, model, kv, toks, budget_s=20.0):
+    oracle, om, okv = _oracle_setup(cfg, model, kv)
+    tok_s, t_head, per_layer = _oracle_token_seconds(oracle, om, okv, cfg, int(toks[0]), 64, budget_s)
+    return {"value": round(cfg.B / tok_s, 5), "unit": "tok/s", "cores": 1, "kind": "oracle",
+            "sample": f"embedding + LM head once ({t_head:.2f} s) and {len(per_layer)} single "
+                      f"layers of the {cfg.name} step at ctx {cfg.ctx}, scaled to {cfg.L} layers "
+                      f"(one token = {tok_s:.1f} s), single-threaded fp32 C",
+            "host_cores_total": os.cpu_count()}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step is one layer of the decode
+    step (cycling through the layers) plus the timed embedding/LM-head share."""
+    ws_, rank, local = dist_env()
+    if rank != 0:
+        return
+    from token_decode_b200 import synth
+    cfg = synth.CONFIGS[args.config]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    model = synth.make_model(cfg, dev, seed=0)
+    kv = synth.make_kv(cfg, dev, seed=0)
+    oracle, om, okv = _oracle_setup(cfg, model, kv)
+    tok = int(synth.start_tokens(cfg, 0)[0])
+    t = time.perf_counter()
+    oracle.decode_token(om, okv, 0, tok, cfg.ctx, layers=(0, 0))
+    t_head = time.perf_counter() - t
+    for i in range(args.warmup):
+        oracle.decode_token(om, okv, 0, tok, cfg.ctx, layers=(i % cfg.L, i % cfg.L + 1))
+    per = []
+    t_all = time.perf_counter()
+    for i in range(args.steps):
+        l = (i * 7) % cfg.L
+        t = time.perf_counter()
+        oracle.decode_token(om, okv, 0, tok, cfg.ctx, layers=(l, l + 1))
+        per.append(max(0.0, time.perf_counter() - t - t_head))
+    wall = time.perf_counter() - t_all
+    tok_s = t_head + cfg.L * statistics.mean(per)
+    value = cfg.B / tok_s
+    line = {"metric": METRIC, "value": round(value, 5), "unit": "tok/s", "n_gpus": ws_,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * wall / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32 (CPU oracle)",
+            "data": "synthetic (seeded random-init weights)", "impl": "reference",
+            "config": {"workload": cfg.name, "batch": cfg.B, "context": cfg.ctx},
+            "cpu_baseline": {"value": round(value, 5), "unit": "tok/s", "cores": 1, "kind": "oracle",
+                             "sample": f"each step = one of the {cfg.L} layers of one decode token "
+                                       f"(+ embedding/LM head timed once, {t_head:.2f} s), scaled "
+                                       f"to a full token"},
+            "e2e": {"value": round(value, 5), "unit": "tok/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=256)
+    ap.add_argument("--warmup", type=int, default=8)
+    ap.add_argument("--config", default="7b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

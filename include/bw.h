@@ -1,0 +1,269 @@
+/*
+ * bw.h -- C ABI of the B200 (sm_100a) decode hot path.
+ *
+ * One call = one piece of one greedy decode step, run asynchronously on a CUDA
+ * stream over caller-owned device memory.  What each call computes, and where
+ * the pages define it:
+ *
+ *   bw_gemv_q4_0 / bw_gemv_nvfp4 -- y = W x over 4-bit block-quantized W, with
+ *       an RMSNorm prologue, residual-add / SiLU-gate epilogues and an argmax
+ *       reduction fused in.  "Rust+CUDA ... bw24 vs llama.cpp" page (devpress),
+ *       section 2.2: linear layer, bias and activation fused in one kernel so
+ *       intermediates stay in registers / shared memory; "bw24" deep-dive page
+ *       (10100.com), section 7 (comparison table): Q4 GGUF weights and native
+ *       NVFP4.  Block formats: GGUF-style Q4_0 (32 weights, fp16 d,
+ *       w = d*(q-8)) and NVFP4 (16 E2M1 codes, E4M3 block scale, fp32 tensor
+ *       scale, w = e2m1*e4m3*ts).
+ *   bw_rmsnorm_fused -- x += add; y = x * rsqrt(mean(x^2) + eps) * gamma.
+ *   bw_paged_attn_decode -- RoPE of the new rows' q and k, fp16 K/V write into
+ *       the paged cache, GQA attention over the cache.  Deep-dive page,
+ *       section 6 ("Paged Cache": logical positions -> physical pages through
+ *       a page table) and section 5, stage 4 (the verify pass expands the K
+ *       draft tokens along the sequence dimension over one shared cache);
+ *       devpress page, section 2.1 (every token reads the whole cache).
+ *   bw_moe_route_gemv -- router GEMV, top-k softmax, grouped expert SwiGLU
+ *       GEMVs and the shared expert.  Deep-dive page, section 7: router
+ *       ordering and expert parallelism without warp divergence.
+ *   bw_argmax -- greedy sampling: the lowest index of the maximum.  Deep-dive
+ *       page, section 1: the argmax token sequence is the correctness gate.
+ *   bw_decode_step -- the whole step (embedding .. argmax) for B sequences of
+ *       n_rows consecutive tokens each (n_rows = 1: decode; n_rows = K+1:
+ *       speculative verify).  Deep-dive page, section 4: an engine facade
+ *       exposing prefill and decode.
+ *
+ * Conventions (all entry points):
+ *  - Pointers are DEVICE pointers owned by the caller unless a comment says
+ *    "host".  The library never allocates, frees or synchronizes on these
+ *    paths (bw_read_error is the one call that synchronizes).
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    kernel call is asynchronous on it.
+ *  - Arguments are validated on the host before any launch; a failed check
+ *    returns BW_ERR_INVALID_ARG or BW_ERR_UNSUPPORTED_SHAPE and launches
+ *    nothing.  A launch failure returns BW_ERR_CUDA.  Conditions only the
+ *    device can see (a page-table entry outside the pool) set a bit in the
+ *    error word at the start of the workspace; read it with bw_read_error
+ *    after the stream has drained.  No exception crosses the ABI.
+ *  - Workspace: scratch device memory of at least the queried size, 256-byte
+ *    aligned, zero-filled ONCE before first use (bw_workspace_init).  Kernels
+ *    leave their counters at zero on return, so the same workspace serves
+ *    any number of later calls and CUDA-graph replays on one stream.  Calls
+ *    sharing a workspace must not run concurrently.
+ *  - Weights live in the GPU layout written by bw_repack_q4_0 /
+ *    bw_repack_nvfp4 from the canonical (file) layout:
+ *      q : nibbles [N][K/2] bytes, row-major (per 32-element chunk the 16
+ *          bytes keep the canonical nibble order of the format)
+ *      s : per group of 8 rows and 32-element chunk, 16 bytes of scales,
+ *          [N/8][K/32][8] fp16 d (Q4_0) or [N/8][K/32][8][2] E4M3 (NVFP4)
+ *    Gate/up matrices are interleaved in groups of 4 rows (rows 8g..8g+3 are
+ *    gate rows 4g..4g+3, rows 8g+4..8g+7 the matching up rows).
+ */
+#ifndef BW_H
+#define BW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BW_ABI_VERSION 1
+
+typedef int bw_status;
+#define BW_OK 0
+#define BW_ERR_INVALID_ARG 1
+#define BW_ERR_UNSUPPORTED_SHAPE 2
+#define BW_ERR_CUDA 3
+#define BW_ERR_DEVICE_TIMEOUT 4
+#define BW_ERR_BAD_PAGE_INDEX 5
+
+/* bits of the device error word (first 4 bytes of a workspace) */
+#define BW_DEVERR_BAD_PAGE 1u
+#define BW_DEVERR_TIMEOUT 2u
+#define BW_DEVERR_BAD_TOKEN 4u
+#define BW_DEVERR_BAD_POS 8u      /* position outside the page table or the RoPE table */
+
+#define BW_FMT_Q4_0 0
+#define BW_FMT_NVFP4 1
+
+/* GEMV flags */
+#define BW_GEMV_RMSNORM 1u    /* prologue: each row of x -> rmsnorm(x) * gamma */
+#define BW_GEMV_RESIDUAL 2u   /* epilogue: y = residual + W x (residual may alias y) */
+#define BW_GEMV_SILU_GATE 4u  /* rows interleaved gate/up: y[m][i] = silu(g_i) * u_i, N/2 outputs */
+#define BW_GEMV_ARGMAX 8u     /* also argmax_out[m] = lowest index of max_n (W x)[m][n] */
+
+/* decode-step flags */
+#define BW_STEP_ADVANCE 1u    /* after the step: tokens_in <- tokens_out, pos += n_rows */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bw_status_string(bw_status s);
+/* BW_ABI_VERSION of the loaded library. */
+int bw_abi_version(void);
+
+/* ------------------------------------------------------------- workspace */
+
+/* Zero-fill `bytes` of workspace on `stream` (once, before first use). */
+bw_status bw_workspace_init(void *ws, size_t bytes, void *stream);
+/* Synchronize `stream`, then copy the device error word of `ws` into
+ * *err_out (host) and clear it on the device. */
+bw_status bw_read_error(void *ws, uint32_t *err_out, void *stream);
+
+/* ---------------------------------------------------------------- layout */
+
+/* Canonical Q4_0 (N x K/32 blocks of 18 bytes) -> GPU layout.
+ * blocks_up != NULL: gate/up interleave of two N x K matrices; the output
+ * then has 2N rows.  q_out: [rows][K/2] bytes; s_out: [rows/8][K/32][8] fp16.
+ * Requires K % 32 == 0, rows % 8 == 0 (N % 4 == 0 for gate/up). */
+bw_status bw_repack_q4_0(const void *blocks, const void *blocks_up, int N, int K,
+                         void *q_out, void *s_out, void *stream);
+/* Canonical NVFP4 (codes [N][K/2], E4M3 scales [N][K/16]) -> GPU layout;
+ * q_up/s_up != NULL: gate/up interleave as above.  s_out: [rows/8][K/32][8][2]. */
+bw_status bw_repack_nvfp4(const void *q, const void *s, const void *q_up, const void *s_up,
+                          int N, int K, void *q_out, void *s_out, void *stream);
+
+/* ------------------------------------------------------------------ GEMV */
+
+/* y[m][n] = sum_k W[n][k] x'[m][k] for m < M, with x' = x or, with
+ * BW_GEMV_RMSNORM, x' = x * rsqrt(mean(x^2) + eps) * gamma.
+ *   x: fp32 [M][K]; y: fp32 [M][N] ([M][N/2] with SILU_GATE; may be NULL
+ *   with ARGMAX); residual: fp32 [M][N] or NULL; argmax_out: int32 [M] or NULL;
+ *   gamma: fp32 [K] or NULL.
+ * Shapes: N % 8 == 0, K % 32 == 0, 1 <= M <= 8.  Pointers 16-byte aligned.
+ * ws must hold bw_gemv_workspace_bytes(N, K, M, flags). */
+bw_status bw_gemv_q4_0(const void *w_q, const void *w_d, int N, int K,
+                       const float *x, int M, const float *gamma, float eps,
+                       const float *residual, float *y, int32_t *argmax_out,
+                       unsigned flags, void *ws, size_t ws_bytes, void *stream);
+/* Same contract; ts is the tensor scale of all rows, or of the gate rows
+ * with SILU_GATE, in which case ts_up scales the up rows. */
+bw_status bw_gemv_nvfp4(const void *w_q, const void *w_s, float ts, float ts_up, int N, int K,
+                        const float *x, int M, const float *gamma, float eps,
+                        const float *residual, float *y, int32_t *argmax_out,
+                        unsigned flags, void *ws, size_t ws_bytes, void *stream);
+size_t bw_gemv_workspace_bytes(int N, int K, int M, unsigned flags);
+
+/* -------------------------------------------------------- small kernels */
+
+/* x [M][H] fp32 in place: x += add (if add != NULL); y = rmsnorm(x) * gamma,
+ * written as fp32 (y_fp16 == 0) or fp16 (y_fp16 != 0) [M][H].  y may be NULL. */
+bw_status bw_rmsnorm_fused(float *x, const float *add, const float *gamma, int M, int H,
+                           float eps, void *y, int y_fp16, void *stream);
+
+/* x[m][:] = dequantized row tokens[m] of the embedding matrix (GPU layout).
+ * A token outside [0, V) sets BW_DEVERR_BAD_TOKEN and writes zeros. */
+bw_status bw_embed(int fmt, const void *e_q, const void *e_s, float ts, int V, int H,
+                   const int32_t *tokens, int M, float *x, void *ws, void *stream);
+
+/* cos/sin of pos * theta^(-2i/hd), evaluated in fp64 and rounded to fp32:
+ * [max_pos][hd/2] each. */
+bw_status bw_rope_table(float theta, int hd, int max_pos, float *cos_out, float *sin_out,
+                        void *stream);
+
+/* idx_out[m] = lowest index of the maximum of logits[m][0..V); margin_out[m]
+ * (optional) = max - second largest value. */
+bw_status bw_argmax(const float *logits, int M, int V, int32_t *idx_out, float *margin_out,
+                    void *stream);
+
+/* ------------------------------------------------------------- attention */
+
+/* Paged GQA decode attention for B sequences x n_rows consecutive query rows.
+ *   qkv: fp32 [B*n_rows][(nq + 2 nkv) hd] raw projections (q heads, k heads,
+ *        v heads); row b*n_rows + r sits at position pos[b] + r.
+ *   rope_cos/rope_sin: fp32 [rope_max_pos][hd/2] (bw_rope_table).
+ *   k_pool/v_pool: fp16 [n_pages][nkv][16][hd] of this layer.  The RoPE'd k
+ *        and the v of every row are rounded to fp16 and written at logical
+ *        position pos[b] + r (physical page page_table[b][pos/16], slot pos%16).
+ *   page_table: int32 [B][max_pages]; pos: int32 [B].
+ *   out: fp32 [B*n_rows][nq hd]; row r of sequence b attends over positions
+ *        0 .. pos[b] + r (causal within the rows); query head h reads kv head
+ *        h / (nq / nkv); scale 1/sqrt(hd); fp32 softmax.
+ * Requires hd == 128 or 64, nq % nkv == 0, (nq/nkv) * n_rows <= 32.
+ * A page-table entry outside [0, n_pages) sets BW_DEVERR_BAD_PAGE; the page
+ * is neither read nor written. */
+bw_status bw_paged_attn_decode(const float *qkv, const float *rope_cos, const float *rope_sin,
+                               int rope_max_pos, void *k_pool, void *v_pool,
+                               const int32_t *page_table, int max_pages, int n_pages,
+                               const int32_t *pos, int B, int n_rows, int nq, int nkv, int hd,
+                               float *out, void *ws, size_t ws_bytes, void *stream);
+size_t bw_attn_workspace_bytes(int B, int n_rows, int nq, int nkv, int hd, int max_pages);
+
+/* ------------------------------------------------------------ whole step */
+
+/* (bw_qweight, bw_layer, bw_model, bw_kv are declared below.) */
+struct bw_model;
+struct bw_layer;
+
+typedef struct bw_qweight {
+    int fmt;         /* BW_FMT_Q4_0 or BW_FMT_NVFP4 */
+    int N, K;        /* rows in the GPU layout (2F for gate/up) and columns */
+    const void *q;   /* GPU-layout nibbles */
+    const void *s;   /* GPU-layout scales */
+    float ts;        /* NVFP4 tensor scale (gate half for gate/up) */
+    float ts_up;     /* NVFP4 tensor scale of the up half (gate/up); else ignored */
+} bw_qweight;
+
+typedef struct bw_layer {
+    const float *attn_norm;  /* gamma [H] */
+    const float *ffn_norm;   /* gamma [H] */
+    bw_qweight wqkv;         /* [(nq + 2 nkv) hd][H] */
+    bw_qweight wo;           /* [H][nq hd] */
+    bw_qweight wgu;          /* dense: gate/up interleaved [2F][H] */
+    bw_qweight wd;           /* dense: [H][F] */
+    /* MoE (n_experts > 0) */
+    const float *router;     /* fp32 [E][H] */
+    const void *egu_q, *egu_s;  /* experts' gate/up, E matrices [2Fe][H] back to back */
+    const void *ed_q, *ed_s;    /* experts' down, E matrices [H][Fe] back to back */
+    const float *egu_ts;     /* fp32 [E][2]: gate and up tensor scales per expert */
+    const float *ed_ts;      /* fp32 [E] */
+    bw_qweight sgu, sd;      /* shared expert (weight 1) */
+} bw_layer;
+
+typedef struct bw_model {
+    int L, H, nq, nkv, hd, F, V;
+    int n_experts, topk, F_exp;  /* n_experts == 0: dense FFN */
+    float eps;
+    bw_qweight embed;            /* [V][H] */
+    bw_qweight lm_head;          /* [V][H] */
+    const float *final_norm;     /* [H] */
+    const float *rope_cos, *rope_sin;
+    int rope_max_pos;
+    const bw_layer *layers;      /* HOST array of L layers */
+} bw_model;
+
+typedef struct bw_kv {
+    void *const *k;              /* HOST array of L device pointers: fp16 [n_pages][nkv][16][hd] */
+    void *const *v;
+    int n_pages;
+    int max_pages;
+    const int32_t *page_table;   /* device int32 [B][max_pages] */
+} bw_kv;
+
+/* Mixture-of-experts feed-forward block of one layer for R token rows, in place:
+ *   y = rmsnorm(x) * ffn_norm;  r = Wr y (router, fp32 [E][H]);
+ *   top-k experts by logit (ties: the lower index); w = softmax over the k
+ *   selected logits;  x += sum_k w_k FFN_{e_k}(y) + FFN_shared(y), where
+ *   FFN(y) = Wd (silu(Wg y) * (Wu y)).
+ *   x: fp32 [R][H]; topk_idx: int32 [R][topk] and topk_w: fp32 [R][topk]
+ *   (optional outputs, in selection order).
+ * Expert weights: m->layers-style bw_layer fields egu_* / ed_* (E matrices
+ * back to back in the GPU layout) and sgu / sd (shared expert).
+ * ws must hold bw_moe_workspace_bytes(m, R). */
+bw_status bw_moe_route_gemv(const struct bw_model *m, const struct bw_layer *ly, float *x, int R,
+                            int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream);
+size_t bw_moe_workspace_bytes(const struct bw_model *m, int R);
+
+/* One greedy decode step for B sequences of n_rows tokens each.
+ *   tokens_in: int32 [B*n_rows]; pos: int32 [B] (position of each sequence's
+ *   first row); tokens_out: int32 [B*n_rows] (argmax after each row);
+ *   logits: fp32 [B*n_rows][V] or NULL.
+ * flags: BW_STEP_ADVANCE (n_rows == 1 only).
+ * ws must hold bw_decode_workspace_bytes(m, kv, B, n_rows). */
+bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in, int32_t *pos,
+                         int B, int n_rows, int32_t *tokens_out, float *logits, unsigned flags,
+                         void *ws, size_t ws_bytes, void *stream);
+size_t bw_decode_workspace_bytes(const bw_model *m, const bw_kv *kv, int B, int n_rows);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BW_H */

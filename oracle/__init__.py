@@ -255,18 +255,32 @@ class Model:
                         vec(m.final_norm), C.cast(layers, C.c_void_p).value)
         self._keep = keep
 
+    def sliced(self, l0: int, l1: int) -> "ModelC":
+        """A model struct over layers [l0, l1) of this one (same memory)."""
+        c = ModelC.from_buffer_copy(self.c)
+        c.L = l1 - l0
+        c.layers = self.c.layers + l0 * C.sizeof(LayerC)
+        return c
+
 
 def decode_token(model: Model, kv: KV, b: int, token: int, pos: int, moe_dense: bool = False,
-                 want_logits: bool = True, want_hidden: bool = False):
+                 want_logits: bool = True, want_hidden: bool = False, layers=None):
     """One greedy token of sequence b at position pos.  Writes K/V of pos into kv.
+    layers=(l0, l1) runs only those layers (a bounded sample of the step).
     Returns dict(token, margin, logits, hidden, moe_idx)."""
     cfg = model.cfg
-    L = model.c.L
+    mc, kc = model.c, kv.c
+    if layers is not None:
+        mc = model.sliced(*layers)
+        kc = KVC.from_buffer_copy(kv.c)
+        kc.k = kv.c.k + layers[0] * C.sizeof(C.c_void_p)
+        kc.v = kv.c.v + layers[0] * C.sizeof(C.c_void_p)
+    L = mc.L
     logits = np.empty(cfg.V, np.float32) if want_logits else None
     hidden = np.empty((L + 1, cfg.H), np.float32) if want_hidden else None
     moe_idx = np.empty((L, cfg.topk), np.int32) if cfg.n_experts else None
     margin = np.zeros(1, np.float32)
-    tok = lib().or_decode_token(C.byref(model.c), C.byref(kv.c), b, int(token), int(pos),
+    tok = lib().or_decode_token(C.byref(mc), C.byref(kc), b, int(token), int(pos),
                                 int(moe_dense),
                                 None if logits is None else _ptr(logits),
                                 None if hidden is None else _ptr(hidden),

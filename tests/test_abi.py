@@ -1,0 +1,91 @@
+"""CPU-side checks of the C ABI: the library builds for sm_100a, loads, exports
+every symbol include/bw.h declares, and rejects bad arguments on the host
+before any launch (no kernel runs here)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from token_decode_b200 import build
+    build.build()
+    from token_decode_b200 import bw
+    return bw.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bw.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bw_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for must in ("bw_gemv_q4_0", "bw_gemv_nvfp4", "bw_rmsnorm_fused", "bw_paged_attn_decode",
+                 "bw_moe_route_gemv", "bw_argmax", "bw_decode_step"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from token_decode_b200 import bw
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert set(_declared()) == set(bw.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", bw.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (bw_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(_declared()) <= exported
+
+
+def test_library_is_built_for_sm_100a(lib):
+    from token_decode_b200 import bw
+    out = subprocess.run(["cuobjdump", "--list-elf", bw.LIB_PATH], capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+
+
+def test_status_strings_and_version(lib):
+    from token_decode_b200 import bw
+    assert lib.bw_abi_version() == 1
+    assert bw.string(0) == "ok"
+    assert "page" in bw.string(5)
+    assert bw.string(99) == "unknown status"
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    p = C.c_void_p
+    fake = p(4096)   # never dereferenced: validation fails first
+    # null weights
+    assert lib.bw_gemv_q4_0(None, fake, 64, 64, fake, 1, None, 1e-6, None, fake, None, 0, fake,
+                            1 << 20, None) == 1
+    # N not a multiple of 8
+    assert lib.bw_gemv_q4_0(fake, fake, 60, 64, fake, 1, None, 1e-6, None, fake, None, 0, fake,
+                            1 << 20, None) == 2
+    # K not a multiple of 32
+    assert lib.bw_gemv_nvfp4(fake, fake, 1.0, 1.0, 64, 48, fake, 1, None, 1e-6, None, fake, None,
+                             0, fake, 1 << 20, None) == 2
+    # RMSNORM without gamma
+    assert lib.bw_gemv_q4_0(fake, fake, 64, 64, fake, 1, None, 1e-6, None, fake, None, 1, fake,
+                            1 << 20, None) == 1
+    # unaligned weights
+    assert lib.bw_gemv_q4_0(p(4097), fake, 64, 64, fake, 1, None, 1e-6, None, fake, None, 0, fake,
+                            1 << 20, None) == 1
+    # attention: unsupported head dim, too many query rows per kv head
+    args = [fake, fake, fake, 128, fake, fake, fake, 8, 8, fake, 1, 1, 8, 2, 96, fake, fake, 1 << 24, None]
+    assert lib.bw_paged_attn_decode(*args) == 2
+    args[11], args[12], args[13], args[14] = 4, 64, 2, 128    # G * n_rows = 128 > 32
+    assert lib.bw_paged_attn_decode(*args) == 2
+    # repack: rows not a multiple of 8
+    assert lib.bw_repack_q4_0(fake, None, 12, 64, fake, fake, None) == 2
+    assert lib.bw_rope_table(C.c_float(-1.0), 64, 16, fake, fake, None) == 1
+    assert lib.bw_decode_step(None, None, None, None, 1, 1, None, None, 0, None, 0, None) == 1
+
+
+def test_workspace_queries_are_host_only(lib):
+    z = lib.bw_gemv_workspace_bytes(4608, 3584, 1, 0)
+    assert z >= 1 << 18
+    assert lib.bw_attn_workspace_bytes(1, 1, 28, 4, 128, 160) > 1 << 18

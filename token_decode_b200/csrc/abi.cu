@@ -1,0 +1,70 @@
+// abi.cu -- status strings, device properties, workspace helpers of libbw.
+#include <stdio.h>
+
+#include "bw_common.cuh"
+
+namespace bw {
+
+int sm_count() {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+bw_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? BW_OK : BW_ERR_CUDA;
+}
+
+}  // namespace bw
+
+extern "C" {
+
+const char *bw_status_string(bw_status s) {
+    switch (s) {
+        case BW_OK: return "ok";
+        case BW_ERR_INVALID_ARG: return "invalid argument";
+        case BW_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case BW_ERR_CUDA: return "CUDA error";
+        case BW_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+        case BW_ERR_BAD_PAGE_INDEX: return "page-table entry outside the KV pool";
+        default: return "unknown status";
+    }
+}
+
+int bw_abi_version(void) { return BW_ABI_VERSION; }
+
+bw_status bw_workspace_init(void *ws, size_t bytes, void *stream) {
+    if (!ws || bytes < BW_WS_HDR_BYTES) return BW_ERR_INVALID_ARG;
+    if (cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BW_ERR_CUDA;
+    }
+    return BW_OK;
+}
+
+bw_status bw_read_error(void *ws, uint32_t *err_out, void *stream) {
+    if (!ws || !err_out) return BW_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BW_ERR_CUDA;
+    }
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemset(ws, 0, sizeof(v)) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BW_ERR_CUDA;
+    }
+    *err_out = v;
+    return BW_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,128 @@
+"""Device-side model and KV cache for the decode step: argument marshalling
+for bw_decode_step.
+
+Takes the seeded inputs (canonical weight bytes already on the GPU), converts
+every matrix to the GPU layout with the library's repack kernels, builds the
+RoPE tables with bw_rope_table, and fills the bw_model / bw_kv descriptors.
+All arithmetic happens in libbw.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import torch
+
+from . import bw
+from .synth import FMT_Q4_0, FMT_NVFP4, PAGE_TOKENS
+
+
+def _gpu_layout(m, up=None):
+    """QMat (+ matching up-projection) -> (bw.QWeight, [tensors to keep alive])."""
+    rows = m.N * (2 if up is not None else 1)
+    q = torch.empty((rows, m.K // 2), dtype=torch.uint8, device=m.q.device)
+    s = torch.empty((rows * (m.K // 16),), dtype=torch.uint8, device=m.q.device)
+    if m.fmt == FMT_Q4_0:
+        bw.repack_q4_0(m.q, m.N, m.K, q, s, blocks_up=None if up is None else up.q)
+    else:
+        bw.repack_nvfp4(m.q, m.s, m.N, m.K, q, s, q_up=None if up is None else up.q,
+                        s_up=None if up is None else up.s)
+    qw = bw.QWeight(m.fmt, rows, m.K, q.data_ptr(), s.data_ptr(), m.ts,
+                    up.ts if up is not None else m.ts)
+    return qw, [q, s]
+
+
+class DeviceModel:
+    """GPU-layout weights + descriptors of one model (see include/bw.h)."""
+
+    def __init__(self, model, max_pos: int):
+        cfg = model.cfg
+        self.cfg = cfg
+        keep = []
+
+        def qw(m, up=None):
+            w, t = _gpu_layout(m, up)
+            keep.extend(t)
+            return w
+
+        L = len(model.layers)
+        self.layers = (bw.Layer * L)()
+        for l, ly in enumerate(model.layers):
+            c = self.layers[l]
+            c.attn_norm = ly.attn_norm.data_ptr()
+            c.ffn_norm = ly.ffn_norm.data_ptr()
+            keep += [ly.attn_norm, ly.ffn_norm]
+            c.wqkv = qw(ly.wqkv)
+            c.wo = qw(ly.wo)
+            if cfg.n_experts == 0:
+                c.wgu = qw(ly.wg, ly.wu)
+                c.wd = qw(ly.wd)
+            else:
+                self._moe_layer(c, ly, keep)
+        self.cos = torch.empty((max_pos, cfg.hd // 2), dtype=torch.float32, device="cuda")
+        self.sin = torch.empty_like(self.cos)
+        bw.rope_table(cfg.theta, cfg.hd, max_pos, self.cos, self.sin)
+        keep += [model.final_norm]
+        self.c = bw.Model(L, cfg.H, cfg.nq, cfg.nkv, cfg.hd, cfg.F, cfg.V, cfg.n_experts, cfg.topk,
+                          cfg.F_exp, cfg.eps, qw(model.embed), qw(model.lm_head),
+                          model.final_norm.data_ptr(), self.cos.data_ptr(), self.sin.data_ptr(),
+                          max_pos, C.cast(self.layers, C.c_void_p).value)
+        self._keep = keep
+        self.weight_bytes = sum(t.numel() * t.element_size() for t in keep)
+
+    def _moe_layer(self, c, ly, keep):
+        E, Fe, H = ly.eg.E, ly.eg.N, ly.eg.K
+        rows = 2 * Fe
+        gq = torch.empty((E, rows, H // 2), dtype=torch.uint8, device="cuda")
+        gs = torch.empty((E, rows * (H // 16)), dtype=torch.uint8, device="cuda")
+        dq = torch.empty((E, H, Fe // 2), dtype=torch.uint8, device="cuda")
+        ds = torch.empty((E, H * (Fe // 16)), dtype=torch.uint8, device="cuda")
+        for e in range(E):
+            g, u, d = ly.eg.mat(e), ly.eu.mat(e), ly.ed.mat(e)
+            if g.fmt == FMT_Q4_0:
+                bw.repack_q4_0(g.q, Fe, H, gq[e], gs[e], blocks_up=u.q)
+                bw.repack_q4_0(d.q, H, Fe, dq[e], ds[e])
+            else:
+                bw.repack_nvfp4(g.q, g.s, Fe, H, gq[e], gs[e], q_up=u.q, s_up=u.s)
+                bw.repack_nvfp4(d.q, d.s, H, Fe, dq[e], ds[e])
+        gts = torch.stack([ly.eg.ts, ly.eu.ts], dim=1).contiguous().to("cuda")
+        dts = ly.ed.ts.contiguous().to("cuda")
+        c.router = ly.router.data_ptr()
+        c.egu_q, c.egu_s, c.ed_q, c.ed_s = gq.data_ptr(), gs.data_ptr(), dq.data_ptr(), ds.data_ptr()
+        c.egu_ts, c.ed_ts = gts.data_ptr(), dts.data_ptr()
+        keep += [ly.router, gq, gs, dq, ds, gts, dts]
+        w, t = _gpu_layout(ly.sg, ly.su)
+        c.sgu = w
+        keep += t
+        w, t = _gpu_layout(ly.sd)
+        c.sd = w
+        keep += t
+
+
+class DeviceKV:
+    """The paged fp16 KV pools (one per layer) + page table as a bw_kv."""
+
+    def __init__(self, kv):
+        self.k = kv.k
+        self.v = kv.v
+        self.page_table = kv.page_table.to(torch.int32).contiguous()
+        L = len(kv.k)
+        self._kp = (C.c_void_p * L)(*[t.data_ptr() for t in kv.k])
+        self._vp = (C.c_void_p * L)(*[t.data_ptr() for t in kv.v])
+        self.c = bw.KV(C.cast(self._kp, C.c_void_p).value, C.cast(self._vp, C.c_void_p).value,
+                       int(kv.n_pages), int(self.page_table.shape[1]), self.page_table.data_ptr())
+
+
+class Decoder:
+    """Owns a workspace and runs bw_decode_step for B sequences x n_rows."""
+
+    def __init__(self, dm: DeviceModel, dkv: DeviceKV, B: int, n_rows: int = 1):
+        self.dm, self.dkv, self.B, self.n_rows = dm, dkv, B, n_rows
+        self.ws = bw.workspace(bw.decode_workspace_bytes(dm.c, dkv.c, B, n_rows))
+        self.tokens_in = torch.zeros(B * n_rows, dtype=torch.int32, device="cuda")
+        self.tokens_out = torch.zeros(B * n_rows, dtype=torch.int32, device="cuda")
+        self.pos = torch.zeros(B, dtype=torch.int32, device="cuda")
+
+    def step(self, logits=None, advance=False, stream=None):
+        bw.decode_step(self.dm.c, self.dkv.c, self.tokens_in, self.pos, self.B, self.n_rows,
+                       self.tokens_out, self.ws, logits=logits,
+                       flags=bw.STEP_ADVANCE if advance else 0, stream=stream)
