@@ -165,12 +165,12 @@ def run_ours(args):
         return out, p
 
     def run(ops):
-        for op in ops:
-            if op == "reset":
-                with torch.cuda.stream(stream):
+        with torch.cuda.stream(stream):
+            for op in ops:
+                if op == "reset":
                     reset()
-            else:
-                graph_for(op).replay()
+                else:
+                    graph_for(op).replay()
 
     torch.cuda.synchronize()
     reset()

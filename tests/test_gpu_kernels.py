@@ -126,7 +126,9 @@ def test_gemv_one_hot_columns_bit_exact(fmt, shape):
     y, _ = _gemv(m, x, 4)
     deq = oracle.dequant(m)
     for i, c in enumerate(cols):
-        assert np.array_equal(bits(y[i]), bits(deq[:, c])), (i, c)
+        # exact equality of values: a zero weight may come out as +0 where the
+        # plain product d*(q-8) gives -0 (same value, different sign bit)
+        assert np.array_equal(y[i], deq[:, c]), (i, c)
 
 
 @pytest.mark.parametrize("fmt", [synth.FMT_Q4_0, synth.FMT_NVFP4])
@@ -139,9 +141,12 @@ def test_gemv_matches_oracle(fmt, shape, M):
     y, _ = _gemv(m, x, M)
     om = oracle.QMat(m)
     xh = x.cpu().numpy()
+    # both sides accumulate K fp32 products in different orders: a normwise
+    # difference of a few sqrt(K) * 2^-24 is rounding, nothing more
+    tol = 2e-7 * np.sqrt(K)
     for r in range(M):
         want = oracle.matvec(om, xh[r])
-        assert rel_err(y[r], want) < 2e-6, rel_err(y[r], want)
+        assert rel_err(y[r], want) < tol, rel_err(y[r], want)
 
 
 @pytest.mark.parametrize("fmt", [synth.FMT_Q4_0, synth.FMT_NVFP4])
@@ -185,7 +190,7 @@ def test_gemv_argmax_lm_head(fmt):
     for r in range(M):
         yn = oracle.rmsnorm(x[r].cpu().numpy(), gamma.cpu().numpy(), 1e-6)
         want = oracle.matvec(om, yn)
-        assert rel_err(y[r], want) < 2e-6
+        assert rel_err(y[r], want) < 2e-7 * np.sqrt(H)
         i, margin = oracle.argmax(want)
         # the GPU's argmax is exact over its own logits
         assert am[r] == int(np.argmax(y[r]))

@@ -288,25 +288,43 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    // combine the splits: gather every split's (max, sum) into shared memory
+    // (the K/V tile buffers are free now), then one coefficient per (split,
+    // query), then each thread sums its output dim over the splits in order.
+    const int nsq = p.n_split * p.Q;
+    float *cm = reinterpret_cast<float *>(att_smem);      // [n_split][Q] maxima -> coefficients
+    float *cl = cm + nsq;                                  // [n_split][Q] sums
+    const size_t gbase = grp * p.n_split * p.Q;
+    for (int i = tid; i < nsq; i += ATT_THREADS) {
+        cm[i] = ld_cg(p.part_m + gbase + i);
+        cl[i] = ld_cg(p.part_l + gbase + i);
+    }
+    __syncthreads();
+    if (tid < p.Q) {
+        float M = -INFINITY;
+        for (int s2 = 0; s2 < p.n_split; s2++) M = fmaxf(M, cm[s2 * p.Q + tid]);
+        float L = 0.0f;
+        for (int s2 = 0; s2 < p.n_split; s2++) {
+            const float ms = cm[s2 * p.Q + tid];
+            const float w = (ms == -INFINITY) ? 0.0f : expf(ms - M);
+            L = fmaf(cl[s2 * p.Q + tid], w, L);
+            cm[s2 * p.Q + tid] = w;
+        }
+        s_l[tid] = L;
+    }
+    __syncthreads();
 #pragma unroll
     for (int i = 0; i < NACC; i++) {
         const int qi = oq0 + i * QSTEP;
         if (qi >= p.Q) continue;
-        float M = -INFINITY;
-        for (int s2 = 0; s2 < p.n_split; s2++)
-            M = fmaxf(M, ld_cg(p.part_m + (grp * p.n_split + s2) * p.Q + qi));
-        float L = 0.0f, O = 0.0f;
-        for (int s2 = 0; s2 < p.n_split; s2++) {
-            const size_t pi = (grp * p.n_split + s2) * p.Q + qi;
-            const float ms = ld_cg(p.part_m + pi);
-            if (ms == -INFINITY) continue;
-            const float w = expf(ms - M);
-            L = fmaf(ld_cg(p.part_l + pi), w, L);
-            O = fmaf(ld_cg(p.part_o + pi * HD + od), w, O);
-        }
+        float O = 0.0f;
+        const float *po = p.part_o + (gbase + qi) * HD + od;
+        const size_t sstride = static_cast<size_t>(p.Q) * HD;
+#pragma unroll 8
+        for (int s2 = 0; s2 < p.n_split; s2++) O = fmaf(ld_cg(po + s2 * sstride), cm[s2 * p.Q + qi], O);
         const int r = qi / p.G, g = qi - r * p.G;
         p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
-              static_cast<size_t>(kvh * p.G + g) * HD + od] = O / L;
+              static_cast<size_t>(kvh * p.G + g) * HD + od] = O / s_l[qi];
     }
     if (tid == 0) p.cnt[grp] = 0u;
 }
@@ -328,11 +346,14 @@ static bw_status attn_go(dim3 grid, cudaStream_t st, const AttnParams &p) {
     return launch_pdl(attn_kernel<HD, QMAX>, grid, dim3(ATT_THREADS), smem, st, p);
 }
 
+// Splits per (sequence, kv head): enough CTAs to cover every SM about once,
+// at least ~4 pages per split, at most 64 splits (the combine keeps
+// n_split * 32 floats of statistics in shared memory).
 static int attn_splits(int B, int nkv, int max_pages) {
     const int groups = B * nkv;
-    int ns = (2 * sm_count() + groups - 1) / groups;
-    ns = max(1, min(ns, max_pages));
-    ns = min(ns, 256);
+    int ns = (sm_count() + groups - 1) / groups;
+    ns = max(1, min(ns, (max_pages + 3) / 4));
+    ns = min(ns, 64);
     return ns;
 }
 
