@@ -142,6 +142,29 @@ bw_status bw_gemv_nvfp4(const void *w_q, const void *w_s, float ts, float ts_up,
                         unsigned flags, void *ws, size_t ws_bytes, void *stream);
 size_t bw_gemv_workspace_bytes(int N, int K, int M, unsigned flags);
 
+/* Size of the fixed device scratch behind bw_gemv_q4_0_noalloc (1 MiB). */
+#define BW_GEMV_NOALLOC_SCRATCH_BYTES (1u << 20)
+/* bw_gemv_q4_0 without a workspace argument, for callers that cannot allocate
+ * device memory (a host framework that owns every allocation and passes a
+ * library only inputs and outputs, or a path where cudaMalloc's implicit
+ * synchronization is not acceptable).  No counterpart in the pages: a
+ * library-interface addition.
+ *   Same arguments, layout and results as bw_gemv_q4_0.  The scratch is a
+ *   file-scope __device__ array of BW_GEMV_NOALLOC_SCRATCH_BYTES that every
+ *   GPU loading the library holds until process exit; nothing is allocated
+ *   or freed (it issues one cudaMemsetAsync to clear its counters).
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   All calls share the one array: calls that overlap on the GPU (other
+ *   streams, other host threads) race and must be serialized by the caller.
+ *   A shape whose split-K scratch exceeds the array returns
+ *   BW_ERR_UNSUPPORTED_SHAPE without launching. */
+bw_status bw_gemv_q4_0_noalloc(const void *w_q, const void *w_d, int N, int K,
+                               const float *x, int M, const float *gamma, float eps,
+                               const float *residual, float *y, int32_t *argmax_out,
+                               unsigned flags, void *stream);
+
 /* -------------------------------------------------------- small kernels */
 
 /* x [M][H] fp32 in place: x += add (if add != NULL); y = rmsnorm(x) * gamma,

@@ -25,7 +25,7 @@ STEP_ADVANCE = 1
 EXPORTS = (
     "bw_status_string", "bw_abi_version", "bw_workspace_init", "bw_read_error",
     "bw_repack_q4_0", "bw_repack_nvfp4", "bw_gemv_q4_0", "bw_gemv_nvfp4",
-    "bw_gemv_workspace_bytes", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
+    "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
     "bw_paged_attn_decode", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
     "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes",
 )
@@ -84,6 +84,7 @@ def lib() -> C.CDLL:
             "bw_gemv_q4_0": (i, [p, p, i, i, p, i, p, f, p, p, p, u, p, z, p]),
             "bw_gemv_nvfp4": (i, [p, p, f, f, i, i, p, i, p, f, p, p, p, u, p, z, p]),
             "bw_gemv_workspace_bytes": (z, [i, i, i, u]),
+            "bw_gemv_q4_0_noalloc": (i, [p, p, i, i, p, i, p, f, p, p, p, u, p]),
             "bw_rmsnorm_fused": (i, [p, p, p, i, i, f, p, i, p]),
             "bw_embed": (i, [i, p, p, f, i, i, p, i, p, p, p]),
             "bw_rope_table": (i, [f, i, i, p, p, p]),
@@ -162,6 +163,15 @@ def gemv_q4_0(w_q, w_d, N, K, x, M, y, ws, gamma=None, eps=1e-6, residual=None, 
     _check(lib().bw_gemv_q4_0(_ptr(w_q), _ptr(w_d), N, K, _ptr(x), M, _ptr(gamma), eps,
                               _ptr(residual), _ptr(y), _ptr(argmax_out), flags, _ptr(ws),
                               ws.numel(), _stream(stream)), "bw_gemv_q4_0")
+
+
+def gemv_q4_0_noalloc(w_q, w_d, N, K, x, M, y, gamma=None, eps=1e-6, residual=None,
+                      argmax_out=None, flags=0, stream=None):
+    """bw_gemv_q4_0 with the library's fixed device scratch instead of a workspace,
+    for callers that cannot allocate device memory."""
+    _check(lib().bw_gemv_q4_0_noalloc(_ptr(w_q), _ptr(w_d), N, K, _ptr(x), M, _ptr(gamma), eps,
+                                      _ptr(residual), _ptr(y), _ptr(argmax_out), flags,
+                                      _stream(stream)), "bw_gemv_q4_0_noalloc")
 
 
 def gemv_nvfp4(w_q, w_s, ts, N, K, x, M, y, ws, ts_up=None, gamma=None, eps=1e-6, residual=None,
