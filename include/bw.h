@@ -48,14 +48,20 @@
  *    leave their counters at zero on return, so the same workspace serves
  *    any number of later calls and CUDA-graph replays on one stream.  Calls
  *    sharing a workspace must not run concurrently.
- *  - Weights live in the GPU layout written by bw_repack_q4_0 /
- *    bw_repack_nvfp4 from the canonical (file) layout:
- *      q : nibbles [N][K/2] bytes, row-major (per 32-element chunk the 16
- *          bytes keep the canonical nibble order of the format)
- *      s : per group of 8 rows and 32-element chunk, 16 bytes of scales,
- *          [N/8][K/32][8] fp16 d (Q4_0) or [N/8][K/32][8][2] E4M3 (NVFP4)
- *    Gate/up matrices are interleaved in groups of 4 rows (rows 8g..8g+3 are
- *    gate rows 4g..4g+3, rows 8g+4..8g+7 the matching up rows).
+ *  - Weights live in the tiled GPU layout written by bw_repack_q4_0 /
+ *    bw_repack_nvfp4 from the canonical (file) layout.  W[N][K] is cut into
+ *    tiles of 128 rows x 512 columns (N padded to a multiple of 128 rows and
+ *    K to a multiple of 512 columns, with zeros); tiles follow each other in
+ *    (row block, column tile) order:
+ *      q : per tile 32 KB: row r at r*256 bytes, 32-column chunk c of that
+ *          row at +c*16 (the chunk's 16 code bytes in the canonical nibble
+ *          order of the format)
+ *      s : per tile 4 KB: 8-row group g at g*256 bytes, chunk c at +c*16:
+ *          the 8 rows' fp16 d (Q4_0) or 8 x 2 E4M3 block scales (NVFP4)
+ *    so every tile is two contiguous blocks (streamed with plain bulk
+ *    copies).  Sizes: bw_repack_bytes.  Gate/up matrices are interleaved in
+ *    groups of 4 rows (rows 8g..8g+3 are gate rows 4g..4g+3, rows 8g+4..8g+7
+ *    the matching up rows).
  */
 #ifndef BW_H
 #define BW_H
@@ -110,14 +116,18 @@ bw_status bw_read_error(void *ws, uint32_t *err_out, void *stream);
 
 /* ---------------------------------------------------------------- layout */
 
-/* Canonical Q4_0 (N x K/32 blocks of 18 bytes) -> GPU layout.
+/* Bytes of the tiled codes (*q_bytes) and scales (*s_bytes) of a matrix of
+ * `rows` rows (2N for gate/up) and K columns in the GPU layout. */
+bw_status bw_repack_bytes(int rows, int K, size_t *q_bytes, size_t *s_bytes);
+/* Canonical Q4_0 (N x K/32 blocks of 18 bytes) -> tiled GPU layout.
  * blocks_up != NULL: gate/up interleave of two N x K matrices; the output
- * then has 2N rows.  q_out: [rows][K/2] bytes; s_out: [rows/8][K/32][8] fp16.
- * Requires K % 32 == 0, rows % 8 == 0 (N % 4 == 0 for gate/up). */
+ * then has 2N rows.  q_out / s_out: bw_repack_bytes() each, 16-byte aligned
+ * (the padding is zero-filled).  Requires K % 32 == 0, rows % 8 == 0
+ * (N % 4 == 0 for gate/up). */
 bw_status bw_repack_q4_0(const void *blocks, const void *blocks_up, int N, int K,
                          void *q_out, void *s_out, void *stream);
-/* Canonical NVFP4 (codes [N][K/2], E4M3 scales [N][K/16]) -> GPU layout;
- * q_up/s_up != NULL: gate/up interleave as above.  s_out: [rows/8][K/32][8][2]. */
+/* Canonical NVFP4 (codes [N][K/2], E4M3 scales [N][K/16]) -> tiled GPU
+ * layout; q_up/s_up != NULL: gate/up interleave as above. */
 bw_status bw_repack_nvfp4(const void *q, const void *s, const void *q_up, const void *s_up,
                           int N, int K, void *q_out, void *s_out, void *stream);
 
@@ -172,7 +182,7 @@ bw_status bw_gemv_q4_0_noalloc(const void *w_q, const void *w_d, int N, int K,
 bw_status bw_rmsnorm_fused(float *x, const float *add, const float *gamma, int M, int H,
                            float eps, void *y, int y_fp16, void *stream);
 
-/* x[m][:] = dequantized row tokens[m] of the embedding matrix (GPU layout).
+/* x[m][:] = dequantized row tokens[m] of the embedding matrix (tiled GPU layout).
  * A token outside [0, V) sets BW_DEVERR_BAD_TOKEN and writes zeros. */
 bw_status bw_embed(int fmt, const void *e_q, const void *e_s, float ts, int V, int H,
                    const int32_t *tokens, int M, float *x, void *ws, void *stream);

@@ -88,4 +88,4 @@ def test_host_validation_rejects_bad_arguments(lib):
 def test_workspace_queries_are_host_only(lib):
     z = lib.bw_gemv_workspace_bytes(4608, 3584, 1, 0)
     assert z >= 1 << 18
-    assert lib.bw_attn_workspace_bytes(1, 1, 28, 4, 128, 160) > 1 << 18
+    assert lib.bw_attn_workspace_bytes(1, 1, 28, 4, 128, 160) >= 1 << 18

@@ -61,10 +61,14 @@ def _run_steps(cfg, steps, seed=0, n_layers=None, B=None, check_kv=True):
         dec.pos += 1
     if check_kv:
         for l in range(len(okv.k)):
-            g = dkv.k[l].cpu().numpy().view(np.uint16)
-            # fp16 K/V of the decoded positions: identical except rare 1-ulp rounding flips
-            diff = np.abs(g.astype(np.int32) - okv.k[l].astype(np.int32))
-            assert np.max(diff) <= 2 and np.mean(diff == 0) > 0.999
+            for gpu_pool, ora_pool in ((dkv.k[l], okv.k[l]), (dkv.v[l], okv.v[l])):
+                g = gpu_pool.cpu().numpy().view(np.uint16)
+                # untouched slots are identical; written rows agree within the
+                # tolerance (fp16 rounding of values that differ by fp32 reordering)
+                assert np.mean(g == ora_pool) > 0.99
+                gv = g.view(np.float16).astype(np.float64)
+                ov = ora_pool.view(np.float16).astype(np.float64)
+                assert rel_err(gv, ov) < TOL
     return worst
 
 
@@ -81,6 +85,48 @@ def test_tiny_nvfp4_two_layers_batch2():
 def test_tiny_batch5_rows_above_gemv_block():
     cfg = synth.CONFIGS["tiny"].with_(B=5)
     _run_steps(cfg, 3)
+
+
+def _tiny_moe(**kw):
+    return synth.CONFIGS["tiny"].with_(name="tiny-moe", fmt=synth.FMT_NVFP4, F=0, n_experts=16,
+                                       topk=4, F_exp=64, B=4, L=2, **kw)
+
+
+def test_tiny_moe_decode_and_router_topk():
+    """MoE decode vs the oracle: logits, tokens and the selected experts."""
+    cfg = _tiny_moe()
+    model, kv, om, okv, dm, dkv = _setup(cfg, seed=3)
+    dec = runtime.Decoder(dm, dkv, cfg.B)
+    toks = synth.start_tokens(cfg, 3)[: cfg.B]
+    dec.tokens_in.copy_(toks)
+    dec.pos.fill_(cfg.ctx)
+    logits = torch.empty((cfg.B, cfg.V), device="cuda")
+    dec.step(logits=logits)
+    assert bw.read_error(dec.ws) == 0
+    for b in range(cfg.B):
+        res = oracle.decode_token(om, okv, b, int(toks[b]), cfg.ctx)
+        assert rel_err(logits[b].cpu().numpy(), res["logits"]) < TOL
+        if res["margin"] > MARGIN:
+            assert int(dec.tokens_out[b]) == res["token"]
+    # the routing kernel alone: same inputs -> same expert choice as the oracle's
+    x = torch.randn((cfg.B, cfg.H), device="cuda")
+    ly = dm.layers[0]
+    idx = torch.empty((cfg.B, cfg.topk), dtype=torch.int32, device="cuda")
+    wts = torch.empty((cfg.B, cfg.topk), device="cuda")
+    ws = bw.workspace(bw.moe_workspace_bytes(dm.c, cfg.B))
+    x0 = x.clone()
+    bw.moe_route_gemv(dm.c, ly, x, cfg.B, ws, topk_idx=idx, topk_w=wts)
+    torch.cuda.synchronize()
+    g = model.layers[0]
+    for b in range(cfg.B):
+        y = oracle.rmsnorm(x0[b].cpu().numpy(), g.ffn_norm.cpu().numpy(), cfg.eps)
+        r = (g.router.cpu().numpy().astype(np.float64) @ y.astype(np.float64))
+        order = np.lexsort((np.arange(cfg.n_experts), -r))
+        gap = r[order[cfg.topk - 1]] - r[order[cfg.topk]]
+        if gap > 1e-3:
+            assert sorted(idx[b].tolist()) == sorted(order[: cfg.topk].tolist())
+        assert abs(float(wts[b].sum()) - 1.0) < 1e-5
+    assert torch.isfinite(x).all() and not torch.equal(x, x0)
 
 
 def test_graph_replay_with_device_advance_matches_eager():
@@ -187,6 +233,13 @@ def test_7b_full_model_two_steps():
     """The benchmark workload itself: all 28 layers at full size, two steps."""
     cfg = synth.CONFIGS["7b"]
     _run_steps(cfg, 2, check_kv=False)
+
+
+@pytest.mark.slow
+def test_moe_full_size_layers_batch32():
+    """35B-A3B-class shapes (256 experts, top-8, shared expert), B = 32, two layers."""
+    cfg = synth.CONFIGS["moe"].with_(L=2)
+    _run_steps(cfg, 1, n_layers=2, check_kv=False)
 
 
 @pytest.mark.slow

@@ -24,7 +24,7 @@ STEP_ADVANCE = 1
 # every symbol include/bw.h declares (checked by the CPU test-suite)
 EXPORTS = (
     "bw_status_string", "bw_abi_version", "bw_workspace_init", "bw_read_error",
-    "bw_repack_q4_0", "bw_repack_nvfp4", "bw_gemv_q4_0", "bw_gemv_nvfp4",
+    "bw_repack_bytes", "bw_repack_q4_0", "bw_repack_nvfp4", "bw_gemv_q4_0", "bw_gemv_nvfp4",
     "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
     "bw_paged_attn_decode", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
     "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes",
@@ -79,6 +79,7 @@ def lib() -> C.CDLL:
             "bw_abi_version": (i, []),
             "bw_workspace_init": (i, [p, z, p]),
             "bw_read_error": (i, [p, p, p]),
+            "bw_repack_bytes": (i, [i, i, p, p]),
             "bw_repack_q4_0": (i, [p, p, i, i, p, p, p]),
             "bw_repack_nvfp4": (i, [p, p, p, p, i, i, p, p, p]),
             "bw_gemv_q4_0": (i, [p, p, i, i, p, i, p, f, p, p, p, u, p, z, p]),
@@ -142,6 +143,13 @@ def read_error(ws: torch.Tensor, stream=None) -> int:
     out = C.c_uint32(0)
     _check(lib().bw_read_error(_ptr(ws), C.byref(out), _stream(stream)), "bw_read_error")
     return out.value
+
+
+def repack_bytes(rows, K):
+    """(code bytes, scale bytes) of a `rows` x K matrix in the tiled GPU layout."""
+    qb, sb = C.c_size_t(0), C.c_size_t(0)
+    _check(lib().bw_repack_bytes(rows, K, C.byref(qb), C.byref(sb)), "bw_repack_bytes")
+    return qb.value, sb.value
 
 
 def repack_q4_0(blocks, N, K, q_out, s_out, blocks_up=None, stream=None):

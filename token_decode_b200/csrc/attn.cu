@@ -1,34 +1,41 @@
 // attn.cu -- paged fp16-KV GQA decode attention with fused RoPE and KV write
 // (sm_100a).
 //
-// One CTA per (split, kv head, sequence).  The split owns a contiguous range
-// of whole pages of the sequence's logical positions (split-KV, so a batch-1
-// step still fills every SM); it
+// One CTA per (split, kv head, sequence); the splits of one (sequence, kv
+// head) form a thread-block cluster.  Each CTA
 //   1. ropes the G = nq/nkv query heads of its kv head for each of the n_rows
 //      query rows (positions pos..pos+n_rows-1),
-//   2. if one of those positions falls in its range, ropes that row's k,
-//      rounds k and v to fp16 and writes them into the paged pool (the
-//      deep-dive page, section 6: positions map to physical pages through
-//      the page table; section 5, stage 4: the K draft rows of a verify pass
-//      share one cache, causally masked),
-//   3. streams its pages through shared memory in 32-token tiles (cp.async,
-//      double-buffered) with an online softmax in fp32,
-//   4. leaves (max, sum, unnormalised output) per query in the workspace; the
-//      last CTA of the (sequence, kv head) -- atomic counter, no waiting --
-//      combines the splits in split order, so results are deterministic and
-//      independent of the physical page order.
-// The K tile is stored with its 16-byte granules XOR-swizzled by token so the
-// lane-per-token score loop reads shared memory without bank conflicts.
+//   2. ropes the new rows' k, rounds k and v to fp16 and writes them into the
+//      paged pool when their position falls in its page range (the deep-dive
+//      page, section 6: logical positions map to physical pages through the
+//      page table; section 5, stage 4: the draft rows of a verify pass share
+//      one cache, causally masked),
+//   3. streams its pages into a ring of shared-memory stages with 1-D bulk
+//      copies (cp.async.bulk, completion on an mbarrier; two pages = 32
+//      tokens per stage) and runs an fp32 online softmax over them,
+//   4. combines the splits through distributed shared memory: after a
+//      cluster barrier every CTA reads the others' (max, sum, partial output)
+//      and writes a slice of the final output, in split order, so results are
+//      deterministic and independent of the physical page order.
+// K rows are read with a per-lane rotation of their 16-byte granules (lane t
+// starts at granule t), which keeps the linear bulk-copied layout free of
+// shared-memory bank conflicts; the query is stored split in two float4
+// planes so its rotated reads are conflict-free too.
+#include <cooperative_groups.h>
 #include <math.h>
 
 #include "bw_common.cuh"
 
+namespace cg = cooperative_groups;
+
 namespace bw {
 
-constexpr int ATT_THREADS = 128;
+constexpr int ATT_THREADS = 256;
 constexpr int ATT_WARPS = ATT_THREADS / 32;
-constexpr int ATT_TT = 32;          // tokens per tile (two pages)
+constexpr int ATT_TT = 32;          // tokens per stage (two pages)
 constexpr int ATT_MAXQ = 32;        // query vectors per CTA (G * n_rows)
+constexpr int ATT_MAXR = 8;         // query rows per sequence (1 + draft tokens)
+constexpr int ATT_MAXNS = 16;       // splits (cluster size) per (sequence, kv head)
 
 struct AttnParams {
     const float *qkv;
@@ -41,18 +48,20 @@ struct AttnParams {
     int B, R, nq, nkv, G, Q, n_split;
     float scale;
     float *out;
-    float *part_m, *part_l, *part_o;   // [B][nkv][n_split][Q] (+ [hd])
-    uint32_t *cnt;                     // [B][nkv]
     uint32_t *err;
 };
 
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+template <int HD>
+__host__ __device__ constexpr int att_stages() { return HD == 128 ? 4 : 6; }
+
+template <int HD, int QMAX>
+constexpr size_t att_smem_bytes() {
+    return static_cast<size_t>(att_stages<HD>()) * 2 * ATT_TT * HD * 2   // K/V ring (fp16)
+           + static_cast<size_t>(QMAX) * HD * 4                          // query planes (fp32)
+           + static_cast<size_t>(QMAX) * ATT_TT * 4                      // probabilities
+           + 2 * static_cast<size_t>(ATT_MAXR) * HD * 2                  // new k, v rows (fp16)
+           + static_cast<size_t>(att_stages<HD>()) * 8;                  // mbarriers
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // rotate-half RoPE of one pair, rounding each product like the plain formula
 __device__ __forceinline__ void rope_pair(float a, float b, float c, float s, float &ra, float &rb) {
@@ -60,21 +69,50 @@ __device__ __forceinline__ void rope_pair(float a, float b, float c, float s, fl
     rb = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
 }
 
+__device__ __forceinline__ float dot8(const float4 lo, const float4 hi, const uint4 k) {
+    const float2 k0 = __half22float2(*reinterpret_cast<const __half2 *>(&k.x));
+    const float2 k1 = __half22float2(*reinterpret_cast<const __half2 *>(&k.y));
+    const float2 k2 = __half22float2(*reinterpret_cast<const __half2 *>(&k.z));
+    const float2 k3 = __half22float2(*reinterpret_cast<const __half2 *>(&k.w));
+    float d = lo.x * k0.x;
+    d = fmaf(lo.y, k0.y, d);
+    d = fmaf(lo.z, k1.x, d);
+    d = fmaf(lo.w, k1.y, d);
+    d = fmaf(hi.x, k2.x, d);
+    d = fmaf(hi.y, k2.y, d);
+    d = fmaf(hi.z, k3.x, d);
+    d = fmaf(hi.w, k3.y, d);
+    return d;
+}
+
 template <int HD, int QMAX>
 __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
-    constexpr int NG = HD / 8;   // 16-byte granules per row
-    extern __shared__ float4 att_smem[];
-    __half (*sk)[ATT_TT * HD] = reinterpret_cast<__half (*)[ATT_TT * HD]>(att_smem);
-    __half (*sv)[ATT_TT * HD] = reinterpret_cast<__half (*)[ATT_TT * HD]>(sk + 2);
-    float *sq = reinterpret_cast<float *>(sv + 2);                       // [QMAX][HD]
-    float (*sp)[ATT_TT] = reinterpret_cast<float (*)[ATT_TT]>(sq + QMAX * HD);  // [QMAX][TT]
+    constexpr int NG = HD / 8;              // 16-byte granules per K/V row
+    constexpr int NST = att_stages<HD>();
+    constexpr int SH = ATT_TT * HD;         // halves per K (or V) stage
+    constexpr int TG = ATT_THREADS / HD;    // P.V token groups: 2 (HD 128) or 4 (HD 64)
+    constexpr int TPG = ATT_TT / TG;        // tokens per group and stage (16 or 8)
+    constexpr int NACC = QMAX;
+    constexpr int QPW = (QMAX + ATT_WARPS - 1) / ATT_WARPS;   // queries owned per warp
+    extern __shared__ __align__(128) unsigned char att_sm[];
+    __half *ring = reinterpret_cast<__half *>(att_sm);                       // [NST][K|V][SH]
+    float4 *q_lo = reinterpret_cast<float4 *>(ring + static_cast<size_t>(NST) * 2 * SH);  // [QMAX][NG]
+    float4 *q_hi = q_lo + QMAX * NG;                                        // [QMAX][NG]
+    float *P = reinterpret_cast<float *>(q_hi + QMAX * NG);                 // [QMAX][TT]
+    __half *newk = reinterpret_cast<__half *>(P + QMAX * ATT_TT);           // [MAXR][HD]
+    __half *newv = newk + ATT_MAXR * HD;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(newv + ATT_MAXR * HD);     // [NST]
     __shared__ float s_m[ATT_MAXQ], s_l[ATT_MAXQ], s_corr[ATT_MAXQ];
-    __shared__ int s_page[2][ATT_TT / 16];
-    __shared__ bool s_last;
+    __shared__ int s_page[NST][2];
 
-    pdl_trigger();
-    const int sp_idx = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    pdl_trigger();
+    if (tid == 0) {
+        for (int s = 0; s < NST; s++) mbar_init(&bar[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
     pdl_wait();
 
     const int p0 = p.pos[b];
@@ -85,12 +123,45 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
     }
     const int n_pg = (len + 15) / 16;
     const int pps = (n_pg + p.n_split - 1) / p.n_split;
-    const int pg0 = min(n_pg, sp_idx * pps), pg1 = min(n_pg, pg0 + pps);
-    const int t0 = pg0 * 16, t1 = min(len, pg1 * 16);
+    const int pg0 = min(n_pg, split * pps), pg1 = min(n_pg, pg0 + pps);
+    const int t1 = min(len, pg1 * 16);
+    const int n_tiles = (pg1 - pg0 + 1) / 2;
     const int32_t *pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
     const size_t row_stride = static_cast<size_t>(p.nq + 2 * p.nkv) * HD;
+    constexpr uint32_t PAGE_BYTES = 16 * HD * 2;
 
-    // ---- 1. roped, unscaled queries into shared memory
+    // one thread streams pages: expect the bytes, then issue the bulk copies
+    auto issue = [&](int tile) {
+        const int st = tile % NST;
+        int pages[2];
+        uint32_t bytes = 0;
+        for (int j = 0; j < 2; j++) {
+            const int lp = pg0 + 2 * tile + j;
+            int page = -1;
+            if (lp < pg1) {
+                page = pt[lp];
+                if (page < 0 || page >= p.n_pages) {
+                    set_error(p.err, BW_DEVERR_BAD_PAGE);
+                    page = -1;
+                }
+            }
+            pages[j] = page;
+            s_page[st][j] = page;
+            if (page >= 0) bytes += 2 * PAGE_BYTES;
+        }
+        mbar_arrive_tx(&bar[st], bytes);
+        __half *sk = ring + static_cast<size_t>(st) * 2 * SH;
+        for (int j = 0; j < 2; j++) {
+            if (pages[j] < 0) continue;
+            const size_t off = (static_cast<size_t>(pages[j]) * p.nkv + kvh) * 16 * HD;
+            bulk_g2s(sk + j * 16 * HD, p.k_pool + off, PAGE_BYTES, &bar[st]);
+            bulk_g2s(sk + SH + j * 16 * HD, p.v_pool + off, PAGE_BYTES, &bar[st]);
+        }
+    };
+    if (tid == 0)
+        for (int t = 0; t < min(NST, n_tiles); t++) issue(t);
+
+    // ---- 1. roped queries, split into two float4 planes per 8-dim granule
     for (int i = tid; i < p.Q * (HD / 2); i += ATT_THREADS) {
         const int qi = i / (HD / 2), d = i - qi * (HD / 2);
         const int r = qi / p.G, g = qi - r * p.G;
@@ -101,281 +172,271 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
         const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
         float ra, rb;
         rope_pair(src[d], src[d + HD / 2], c, s, ra, rb);
-        sq[qi * HD + d] = ra;
-        sq[qi * HD + d + HD / 2] = rb;
-    }
-    if (tid < ATT_MAXQ) {
-        s_m[tid] = -INFINITY;
-        s_l[tid] = 0.0f;
+        float *lo = reinterpret_cast<float *>(q_lo + qi * NG);
+        float *hi = reinterpret_cast<float *>(q_hi + qi * NG);
+        const int da = d, db = d + HD / 2;
+        ((da & 7) < 4 ? lo : hi)[(da >> 3) * 4 + (da & 3)] = ra;
+        ((db & 7) < 4 ? lo : hi)[(db >> 3) * 4 + (db & 3)] = rb;
     }
 
-    // ---- 2. the new rows' k (roped) and v, rounded to fp16, into the pool
+    // ---- 2. the new rows' k (roped) and v, rounded to fp16: kept for this
+    //         CTA's stages and written into the pool
     for (int r = 0; r < p.R; r++) {
         const int ppos = p0 + r;
-        if (ppos < t0 || ppos >= t1) continue;   // t1 <= max_pages * 16
+        if (ppos < pg0 * 16 || ppos >= t1) continue;
         const int page = pt[ppos / 16];
-        if (page < 0 || page >= p.n_pages) {
-            if (tid == 0) set_error(p.err, BW_DEVERR_BAD_PAGE);
-            continue;
-        }
-        const size_t off = ((static_cast<size_t>(page) * p.nkv + kvh) * 16 + (ppos & 15)) * HD;
+        const bool ok = page >= 0 && page < p.n_pages;
+        if (!ok && tid == 0) set_error(p.err, BW_DEVERR_BAD_PAGE);
+        const size_t off = ((static_cast<size_t>(ok ? page : 0) * p.nkv + kvh) * 16 + (ppos & 15)) * HD;
         const float *krow = p.qkv + (static_cast<size_t>(b) * p.R + r) * row_stride +
                             static_cast<size_t>(p.nq + kvh) * HD;
         const float *vrow = krow + static_cast<size_t>(p.nkv) * HD;
-        const int rp = ppos;
         for (int d = tid; d < HD / 2; d += ATT_THREADS) {
-            const float c = p.rope_cos[static_cast<size_t>(rp) * (HD / 2) + d];
-            const float s = p.rope_sin[static_cast<size_t>(rp) * (HD / 2) + d];
+            const float c = p.rope_cos[static_cast<size_t>(ppos) * (HD / 2) + d];
+            const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
             float ra, rb;
             rope_pair(krow[d], krow[d + HD / 2], c, s, ra, rb);
-            p.k_pool[off + d] = __float2half_rn(ra);
-            p.k_pool[off + d + HD / 2] = __float2half_rn(rb);
+            const __half ha = __float2half_rn(ra), hb = __float2half_rn(rb);
+            newk[r * HD + d] = ha;
+            newk[r * HD + d + HD / 2] = hb;
+            if (ok) {
+                p.k_pool[off + d] = ha;
+                p.k_pool[off + d + HD / 2] = hb;
+            }
         }
-        for (int d = tid; d < HD; d += ATT_THREADS) p.v_pool[off + d] = __float2half_rn(vrow[d]);
+        for (int d = tid; d < HD; d += ATT_THREADS) {
+            const __half hv = __float2half_rn(vrow[d]);
+            newv[r * HD + d] = hv;
+            if (ok) p.v_pool[off + d] = hv;
+        }
     }
     __syncthreads();
 
-    // ---- 3. tiles of 32 tokens: scores, online softmax, P.V
-    const int n_tiles = (t1 - t0 + ATT_TT - 1) / ATT_TT;
-    auto issue_tile = [&](int tile, int buf) {
-        const int tb = t0 + tile * ATT_TT;
-        if (tid < ATT_TT / 16) {
-            const int lp = tb / 16 + tid;
-            int page = -1;
-            if (lp * 16 < t1) {
-                page = pt[lp];
-                if (page < 0 || page >= p.n_pages) {
-                    set_error(p.err, BW_DEVERR_BAD_PAGE);
-                    page = -1;
-                }
-            }
-            s_page[buf][tid] = page;
-        }
-        __syncthreads();
-        for (int i = tid; i < ATT_TT * NG; i += ATT_THREADS) {
-            const int t = i / NG, g = i - t * NG;
-            const int page = s_page[buf][t / 16];
-            if (page < 0) continue;
-            const size_t off = ((static_cast<size_t>(page) * p.nkv + kvh) * 16 + (t & 15)) * HD + g * 8;
-            cp_async16(&sk[buf][t * HD + 8 * (g ^ (t & 7))], p.k_pool + off);
-            cp_async16(&sv[buf][t * HD + 8 * g], p.v_pool + off);
-        }
-        cp_async_commit();
-    };
-
-    // thread -> output dims: HD == 128: one dim per thread for every query;
-    // HD == 64: dim tid % 64 for the queries of parity tid / 64
-    constexpr int QSTEP = ATT_THREADS / HD;            // 1 or 2
-    constexpr int NACC = QMAX / QSTEP;
+    // ---- 3. stages of 32 tokens: scores, online softmax, P.V
+    float m_run[QPW], l_run[QPW];
+#pragma unroll
+    for (int j = 0; j < QPW; j++) {
+        m_run[j] = -INFINITY;
+        l_run[j] = 0.0f;
+    }
     float acc[NACC];
 #pragma unroll
     for (int i = 0; i < NACC; i++) acc[i] = 0.0f;
-    const int od = tid % HD, oq0 = tid / HD;
+    const int od = tid % HD, tq = tid / HD;   // output dim, token group
 
-    if (n_tiles > 0) issue_tile(0, 0);
     for (int tile = 0; tile < n_tiles; tile++) {
-        const int buf = tile & 1;
-        if (tile + 1 < n_tiles) {
-            issue_tile(tile + 1, buf ^ 1);
-            cp_async_wait<1>();
-        } else {
-            cp_async_wait<0>();
+        const int st = tile % NST;
+        mbar_wait(&bar[st], static_cast<uint32_t>((tile / NST) & 1), p.err);
+        __half *sk = ring + static_cast<size_t>(st) * 2 * SH;
+        __half *sv = sk + SH;
+        const int tb = (pg0 + 2 * tile) * 16;
+        // the rows written by this step replace what the copy brought
+        for (int r = 0; r < p.R; r++) {
+            const int slot = p0 + r - tb;
+            if (slot < 0 || slot >= ATT_TT || p0 + r >= t1 || s_page[st][slot >> 4] < 0) continue;
+            for (int d = tid; d < HD; d += ATT_THREADS) {
+                sk[slot * HD + d] = newk[r * HD + d];
+                sv[slot * HD + d] = newv[r * HD + d];
+            }
         }
         __syncthreads();
-        const int tb = t0 + tile * ATT_TT;
-        // scores: lane = token, warp strides over queries
+        // scores: lane = token, warp w owns queries w, w + 4, ...
         {
             const int t = lane;
             const int tpos = tb + t;
-            const bool tok_ok = tpos < t1 && s_page[buf][t / 16] >= 0;
+            const bool tok_ok = tpos < t1 && s_page[st][t >> 4] >= 0;
             uint4 kr[NG];
-            if (tok_ok) {
 #pragma unroll
-                for (int g = 0; g < NG; g++)
-                    kr[g] = *reinterpret_cast<const uint4 *>(&sk[buf][t * HD + 8 * (g ^ (t & 7))]);
+            for (int g = 0; g < NG; g++) {
+                const int g2 = (g + t) & (NG - 1);
+                kr[g] = *reinterpret_cast<const uint4 *>(sk + t * HD + g2 * 8);
             }
-            for (int qi = warp; qi < p.Q; qi += ATT_WARPS) {
+#pragma unroll
+            for (int j = 0; j < QPW; j++) {
+                const int qi = warp + ATT_WARPS * j;
+                if (qi >= p.Q) break;
                 const int r = qi / p.G;
                 float s = -INFINITY;
                 if (tok_ok && tpos <= p0 + r) {
                     float dot = 0.0f;
 #pragma unroll
                     for (int g = 0; g < NG; g++) {
-                        const float4 qa = *reinterpret_cast<const float4 *>(&sq[qi * HD + 8 * g]);
-                        const float4 qb = *reinterpret_cast<const float4 *>(&sq[qi * HD + 8 * g + 4]);
-                        const float2 k0 = __half22float2(*reinterpret_cast<const __half2 *>(&kr[g].x));
-                        const float2 k1 = __half22float2(*reinterpret_cast<const __half2 *>(&kr[g].y));
-                        const float2 k2 = __half22float2(*reinterpret_cast<const __half2 *>(&kr[g].z));
-                        const float2 k3 = __half22float2(*reinterpret_cast<const __half2 *>(&kr[g].w));
-                        dot = fmaf(qa.x, k0.x, dot);
-                        dot = fmaf(qa.y, k0.y, dot);
-                        dot = fmaf(qa.z, k1.x, dot);
-                        dot = fmaf(qa.w, k1.y, dot);
-                        dot = fmaf(qb.x, k2.x, dot);
-                        dot = fmaf(qb.y, k2.y, dot);
-                        dot = fmaf(qb.z, k3.x, dot);
-                        dot = fmaf(qb.w, k3.y, dot);
+                        const int g2 = (g + t) & (NG - 1);
+                        dot += dot8(q_lo[qi * NG + g2], q_hi[qi * NG + g2], kr[g]);
                     }
                     s = dot * p.scale;
                 }
-                // online softmax update of this query (one warp owns it)
-                const float m_old = s_m[qi];
-                const float m_new = fmaxf(m_old, warp_max(s));
+                const float m_new = fmaxf(m_run[j], warp_max(s));
                 const float pr = (s == -INFINITY) ? 0.0f : expf(s - m_new);
                 const float lsum = warp_sum(pr);
-                sp[qi][t] = pr;
-                if (lane == 0) {
-                    const float corr = (m_old == -INFINITY) ? 0.0f : expf(m_old - m_new);
-                    s_corr[qi] = corr;
-                    s_l[qi] = s_l[qi] * corr + lsum;
-                    s_m[qi] = m_new;
-                }
+                const float corr = (m_run[j] == -INFINITY) ? 0.0f : expf(m_run[j] - m_new);
+                l_run[j] = l_run[j] * corr + lsum;
+                m_run[j] = m_new;
+                P[qi * ATT_TT + t] = pr;
+                if (lane == 0) s_corr[qi] = corr;
             }
         }
         __syncthreads();
-        // P.V: thread owns dim od for queries oq0, oq0 + QSTEP, ...
+        // P.V: thread (od, tq) sums tokens [tq*TPG, tq*TPG + TPG) of the stage
 #pragma unroll
-        for (int i = 0; i < NACC; i++) {
-            const int qi = oq0 + i * QSTEP;
-            if (qi < p.Q) acc[i] *= s_corr[qi];
-        }
+        for (int i = 0; i < NACC; i++)
+            if (i < p.Q) acc[i] *= s_corr[i];
         {
             const int nt = min(ATT_TT, t1 - tb);
-            for (int pg = 0; pg < ATT_TT / 16; pg++) {
-                if (s_page[buf][pg] < 0) continue;
-                const int te = min(nt, pg * 16 + 16);
-                for (int t = pg * 16; t < te; t++) {
-                    const float v = __half2float(sv[buf][t * HD + od]);
+            const int ta = tq * TPG;
+            const int te = min(nt, ta + TPG);
+            if (ta < te && s_page[st][ta >> 4] >= 0) {
+                for (int t4 = ta; t4 < te; t4 += 4) {
+                    float v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; u++)
+                        v[u] = (t4 + u < te) ? __half2float(sv[(t4 + u) * HD + od]) : 0.0f;
 #pragma unroll
                     for (int i = 0; i < NACC; i++) {
-                        const int qi = oq0 + i * QSTEP;
-                        if (qi < p.Q) acc[i] = fmaf(sp[qi][t], v, acc[i]);
+                        if (i < p.Q) {
+                            const float4 pr = *reinterpret_cast<const float4 *>(&P[i * ATT_TT + t4]);
+                            float a = acc[i];
+                            a = fmaf(pr.x, v[0], a);
+                            a = fmaf(pr.y, v[1], a);
+                            a = fmaf(pr.z, v[2], a);
+                            a = fmaf(pr.w, v[3], a);
+                            acc[i] = a;
+                        }
                     }
                 }
             }
         }
         __syncthreads();
+        if (tid == 0 && tile + NST < n_tiles) issue(tile + NST);
     }
-
-    // ---- 4. partial results, then the last CTA combines the splits
-    const size_t grp = static_cast<size_t>(b) * p.nkv + kvh;
-    if (p.n_split == 1) {
+    if (lane == 0) {
 #pragma unroll
-        for (int i = 0; i < NACC; i++) {
-            const int qi = oq0 + i * QSTEP;
+        for (int j = 0; j < QPW; j++) {
+            const int qi = warp + ATT_WARPS * j;
             if (qi < p.Q) {
-                const int r = qi / p.G, g = qi - r * p.G;
-                const float l = s_l[qi];
-                p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
-                      static_cast<size_t>(kvh * p.G + g) * HD + od] = acc[i] / l;
+                s_m[qi] = m_run[j];
+                s_l[qi] = l_run[j];
             }
         }
-        return;
     }
-    const size_t pbase = (grp * p.n_split + sp_idx) * p.Q;
+    __syncthreads();
+
+    // ---- 4. outputs: merge the token groups (in group order), then write
+    //         directly or combine across the cluster's splits
+    float *s_o = reinterpret_cast<float *>(att_sm);   // [TG][Q][HD]: the ring is drained
 #pragma unroll
-    for (int i = 0; i < NACC; i++) {
-        const int qi = oq0 + i * QSTEP;
-        if (qi < p.Q) __stcg(p.part_o + (pbase + qi) * HD + od, acc[i]);
-    }
-    if (tid < p.Q) {
-        __stcg(p.part_m + pbase + tid, s_m[tid]);
-        __stcg(p.part_l + pbase + tid, s_l[tid]);
-    }
-    __threadfence();
+    for (int i = 0; i < NACC; i++)
+        if (i < p.Q) s_o[(tq * QMAX + i) * HD + od] = acc[i];
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(p.cnt + grp, 1u) == static_cast<uint32_t>(p.n_split - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    // combine the splits: gather every split's (max, sum) into shared memory
-    // (the K/V tile buffers are free now), then one coefficient per (split,
-    // query), then each thread sums its output dim over the splits in order.
-    const int nsq = p.n_split * p.Q;
-    float *cm = reinterpret_cast<float *>(att_smem);      // [n_split][Q] maxima -> coefficients
-    float *cl = cm + nsq;                                  // [n_split][Q] sums
-    const size_t gbase = grp * p.n_split * p.Q;
-    for (int i = tid; i < nsq; i += ATT_THREADS) {
-        cm[i] = ld_cg(p.part_m + gbase + i);
-        cl[i] = ld_cg(p.part_l + gbase + i);
-    }
-    __syncthreads();
-    if (tid < p.Q) {
-        float M = -INFINITY;
-        for (int s2 = 0; s2 < p.n_split; s2++) M = fmaxf(M, cm[s2 * p.Q + tid]);
-        float L = 0.0f;
-        for (int s2 = 0; s2 < p.n_split; s2++) {
-            const float ms = cm[s2 * p.Q + tid];
-            const float w = (ms == -INFINITY) ? 0.0f : expf(ms - M);
-            L = fmaf(cl[s2 * p.Q + tid], w, L);
-            cm[s2 * p.Q + tid] = w;
+    for (int e = tid; e < p.Q * HD; e += ATT_THREADS) {
+        const int qi = e / HD, d = e - qi * HD;
+        float o = s_o[qi * HD + d];
+#pragma unroll
+        for (int g = 1; g < TG; g++) o += s_o[(g * QMAX + qi) * HD + d];
+        if (p.n_split == 1) {
+            const int r = qi / p.G, gq = qi - r * p.G;
+            p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
+                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = o / s_l[qi];
+        } else {
+            s_o[(TG * QMAX) * HD + e] = o;   // merged partial after the group planes
         }
-        s_l[tid] = L;
     }
+    if (p.n_split == 1) return;
+    float *s_om = s_o + (TG * QMAX) * HD;
     __syncthreads();
-#pragma unroll
-    for (int i = 0; i < NACC; i++) {
-        const int qi = oq0 + i * QSTEP;
-        if (qi >= p.Q) continue;
-        float O = 0.0f;
-        const float *po = p.part_o + (gbase + qi) * HD + od;
-        const size_t sstride = static_cast<size_t>(p.Q) * HD;
-#pragma unroll 8
-        for (int s2 = 0; s2 < p.n_split; s2++) O = fmaf(ld_cg(po + s2 * sstride), cm[s2 * p.Q + qi], O);
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    const int ns = p.n_split;
+    for (int e = split * ATT_THREADS + tid; e < p.Q * HD; e += ns * ATT_THREADS) {
+        const int qi = e / HD, d = e - qi * HD;
+        float ms[ATT_MAXNS];
+        float M = -INFINITY;
+        for (int r2 = 0; r2 < ns; r2++) {
+            ms[r2] = cluster.map_shared_rank(s_m, r2)[qi];
+            M = fmaxf(M, ms[r2]);
+        }
+        float L = 0.0f, O = 0.0f;
+        for (int r2 = 0; r2 < ns; r2++) {
+            if (ms[r2] == -INFINITY) continue;
+            const float w = expf(ms[r2] - M);
+            L = fmaf(cluster.map_shared_rank(s_l, r2)[qi], w, L);
+            O = fmaf(cluster.map_shared_rank(s_om, r2)[qi * HD + d], w, O);
+        }
         const int r = qi / p.G, g = qi - r * p.G;
         p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
-              static_cast<size_t>(kvh * p.G + g) * HD + od] = O / s_l[qi];
+              static_cast<size_t>(kvh * p.G + g) * HD + d] = O / L;
     }
-    if (tid == 0) p.cnt[grp] = 0u;
+    cluster.sync();   // keep this CTA's shared memory alive until every reader is done
+}
+
+// Splits per (sequence, kv head) = cluster size: about one CTA per SM in
+// total, at least one stage (two pages) each, at most 16.
+static int attn_splits(int B, int nkv, int max_pages) {
+    const int groups = B * nkv;
+    int ns = (sm_count() + groups / 2) / groups;
+    ns = max(1, min(ns, ATT_MAXNS));
+    ns = min(ns, max(1, (max_pages + 1) / 2));
+    return ns;
+}
+
+size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages) {
+    (void)B; (void)R; (void)nq; (void)nkv; (void)hd; (void)max_pages;
+    return 0;
 }
 
 template <int HD, int QMAX>
-static bw_status attn_go(dim3 grid, cudaStream_t st, const AttnParams &p) {
-    const size_t smem = 4u * ATT_TT * HD * sizeof(__half) + static_cast<size_t>(QMAX) * HD * 4 +
-                        static_cast<size_t>(QMAX) * ATT_TT * 4;
+static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnParams &p) {
+    constexpr size_t smem = att_smem_bytes<HD, QMAX>();
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(attn_kernel<HD, QMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess)
+                                 static_cast<int>(smem)) != cudaSuccess ||
+            cudaFuncSetAttribute(attn_kernel<HD, QMAX>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess) {
+            (void)cudaGetLastError();
             return BW_ERR_CUDA;
+        }
         attr_set[dev] = true;
     }
-    return launch_pdl(attn_kernel<HD, QMAX>, grid, dim3(ATT_THREADS), smem, st, p);
-}
-
-// Splits per (sequence, kv head): enough CTAs to cover every SM about once,
-// at least ~4 pages per split, at most 64 splits (the combine keeps
-// n_split * 32 floats of statistics in shared memory).
-static int attn_splits(int B, int nkv, int max_pages) {
-    const int groups = B * nkv;
-    int ns = (sm_count() + groups - 1) / groups;
-    ns = max(1, min(ns, (max_pages + 3) / 4));
-    ns = min(ns, 64);
-    return ns;
-}
-
-size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages) {
-    const int ns = attn_splits(B, nkv, max_pages);
-    const size_t Q = static_cast<size_t>(nq / nkv) * R;
-    const size_t n = static_cast<size_t>(B) * nkv * ns * Q;
-    return 2 * align_up(n * 4, BW_WS_ALIGN) + align_up(n * hd * 4, BW_WS_ALIGN);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ns, nkv, B);
+    cfg.blockDim = dim3(ATT_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = ns;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    AttnParams q = p;
+    q.n_split = ns;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<HD, QMAX>, q);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BW_ERR_CUDA;
+    }
+    return BW_OK;
 }
 
 bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
                       void *k_pool, void *v_pool, const int32_t *page_table, int max_pages,
                       int n_pages, const int32_t *pos, int B, int R, int nq, int nkv, int hd,
                       float *out, const Scratch &sc, cudaStream_t st) {
-    if (!qkv || !rope_cos || !rope_sin || !k_pool || !v_pool || !page_table || !pos || !out || !sc.cnt)
+    if (!qkv || !rope_cos || !rope_sin || !k_pool || !v_pool || !page_table || !pos || !out)
         return BW_ERR_INVALID_ARG;
     if (B <= 0 || R <= 0 || nq <= 0 || nkv <= 0 || max_pages <= 0 || n_pages <= 0 || rope_max_pos <= 0)
         return BW_ERR_INVALID_ARG;
-    if ((hd != 128 && hd != 64) || nq % nkv || (nq / nkv) * R > ATT_MAXQ) return BW_ERR_UNSUPPORTED_SHAPE;
+    if ((hd != 128 && hd != 64) || nq % nkv || (nq / nkv) * R > ATT_MAXQ || R > ATT_MAXR)
+        return BW_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(qkv)) return BW_ERR_INVALID_ARG;
-    if (B * nkv + CNT_ATTN > BW_WS_COUNTERS) return BW_ERR_UNSUPPORTED_SHAPE;
-    if (sc.bytes < attn_scratch_bytes(B, R, nq, nkv, hd, max_pages)) return BW_ERR_INVALID_ARG;
+    if (nkv > 65535 || B > 65535) return BW_ERR_UNSUPPORTED_SHAPE;
     AttnParams p;
     p.qkv = qkv;
     p.rope_cos = rope_cos;
@@ -393,25 +454,18 @@ bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope
     p.nkv = nkv;
     p.G = nq / nkv;
     p.Q = p.G * R;
-    p.n_split = attn_splits(B, nkv, max_pages);
     p.scale = 1.0f / sqrtf(static_cast<float>(hd));
     p.out = out;
-    const size_t n = static_cast<size_t>(B) * nkv * p.n_split * p.Q;
-    Carver cv(sc.base);
-    p.part_m = cv.take<float>(n);
-    p.part_l = cv.take<float>(n);
-    p.part_o = cv.take<float>(n * hd);
-    p.cnt = sc.cnt + CNT_ATTN;
     p.err = sc.err;
-    dim3 grid(p.n_split, nkv, B);
+    const int ns = attn_splits(B, nkv, max_pages);
     if (hd == 128) {
-        if (p.Q <= 4) return attn_go<128, 4>(grid, st, p);
-        if (p.Q <= 8) return attn_go<128, 8>(grid, st, p);
-        if (p.Q <= 16) return attn_go<128, 16>(grid, st, p);
-        return attn_go<128, 32>(grid, st, p);
+        if (p.Q <= 4) return attn_go<128, 4>(ns, nkv, B, st, p);
+        if (p.Q <= 8) return attn_go<128, 8>(ns, nkv, B, st, p);
+        if (p.Q <= 16) return attn_go<128, 16>(ns, nkv, B, st, p);
+        return attn_go<128, 32>(ns, nkv, B, st, p);
     }
-    if (p.Q <= 8) return attn_go<64, 8>(grid, st, p);
-    return attn_go<64, 32>(grid, st, p);
+    if (p.Q <= 8) return attn_go<64, 8>(ns, nkv, B, st, p);
+    return attn_go<64, 32>(ns, nkv, B, st, p);
 }
 
 }  // namespace bw

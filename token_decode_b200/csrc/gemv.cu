@@ -4,53 +4,57 @@
 // bw.h).  Fused: RMSNorm prologue, residual-add / SiLU-gate epilogues, greedy
 // argmax over the outputs.  The fusion follows the devpress bw24 page,
 // section 2.2 (linear + activation in one kernel, intermediates in registers
-// and shared memory).
+// and shared memory); the TMA staging follows the deep-dive page, section 2
+// (asynchronous global->shared prefetch while computing).
 //
-// Work decomposition.  Rows come in groups of 8 ("row groups", rg); the K
-// axis in 32-element chunks.  K is cut into S slices so that RG*S work items
-// cover ~2 CTAs x 8 warps per SM; one warp owns one (rg, slice) item at a
-// time and each lane streams whole chunks of that item: 8 rows x 16 bytes of
-// nibbles + 16 bytes of scales per chunk, with every warp-wide load
-// instruction covering 512 contiguous bytes.  The activation slice is staged
-// once per CTA in shared memory (16-byte granules XOR-swizzled by chunk so
-// the 32 lanes of a warp hit distinct banks).  Items with S > 1 leave their
-// partial sums in the workspace; the last warp to finish a row group (atomic
-// counter, no waiting) adds the slices in slice order, so results are
-// deterministic run to run.
+// Warp-specialized CTA: a producer warp streams weight tiles of 128 rows x
+// 512 columns -- in the tiled layout each is one contiguous 32 KB block of
+// codes plus one 4 KB block of scales, i.e. two plain bulk copies
+// (cp.async.bulk) -- into a ring of shared-memory stages (mbarrier
+// full/empty pairs); eight consumer warps each own two 8-row groups of the
+// tile (one per half-warp), one 32-column chunk per lane.  The producer
+// touches only constant weights, so it starts streaming before
+// griddepcontrol.wait, while the previous kernel drains.
+//
+// Work decomposition: 128-row blocks x K slices.  The slice count S is chosen
+// on the host by a makespan search over the SM count; slices leave partial
+// sums in the workspace and the last warp to finish a row group (atomic
+// counter, no waiting) adds them in slice order, so results are
+// deterministic.  The activation slice of a CTA is staged once in shared
+// memory (16-byte granules XOR-swizzled by chunk, conflict-free per warp).
 //
 // Q4_0 arithmetic without integer->float conversions: a nibble q masked in
 // place into the low bits of an fp32 word is the denormal q * 2^(4p-149)
 // (p = its nibble slot within a 16-bit half).  The activation is pre-scaled
-// by 2^(101-4p), so the product is exactly q*x*2^-48 and the FMA accumulates
-// it in the normal fp32 range.  The -8 offset enters once per chunk through
-// the activation's chunk sum.  With one-hot x the result is exactly d*(q-8),
-// i.e. the dequantized weight, bit for bit.
+// by 2^(101-4p), so each product is exactly q*x*2^-48 and packed fp32x2 FMAs
+// accumulate in the normal range.  The -8 offset enters once per chunk
+// through the activation's chunk sum.  With one-hot x the result is exactly
+// d*(q-8), the dequantized weight.
 //
 // NVFP4: the sm_100a e2m1x2 -> f16x2 conversion gives exact values; the E4M3
 // block scale multiplies each 16-element block dot, the tensor scale the
 // final sum.
-//
-// Programmatic dependent launch: weights are constant, so every warp issues
-// the loads of its first chunk before griddepcontrol.wait; only the
-// activations and the outputs depend on the previous kernel.
-#include <math.h>
-#include <stdio.h>
-
-#include "bw_common.cuh"
+#include "gemv_core.cuh"
 
 namespace bw {
 
-constexpr int GEMV_THREADS = 256;
-constexpr int GEMV_WARPS = GEMV_THREADS / 32;
-constexpr int GEMV_MAX_M = 4;
+// One activation row: a CTA is half an SM (2 stages, <= 32 KB of staged
+// activations, <= 113 registers), so two CTAs share an SM -- two of this
+// kernel, or this one and the next kernel on the stream starting early.
+// More rows need the registers of a whole SM.
+template <int M>
+__host__ __device__ constexpr int gv_ctas_per_sm() { return M == 1 ? 2 : 1; }
+__host__ __device__ constexpr int gv_stages(int M) { return M == 1 ? 2 : 3; }
+__host__ __device__ constexpr size_t gv_xs_limit(int M) { return M == 1 ? 38 * 1024 : 66 * 1024; }
 
 struct GemvParams {
-    const uint8_t *q;      // [N][K/2]
-    const uint4 *s;        // [N/8][K/32] x 16 bytes
+    const uint8_t *q;      // tiled codes
+    const uint8_t *s;      // tiled scales
     int N, K, M;
-    int NC, RG;            // chunks per row, row groups
-    int S, CS;             // slices, chunks per slice
-    int grid_rg;           // CTAs per slice
+    int NC, RG, RB, KT;    // chunks per row, row groups, row blocks, column tiles
+    int S, CT;             // slices, column tiles per slice
+    int per_slice;         // CTAs per slice
+    int nst;               // pipeline stages
     const float *x;        // [M][K]
     const float *gamma;    // [K] or null
     float eps;
@@ -66,168 +70,16 @@ struct GemvParams {
     uint32_t *am_cnt;      // [1]
     int32_t *adv_tokens;   // [M] or null: also receives the argmax (next step's input)
     int32_t *adv_pos;      // [M] or null: incremented after the argmax
+    uint32_t *err;
 };
 
-// x'[m][e] for element e of chunk c lives at granule (g ^ (c & 7)) of the
-// chunk, g = idx / 4, idx = position of e in the kernel's consumption order.
-__device__ __forceinline__ int q4_order(int e) {
-    // byte j = e % 16 of the block: word j/4, nibble 2*(j%4) (+1 for the high half)
-    const int j = e & 15;
-    return 8 * (j >> 2) + 2 * (j & 3) + (e >> 4);
-}
-
-__device__ __forceinline__ float4 ld_gran(const float *xs_chunk, int g, int c) {
-    return *reinterpret_cast<const float4 *>(xs_chunk + 4 * (g ^ (c & 7)));
-}
-
-template <int FMT>
-__device__ __forceinline__ void load_chunk(const GemvParams &p, int rg, int kc, uint4 (&w)[9]) {
-    const uint8_t *base = p.q + static_cast<size_t>(rg) * 8u * static_cast<size_t>(p.K / 2) +
-                          static_cast<size_t>(kc) * 16u;
-    const size_t rs = static_cast<size_t>(p.K / 2);
-#pragma unroll
-    for (int r = 0; r < 8; r++) w[r] = ld_stream16(base + r * rs);
-    w[8] = ld_stream16(p.s + static_cast<size_t>(rg) * p.NC + kc);
-}
-
-__device__ __forceinline__ uint32_t u4_get(const uint4 &v, int i) {
-    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
-}
-
-// acc[r][m] += dot(row r of this chunk, x'[m] of this chunk)
-template <int FMT, int M>
-__device__ __forceinline__ void compute_chunk(const uint4 (&w)[9], const float *xs, const float *ct,
-                                              int cl, int chunk_stride, float (&acc)[8][M]) {
-    if constexpr (FMT == BW_FMT_Q4_0) {
-        float bd[8][M];
-#pragma unroll
-        for (int r = 0; r < 8; r++)
-#pragma unroll
-            for (int m = 0; m < M; m++) bd[r][m] = ct[m * chunk_stride];
-#pragma unroll
-        for (int wd = 0; wd < 4; wd++) {
-            float4 xa[M], xb[M];
-#pragma unroll
-            for (int m = 0; m < M; m++) {
-                const float *xc = xs + static_cast<size_t>(m) * chunk_stride * 32 + cl * 32;
-                xa[m] = ld_gran(xc, 2 * wd, cl);
-                xb[m] = ld_gran(xc, 2 * wd + 1, cl);
-            }
-#pragma unroll
-            for (int r = 0; r < 8; r++) {
-                const uint32_t v = u4_get(w[r], wd);
-                const uint32_t h = v >> 16;
-                const float f0 = __uint_as_float(v & 0xfu), f1 = __uint_as_float(v & 0xf0u);
-                const float f2 = __uint_as_float(v & 0xf00u), f3 = __uint_as_float(v & 0xf000u);
-                const float f4 = __uint_as_float(h & 0xfu), f5 = __uint_as_float(h & 0xf0u);
-                const float f6 = __uint_as_float(h & 0xf00u), f7 = __uint_as_float(h & 0xf000u);
-#pragma unroll
-                for (int m = 0; m < M; m++) {
-                    float b = bd[r][m];
-                    b = fma_rn(f0, xa[m].x, b);
-                    b = fma_rn(f1, xa[m].y, b);
-                    b = fma_rn(f2, xa[m].z, b);
-                    b = fma_rn(f3, xa[m].w, b);
-                    b = fma_rn(f4, xb[m].x, b);
-                    b = fma_rn(f5, xb[m].y, b);
-                    b = fma_rn(f6, xb[m].z, b);
-                    b = fma_rn(f7, xb[m].w, b);
-                    bd[r][m] = b;
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < 8; r++) {
-            const float d = half_bits_to_f((u4_get(w[8], r >> 1) >> (16 * (r & 1))) & 0xffffu);
-#pragma unroll
-            for (int m = 0; m < M; m++) acc[r][m] = fma_rn(d, bd[r][m], acc[r][m]);
-        }
-    } else {
-#pragma unroll
-        for (int half = 0; half < 2; half++) {
-            float bd[8][M];
-#pragma unroll
-            for (int r = 0; r < 8; r++)
-#pragma unroll
-                for (int m = 0; m < M; m++) bd[r][m] = 0.0f;
-#pragma unroll
-            for (int wd = 2 * half; wd < 2 * half + 2; wd++) {
-                float4 xa[M], xb[M];
-#pragma unroll
-                for (int m = 0; m < M; m++) {
-                    const float *xc = xs + static_cast<size_t>(m) * chunk_stride * 32 + cl * 32;
-                    xa[m] = ld_gran(xc, 2 * wd, cl);
-                    xb[m] = ld_gran(xc, 2 * wd + 1, cl);
-                }
-#pragma unroll
-                for (int r = 0; r < 8; r++) {
-                    const uint32_t v = u4_get(w[r], wd);
-                    const float2 e0 = e2m1x2_to_f2(v & 0xffu);
-                    const float2 e1 = e2m1x2_to_f2((v >> 8) & 0xffu);
-                    const float2 e2 = e2m1x2_to_f2((v >> 16) & 0xffu);
-                    const float2 e3 = e2m1x2_to_f2(v >> 24);
-#pragma unroll
-                    for (int m = 0; m < M; m++) {
-                        float b = bd[r][m];
-                        b = fma_rn(e0.x, xa[m].x, b);
-                        b = fma_rn(e0.y, xa[m].y, b);
-                        b = fma_rn(e1.x, xa[m].z, b);
-                        b = fma_rn(e1.y, xa[m].w, b);
-                        b = fma_rn(e2.x, xb[m].x, b);
-                        b = fma_rn(e2.y, xb[m].y, b);
-                        b = fma_rn(e3.x, xb[m].z, b);
-                        b = fma_rn(e3.y, xb[m].w, b);
-                        bd[r][m] = b;
-                    }
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < 8; r++) {
-                const uint32_t two = (u4_get(w[8], r >> 1) >> (16 * (r & 1))) & 0xffffu;
-                const float2 sc = e4m3x2_to_f2(two);
-                const float s = half ? sc.y : sc.x;
-#pragma unroll
-                for (int m = 0; m < M; m++) acc[r][m] = fma_rn(s, bd[r][m], acc[r][m]);
-            }
-        }
-    }
-}
-
-// Reduce acc[8][M] over the 32 lanes.  Afterwards lane l with (l & 3) == 0
-// holds the totals of row (l >> 2) in out[m].
-template <int M>
-__device__ __forceinline__ void reduce_rows(float (&acc)[8][M], int lane, float (&out)[M]) {
-    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
-#pragma unroll
-    for (int m = 0; m < M; m++) {
-        float b[4], c[2];
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const float send = b4 ? acc[i][m] : acc[i + 4][m];
-            const float keep = b4 ? acc[i + 4][m] : acc[i][m];
-            b[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-        }
-#pragma unroll
-        for (int i = 0; i < 2; i++) {
-            const float send = b3 ? b[i] : b[i + 2];
-            const float keep = b3 ? b[i + 2] : b[i];
-            c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-        }
-        const float send = b2 ? c[0] : c[1];
-        const float keep = b2 ? c[1] : c[0];
-        float d = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-        d += __shfl_xor_sync(0xffffffffu, d, 2);
-        d += __shfl_xor_sync(0xffffffffu, d, 1);
-        out[m] = d;
-    }
-}
-
-// Final values of row group rg (lanes with (lane & 3) == 0 hold row lane>>2):
-// scale, epilogue, outputs, argmax tracking.
+// Final values of row group rg (lanes with (lane & 1) == 0 hold row
+// (lane >> 1) & 7): scale, epilogue, outputs, argmax tracking.
+// All lanes must call it (it shuffles); `act` gates the stores.
 template <int FMT, int M>
 __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, const float (&tot)[M],
-                                         float (&bestv)[M], int (&besti)[M]) {
-    const int r = lane >> 2;
+                                         float (&bestv)[M], int (&besti)[M], bool act) {
+    const int r = (lane >> 1) & 7;
     const bool gu = p.flags & BW_GEMV_SILU_GATE;
     float val[M];
 #pragma unroll
@@ -241,11 +93,11 @@ __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, 
         val[m] = v;
     }
     if (gu) {
-        // gate row r (< 4) pairs with up row r + 4, held by lane + 16
+        // gate row r (< 4) pairs with up row r + 4, held by lane + 8
 #pragma unroll
         for (int m = 0; m < M; m++) {
-            const float up = __shfl_down_sync(0xffffffffu, val[m], 16);
-            if ((lane & 3) == 0 && r < 4 && m < p.M) {
+            const float up = __shfl_down_sync(0xffffffffu, val[m], 8);
+            if (act && (lane & 1) == 0 && r < 4 && m < p.M && rg < p.RG) {
                 const float g = val[m];
                 const float a = (g / (1.0f + expf(-g))) * up;
                 p.y[static_cast<size_t>(m) * (p.N / 2) + rg * 4 + r] = a;
@@ -253,7 +105,7 @@ __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, 
         }
         return;
     }
-    if ((lane & 3) != 0) return;
+    if (!act || (lane & 1) != 0 || rg >= p.RG) return;
     const int n = rg * 8 + r;
 #pragma unroll
     for (int m = 0; m < M; m++) {
@@ -269,86 +121,118 @@ __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, 
     }
 }
 
-// CTAs resident per SM the launch plan assumes (register budget 128 at M = 1)
-template <int M>
-constexpr int gemv_ctas_per_sm() { return M == 1 ? 2 : 1; }
-
 template <int FMT, int M>
-__global__ void __launch_bounds__(GEMV_THREADS, gemv_ctas_per_sm<M>()) gemv_kernel(const GemvParams p) {
-    extern __shared__ float4 smem4[];
-    float *xs = reinterpret_cast<float *>(smem4);      // [M][CS][32] swizzled
-    float *ct = xs + static_cast<size_t>(M) * p.CS * 32; // [M][CS] chunk terms (Q4_0)
-    __shared__ float s_red[GEMV_WARPS][M];
+__global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(const GemvParams p) {
+    extern __shared__ __align__(128) unsigned char gv_smem[];
+    const int nst = p.nst;
+    unsigned char *stages = gv_smem;                                                     // nst x 36 KB
+    float *xs = reinterpret_cast<float *>(gv_smem + static_cast<size_t>(nst) * GV_STAGE_BYTES);  // [M][CS][32]
+    const int CS = p.CT * GV_TC;                                                          // chunks per slice
+    float *ct = xs + static_cast<size_t>(M) * CS * 32;                                   // [M][CS]
+    float *gt = ct + ((static_cast<size_t>(M) * CS + 3) & ~static_cast<size_t>(3));      // [CS*32] gains (RMSNorm)
+    uint64_t *full = reinterpret_cast<uint64_t *>(gt + ((p.flags & BW_GEMV_RMSNORM) ? CS * 32 : 0));
+    uint64_t *empty = full + nst;
+    const uint32_t stages_a = smem_u32(stages), xs_a = smem_u32(xs), ct_a = smem_u32(ct);
+    __shared__ float s_red[GV_CW][M];
     __shared__ float s_rnorm[M];
-    __shared__ float s_bv[GEMV_WARPS][M];
-    __shared__ int s_bi[GEMV_WARPS][M];
+    __shared__ float s_bv[GV_CW][M];
+    __shared__ int s_bi[GV_CW][M];
     __shared__ bool s_last;
 
-    pdl_trigger();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int slice = blockIdx.x % p.S;
-    const int cta_in_slice = blockIdx.x / p.S;
-    const int c0 = slice * p.CS;
-    const int nc = min(p.CS, p.NC - c0);
-    const int u = (nc + 31) >> 5;
-    const int rg_stride = p.grid_rg * GEMV_WARPS;
+    const int j0 = blockIdx.x / p.S;
+    const int kt0 = slice * p.CT;
+    const int T = min(p.CT, p.KT - kt0);                  // column tiles of this slice
+    const int c0 = kt0 * GV_TC;
+    const int nc = min(T * GV_TC, p.NC - c0);             // real chunks of this slice
+    const int n_items = j0 < p.RB ? (p.RB - 1 - j0) / p.per_slice + 1 : 0;
+    const int n_steps = n_items * T;
 
-    // ---- prefetch the first chunk of this warp's first item (constant data)
-    int rg = cta_in_slice * GEMV_WARPS + warp;
-    int j = 0;
-    uint4 cur[9];
-    if (rg < p.RG && lane < nc) load_chunk<FMT>(p, rg, c0 + lane, cur);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nst; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], GV_CW);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    pdl_trigger();
 
+    if (warp == GV_CW) {
+        // ---- producer: constant weights only, so no dependency wait
+        if (lane == 0) {
+            for (int step = 0; step < n_steps; step++) {
+                const int s = step % nst;
+                if (step >= nst) mbar_wait(&empty[s], static_cast<uint32_t>((step / nst - 1) & 1), p.err);
+                const int item = step / T, kt = kt0 + (step - item * T);
+                const int rb = j0 + item * p.per_slice;
+                const size_t tile = static_cast<size_t>(rb) * p.KT + kt;
+                unsigned char *st = stages + static_cast<size_t>(s) * GV_STAGE_BYTES;
+                mbar_arrive_tx_relaxed(&full[s], GV_STAGE_BYTES);
+                bulk_g2s(st, p.q + tile * GV_NIB_BYTES, GV_NIB_BYTES, &full[s]);
+                bulk_g2s(st + GV_NIB_BYTES, p.s + tile * GV_SC_BYTES, GV_SC_BYTES, &full[s]);
+            }
+        }
+        return;
+    }
+
+    // ---- consumers
     pdl_wait();
-
-    // ---- prologue: activations of this slice into shared memory
-    if (p.flags & BW_GEMV_RMSNORM) {
-        float ss[M];
+    const int ctid = threadIdx.x;   // 0 .. 255
+    const bool norm = p.flags & BW_GEMV_RMSNORM;
+    // pass 1: the slice's activations (and gains) in natural order, all loads
+    // issued back to back; the RMSNorm sum of squares on the way
+    const int ne = nc * 32;
+    float ss[M];
 #pragma unroll
-        for (int m = 0; m < M; m++) ss[m] = 0.0f;
-        for (int k = threadIdx.x; k < p.K; k += GEMV_THREADS)
+    for (int m = 0; m < M; m++) {
+        ss[m] = 0.0f;
+        if (m >= p.M) {
+            for (int e = ctid; e < ne; e += GV_CW * 32) xs[static_cast<size_t>(m) * CS * 32 + e] = 0.0f;
+            continue;
+        }
+        const float *xr = p.x + static_cast<size_t>(m) * p.K + c0 * 32;
+#pragma unroll 4
+        for (int e = ctid; e < ne; e += GV_CW * 32) {
+            const float v = xr[e];
+            xs[static_cast<size_t>(m) * CS * 32 + e] = v;
+            ss[m] = fma_rn(v, v, ss[m]);
+        }
+    }
+    if (norm) {
+#pragma unroll 4
+        for (int e = ctid; e < ne; e += GV_CW * 32) gt[e] = p.gamma[c0 * 32 + e];
+        if (p.S > 1) {
+            // the norm needs the whole row, not just this slice
 #pragma unroll
-            for (int m = 0; m < M; m++)
-                if (m < p.M) {
-                    const float v = p.x[static_cast<size_t>(m) * p.K + k];
-                    ss[m] = fma_rn(v, v, ss[m]);
-                }
+            for (int m = 0; m < M; m++) {
+                ss[m] = 0.0f;
+                if (m < p.M)
+#pragma unroll 4
+                    for (int k = ctid; k < p.K; k += GV_CW * 32) {
+                        const float v = p.x[static_cast<size_t>(m) * p.K + k];
+                        ss[m] = fma_rn(v, v, ss[m]);
+                    }
+            }
+        }
 #pragma unroll
         for (int m = 0; m < M; m++) {
             ss[m] = warp_sum(ss[m]);
             if (lane == 0) s_red[warp][m] = ss[m];
         }
-        __syncthreads();
-        if (threadIdx.x < M) {
+        consumer_sync();
+        if (ctid < M) {
             float t = 0.0f;
-            for (int w2 = 0; w2 < GEMV_WARPS; w2++) t += s_red[w2][threadIdx.x];
-            s_rnorm[threadIdx.x] = 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps);
-        }
-        __syncthreads();
-    }
-    for (int pair = warp; pair < M * nc; pair += GEMV_WARPS) {
-        const int m = pair / nc, cl = pair - m * nc;
-        const int e = lane;
-        const int k = (c0 + cl) * 32 + e;
-        float v = 0.0f;
-        if (m < p.M) {
-            v = p.x[static_cast<size_t>(m) * p.K + k];
-            if (p.flags & BW_GEMV_RMSNORM) v = (v * s_rnorm[m]) * p.gamma[k];
-        }
-        float *xc = xs + static_cast<size_t>(m) * p.CS * 32 + cl * 32;
-        if constexpr (FMT == BW_FMT_Q4_0) {
-            const int idx = q4_order(e);
-            const float scale = __int_as_float((127 + 101 - 4 * (idx & 3)) << 23);
-            xc[4 * ((idx >> 2) ^ (cl & 7)) + (idx & 3)] = v * scale;
-            const float sum = warp_sum(v);
-            if (lane == 0) ct[m * p.CS + cl] = sum * -2.8421709430404007e-14f;  // -8 * 2^-48
-        } else {
-            xc[4 * ((e >> 2) ^ (cl & 7)) + (e & 3)] = v;
+            for (int w2 = 0; w2 < GV_CW; w2++) t += s_red[w2][ctid];
+            s_rnorm[ctid] = 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps);
         }
     }
-    __syncthreads();
+    consumer_sync();
+    // pass 2: swizzle and pre-scale in place
+    stage_pass2<FMT, M>(xs, ct, norm ? gt : nullptr, s_rnorm, CS, nc, warp, lane);
+    consumer_sync();
 
-    // ---- main loop over (item, chunk) steps with a one-step prefetch
     float acc[8][M];
 #pragma unroll
     for (int r = 0; r < 8; r++)
@@ -362,58 +246,59 @@ __global__ void __launch_bounds__(GEMV_THREADS, gemv_ctas_per_sm<M>()) gemv_kern
         besti[m] = 0x7fffffff;
     }
 
-    while (rg < p.RG) {
-        int nrg = rg, nj = j + 1;
-        if (nj == u) {
-            nj = 0;
-            nrg = rg + rg_stride;
+    int step = 0;
+    for (int item = 0; item < n_items; item++) {
+        const int rb = j0 + item * p.per_slice;
+        const int rg = rb * (GV_TR / 8) + 2 * warp + (lane >> 4);
+        for (int kt = 0; kt < T; kt++, step++) {
+            const int s = step % nst;
+            mbar_wait(&full[s], static_cast<uint32_t>((step / nst) & 1), p.err);
+            const int cl = kt * GV_TC + (lane & 15);
+            if (cl < nc)
+                stage_chunk<FMT, M>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, warp, lane, xs_a, ct_a,
+                                    cl, CS, acc);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_relaxed(&empty[s]);
         }
-        uint4 nxt[9];
-        const int ncl = lane + 32 * nj;
-        if (nrg < p.RG && ncl < nc) load_chunk<FMT>(p, nrg, c0 + ncl, nxt);
-        const int cl = lane + 32 * j;
-        if (cl < nc) compute_chunk<FMT, M>(cur, xs, ct + cl, cl, p.CS, acc);
-        if (j == u - 1) {
-            float tot[M];
-            reduce_rows<M>(acc, lane, tot);
+        float tot[M];
+        reduce_rows16<M>(acc, lane, tot);
 #pragma unroll
-            for (int r = 0; r < 8; r++)
+        for (int r = 0; r < 8; r++)
 #pragma unroll
-                for (int m = 0; m < M; m++) acc[r][m] = 0.0f;
-            if (p.S == 1) {
-                epilogue<FMT, M>(p, rg, lane, tot, bestv, besti);
-            } else {
-                const int r = lane >> 2;
-                if ((lane & 3) == 0) {
-                    float *dst = p.partial + ((static_cast<size_t>(slice) * p.RG + rg) * 8 + r) * M;
+            for (int m = 0; m < M; m++) acc[r][m] = 0.0f;
+        if (p.S == 1) {
+            epilogue<FMT, M>(p, rg, lane, tot, bestv, besti, true);
+        } else {
+            // split K: leave the partial sums; the last slice to finish a row
+            // group (per half-warp) adds them in slice order and runs the epilogue
+            const int r = (lane >> 1) & 7;
+            const bool real = rg < p.RG;
+            if ((lane & 1) == 0 && real) {
+                float *dst = p.partial + ((static_cast<size_t>(slice) * p.RG + rg) * 8 + r) * M;
 #pragma unroll
-                    for (int m = 0; m < M; m++) __stcg(dst + m, tot[m]);
-                }
-                __threadfence();
-                __syncwarp();
-                uint32_t old = 0;
-                if (lane == 0) old = atomicAdd(p.rg_cnt + rg, 1u);
-                old = __shfl_sync(0xffffffffu, old, 0);
-                if (old == static_cast<uint32_t>(p.S - 1)) {
-                    __threadfence();
-                    float sum[M];
-#pragma unroll
-                    for (int m = 0; m < M; m++) sum[m] = 0.0f;
-                    if ((lane & 3) == 0)
-                        for (int s2 = 0; s2 < p.S; s2++) {
-                            const float *src = p.partial + ((static_cast<size_t>(s2) * p.RG + rg) * 8 + r) * M;
-#pragma unroll
-                            for (int m = 0; m < M; m++) sum[m] += ld_cg(src + m);
-                        }
-                    epilogue<FMT, M>(p, rg, lane, sum, bestv, besti);
-                    if (lane == 0) p.rg_cnt[rg] = 0u;
-                }
+                for (int m = 0; m < M; m++) __stcg(dst + m, tot[m]);
             }
-        }
-        rg = nrg;
-        j = nj;
+            __threadfence();
+            __syncwarp();
+            uint32_t old = 0;
+            if ((lane & 15) == 0 && real) old = atomicAdd(p.rg_cnt + rg, 1u);
+            old = __shfl_sync(0xffffffffu, old, lane & 16);
+            const bool last = real && old == static_cast<uint32_t>(p.S - 1);
+            float sum[M];
 #pragma unroll
-        for (int i = 0; i < 9; i++) cur[i] = nxt[i];
+            for (int m = 0; m < M; m++) sum[m] = 0.0f;
+            if (last) {
+                __threadfence();
+                if ((lane & 1) == 0)
+                    for (int s2 = 0; s2 < p.S; s2++) {
+                        const float *src = p.partial + ((static_cast<size_t>(s2) * p.RG + rg) * 8 + r) * M;
+#pragma unroll
+                        for (int m = 0; m < M; m++) sum[m] += ld_cg(src + m);
+                    }
+            }
+            epilogue<FMT, M>(p, rg, lane, sum, bestv, besti, last);
+            if (last && (lane & 15) == 0) p.rg_cnt[rg] = 0u;
+        }
     }
 
     // ---- greedy argmax over all outputs
@@ -436,12 +321,12 @@ __global__ void __launch_bounds__(GEMV_THREADS, gemv_ctas_per_sm<M>()) gemv_kern
                 s_bi[warp][m] = i;
             }
         }
-        __syncthreads();
-        if (threadIdx.x < M) {
-            const int m = threadIdx.x;
+        consumer_sync();
+        if (ctid < M) {
+            const int m = ctid;
             float v = s_bv[0][m];
             int i = s_bi[0][m];
-            for (int w2 = 1; w2 < GEMV_WARPS; w2++)
+            for (int w2 = 1; w2 < GV_CW; w2++)
                 if (better(s_bv[w2][m], s_bi[w2][m], v, i)) {
                     v = s_bv[w2][m];
                     i = s_bi[w2][m];
@@ -450,12 +335,12 @@ __global__ void __launch_bounds__(GEMV_THREADS, gemv_ctas_per_sm<M>()) gemv_kern
             __stcg(p.am_idx + blockIdx.x * M + m, i);
         }
         __threadfence();
-        __syncthreads();
-        if (threadIdx.x == 0) s_last = atomicAdd(p.am_cnt, 1u) == gridDim.x - 1;
-        __syncthreads();
+        consumer_sync();
+        if (ctid == 0) s_last = atomicAdd(p.am_cnt, 1u) == gridDim.x - 1;
+        consumer_sync();
         if (s_last) {
             __threadfence();
-            for (int m = warp; m < p.M; m += GEMV_WARPS) {
+            for (int m = warp; m < p.M; m += GV_CW) {
                 float v = -INFINITY;
                 int i = 0x7fffffff;
                 for (int b = lane; b < static_cast<int>(gridDim.x); b += 32) {
@@ -482,7 +367,7 @@ __global__ void __launch_bounds__(GEMV_THREADS, gemv_ctas_per_sm<M>()) gemv_kern
                     if (p.adv_pos) p.adv_pos[m] += 1;
                 }
             }
-            if (threadIdx.x == 0) *p.am_cnt = 0u;
+            if (ctid == 0) *p.am_cnt = 0u;
         }
     }
 }
@@ -490,68 +375,80 @@ __global__ void __launch_bounds__(GEMV_THREADS, gemv_ctas_per_sm<M>()) gemv_kern
 // ------------------------------------------------------------------- host
 
 struct GemvPlan {
-    int S, CS, grid_rg, grid;
+    int S, CT, per_slice, grid, nst;
     size_t smem;
     size_t partial_floats;
 };
 
-static GemvPlan plan_gemv(int N, int K, int Mk) {
+static int kernel_m(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
+
+// Slices: minimise (rounds of items over the CTA slots) x (column tiles per
+// item), with a small cost per extra slice (the partial-sum pass), subject to
+// the staged activations fitting in shared memory.
+static GemvPlan plan_gemv(int N, int K, int Mk, bool norm) {
     GemvPlan pl;
-    const int RG = N / 8, NC = K / 32;
-    const int per_sm = Mk == 1 ? gemv_ctas_per_sm<1>() : gemv_ctas_per_sm<2>();
-    const int target_warps = sm_count() * per_sm * GEMV_WARPS;
-    int S = 1;
-    if (RG < target_warps) {
-        S = (target_warps + RG / 2) / RG;
-        S = max(1, min(S, max(1, NC / 16)));
+    const int RB = gv_row_blocks(N), KT = gv_col_tiles(K), RG = N / 8;
+    const int G = sm_count() * (Mk == 1 ? gv_ctas_per_sm<1>() : gv_ctas_per_sm<2>());
+    int bestS = 1, bestCT = KT;
+    double best = 1e30;
+    for (int S = 1; S <= min(64, KT); S++) {
+        const int CT = (KT + S - 1) / S;
+        if ((KT + CT - 1) / CT != S) continue;
+        if (static_cast<size_t>(Mk) * CT * GV_TC * 33 * 4 + (norm ? static_cast<size_t>(CT) * GV_TC * 32 * 4 : 0) >
+            gv_xs_limit(Mk))
+            continue;
+        const int per_slice = max(1, min(RB, G / S));
+        const int rounds = (RB + per_slice - 1) / per_slice;
+        // an item costs its column tiles plus its epilogue (more with split K:
+        // partial sums, a fence and a counter per row group)
+        const double cost = static_cast<double>(rounds) * (CT + (S > 1 ? 1.5 : 0.5));
+        if (cost < best - 1e-9) {
+            best = cost;
+            bestS = S;
+            bestCT = CT;
+        }
     }
-    int CS = (NC + S - 1) / S;
-    S = (NC + CS - 1) / CS;
-    // keep the staged activations within 96 KB
-    while (static_cast<size_t>(Mk) * CS * 33 * 4 > 96u * 1024u && CS > 32) {
-        S++;
-        CS = (NC + S - 1) / S;
-        S = (NC + CS - 1) / CS;
-    }
-    const int target_ctas = sm_count() * per_sm;
-    int grid_rg = (RG + GEMV_WARPS - 1) / GEMV_WARPS;
-    grid_rg = max(1, min(grid_rg, target_ctas / S));
-    pl.S = S;
-    pl.CS = CS;
-    pl.grid_rg = grid_rg;
-    pl.grid = S * grid_rg;
-    pl.smem = static_cast<size_t>(Mk) * CS * 32 * 4 + static_cast<size_t>(Mk) * CS * 4;
-    pl.partial_floats = S > 1 ? static_cast<size_t>(S) * RG * 8 * Mk : 0;
+    pl.S = bestS;
+    pl.CT = bestCT;
+    pl.per_slice = max(1, min(RB, G / bestS));
+    pl.grid = pl.S * pl.per_slice;
+    pl.nst = gv_stages(Mk);
+    pl.smem = static_cast<size_t>(pl.nst) * GV_STAGE_BYTES + static_cast<size_t>(Mk) * bestCT * GV_TC * 33 * 4 + 16 +
+              (norm ? static_cast<size_t>(bestCT) * GV_TC * 32 * 4 : 0) + 2 * static_cast<size_t>(pl.nst) * 8;
+    pl.partial_floats = pl.S > 1 ? static_cast<size_t>(pl.S) * RG * 8 * Mk : 0;
     return pl;
 }
 
-static int kernel_m(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : 4; }
-
 size_t gemv_scratch_bytes(int N, int K, int M) {
     size_t tot = 0;
-    for (int m0 = 0; m0 < M; m0 += GEMV_MAX_M) {
-        const int Mk = kernel_m(min(GEMV_MAX_M, M - m0));
-        const GemvPlan pl = plan_gemv(N, K, Mk);
+    for (int m0 = 0; m0 < M; m0 += GV_MAX_M) {
+        const int Mk = kernel_m(min(GV_MAX_M, M - m0));
+        for (int norm = 0; norm < 2; norm++) {
+        const GemvPlan pl = plan_gemv(N, K, Mk, norm != 0);
         size_t b = align_up(pl.partial_floats * 4, BW_WS_ALIGN) +
                    2 * align_up(static_cast<size_t>(pl.grid) * Mk * 4, BW_WS_ALIGN);
         tot = max(tot, b);
+        }
     }
     return tot;
 }
 
 template <int FMT, int M>
 static bw_status launch_gemv_m(const GemvParams &p0, const GemvPlan &pl, cudaStream_t st) {
-    static bool attr_set[64] = {};
+    // raise the kernel's dynamic shared-memory limit to what this plan needs
+    static size_t attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
-    if (!attr_set[dev]) {
+    if (attr_set[dev] < pl.smem) {
         if (cudaFuncSetAttribute(gemv_kernel<FMT, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 100 * 1024) != cudaSuccess)
+                                 static_cast<int>(pl.smem)) != cudaSuccess) {
+            (void)cudaGetLastError();
             return BW_ERR_CUDA;
-        attr_set[dev] = true;
+        }
+        attr_set[dev] = pl.smem;
     }
-    return launch_pdl(gemv_kernel<FMT, M>, dim3(pl.grid), dim3(GEMV_THREADS), pl.smem, st, p0);
+    return launch_pdl(gemv_kernel<FMT, M>, dim3(pl.grid), dim3(GV_THREADS), pl.smem, st, p0);
 }
 
 bw_status gemv_launch(int fmt, const void *wq, const void *ws_scales, float ts, float ts_up, int N,
@@ -569,22 +466,25 @@ bw_status gemv_launch(int fmt, const void *wq, const void *ws_scales, float ts, 
     if (!(flags & BW_GEMV_ARGMAX) && !y) return BW_ERR_INVALID_ARG;
     if (sc.bytes < gemv_scratch_bytes(N, K, M)) return BW_ERR_INVALID_ARG;
     const int ncols = (flags & BW_GEMV_SILU_GATE) ? N / 2 : N;
-    for (int m0 = 0; m0 < M; m0 += GEMV_MAX_M) {
-        const int Mr = min(GEMV_MAX_M, M - m0);
+    for (int m0 = 0; m0 < M; m0 += GV_MAX_M) {
+        const int Mr = min(GV_MAX_M, M - m0);
         const int Mk = kernel_m(Mr);
-        const GemvPlan pl = plan_gemv(N, K, Mk);
+        const GemvPlan pl = plan_gemv(N, K, Mk, (flags & BW_GEMV_RMSNORM) != 0);
         Carver cv(sc.base);
         GemvParams p;
         p.q = static_cast<const uint8_t *>(wq);
-        p.s = static_cast<const uint4 *>(ws_scales);
+        p.s = static_cast<const uint8_t *>(ws_scales);
         p.N = N;
         p.K = K;
         p.M = Mr;
         p.NC = K / 32;
         p.RG = N / 8;
+        p.RB = gv_row_blocks(N);
+        p.KT = gv_col_tiles(K);
         p.S = pl.S;
-        p.CS = pl.CS;
-        p.grid_rg = pl.grid_rg;
+        p.CT = pl.CT;
+        p.per_slice = pl.per_slice;
+        p.nst = pl.nst;
         p.x = x + static_cast<size_t>(m0) * K;
         p.gamma = gamma;
         p.eps = eps;
@@ -601,6 +501,7 @@ bw_status gemv_launch(int fmt, const void *wq, const void *ws_scales, float ts, 
         p.am_cnt = sc.cnt + CNT_ARGMAX;
         p.adv_tokens = adv_tokens ? adv_tokens + m0 : nullptr;
         p.adv_pos = adv_pos ? adv_pos + m0 : nullptr;
+        p.err = sc.err;
         if (pl.S > 1 && p.RG + CNT_GEMV_RG > CNT_ATTN) return BW_ERR_UNSUPPORTED_SHAPE;
         bw_status stt;
         if (fmt == BW_FMT_Q4_0) {

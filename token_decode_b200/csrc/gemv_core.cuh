@@ -1,0 +1,272 @@
+// gemv_core.cuh -- device core shared by the dense and the grouped-expert
+// dequant-GEMV kernels (sm_100a): the tiled weight layout, the stage
+// pipeline helpers, the 4-bit dequant-dot inner loop and the lane
+// reduction.
+//
+// Tiled GPU layout (written by the repack kernels).  A matrix W[N][K] is cut
+// into tiles of 128 rows x 512 columns (16 chunks of 32 columns); N is padded
+// to a multiple of 128 rows and K to a multiple of 512 columns with zeros.
+// Tile (rb, kt) of the codes is one contiguous 32 KB block: row r of the tile
+// at r*256 bytes, chunk c of that row at +c*16 (the 16 code bytes of the
+// chunk in the canonical nibble order).  Tile (rb, kt) of the scales is one
+// contiguous 4 KB block: row group g (rows 8g..8g+7 of the tile) at g*256,
+// chunk c at +c*16: the 8 rows' fp16 d (Q4_0) or 8 x 2 E4M3 block scales
+// (NVFP4).  Tiles follow each other in (rb, kt) order.  Every pipeline stage
+// is therefore two plain contiguous bulk copies that stream at full HBM
+// rate.
+#pragma once
+
+#include <math.h>
+
+#include "bw_common.cuh"
+
+namespace bw {
+
+constexpr int GV_CW = 8;                          // consumer warps
+constexpr int GV_THREADS = (GV_CW + 1) * 32;      // + one producer warp
+constexpr int GV_MAX_M = 4;
+constexpr int GV_TR = 128;                        // tile rows (16 row groups)
+constexpr int GV_TC = 16;                         // tile chunks (of 32 columns)
+constexpr uint32_t GV_NIB_BYTES = GV_TR * GV_TC * 16;        // 32 KB
+constexpr uint32_t GV_SC_BYTES = (GV_TR / 8) * GV_TC * 16;   // 4 KB
+constexpr uint32_t GV_STAGE_BYTES = GV_NIB_BYTES + GV_SC_BYTES;
+
+__host__ __device__ constexpr int gv_row_blocks(int N) { return (N + GV_TR - 1) / GV_TR; }
+__host__ __device__ constexpr int gv_col_tiles(int K) { return (K / 32 + GV_TC - 1) / GV_TC; }
+
+// Producer arrival that only announces the bytes its bulk copies will
+// deliver; it publishes no data of its own, so it needs no release fence.
+__device__ __forceinline__ void mbar_arrive_tx_relaxed(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.relaxed.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// Consumer release of a stage.  Relaxed: every shared-memory load of the
+// stage has already been consumed by the arithmetic before this point, so
+// the loads are complete and no release fence is needed.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void consumer_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(GV_CW * 32) : "memory");
+}
+
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+// Position of element e (0..31) of a Q4_0 chunk in the kernel's consumption
+// order: byte j = e % 16 is word j/4, nibble 2*(j%4), +1 for the high half.
+__device__ __forceinline__ int q4_order(int e) {
+    const int j = e & 15;
+    return 8 * (j >> 2) + 2 * (j & 3) + (e >> 4);
+}
+
+// Explicit shared-memory loads (32-bit shared addresses).  Volatile so they
+// stay after the mbarrier wait that publishes the stage they read.
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float4 lds_f4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float lds_f(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+
+// Staged activations: chunk c of row m at (m*chunk_stride + c)*128 bytes; its
+// 16-byte granule g is stored at granule (g ^ (c & 7)), so 8 lanes reading
+// granule g of 8 consecutive chunks hit 8 different bank groups.
+__device__ __forceinline__ uint32_t gran_addr(uint32_t chunk_a, int g, int c) {
+    return chunk_a + 16u * static_cast<uint32_t>(g ^ (c & 7));
+}
+
+// Writes activation value v of element e of local chunk cl (row m) into the
+// staged layout: Q4_0 pre-scaled per nibble slot, plus the chunk's -8 term.
+template <int FMT>
+__device__ __forceinline__ void stage_x(float *xs, float *ct, int chunk_stride, int m, int cl, int lane, float v) {
+    float *xc = xs + static_cast<size_t>(m * chunk_stride + cl) * 32;
+    if constexpr (FMT == BW_FMT_Q4_0) {
+        const int idx = q4_order(lane);
+        const float scale = __int_as_float((127 + 101 - 4 * (idx & 3)) << 23);   // 2^(101-4p)
+        xc[4 * ((idx >> 2) ^ (cl & 7)) + (idx & 3)] = v * scale;
+        const float sum = warp_sum(v);
+        if (lane == 0) ct[m * chunk_stride + cl] = sum * -2.8421709430404007e-14f;   // -8 * 2^-48
+    } else {
+        xc[4 * ((lane >> 2) ^ (cl & 7)) + (lane & 3)] = v;
+    }
+}
+
+// Second staging pass: the slice's activations sit in natural order at the
+// start of each chunk's slot (first pass: one wide burst of independent
+// global loads); each warp turns its chunks into the swizzled, pre-scaled
+// form in place, applying the RMSNorm (x * rnorm) * gamma when gt != null.
+template <int FMT, int M>
+__device__ __forceinline__ void stage_pass2(float *xs, float *ct, const float *gt, const float *rnorm, int CS,
+                                            int nc, int warp, int lane) {
+    for (int pair = warp; pair < M * nc; pair += GV_CW) {
+        const int m = pair / nc, cl = pair - m * nc;
+        float v = xs[static_cast<size_t>(m * CS + cl) * 32 + lane];
+        if (gt) v = (v * rnorm[m]) * gt[cl * 32 + lane];
+        __syncwarp();
+        stage_x<FMT>(xs, ct, CS, m, cl, lane, v);
+    }
+}
+
+__device__ __forceinline__ uint32_t u4_get(const uint4 &v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
+// acc[r][m] += dot(row r of this chunk, x'[m] of this chunk).
+//   w: 8 rows x 16 bytes of codes + 16 bytes of scales (this lane's chunk)
+//   xs_a: shared address of the staged activations [M][chunk_stride][32]
+//   ctv[m]: the chunk's -8 * 2^-48 * sum(x) term (Q4_0)
+template <int FMT, int M>
+__device__ __forceinline__ void compute_chunk(const uint4 (&w)[9], uint32_t xs_a, const float (&ctv)[M], int cl,
+                                              int chunk_stride, float (&acc)[8][M]) {
+    if constexpr (FMT == BW_FMT_Q4_0) {
+        float2 bd[8][M];
+#pragma unroll
+        for (int r = 0; r < 8; r++)
+#pragma unroll
+            for (int m = 0; m < M; m++) bd[r][m] = make_float2(ctv[m], 0.0f);
+#pragma unroll
+        for (int wd = 0; wd < 4; wd++) {
+            float4 xa[M], xb[M];
+#pragma unroll
+            for (int m = 0; m < M; m++) {
+                const uint32_t xc = xs_a + 128u * static_cast<uint32_t>(m * chunk_stride + cl);
+                xa[m] = lds_f4(gran_addr(xc, 2 * wd, cl));
+                xb[m] = lds_f4(gran_addr(xc, 2 * wd + 1, cl));
+            }
+#pragma unroll
+            for (int r = 0; r < 8; r++) {
+                const uint32_t v = u4_get(w[r], wd);
+                const uint32_t h = v >> 16;
+                const float2 f01 = make_float2(__uint_as_float(v & 0xfu), __uint_as_float(v & 0xf0u));
+                const float2 f23 = make_float2(__uint_as_float(v & 0xf00u), __uint_as_float(v & 0xf000u));
+                const float2 f45 = make_float2(__uint_as_float(h & 0xfu), __uint_as_float(h & 0xf0u));
+                const float2 f67 = make_float2(__uint_as_float(h & 0xf00u), __uint_as_float(h & 0xf000u));
+#pragma unroll
+                for (int m = 0; m < M; m++) {
+                    float2 b = bd[r][m];
+                    b = ffma2(f01, make_float2(xa[m].x, xa[m].y), b);
+                    b = ffma2(f23, make_float2(xa[m].z, xa[m].w), b);
+                    b = ffma2(f45, make_float2(xb[m].x, xb[m].y), b);
+                    b = ffma2(f67, make_float2(xb[m].z, xb[m].w), b);
+                    bd[r][m] = b;
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+            const float d = half_bits_to_f((u4_get(w[8], r >> 1) >> (16 * (r & 1))) & 0xffffu);
+#pragma unroll
+            for (int m = 0; m < M; m++) acc[r][m] = fma_rn(d, bd[r][m].x + bd[r][m].y, acc[r][m]);
+        }
+    } else {
+#pragma unroll
+        for (int half = 0; half < 2; half++) {
+            float2 bd[8][M];
+#pragma unroll
+            for (int r = 0; r < 8; r++)
+#pragma unroll
+                for (int m = 0; m < M; m++) bd[r][m] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int wd = 2 * half; wd < 2 * half + 2; wd++) {
+                float4 xa[M], xb[M];
+#pragma unroll
+                for (int m = 0; m < M; m++) {
+                    const uint32_t xc = xs_a + 128u * static_cast<uint32_t>(m * chunk_stride + cl);
+                    xa[m] = lds_f4(gran_addr(xc, 2 * wd, cl));
+                    xb[m] = lds_f4(gran_addr(xc, 2 * wd + 1, cl));
+                }
+#pragma unroll
+                for (int r = 0; r < 8; r++) {
+                    const uint32_t v = u4_get(w[r], wd);
+                    const float2 e0 = e2m1x2_to_f2(v & 0xffu);
+                    const float2 e1 = e2m1x2_to_f2((v >> 8) & 0xffu);
+                    const float2 e2 = e2m1x2_to_f2((v >> 16) & 0xffu);
+                    const float2 e3 = e2m1x2_to_f2(v >> 24);
+#pragma unroll
+                    for (int m = 0; m < M; m++) {
+                        float2 b = bd[r][m];
+                        b = ffma2(e0, make_float2(xa[m].x, xa[m].y), b);
+                        b = ffma2(e1, make_float2(xa[m].z, xa[m].w), b);
+                        b = ffma2(e2, make_float2(xb[m].x, xb[m].y), b);
+                        b = ffma2(e3, make_float2(xb[m].z, xb[m].w), b);
+                        bd[r][m] = b;
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < 8; r++) {
+                const uint32_t two = (u4_get(w[8], r >> 1) >> (16 * (r & 1))) & 0xffffu;
+                const float2 sc = e4m3x2_to_f2(two);
+                const float s = half ? sc.y : sc.x;
+#pragma unroll
+                for (int m = 0; m < M; m++) acc[r][m] = fma_rn(s, bd[r][m].x + bd[r][m].y, acc[r][m]);
+            }
+        }
+    }
+}
+
+// One lane's chunk of one stage.  Warp w owns row groups 2w (lanes 0..15)
+// and 2w+1 (lanes 16..31) of the 128-row tile; lane & 15 is the chunk.
+template <int FMT, int M>
+__device__ __forceinline__ void stage_chunk(uint32_t stage_a, int warp, int lane, uint32_t xs_a, uint32_t ct_a,
+                                            int cl, int chunk_stride, float (&acc)[8][M]) {
+    const int g = 2 * warp + (lane >> 4), c = lane & 15;
+    uint4 w[9];
+#pragma unroll
+    for (int r = 0; r < 8; r++) w[r] = lds_u4(stage_a + (g * 8 + r) * (GV_TC * 16) + c * 16);
+    w[8] = lds_u4(stage_a + GV_NIB_BYTES + g * (GV_TC * 16) + c * 16);
+    float ctv[M];
+#pragma unroll
+    for (int m = 0; m < M; m++)
+        ctv[m] = (FMT == BW_FMT_Q4_0) ? lds_f(ct_a + 4u * static_cast<uint32_t>(m * chunk_stride + cl)) : 0.0f;
+    compute_chunk<FMT, M>(w, xs_a, ctv, cl, chunk_stride, acc);
+}
+
+// Reduce acc[8][M] over each half-warp (16 lanes, one row group each).
+// Afterwards lane l with (l & 1) == 0 holds the totals of row ((l >> 1) & 7)
+// of its half's row group in out[m].
+template <int M>
+__device__ __forceinline__ void reduce_rows16(float (&acc)[8][M], int lane, float (&out)[M]) {
+    const bool b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+    for (int m = 0; m < M; m++) {
+        float b[4], c[2];
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float send = b3 ? acc[i][m] : acc[i + 4][m];
+            const float keep = b3 ? acc[i + 4][m] : acc[i][m];
+            b[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+#pragma unroll
+        for (int i = 0; i < 2; i++) {
+            const float send = b2 ? b[i] : b[i + 2];
+            const float keep = b2 ? b[i + 2] : b[i];
+            c[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+        }
+        const float send = b1 ? c[0] : c[1];
+        const float keep = b1 ? c[1] : c[0];
+        float d = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+        d += __shfl_xor_sync(0xffffffffu, d, 1);
+        out[m] = d;
+    }
+}
+
+}  // namespace bw

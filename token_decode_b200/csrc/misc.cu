@@ -2,7 +2,7 @@
 // kernels of libbw (sm_100a).
 #include <math.h>
 
-#include "bw_common.cuh"
+#include "gemv_core.cuh"
 
 namespace bw {
 
@@ -21,8 +21,19 @@ __device__ __forceinline__ void src_row(int R, bool inter, int &row, int &which)
     which = i >> 2;
 }
 
-__global__ void repack_q4_0_kernel(const uint8_t *blocks, const uint8_t *blocks_up, int rows, int NC,
-                                   uint8_t *q_out, uint16_t *s_out) {
+// Tiled layout offsets (see gemv_core.cuh): codes of (row R, chunk c) and the
+// byte offset of row R's scale slot for chunk c.
+__device__ __forceinline__ size_t tile_code_off(int R, int c, int KT) {
+    const size_t tile = static_cast<size_t>(R / GV_TR) * KT + c / GV_TC;
+    return tile * GV_NIB_BYTES + static_cast<size_t>(R % GV_TR) * (GV_TC * 16) + (c % GV_TC) * 16;
+}
+__device__ __forceinline__ size_t tile_scale_off(int R, int c, int KT) {
+    const size_t tile = static_cast<size_t>(R / GV_TR) * KT + c / GV_TC;
+    return tile * GV_SC_BYTES + static_cast<size_t>((R % GV_TR) / 8) * (GV_TC * 16) + (c % GV_TC) * 16 + (R % 8) * 2;
+}
+
+__global__ void repack_q4_0_kernel(const uint8_t *blocks, const uint8_t *blocks_up, int rows, int NC, int KT,
+                                   uint8_t *q_out, uint8_t *s_out) {
     const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= static_cast<size_t>(rows) * NC) return;
     const int R = static_cast<int>(i / NC), c = static_cast<int>(i % NC);
@@ -33,13 +44,12 @@ __global__ void repack_q4_0_kernel(const uint8_t *blocks, const uint8_t *blocks_
     uint32_t w[4];
 #pragma unroll
     for (int k = 0; k < 4; k++) w[k] = static_cast<uint32_t>(s16[1 + 2 * k]) | (static_cast<uint32_t>(s16[2 + 2 * k]) << 16);
-    *reinterpret_cast<uint4 *>(q_out + static_cast<size_t>(R) * NC * 16 + static_cast<size_t>(c) * 16) =
-        make_uint4(w[0], w[1], w[2], w[3]);
-    s_out[(static_cast<size_t>(R >> 3) * NC + c) * 8 + (R & 7)] = s16[0];
+    *reinterpret_cast<uint4 *>(q_out + tile_code_off(R, c, KT)) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint16_t *>(s_out + tile_scale_off(R, c, KT)) = s16[0];
 }
 
 __global__ void repack_nvfp4_kernel(const uint8_t *q, const uint8_t *s, const uint8_t *q_up,
-                                    const uint8_t *s_up, int rows, int NC, uint8_t *q_out, uint8_t *s_out) {
+                                    const uint8_t *s_up, int rows, int NC, int KT, uint8_t *q_out, uint8_t *s_out) {
     const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i >= static_cast<size_t>(rows) * NC) return;
     const int R = static_cast<int>(i / NC), c = static_cast<int>(i % NC);
@@ -47,9 +57,9 @@ __global__ void repack_nvfp4_kernel(const uint8_t *q, const uint8_t *s, const ui
     src_row(R, q_up != nullptr, row, which);
     const uint8_t *qs = which ? q_up : q;
     const uint8_t *ss = which ? s_up : s;
-    *reinterpret_cast<uint4 *>(q_out + static_cast<size_t>(R) * NC * 16 + static_cast<size_t>(c) * 16) =
+    *reinterpret_cast<uint4 *>(q_out + tile_code_off(R, c, KT)) =
         *reinterpret_cast<const uint4 *>(qs + static_cast<size_t>(row) * NC * 16 + static_cast<size_t>(c) * 16);
-    uint8_t *d = s_out + (static_cast<size_t>(R >> 3) * NC + c) * 16 + (R & 7) * 2;
+    uint8_t *d = s_out + tile_scale_off(R, c, KT);
     d[0] = ss[static_cast<size_t>(row) * NC * 2 + 2 * c];
     d[1] = ss[static_cast<size_t>(row) * NC * 2 + 2 * c + 1];
 }
@@ -67,21 +77,22 @@ __global__ void embed_kernel(int fmt, const uint8_t *eq, const uint8_t *es, floa
     const int tok = tokens[m];
     const bool ok = tok >= 0 && tok < V;
     if (!ok && threadIdx.x == 0) set_error(err, BW_DEVERR_BAD_TOKEN);
-    const int NC = H / 32;
+    const int KT = gv_col_tiles(H);
     for (int k = threadIdx.x; k < H; k += blockDim.x) {
         float w = 0.0f;
         if (ok) {
             const int c = k >> 5, e = k & 31;
+            const size_t qo = tile_code_off(tok, c, KT), so = tile_scale_off(tok, c, KT);
             if (fmt == BW_FMT_Q4_0) {
-                const uint8_t byte = eq[static_cast<size_t>(tok) * (H / 2) + c * 16 + (e & 15)];
+                const uint8_t byte = eq[qo + (e & 15)];
                 const int q = (e >> 4) ? (byte >> 4) : (byte & 15);
-                const uint16_t dh = reinterpret_cast<const uint16_t *>(es)[(static_cast<size_t>(tok >> 3) * NC + c) * 8 + (tok & 7)];
+                const uint16_t dh = *reinterpret_cast<const uint16_t *>(es + so);
                 w = __fmul_rn(half_bits_to_f(dh), static_cast<float>(q - 8));
             } else {
-                const uint8_t byte = eq[static_cast<size_t>(tok) * (H / 2) + c * 16 + (e >> 1)];
+                const uint8_t byte = eq[qo + (e >> 1)];
                 const float2 v2 = e2m1x2_to_f2(byte);
                 const float ev = (e & 1) ? v2.y : v2.x;
-                const float sv = e4m3_to_f(es[(static_cast<size_t>(tok >> 3) * NC + c) * 16 + (tok & 7) * 2 + (e >> 4)]);
+                const float sv = e4m3_to_f(es[so + (e >> 4)]);
                 w = __fmul_rn(__fmul_rn(ev, sv), ts);
             }
         }
@@ -192,7 +203,7 @@ __global__ void rmsnorm_kernel(float *x, const float *add, const float *gamma, i
 bw_status embed_launch(int fmt, const void *e_q, const void *e_s, float ts, int V, int H,
                        const int32_t *tokens, int M, float *x, uint32_t *err, cudaStream_t st) {
     if (!e_q || !e_s || !tokens || !x || V <= 0 || H <= 0 || M <= 0) return BW_ERR_INVALID_ARG;
-    if (H % 32 || V % 8) return BW_ERR_UNSUPPORTED_SHAPE;
+    if (H % 32) return BW_ERR_UNSUPPORTED_SHAPE;
     if (fmt != BW_FMT_Q4_0 && fmt != BW_FMT_NVFP4) return BW_ERR_INVALID_ARG;
     return launch_pdl(embed_kernel, dim3(M), dim3(256), 0, st, fmt, static_cast<const uint8_t *>(e_q),
                       static_cast<const uint8_t *>(e_s), ts, V, H, tokens, x, err);
@@ -208,19 +219,34 @@ bw_status rmsnorm_launch(float *x, const float *add, const float *gamma, int M, 
 
 extern "C" {
 
+bw_status bw_repack_bytes(int rows, int K, size_t *q_bytes, size_t *s_bytes) {
+    if (rows <= 0 || K <= 0 || K % 32 || !q_bytes || !s_bytes) return BW_ERR_INVALID_ARG;
+    const size_t tiles = static_cast<size_t>(bw::gv_row_blocks(rows)) * bw::gv_col_tiles(K);
+    *q_bytes = tiles * bw::GV_NIB_BYTES;
+    *s_bytes = tiles * bw::GV_SC_BYTES;
+    return BW_OK;
+}
+
 bw_status bw_repack_q4_0(const void *blocks, const void *blocks_up, int N, int K, void *q_out, void *s_out,
                          void *stream) {
     if (!blocks || !q_out || !s_out || N <= 0 || K <= 0) return BW_ERR_INVALID_ARG;
     const int rows = blocks_up ? 2 * N : N;
     if (K % 32 || rows % 8 || (blocks_up && N % 4)) return BW_ERR_UNSUPPORTED_SHAPE;
-    if (!bw::aligned16(q_out) || (reinterpret_cast<uintptr_t>(blocks) & 1) ||
-        (blocks_up && (reinterpret_cast<uintptr_t>(blocks_up) & 1)) || (reinterpret_cast<uintptr_t>(s_out) & 1))
+    if (!bw::aligned16(q_out) || !bw::aligned16(s_out) || (reinterpret_cast<uintptr_t>(blocks) & 1) ||
+        (blocks_up && (reinterpret_cast<uintptr_t>(blocks_up) & 1)))
         return BW_ERR_INVALID_ARG;
-    const int NC = K / 32;
+    const int NC = K / 32, KT = bw::gv_col_tiles(K);
+    size_t qb = 0, sb = 0;
+    bw_repack_bytes(rows, K, &qb, &sb);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(q_out, 0, qb, st) != cudaSuccess || cudaMemsetAsync(s_out, 0, sb, st) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BW_ERR_CUDA;
+    }
     const size_t n = static_cast<size_t>(rows) * NC;
-    bw::repack_q4_0_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint8_t *>(blocks), static_cast<const uint8_t *>(blocks_up), rows, NC,
-        static_cast<uint8_t *>(q_out), static_cast<uint16_t *>(s_out));
+    bw::repack_q4_0_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        static_cast<const uint8_t *>(blocks), static_cast<const uint8_t *>(blocks_up), rows, NC, KT,
+        static_cast<uint8_t *>(q_out), static_cast<uint8_t *>(s_out));
     return bw::launch_status();
 }
 
@@ -229,12 +255,20 @@ bw_status bw_repack_nvfp4(const void *q, const void *s, const void *q_up, const 
     if (!q || !s || !q_out || !s_out || N <= 0 || K <= 0 || (!q_up) != (!s_up)) return BW_ERR_INVALID_ARG;
     const int rows = q_up ? 2 * N : N;
     if (K % 32 || rows % 8 || (q_up && N % 4)) return BW_ERR_UNSUPPORTED_SHAPE;
-    if (!bw::aligned16(q) || !bw::aligned16(q_out) || (q_up && !bw::aligned16(q_up))) return BW_ERR_INVALID_ARG;
-    const int NC = K / 32;
+    if (!bw::aligned16(q) || !bw::aligned16(q_out) || !bw::aligned16(s_out) || (q_up && !bw::aligned16(q_up)))
+        return BW_ERR_INVALID_ARG;
+    const int NC = K / 32, KT = bw::gv_col_tiles(K);
+    size_t qb = 0, sb = 0;
+    bw_repack_bytes(rows, K, &qb, &sb);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(q_out, 0, qb, st) != cudaSuccess || cudaMemsetAsync(s_out, 0, sb, st) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BW_ERR_CUDA;
+    }
     const size_t n = static_cast<size_t>(rows) * NC;
-    bw::repack_nvfp4_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+    bw::repack_nvfp4_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
         static_cast<const uint8_t *>(q), static_cast<const uint8_t *>(s), static_cast<const uint8_t *>(q_up),
-        static_cast<const uint8_t *>(s_up), rows, NC, static_cast<uint8_t *>(q_out), static_cast<uint8_t *>(s_out));
+        static_cast<const uint8_t *>(s_up), rows, NC, KT, static_cast<uint8_t *>(q_out), static_cast<uint8_t *>(s_out));
     return bw::launch_status();
 }
 

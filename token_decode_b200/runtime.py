@@ -19,8 +19,9 @@ from .synth import FMT_Q4_0, FMT_NVFP4, PAGE_TOKENS
 def _gpu_layout(m, up=None):
     """QMat (+ matching up-projection) -> (bw.QWeight, [tensors to keep alive])."""
     rows = m.N * (2 if up is not None else 1)
-    q = torch.empty((rows, m.K // 2), dtype=torch.uint8, device=m.q.device)
-    s = torch.empty((rows * (m.K // 16),), dtype=torch.uint8, device=m.q.device)
+    qb, sb = bw.repack_bytes(rows, m.K)
+    q = torch.empty((qb,), dtype=torch.uint8, device=m.q.device)
+    s = torch.empty((sb,), dtype=torch.uint8, device=m.q.device)
     if m.fmt == FMT_Q4_0:
         bw.repack_q4_0(m.q, m.N, m.K, q, s, blocks_up=None if up is None else up.q)
     else:
@@ -71,11 +72,12 @@ class DeviceModel:
 
     def _moe_layer(self, c, ly, keep):
         E, Fe, H = ly.eg.E, ly.eg.N, ly.eg.K
-        rows = 2 * Fe
-        gq = torch.empty((E, rows, H // 2), dtype=torch.uint8, device="cuda")
-        gs = torch.empty((E, rows * (H // 16)), dtype=torch.uint8, device="cuda")
-        dq = torch.empty((E, H, Fe // 2), dtype=torch.uint8, device="cuda")
-        ds = torch.empty((E, H * (Fe // 16)), dtype=torch.uint8, device="cuda")
+        gqb, gsb = bw.repack_bytes(2 * Fe, H)
+        dqb, dsb = bw.repack_bytes(H, Fe)
+        gq = torch.empty((E, gqb), dtype=torch.uint8, device="cuda")
+        gs = torch.empty((E, gsb), dtype=torch.uint8, device="cuda")
+        dq = torch.empty((E, dqb), dtype=torch.uint8, device="cuda")
+        ds = torch.empty((E, dsb), dtype=torch.uint8, device="cuda")
         for e in range(E):
             g, u, d = ly.eg.mat(e), ly.eu.mat(e), ly.ed.mat(e)
             if g.fmt == FMT_Q4_0:
