@@ -110,6 +110,42 @@ def step_bytes(cfg, model, avg_ctx):
     return model.weight_bytes_dense() + kv_read + kv_write
 
 
+# ncu summaries of the dominant kernel: DRAM traffic per launch, valid while the
+# kernel's sources hash to the recorded value
+_PROFILE_FILES = {("gu", "7b"): "gemv_gate_up_7b.md"}
+_KERNEL_SOURCES = {"gu": ("gemv.cu", "gemv_core.cuh", "bw_common.cuh")}
+
+
+def kernel_sources_sha(kind):
+    import hashlib
+    h = hashlib.sha256()
+    for f in _KERNEL_SOURCES[kind]:
+        with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "token_decode_b200",
+                               "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(kind, cfg_name):
+    name = _PROFILE_FILES.get((kind, cfg_name))
+    if name is None:
+        return None
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", name)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for ln in open(path):
+        if ln.startswith("- ") and ":" in ln:
+            k, v = ln[2:].split(":", 1)
+            vals[k.strip().strip("`")] = v.strip().strip("`")
+    if vals.get("kernel_sources_sha") != kernel_sources_sha(kind):
+        return None
+    try:
+        return int(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def run_ours(args):
     from token_decode_b200 import build, bw, runtime, synth
     ws_, rank, local = dist_env()
@@ -247,36 +283,14 @@ def run_ours(args):
     e2e_ms = f0.elapsed_time(f1)
     e2e_value = n_e2e * cfg.B / (e2e_ms / 1000.0) * ws_
 
-    # ---- dominant kernel: the fused gate/up GEMV, every layer back to back
-    gu_bytes = sum(dm.layers[l].wgu.N * dm.layers[l].wgu.K * 9 // 16 for l in range(cfg.L))
-    gu_bytes += 0  # (9/16 byte per weight: 4-bit codes + a 2-byte scale per 32)
-    kws = bw.workspace(bw.gemv_workspace_bytes(2 * cfg.F, cfg.H, cfg.B, 0))
-    xin = torch.randn((cfg.B, cfg.H), device="cuda")
-    gam = torch.ones(cfg.H, device="cuda")
-    act = torch.empty((cfg.B, cfg.F), device="cuda")
-
-    def gu_all():
-        for l in range(cfg.L):
-            w = dm.layers[l].wgu
-            if cfg.fmt == synth.FMT_Q4_0:
-                bw.gemv_q4_0(w.q, w.s, w.N, w.K, xin, cfg.B, act, kws, gamma=gam,
-                             flags=bw.GEMV_RMSNORM | bw.GEMV_SILU_GATE, stream=stream)
-            else:
-                bw.gemv_nvfp4(w.q, w.s, w.ts, w.N, w.K, xin, cfg.B, act, kws, ts_up=w.ts_up,
-                              gamma=gam, flags=bw.GEMV_RMSNORM | bw.GEMV_SILU_GATE, stream=stream)
-    for _ in range(3):
-        gu_all()
-    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reps = 5
-    k0.record(stream)
-    for _ in range(reps):
-        gu_all()
-    k1.record(stream)
-    k1.synchronize()
-    gu_ms = k0.elapsed_time(k1) / (reps * cfg.L)
-    gu_launch_bytes = gu_bytes / cfg.L
+    # ---- per kernel: every launch kind of the step over all layers, graph-replayed;
+    # the dominant one (gate/up GEMV, or the MoE FFN) gives the roofline figure
+    from token_decode_b200 import kernel_bench
+    kern = kernel_bench.run_all(dm, dkv, cfg.B, stream, cfg.ctx + cfg.steps // 2, reps=5)
+    dom = "gu" if "gu" in kern else "moe"
     peak, peak_kind = _peaks()
-    achieved = gu_launch_bytes / (gu_ms / 1000.0) / 1e9
+    achieved = kern[dom]["GBps"]
+    traffic = _ncu_traffic(dom, cfg.name)
 
     avg_ctx = cfg.ctx + (cfg.steps + 1) / 2
     sb = step_bytes(cfg, model, avg_ctx)
@@ -308,10 +322,14 @@ def run_ours(args):
         "roofline_step_frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4),
         "roofline_step_frac_of_measured": round(step_gbs / peak, 4),
         "bytes_per_step": int(sb),
-        "roofline": {"bound": "hbm", "kernel": "gemv_kernel (fused RMSNorm + gate/up + SiLU gate)",
-                     "achieved": round(achieved, 1), "peak": peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
-                     "bytes_per_launch": int(gu_launch_bytes), "avg_launch_us": round(gu_ms * 1000, 3)},
+        "roofline": {"bound": "hbm",
+                     "kernel": "gemv_kernel (fused RMSNorm + gate/up + SiLU gate)" if dom == "gu"
+                               else "MoE FFN (route + grouped expert GEMVs + combine)",
+                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "bytes_per_launch": kern[dom]["bytes_per_launch"],
+                     "avg_launch_us": kern[dom]["us_per_launch"]},
+        "kernels": kern,
         "e2e": {"value": round(e2e_value, 3), "unit": "tok/s", "steps": n_e2e,
                 "h2d_bytes_per_step": 4 * cfg.B, "d2h_bytes_per_step": 4 * cfg.B,
                 "path": "bw_decode_step via the C ABI, pinned host token in/out, sync each step"},

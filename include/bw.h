@@ -26,6 +26,7 @@
  *       ordering and expert parallelism without warp divergence.
  *   bw_argmax -- greedy sampling: the lowest index of the maximum.  Deep-dive
  *       page, section 1: the argmax token sequence is the correctness gate.
+ *   bw_spec_accept -- the accepted draft count after a verify pass.
  *   bw_decode_step -- the whole step (embedding .. argmax) for B sequences of
  *       n_rows consecutive tokens each (n_rows = 1: decode; n_rows = K+1:
  *       speculative verify).  Deep-dive page, section 4: an engine facade
@@ -54,8 +55,8 @@
  *    K to a multiple of 512 columns, with zeros); tiles follow each other in
  *    (row block, column tile) order:
  *      q : per tile 32 KB: row r at r*256 bytes, 32-column chunk c of that
- *          row at +c*16 (the chunk's 16 code bytes in the canonical nibble
- *          order of the format)
+ *          row in the 16-byte slot c ^ (r & 7) (the chunk's 16 code bytes in
+ *          the canonical nibble order of the format)
  *      s : per tile 4 KB: 8-row group g at g*256 bytes, chunk c at +c*16:
  *          the 8 rows' fp16 d (Q4_0) or 8 x 2 E4M3 block scales (NVFP4)
  *    so every tile is two contiguous blocks (streamed with plain bulk
@@ -100,6 +101,7 @@ typedef int bw_status;
 
 /* decode-step flags */
 #define BW_STEP_ADVANCE 1u    /* after the step: tokens_in <- tokens_out, pos += n_rows */
+#define BW_MAX_VERIFY_ROWS 8  /* n_rows limit of a verify pass (the last token + up to 7 drafts) */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *bw_status_string(bw_status s);
@@ -295,6 +297,24 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
                          int B, int n_rows, int32_t *tokens_out, float *logits, unsigned flags,
                          void *ws, size_t ws_bytes, void *stream);
 size_t bw_decode_workspace_bytes(const bw_model *m, const bw_kv *kv, int B, int n_rows);
+
+/* Acceptance after a speculative verify pass.  "bw24" deep-dive page
+ * (10100.com), section 5, stage 4 (the verify kernel unrolls the drafts as
+ * sequence rows and masks every row after the first mismatch) and section 1
+ * (the speculative output equals plain greedy decoding token for token).
+ *   tokens_in:  int32 [B*n_rows], the rows the pass ran: t0, d1 .. dK;
+ *   tokens_out: int32 [B*n_rows], its greedy token a_r after each row r.
+ *   n_accept:   int32 [B] out: n = the largest count with d_i == a_{i-1} for
+ *               every i <= n.  The pass has then produced d1..dn, a_n.
+ *   next_out:   optional; next_out[b*next_stride] = a_n (the next pass's t0).
+ *               It may be tokens_in itself with stride n_rows.
+ *   pos:        optional int32 [B]; pos[b] += n + 1 (KV rows past the accepted
+ *               ones are stale and are overwritten by later passes).
+ * Requires 1 <= n_rows <= BW_MAX_VERIFY_ROWS.  Device pointers; asynchronous
+ * on stream; graph capturable. */
+bw_status bw_spec_accept(const int32_t *tokens_in, const int32_t *tokens_out, int B, int n_rows,
+                         int32_t *n_accept, int32_t *next_out, int next_stride, int32_t *pos,
+                         void *stream);
 
 #ifdef __cplusplus
 }

@@ -81,6 +81,7 @@ def lib():
             "or_attend_head": (None, [p, p, p, p, i, i, i, i, i, p]),
             "or_topk_softmax": (None, [p, i, i, p, p]),
             "or_argmax": (C.c_int32, [p, i, p]),
+            "or_spec_accept": (C.c_int32, [p, p, i, p]),
             "or_decode_token": (C.c_int32, [p, p, i, C.c_int32, i, i, p, p, p, p]),
         }
         for name, (res, args) in sig.items():
@@ -208,6 +209,17 @@ def argmax(v):
     margin = np.zeros(1, np.float32)
     i = lib().or_argmax(_ptr(v), v.size, _ptr(margin))
     return int(i), float(margin[0])
+
+
+def spec_accept(rows, greedy):
+    """(n accepted drafts, next token) of one verify pass; rows = [t0, d1..dK],
+    greedy = the greedy token after each row."""
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    g = np.ascontiguousarray(np.asarray(greedy, dtype=np.int32))
+    assert r.size == g.size and r.size >= 1
+    nxt = np.zeros(1, np.int32)
+    n = lib().or_spec_accept(_ptr(r), _ptr(g), r.size, _ptr(nxt))
+    return int(n), int(nxt[0])
 
 
 # --------------------------------------------------------------- the model

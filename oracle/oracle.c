@@ -258,6 +258,18 @@ int32_t or_argmax(const float *v, int n, float *margin)
     return best;
 }
 
+int32_t or_spec_accept(const int32_t *rows, const int32_t *greedy, int n_rows, int32_t *next)
+{
+    int32_t n = 0;
+    for (int i = 1; i < n_rows; i++) {
+        if (rows[i] != greedy[i - 1])
+            break;          /* first rejected draft: nothing after it stands */
+        n++;
+    }
+    *next = greedy[n];
+    return n;
+}
+
 /* ------------------------------------------------------------- decode step */
 
 /* SwiGLU feed-forward: Wd (silu(Wg y) * (Wu y)) */

@@ -120,6 +120,13 @@ void or_attend_head(const float *q, const uint16_t *kpool, const uint16_t *vpool
 void or_topk_softmax(const float *r, int E, int k, int32_t *idx, float *w);
 /* lowest index of the maximum; *margin = max - second largest value */
 int32_t or_argmax(const float *v, int n, float *margin);
+/* Speculative verify acceptance ("bw24" deep-dive page, section 5, stage 4;
+ * section 1: speculative output == greedy output).  rows[0..n_rows) are the
+ * tokens the verify pass ran (the last accepted token, then the drafts);
+ * greedy[r] is the greedy token after row r.  Returns the number of drafts
+ * accepted, n: drafts are taken in order while each one equals the greedy
+ * token of the row before it.  *next = greedy[n]. */
+int32_t or_spec_accept(const int32_t *rows, const int32_t *greedy, int n_rows, int32_t *next);
 
 /* One greedy decode token of sequence b at position pos (writes its K/V into
  * the cache, attends over positions 0..pos).  logits [V] may be NULL;

@@ -24,3 +24,25 @@ def cuda_ok() -> bool:
 TOL = 2e-3
 # argmax tokens must agree whenever the oracle's top-2 margin exceeds this
 MARGIN = 1e-2
+
+
+def check_kv(gpu_pools, ora_pools, page_table, B, first_pos, n_new, page_tokens=16):
+    """The KV cache after a step: every slot the step did not write is
+    bit-identical to the oracle's; the rows it wrote (positions first_pos ..
+    first_pos + n_new - 1 of each sequence) agree within the tolerance (fp16
+    roundings of values whose fp32 sums differ only by summation order, or by
+    the tensor-core path's fp16 activations)."""
+    pt = np.asarray(page_table.cpu() if hasattr(page_table, "cpu") else page_table)
+    for gpu_pool, ora_pool in zip(gpu_pools, ora_pools):
+        # pools are [page][kv head][slot][dim]: bring (page, slot) to the front
+        g = gpu_pool.cpu().numpy().view(np.uint16).transpose(0, 2, 1, 3)
+        o = np.asarray(ora_pool).view(np.uint16).transpose(0, 2, 1, 3)
+        written = np.zeros((g.shape[0], g.shape[1]), dtype=bool)   # [page][slot]
+        for b in range(B):
+            for p in range(first_pos, first_pos + n_new):
+                written[pt[b, p // page_tokens], p % page_tokens] = True
+        untouched = ~written
+        assert np.array_equal(g[untouched], o[untouched])
+        gw = g[written].view(np.float16).astype(np.float64)
+        ow = o[written].view(np.float16).astype(np.float64)
+        assert rel_err(gw, ow) < TOL

@@ -83,6 +83,10 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.bw_repack_q4_0(fake, None, 12, 64, fake, fake, None) == 2
     assert lib.bw_rope_table(C.c_float(-1.0), 64, 16, fake, fake, None) == 1
     assert lib.bw_decode_step(None, None, None, None, 1, 1, None, None, 0, None, 0, None) == 1
+    # verify acceptance: too many rows, no sequences, a zero stride for next_out
+    assert lib.bw_spec_accept(fake, fake, 1, 9, fake, None, 1, None, None) == 1
+    assert lib.bw_spec_accept(fake, fake, 0, 4, fake, None, 1, None, None) == 1
+    assert lib.bw_spec_accept(fake, fake, 1, 4, fake, fake, 0, None, None) == 1
 
 
 def test_workspace_queries_are_host_only(lib):

@@ -9,6 +9,7 @@ import torch
 import oracle
 from token_decode_b200 import bw, runtime, synth
 from gpu_util import MARGIN, TOL, rel_err
+from gpu_util import check_kv as check_kv_pools
 
 pytestmark = pytest.mark.gpu
 
@@ -60,15 +61,8 @@ def _run_steps(cfg, steps, seed=0, n_layers=None, B=None, check_kv=True):
         cur = got_tok
         dec.pos += 1
     if check_kv:
-        for l in range(len(okv.k)):
-            for gpu_pool, ora_pool in ((dkv.k[l], okv.k[l]), (dkv.v[l], okv.v[l])):
-                g = gpu_pool.cpu().numpy().view(np.uint16)
-                # untouched slots are identical; written rows agree within the
-                # tolerance (fp16 rounding of values that differ by fp32 reordering)
-                assert np.mean(g == ora_pool) > 0.99
-                gv = g.view(np.float16).astype(np.float64)
-                ov = ora_pool.view(np.float16).astype(np.float64)
-                assert rel_err(gv, ov) < TOL
+        check_kv_pools(list(dkv.k) + list(dkv.v), list(okv.k) + list(okv.v), dkv.page_table, B,
+                       cfg.ctx, steps)
     return worst
 
 
@@ -80,6 +74,12 @@ def test_tiny_decode_8_steps():
 def test_tiny_nvfp4_two_layers_batch2():
     cfg = synth.CONFIGS["tiny"].with_(fmt=synth.FMT_NVFP4, L=2, B=2)
     _run_steps(cfg, 4)
+
+
+def test_tiny_nvfp4_batch8_tensor_core_path():
+    """8 rows of NVFP4: every projection runs on the tcgen05 GEMM."""
+    cfg = synth.CONFIGS["tiny"].with_(fmt=synth.FMT_NVFP4, B=8)
+    _run_steps(cfg, 3)
 
 
 def test_tiny_batch5_rows_above_gemv_block():
@@ -243,7 +243,7 @@ def test_moe_full_size_layers_batch32():
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("name,layers", [("9b", 3), ("27b", 2)])
+@pytest.mark.parametrize("name,layers", [("9b", 3), ("27b", 2), ("9b_b32", 2)])
 def test_full_size_layers_nvfp4(name, layers):
     """Full-size layer shapes of the NVFP4 models (a few layers, one step)."""
     cfg = synth.CONFIGS[name].with_(L=layers)

@@ -153,6 +153,10 @@ def test_gemv_matches_oracle(fmt, shape, M):
 @pytest.mark.parametrize("M", [1, 2, 4, 6])
 def test_gemv_fused_rmsnorm_residual_silu(fmt, M):
     H, F = 3584, 1024
+    # NVFP4 with more than 4 rows runs on the tensor cores with fp16
+    # activations (tests/test_gpu_mma.py checks that path tightly); here it
+    # gets the graded tolerance, the CUDA-core path the fp32-reordering one
+    tol = 2e-3 if (fmt == synth.FMT_NVFP4 and M > 4) else 1e-5
     wg = synth.quantize(synth.randn((F, H), 0.02, "cuda", 3, "wg"), fmt)
     wu = synth.quantize(synth.randn((F, H), 0.02, "cuda", 3, "wu"), fmt)
     wd = synth.quantize(synth.randn((H, F), 0.02, "cuda", 3, "wd"), fmt)
@@ -168,7 +172,7 @@ def test_gemv_fused_rmsnorm_residual_silu(fmt, M):
         g = oracle.matvec(ogu[0], yn)
         u = oracle.matvec(ogu[1], yn)
         want = np.array([oracle.silu(float(v)) for v in g], np.float32) * u
-        assert rel_err(a[r], want) < 1e-5, rel_err(a[r], want)
+        assert rel_err(a[r], want) < tol, rel_err(a[r], want)
     # down with the residual epilogue (in place)
     act = torch.from_numpy(a).cuda()
     res = torch.randn((M, H), device="cuda")
@@ -176,7 +180,7 @@ def test_gemv_fused_rmsnorm_residual_silu(fmt, M):
     od = oracle.QMat(wd)
     for r in range(M):
         want = res[r].cpu().numpy() + oracle.matvec(od, a[r])
-        assert rel_err(y[r], want) < 1e-5
+        assert rel_err(y[r], want) < tol
 
 
 @pytest.mark.parametrize("fmt", [synth.FMT_Q4_0, synth.FMT_NVFP4])

@@ -479,3 +479,51 @@ def test_moe_all_experts_equal_weights_is_dense_mixture():
     _, want_x = _np_forward(model, kv_np, 0, 5, cfg.ctx)
     assert np.max(np.abs(res["hidden"][-1] - want_x)) < 2e-5 * np.max(np.abs(want_x))
     assert sorted(res["moe_idx"][0].tolist()) == list(range(8))
+
+
+# --------------------------------------------------------- speculative verify
+
+def test_spec_accept_golden():
+    """Hand-worked acceptance cases (tests/golden/spec_accept.txt)."""
+    n_cases = 0
+    for line in _golden_lines("spec_accept.txt"):
+        rows, greedy, want = (part.split() for part in line.split("|"))
+        got = oracle.spec_accept([int(t) for t in rows], [int(t) for t in greedy])
+        assert got == (int(want[0]), int(want[1])), line
+        n_cases += 1
+    assert n_cases == 6
+
+
+def test_spec_accept_reproduces_greedy_sequence():
+    """The section-1 invariant by brute force: with a deterministic next-token
+    function standing in for the model, the tokens a verify pass emits
+    (accepted drafts, then the next token) are exactly the next tokens of
+    plain sequential greedy decoding, for drafts that are right, partly right
+    or wrong."""
+    rng = np.random.default_rng(11)
+    V = 7
+
+    def greedy_next(prefix):
+        h = 2166136261
+        for t in prefix:
+            h = ((h ^ int(t)) * 16777619) & 0xFFFFFFFF
+        return h % V
+
+    for _ in range(400):
+        ctx = list(rng.integers(0, V, size=int(rng.integers(1, 5))))
+        K = int(rng.integers(0, 7))
+        truth = []
+        seq = list(ctx)
+        for _ in range(K + 1):
+            seq.append(greedy_next(seq))
+            truth.append(seq[-1])
+        # drafts: the true continuation with random corruptions
+        drafts = [t if rng.random() < 0.7 else int(rng.integers(0, V)) for t in truth[:K]]
+        rows = [ctx[-1]] + drafts
+        greedy = [greedy_next(ctx + drafts[:r]) for r in range(K + 1)]
+        n, nxt = oracle.spec_accept(rows, greedy)
+        emitted = drafts[:n] + [nxt]
+        assert emitted == truth[: n + 1]
+        # maximal: the next draft, if any, was wrong
+        if n < K:
+            assert drafts[n] != truth[n]

@@ -20,6 +20,7 @@ DEVERR_BAD_PAGE, DEVERR_TIMEOUT, DEVERR_BAD_TOKEN, DEVERR_BAD_POS = 1, 2, 4, 8
 FMT_Q4_0, FMT_NVFP4 = 0, 1
 GEMV_RMSNORM, GEMV_RESIDUAL, GEMV_SILU_GATE, GEMV_ARGMAX = 1, 2, 4, 8
 STEP_ADVANCE = 1
+MAX_VERIFY_ROWS = 8
 
 # every symbol include/bw.h declares (checked by the CPU test-suite)
 EXPORTS = (
@@ -27,7 +28,7 @@ EXPORTS = (
     "bw_repack_bytes", "bw_repack_q4_0", "bw_repack_nvfp4", "bw_gemv_q4_0", "bw_gemv_nvfp4",
     "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
     "bw_paged_attn_decode", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
-    "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes",
+    "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes", "bw_spec_accept",
 )
 
 
@@ -96,6 +97,7 @@ def lib() -> C.CDLL:
             "bw_moe_workspace_bytes": (z, [p, i]),
             "bw_decode_step": (i, [p, p, p, p, i, i, p, p, u, p, z, p]),
             "bw_decode_workspace_bytes": (z, [p, p, i, i]),
+            "bw_spec_accept": (i, [p, p, i, i, p, p, i, p, p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -241,3 +243,11 @@ def decode_step(model: Model, kv: KV, tokens_in, pos, B, n_rows, tokens_out, ws,
     _check(lib().bw_decode_step(C.byref(model), C.byref(kv), _ptr(tokens_in), _ptr(pos), B, n_rows,
                                 _ptr(tokens_out), _ptr(logits), flags, _ptr(ws), ws.numel(),
                                 _stream(stream)), "bw_decode_step")
+
+
+def spec_accept(tokens_in, tokens_out, B, n_rows, n_accept, next_out=None, next_stride=1, pos=None,
+                stream=None):
+    """Accepted draft count per sequence after a verify pass (see bw.h)."""
+    _check(lib().bw_spec_accept(_ptr(tokens_in), _ptr(tokens_out), B, n_rows, _ptr(n_accept),
+                                _ptr(next_out), next_stride, _ptr(pos), _stream(stream)),
+           "bw_spec_accept")

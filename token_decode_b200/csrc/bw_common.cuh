@@ -67,6 +67,11 @@ bw_status gemv_launch(int fmt, const void *wq, const void *wscales, float ts, fl
                       const float *x, int M, const float *gamma, float eps, const float *residual,
                       float *y, int32_t *argmax_out, unsigned flags, const Scratch &sc,
                       cudaStream_t st, int32_t *adv_tokens = nullptr, int32_t *adv_pos = nullptr);
+size_t mma_scratch_bytes(int N, int K, int M);
+bw_status mma_gemm_launch(const void *wq, const void *wscales, float ts, float ts_up, int N, int K,
+                          const float *x, int M, const float *gamma, float eps, const float *residual,
+                          float *y, int32_t *argmax_out, unsigned flags, const Scratch &sc, cudaStream_t st,
+                          int32_t *adv_tokens, int32_t *adv_pos);
 size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages);
 bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
                       void *k_pool, void *v_pool, const int32_t *page_table, int max_pages, int n_pages,

@@ -419,8 +419,11 @@ static GemvPlan plan_gemv(int N, int K, int Mk, bool norm) {
     return pl;
 }
 
+// NVFP4 with more rows than a CUDA-core pass takes goes to the tensor cores
+static bool use_mma(int fmt, int M) { return fmt == BW_FMT_NVFP4 && M > GV_MAX_M; }
+
 size_t gemv_scratch_bytes(int N, int K, int M) {
-    size_t tot = 0;
+    size_t tot = M > GV_MAX_M ? mma_scratch_bytes(N, K, M) : 0;
     for (int m0 = 0; m0 < M; m0 += GV_MAX_M) {
         const int Mk = kernel_m(min(GV_MAX_M, M - m0));
         for (int norm = 0; norm < 2; norm++) {
@@ -465,6 +468,9 @@ bw_status gemv_launch(int fmt, const void *wq, const void *ws_scales, float ts, 
         return BW_ERR_INVALID_ARG;
     if (!(flags & BW_GEMV_ARGMAX) && !y) return BW_ERR_INVALID_ARG;
     if (sc.bytes < gemv_scratch_bytes(N, K, M)) return BW_ERR_INVALID_ARG;
+    if (use_mma(fmt, M))
+        return mma_gemm_launch(wq, ws_scales, ts, ts_up, N, K, x, M, gamma, eps, residual, y, argmax_out, flags, sc,
+                               st, adv_tokens, adv_pos);
     const int ncols = (flags & BW_GEMV_SILU_GATE) ? N / 2 : N;
     for (int m0 = 0; m0 < M; m0 += GV_MAX_M) {
         const int Mr = min(GV_MAX_M, M - m0);

@@ -7,8 +7,10 @@
 // into tiles of 128 rows x 512 columns (16 chunks of 32 columns); N is padded
 // to a multiple of 128 rows and K to a multiple of 512 columns with zeros.
 // Tile (rb, kt) of the codes is one contiguous 32 KB block: row r of the tile
-// at r*256 bytes, chunk c of that row at +c*16 (the 16 code bytes of the
-// chunk in the canonical nibble order).  Tile (rb, kt) of the scales is one
+// at r*256 bytes, chunk c of that row in 16-byte slot c ^ (r & 7) (the 16
+// code bytes of the chunk in the canonical nibble order).  The XOR keeps both
+// access patterns free of shared-memory bank conflicts: 16 lanes reading the
+// 16 chunks of one row, and 8 lanes reading one chunk of 8 consecutive rows.  Tile (rb, kt) of the scales is one
 // contiguous 4 KB block: row group g (rows 8g..8g+7 of the tile) at g*256,
 // chunk c at +c*16: the 8 rows' fp16 d (Q4_0) or 8 x 2 E4M3 block scales
 // (NVFP4).  Tiles follow each other in (rb, kt) order.  Every pipeline stage
@@ -231,7 +233,7 @@ __device__ __forceinline__ void stage_chunk(uint32_t stage_a, int warp, int lane
     const int g = 2 * warp + (lane >> 4), c = lane & 15;
     uint4 w[9];
 #pragma unroll
-    for (int r = 0; r < 8; r++) w[r] = lds_u4(stage_a + (g * 8 + r) * (GV_TC * 16) + c * 16);
+    for (int r = 0; r < 8; r++) w[r] = lds_u4(stage_a + (g * 8 + r) * (GV_TC * 16) + ((c ^ r) * 16));
     w[8] = lds_u4(stage_a + GV_NIB_BYTES + g * (GV_TC * 16) + c * 16);
     float ctv[M];
 #pragma unroll

@@ -25,7 +25,7 @@ __device__ __forceinline__ void src_row(int R, bool inter, int &row, int &which)
 // byte offset of row R's scale slot for chunk c.
 __device__ __forceinline__ size_t tile_code_off(int R, int c, int KT) {
     const size_t tile = static_cast<size_t>(R / GV_TR) * KT + c / GV_TC;
-    return tile * GV_NIB_BYTES + static_cast<size_t>(R % GV_TR) * (GV_TC * 16) + (c % GV_TC) * 16;
+    return tile * GV_NIB_BYTES + static_cast<size_t>(R % GV_TR) * (GV_TC * 16) + ((c % GV_TC) ^ (R % 8)) * 16;
 }
 __device__ __forceinline__ size_t tile_scale_off(int R, int c, int KT) {
     const size_t tile = static_cast<size_t>(R / GV_TR) * KT + c / GV_TC;
