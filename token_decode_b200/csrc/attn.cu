@@ -1,8 +1,8 @@
 // attn.cu -- paged fp16-KV GQA decode attention with fused RoPE and KV write
 // (sm_100a).
 //
-// One CTA per (split, kv head, sequence); the splits of one (sequence, kv
-// head) form a thread-block cluster.  Each CTA
+// One CTA per (split, kv head, sequence).  A split is a contiguous range of
+// the sequence's logical pages.  Each CTA
 //   1. ropes the G = nq/nkv query heads of its kv head for each of the n_rows
 //      query rows (positions pos..pos+n_rows-1),
 //   2. ropes the new rows' k, rounds k and v to fp16 and writes them into the
@@ -10,32 +10,42 @@
 //      page, section 6: logical positions map to physical pages through the
 //      page table; section 5, stage 4: the draft rows of a verify pass share
 //      one cache, causally masked),
-//   3. streams its pages into a ring of shared-memory stages with 1-D bulk
-//      copies (cp.async.bulk, completion on an mbarrier; two pages = 32
-//      tokens per stage) and runs an fp32 online softmax over them,
-//   4. combines the splits through distributed shared memory: after a
-//      cluster barrier every CTA reads the others' (max, sum, partial output)
-//      and writes a slice of the final output, in split order, so results are
+//   3. streams its pages into a ring of shared-memory stages: a producer warp
+//      issues 1-D bulk copies (cp.async.bulk, completion on a "full"
+//      mbarrier) and refills a stage when the consumer warps have released it
+//      (an "empty" mbarrier), so the ring needs no block-wide barrier;
+//   4. runs the scores and P.V of each 64-token stage on the tensor cores
+//      (warp-level mma.m16n8k16, fp32 accumulate): the query rows are padded
+//      to 16 (or 32); q and the probabilities are split into fp16 hi + lo
+//      parts (hi + lo reproduces an fp32 value to ~22 bits) and multiplied by
+//      the exact fp16 K and V in two MMAs each, so the products keep fp32
+//      accuracy; the online softmax keeps one running max and sum per query
+//      row, exchanged between warps through shared memory (two barriers per
+//      stage, double-buffered);
+//   5. writes the output (one split) or leaves (max, sum, partial output) in
+//      the workspace; the last CTA of a
+//      (sequence, kv head) to finish -- an atomic counter, no waiting --
+//      combines the splits in split order.  Results are therefore
 //      deterministic and independent of the physical page order.
-// K rows are read with a per-lane rotation of their 16-byte granules (lane t
-// starts at granule t), which keeps the linear bulk-copied layout free of
-// shared-memory bank conflicts; the query is stored split in two float4
-// planes so its rotated reads are conflict-free too.
-#include <cooperative_groups.h>
+// The q and P planes have padded rows, so their 8x8 fragment loads are free
+// of shared-memory bank conflicts.
 #include <math.h>
 
 #include "bw_common.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace bw {
 
-constexpr int ATT_THREADS = 256;
-constexpr int ATT_WARPS = ATT_THREADS / 32;
-constexpr int ATT_TT = 32;          // tokens per stage (two pages)
-constexpr int ATT_MAXQ = 32;        // query vectors per CTA (G * n_rows)
-constexpr int ATT_MAXR = 8;         // query rows per sequence (1 + draft tokens)
-constexpr int ATT_MAXNS = 16;       // splits (cluster size) per (sequence, kv head)
+constexpr int ATT_CW = 8;                       // consumer warps
+constexpr int ATT_THREADS = (ATT_CW + 1) * 32;  // + one producer warp
+constexpr int ATT_CT = ATT_CW * 32;             // consumer threads
+constexpr int ATT_MAXQ = 32;                    // query vectors per CTA (G * n_rows)
+constexpr int ATT_MAXR = 8;                     // query rows per sequence (1 + draft tokens)
+constexpr int ATT_MAXNS = 64;                   // splits per (sequence, kv head)
+constexpr int ATT_MAXPAGES = 8192;              // page-table width the CTA's page list holds
+constexpr int ATT_ST = 64;                      // tokens per stage: 4 pages, 8 per consumer warp
+constexpr int ATT_PPS = ATT_ST / 16;
+constexpr int ATT_NST = 2;                      // stages in the ring (two CTAs fit an SM)
+constexpr int ATT_PST = ATT_ST + 8;             // padded row of the probability planes (halves)
 
 struct AttnParams {
     const float *qkv;
@@ -48,19 +58,22 @@ struct AttnParams {
     int B, R, nq, nkv, G, Q, n_split;
     float scale;
     float *out;
+    float *part_o;        // [B][nkv][n_split][Q][HD]
+    float *part_ml;       // [B][nkv][n_split][Q][2]
+    uint32_t *cnt;        // [B][nkv] arrival counters (zero between launches)
     uint32_t *err;
 };
 
-template <int HD>
-__host__ __device__ constexpr int att_stages() { return HD == 128 ? 4 : 6; }
-
-template <int HD, int QMAX>
-constexpr size_t att_smem_bytes() {
-    return static_cast<size_t>(att_stages<HD>()) * 2 * ATT_TT * HD * 2   // K/V ring (fp16)
-           + static_cast<size_t>(QMAX) * HD * 4                          // query planes (fp32)
-           + static_cast<size_t>(QMAX) * ATT_TT * 4                      // probabilities
-           + 2 * static_cast<size_t>(ATT_MAXR) * HD * 2                  // new k, v rows (fp16)
-           + static_cast<size_t>(att_stages<HD>()) * 8;                  // mbarriers
+// shared memory: K/V ring, q hi/lo planes, P hi/lo planes (double buffered),
+// row max / row sum exchange (double buffered), new k/v rows, barriers
+template <int HD, int MT>
+__host__ __device__ constexpr size_t att_smem_fixed() {
+    return static_cast<size_t>(ATT_NST) * 2 * ATT_ST * HD * 2            // K/V ring (fp16)
+           + 2 * static_cast<size_t>(16 * MT) * (HD + 8) * 2              // q hi, lo
+           + 2 * 2 * static_cast<size_t>(16 * MT) * ATT_PST * 2           // P hi, lo x 2 buffers
+           + 2 * 2 * static_cast<size_t>(ATT_CW) * (16 * MT) * 4          // row max, row sum x 2 buffers
+           + 2 * static_cast<size_t>(ATT_MAXR) * HD * 2                   // new k, v rows
+           + 2 * static_cast<size_t>(ATT_NST) * 8;                        // mbarriers
 }
 
 // rotate-half RoPE of one pair, rounding each product like the plain formula
@@ -69,50 +82,75 @@ __device__ __forceinline__ void rope_pair(float a, float b, float c, float s, fl
     rb = __fadd_rn(__fmul_rn(b, c), __fmul_rn(a, s));
 }
 
-__device__ __forceinline__ float dot8(const float4 lo, const float4 hi, const uint4 k) {
-    const float2 k0 = __half22float2(*reinterpret_cast<const __half2 *>(&k.x));
-    const float2 k1 = __half22float2(*reinterpret_cast<const __half2 *>(&k.y));
-    const float2 k2 = __half22float2(*reinterpret_cast<const __half2 *>(&k.z));
-    const float2 k3 = __half22float2(*reinterpret_cast<const __half2 *>(&k.w));
-    float d = lo.x * k0.x;
-    d = fmaf(lo.y, k0.y, d);
-    d = fmaf(lo.z, k1.x, d);
-    d = fmaf(lo.w, k1.y, d);
-    d = fmaf(hi.x, k2.x, d);
-    d = fmaf(hi.y, k2.y, d);
-    d = fmaf(hi.z, k3.x, d);
-    d = fmaf(hi.w, k3.y, d);
-    return d;
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(ATT_CT) : "memory"); }
+
+// warp-level tensor-core MMA (m16n8k16, f16 inputs, f32 accumulate) and the
+// 8x8 shared-memory matrix loads that feed it
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t &r0, uint32_t &r1, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t &r0, uint32_t &r1, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
 }
 
-template <int HD, int QMAX>
+// Splits a value into fp16 hi + lo: hi + lo reproduces v to ~22 bits, so two
+// MMAs (hi and lo) against exact fp16 K/V give products at fp32-level accuracy.
+__device__ __forceinline__ void split_f16(float v, __half &hi, __half &lo) {
+    hi = __float2half_rn(v);
+    lo = __float2half_rn(v - __half2float(hi));
+}
+
+template <int HD, int MT>
 __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
-    constexpr int NG = HD / 8;              // 16-byte granules per K/V row
-    constexpr int NST = att_stages<HD>();
-    constexpr int SH = ATT_TT * HD;         // halves per K (or V) stage
-    constexpr int TG = ATT_THREADS / HD;    // P.V token groups: 2 (HD 128) or 4 (HD 64)
-    constexpr int TPG = ATT_TT / TG;        // tokens per group and stage (16 or 8)
-    constexpr int NACC = QMAX;
-    constexpr int QPW = (QMAX + ATT_WARPS - 1) / ATT_WARPS;   // queries owned per warp
+    constexpr int QM = 16 * MT;             // query rows of the MMA tiles (padded)
+    constexpr int QS = HD + 8;              // padded q row (halves)
+    constexpr int NKS = HD / 16;            // k-steps of the score MMA
+    constexpr int WD = HD / ATT_CW;         // output dims per warp in P.V
+    constexpr int NT = WD / 8;              // n-tiles per warp in P.V
+    constexpr int SH = ATT_ST * HD;         // halves per K (or V) stage
+    constexpr uint32_t PAGE_BYTES = 16 * HD * 2;
     extern __shared__ __align__(128) unsigned char att_sm[];
-    __half *ring = reinterpret_cast<__half *>(att_sm);                       // [NST][K|V][SH]
-    float4 *q_lo = reinterpret_cast<float4 *>(ring + static_cast<size_t>(NST) * 2 * SH);  // [QMAX][NG]
-    float4 *q_hi = q_lo + QMAX * NG;                                        // [QMAX][NG]
-    float *P = reinterpret_cast<float *>(q_hi + QMAX * NG);                 // [QMAX][TT]
-    __half *newk = reinterpret_cast<__half *>(P + QMAX * ATT_TT);           // [MAXR][HD]
+    __half *ring = reinterpret_cast<__half *>(att_sm);                                  // [NST][K|V][SH]
+    __half *qh = ring + static_cast<size_t>(ATT_NST) * 2 * SH;                          // [QM][QS]
+    __half *ql = qh + QM * QS;
+    __half *Ph = ql + QM * QS;                                                        // [2][QM][PST]
+    __half *Pl = Ph + 2 * QM * ATT_PST;
+    float *rmax = reinterpret_cast<float *>(Pl + 2 * QM * ATT_PST);                   // [2][CW][QM]
+    float *rsum = rmax + 2 * ATT_CW * QM;
+    __half *newk = reinterpret_cast<__half *>(rsum + 2 * ATT_CW * QM);                // [MAXR][HD]
     __half *newv = newk + ATT_MAXR * HD;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(newv + ATT_MAXR * HD);     // [NST]
-    __shared__ float s_m[ATT_MAXQ], s_l[ATT_MAXQ], s_corr[ATT_MAXQ];
-    __shared__ int s_page[NST][2];
+    uint64_t *full = reinterpret_cast<uint64_t *>(newv + ATT_MAXR * HD);              // [NST]
+    uint64_t *empty = full + ATT_NST;                                                 // [NST]
+    int *pages = reinterpret_cast<int *>(empty + ATT_NST);                            // this split's pages
+    __shared__ bool s_last;
 
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    pdl_trigger();
     if (tid == 0) {
-        for (int s = 0; s < NST; s++) mbar_init(&bar[s], 1);
+        for (int s = 0; s < ATT_NST; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], ATT_CW);
+        }
         fence_mbar_init();
     }
-    __syncthreads();
+    pdl_trigger();
     pdl_wait();
 
     const int p0 = p.pos[b];
@@ -124,59 +162,68 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
     const int n_pg = (len + 15) / 16;
     const int pps = (n_pg + p.n_split - 1) / p.n_split;
     const int pg0 = min(n_pg, split * pps), pg1 = min(n_pg, pg0 + pps);
+    const int npl = pg1 - pg0;                          // pages of this split
     const int t1 = min(len, pg1 * 16);
-    const int n_tiles = (pg1 - pg0 + 1) / 2;
+    const int n_stages = (npl + ATT_PPS - 1) / ATT_PPS;
     const int32_t *pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
     const size_t row_stride = static_cast<size_t>(p.nq + 2 * p.nkv) * HD;
-    constexpr uint32_t PAGE_BYTES = 16 * HD * 2;
 
-    // one thread streams pages: expect the bytes, then issue the bulk copies
-    auto issue = [&](int tile) {
-        const int st = tile % NST;
-        int pages[2];
-        uint32_t bytes = 0;
-        for (int j = 0; j < 2; j++) {
-            const int lp = pg0 + 2 * tile + j;
-            int page = -1;
-            if (lp < pg1) {
-                page = pt[lp];
-                if (page < 0 || page >= p.n_pages) {
-                    set_error(p.err, BW_DEVERR_BAD_PAGE);
-                    page = -1;
+    // the split's physical pages, validated once, in parallel
+    for (int i = tid; i < npl; i += ATT_THREADS) {
+        int page = pt[pg0 + i];
+        if (page < 0 || page >= p.n_pages) {
+            set_error(p.err, BW_DEVERR_BAD_PAGE);
+            page = -1;
+        }
+        pages[i] = page;
+    }
+    __syncthreads();
+
+    if (warp == ATT_CW) {
+        // ---- producer: one lane streams the stages
+        if (lane == 0) {
+            for (int s = 0; s < n_stages; s++) {
+                const int st = s % ATT_NST;
+                if (s >= ATT_NST) mbar_wait(&empty[st], static_cast<uint32_t>((s / ATT_NST - 1) & 1), p.err);
+                uint32_t bytes = 0;
+                for (int j = 0; j < ATT_PPS; j++) {
+                    const int lp = s * ATT_PPS + j;
+                    if (lp < npl && pages[lp] >= 0) bytes += 2 * PAGE_BYTES;
+                }
+                mbar_arrive_tx(&full[st], bytes);
+                __half *sk = ring + static_cast<size_t>(st) * 2 * SH;
+                for (int j = 0; j < ATT_PPS; j++) {
+                    const int lp = s * ATT_PPS + j;
+                    if (lp >= npl || pages[lp] < 0) continue;
+                    const size_t off = (static_cast<size_t>(pages[lp]) * p.nkv + kvh) * 16 * HD;
+                    bulk_g2s(sk + j * 16 * HD, p.k_pool + off, PAGE_BYTES, &full[st]);
+                    bulk_g2s(sk + SH + j * 16 * HD, p.v_pool + off, PAGE_BYTES, &full[st]);
                 }
             }
-            pages[j] = page;
-            s_page[st][j] = page;
-            if (page >= 0) bytes += 2 * PAGE_BYTES;
         }
-        mbar_arrive_tx(&bar[st], bytes);
-        __half *sk = ring + static_cast<size_t>(st) * 2 * SH;
-        for (int j = 0; j < 2; j++) {
-            if (pages[j] < 0) continue;
-            const size_t off = (static_cast<size_t>(pages[j]) * p.nkv + kvh) * 16 * HD;
-            bulk_g2s(sk + j * 16 * HD, p.k_pool + off, PAGE_BYTES, &bar[st]);
-            bulk_g2s(sk + SH + j * 16 * HD, p.v_pool + off, PAGE_BYTES, &bar[st]);
-        }
-    };
-    if (tid == 0)
-        for (int t = 0; t < min(NST, n_tiles); t++) issue(t);
+        return;
+    }
 
-    // ---- 1. roped queries, split into two float4 planes per 8-dim granule
-    for (int i = tid; i < p.Q * (HD / 2); i += ATT_THREADS) {
+    // ---- 1. roped queries as fp16 hi/lo planes (padding rows are zero)
+    for (int i = tid; i < QM * (HD / 2); i += ATT_CT) {
         const int qi = i / (HD / 2), d = i - qi * (HD / 2);
-        const int r = qi / p.G, g = qi - r * p.G;
-        const int h = kvh * p.G + g;
-        const int ppos = max(0, min(p0 + r, p.rope_max_pos - 1));
-        const float *src = p.qkv + (static_cast<size_t>(b) * p.R + r) * row_stride + static_cast<size_t>(h) * HD;
-        const float c = p.rope_cos[static_cast<size_t>(ppos) * (HD / 2) + d];
-        const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
-        float ra, rb;
-        rope_pair(src[d], src[d + HD / 2], c, s, ra, rb);
-        float *lo = reinterpret_cast<float *>(q_lo + qi * NG);
-        float *hi = reinterpret_cast<float *>(q_hi + qi * NG);
-        const int da = d, db = d + HD / 2;
-        ((da & 7) < 4 ? lo : hi)[(da >> 3) * 4 + (da & 3)] = ra;
-        ((db & 7) < 4 ? lo : hi)[(db >> 3) * 4 + (db & 3)] = rb;
+        float ra = 0.0f, rb = 0.0f;
+        if (qi < p.Q) {
+            const int r = qi / p.G, g = qi - r * p.G;
+            const int h = kvh * p.G + g;
+            const int ppos = max(0, min(p0 + r, p.rope_max_pos - 1));
+            const float *src = p.qkv + (static_cast<size_t>(b) * p.R + r) * row_stride + static_cast<size_t>(h) * HD;
+            const float c = p.rope_cos[static_cast<size_t>(ppos) * (HD / 2) + d];
+            const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
+            rope_pair(src[d], src[d + HD / 2], c, s, ra, rb);
+        }
+        __half h0, l0, h1, l1;
+        split_f16(ra, h0, l0);
+        split_f16(rb, h1, l1);
+        qh[qi * QS + d] = h0;
+        ql[qi * QS + d] = l0;
+        qh[qi * QS + d + HD / 2] = h1;
+        ql[qi * QS + d + HD / 2] = l1;
     }
 
     // ---- 2. the new rows' k (roped) and v, rounded to fp16: kept for this
@@ -184,14 +231,13 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
     for (int r = 0; r < p.R; r++) {
         const int ppos = p0 + r;
         if (ppos < pg0 * 16 || ppos >= t1) continue;
-        const int page = pt[ppos / 16];
-        const bool ok = page >= 0 && page < p.n_pages;
-        if (!ok && tid == 0) set_error(p.err, BW_DEVERR_BAD_PAGE);
+        const int page = pages[ppos / 16 - pg0];
+        const bool ok = page >= 0;
         const size_t off = ((static_cast<size_t>(ok ? page : 0) * p.nkv + kvh) * 16 + (ppos & 15)) * HD;
         const float *krow = p.qkv + (static_cast<size_t>(b) * p.R + r) * row_stride +
                             static_cast<size_t>(p.nq + kvh) * HD;
         const float *vrow = krow + static_cast<size_t>(p.nkv) * HD;
-        for (int d = tid; d < HD / 2; d += ATT_THREADS) {
+        for (int d = tid; d < HD / 2; d += ATT_CT) {
             const float c = p.rope_cos[static_cast<size_t>(ppos) * (HD / 2) + d];
             const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
             float ra, rb;
@@ -204,239 +250,330 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
                 p.k_pool[off + d + HD / 2] = hb;
             }
         }
-        for (int d = tid; d < HD; d += ATT_THREADS) {
+        for (int d = tid; d < HD; d += ATT_CT) {
             const __half hv = __float2half_rn(vrow[d]);
             newv[r * HD + d] = hv;
             if (ok) p.v_pool[off + d] = hv;
         }
     }
-    __syncthreads();
+    consumers_sync();
 
-    // ---- 3. stages of 32 tokens: scores, online softmax, P.V
-    float m_run[QPW], l_run[QPW];
+    // ---- 3. stages of 64 tokens on the tensor cores
+    const int gid = lane >> 2, tig = lane & 3;          // fragment row group / thread in group
+    const uint32_t qh_a = smem_u32(qh), ql_a = smem_u32(ql);
+    float m_run[MT][2], l_run[MT][2];
+    float o[MT][NT][4];
 #pragma unroll
-    for (int j = 0; j < QPW; j++) {
-        m_run[j] = -INFINITY;
-        l_run[j] = 0.0f;
+    for (int mt = 0; mt < MT; mt++) {
+#pragma unroll
+        for (int h = 0; h < 2; h++) {
+            m_run[mt][h] = -INFINITY;
+            l_run[mt][h] = 0.0f;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; nt++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) o[mt][nt][i] = 0.0f;
     }
-    float acc[NACC];
-#pragma unroll
-    for (int i = 0; i < NACC; i++) acc[i] = 0.0f;
-    const int od = tid % HD, tq = tid / HD;   // output dim, token group
 
-    for (int tile = 0; tile < n_tiles; tile++) {
-        const int st = tile % NST;
-        mbar_wait(&bar[st], static_cast<uint32_t>((tile / NST) & 1), p.err);
+    for (int s = 0; s < n_stages; s++) {
+        const int st = s % ATT_NST, buf = s & 1;
+        mbar_wait(&full[st], static_cast<uint32_t>((s / ATT_NST) & 1), p.err);
         __half *sk = ring + static_cast<size_t>(st) * 2 * SH;
         __half *sv = sk + SH;
-        const int tb = (pg0 + 2 * tile) * 16;
-        // the rows written by this step replace what the copy brought
-        for (int r = 0; r < p.R; r++) {
-            const int slot = p0 + r - tb;
-            if (slot < 0 || slot >= ATT_TT || p0 + r >= t1 || s_page[st][slot >> 4] < 0) continue;
-            for (int d = tid; d < HD; d += ATT_THREADS) {
-                sk[slot * HD + d] = newk[r * HD + d];
-                sv[slot * HD + d] = newv[r * HD + d];
-            }
+        const int tb = (pg0 + s * ATT_PPS) * 16;       // position of the stage's first token
+        const int nvalid = min(ATT_ST, t1 - tb);
+        bool missing = false;
+        for (int j = 0; j < ATT_PPS; j++) {
+            const int lp = s * ATT_PPS + j;
+            if (lp < npl && pages[lp] < 0) missing = true;
         }
-        __syncthreads();
-        // scores: lane = token, warp w owns queries w, w + 4, ...
-        {
-            const int t = lane;
-            const int tpos = tb + t;
-            const bool tok_ok = tpos < t1 && s_page[st][t >> 4] >= 0;
-            uint4 kr[NG];
-#pragma unroll
-            for (int g = 0; g < NG; g++) {
-                const int g2 = (g + t) & (NG - 1);
-                kr[g] = *reinterpret_cast<const uint4 *>(sk + t * HD + g2 * 8);
-            }
-#pragma unroll
-            for (int j = 0; j < QPW; j++) {
-                const int qi = warp + ATT_WARPS * j;
-                if (qi >= p.Q) break;
-                const int r = qi / p.G;
-                float s = -INFINITY;
-                if (tok_ok && tpos <= p0 + r) {
-                    float dot = 0.0f;
-#pragma unroll
-                    for (int g = 0; g < NG; g++) {
-                        const int g2 = (g + t) & (NG - 1);
-                        dot += dot8(q_lo[qi * NG + g2], q_hi[qi * NG + g2], kr[g]);
-                    }
-                    s = dot * p.scale;
+        const bool fix_new = p0 + p.R > tb && p0 < tb + ATT_ST;
+        if (fix_new || missing || nvalid < ATT_ST) {
+            // rows written by this step replace what the copy brought; V rows the
+            // copy did not fill are zeroed (their probability is 0, 0 * stale could be NaN)
+            for (int r = 0; r < p.R; r++) {
+                const int slot = p0 + r - tb;
+                if (slot < 0 || slot >= nvalid || pages[s * ATT_PPS + (slot >> 4)] < 0) continue;
+                for (int d = tid; d < HD; d += ATT_CT) {
+                    sk[slot * HD + d] = newk[r * HD + d];
+                    sv[slot * HD + d] = newv[r * HD + d];
                 }
-                const float m_new = fmaxf(m_run[j], warp_max(s));
-                const float pr = (s == -INFINITY) ? 0.0f : expf(s - m_new);
-                const float lsum = warp_sum(pr);
-                const float corr = (m_run[j] == -INFINITY) ? 0.0f : expf(m_run[j] - m_new);
-                l_run[j] = l_run[j] * corr + lsum;
-                m_run[j] = m_new;
-                P[qi * ATT_TT + t] = pr;
-                if (lane == 0) s_corr[qi] = corr;
             }
+            for (int e = tid; e < ATT_ST * HD; e += ATT_CT) {
+                const int t = e / HD;
+                const bool hole = t >= nvalid || pages[s * ATT_PPS + (t >> 4)] < 0;
+                if (hole) sv[e] = __float2half_rn(0.0f);
+            }
+            consumers_sync();
         }
-        __syncthreads();
-        // P.V: thread (od, tq) sums tokens [tq*TPG, tq*TPG + TPG) of the stage
+        // scores: warp w takes tokens 8w .. 8w+7 (one n-tile) for every query row
+        const int t0 = warp * 8;
+        float sc[MT][4];
 #pragma unroll
-        for (int i = 0; i < NACC; i++)
-            if (i < p.Q) acc[i] *= s_corr[i];
+        for (int mt = 0; mt < MT; mt++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) sc[mt][i] = 0.0f;
         {
-            const int nt = min(ATT_TT, t1 - tb);
-            const int ta = tq * TPG;
-            const int te = min(nt, ta + TPG);
-            if (ta < te && s_page[st][ta >> 4] >= 0) {
-                for (int t4 = ta; t4 < te; t4 += 4) {
-                    float v[4];
+            const uint32_t k_a = smem_u32(sk) + static_cast<uint32_t>(((t0 + (lane & 7)) * HD + ((lane >> 3) & 1) * 8) * 2);
+            const int arow = (lane & 7) + ((lane >> 3) & 1) * 8, acol = (lane >> 4) * 8;
 #pragma unroll
-                    for (int u = 0; u < 4; u++)
-                        v[u] = (t4 + u < te) ? __half2float(sv[(t4 + u) * HD + od]) : 0.0f;
+            for (int kk = 0; kk < NKS; kk++) {
+                uint32_t b0, b1;
+                ldsm_x2(b0, b1, k_a + kk * 32);
 #pragma unroll
-                    for (int i = 0; i < NACC; i++) {
-                        if (i < p.Q) {
-                            const float4 pr = *reinterpret_cast<const float4 *>(&P[i * ATT_TT + t4]);
-                            float a = acc[i];
-                            a = fmaf(pr.x, v[0], a);
-                            a = fmaf(pr.y, v[1], a);
-                            a = fmaf(pr.z, v[2], a);
-                            a = fmaf(pr.w, v[3], a);
-                            acc[i] = a;
-                        }
-                    }
+                for (int mt = 0; mt < MT; mt++) {
+                    const uint32_t off = static_cast<uint32_t>(((mt * 16 + arow) * QS + kk * 16 + acol) * 2);
+                    uint32_t a[4];
+                    ldsm_x4(a, qh_a + off);
+                    mma16816(sc[mt], a, b0, b1);
+                    ldsm_x4(a, ql_a + off);
+                    mma16816(sc[mt], a, b0, b1);
                 }
             }
         }
-        __syncthreads();
-        if (tid == 0 && tile + NST < n_tiles) issue(tile + NST);
-    }
-    if (lane == 0) {
+        // mask, row maxima over this warp's 8 tokens
+        const int tok0 = t0 + tig * 2;                  // tokens of fragment columns 0, 1
 #pragma unroll
-        for (int j = 0; j < QPW; j++) {
-            const int qi = warp + ATT_WARPS * j;
-            if (qi < p.Q) {
-                s_m[qi] = m_run[j];
-                s_l[qi] = l_run[j];
+        for (int mt = 0; mt < MT; mt++) {
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int qi = mt * 16 + gid + 8 * h;
+                const int lim = (qi < p.Q) ? min(t1, p0 + qi / p.G + 1) : 0;   // causal limit (exclusive)
+#pragma unroll
+                for (int c = 0; c < 2; c++) {
+                    const int t = tok0 + c;
+                    const bool ok = tb + t < lim && pages[s * ATT_PPS + (t >> 4)] >= 0;
+                    sc[mt][2 * h + c] = ok ? sc[mt][2 * h + c] * p.scale : -INFINITY;
+                }
+                float mx = fmaxf(sc[mt][2 * h], sc[mt][2 * h + 1]);
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                if (tig == 0) rmax[(buf * ATT_CW + warp) * QM + qi] = mx;
             }
         }
+        consumers_sync();
+        // probabilities against the new running max; row sums
+        float corr[MT][2];
+        __half *ph = Ph + buf * QM * ATT_PST, *pl = Pl + buf * QM * ATT_PST;
+#pragma unroll
+        for (int mt = 0; mt < MT; mt++) {
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int qi = mt * 16 + gid + 8 * h;
+                float ms = -INFINITY;
+#pragma unroll
+                for (int w2 = 0; w2 < ATT_CW; w2++) ms = fmaxf(ms, rmax[(buf * ATT_CW + w2) * QM + qi]);
+                const float m_new = fmaxf(m_run[mt][h], ms);
+                corr[mt][h] = (m_run[mt][h] == -INFINITY) ? 0.0f : expf(m_run[mt][h] - m_new);
+                m_run[mt][h] = m_new;
+                float sum = 0.0f;
+#pragma unroll
+                for (int c = 0; c < 2; c++) {
+                    const float v = sc[mt][2 * h + c];
+                    const float pr = (v == -INFINITY) ? 0.0f : expf(v - m_new);
+                    sum += pr;
+                    __half hi, lo;
+                    split_f16(pr, hi, lo);
+                    ph[qi * ATT_PST + tok0 + c] = hi;
+                    pl[qi * ATT_PST + tok0 + c] = lo;
+                }
+                sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                if (tig == 0) rsum[(buf * ATT_CW + warp) * QM + qi] = sum;
+            }
+        }
+        consumers_sync();
+#pragma unroll
+        for (int mt = 0; mt < MT; mt++) {
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int qi = mt * 16 + gid + 8 * h;
+                float ss = 0.0f;
+#pragma unroll
+                for (int w2 = 0; w2 < ATT_CW; w2++) ss += rsum[(buf * ATT_CW + w2) * QM + qi];
+                l_run[mt][h] = l_run[mt][h] * corr[mt][h] + ss;
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) {
+                    o[mt][nt][2 * h] *= corr[mt][h];
+                    o[mt][nt][2 * h + 1] *= corr[mt][h];
+                }
+            }
+        }
+        // P.V: warp w produces output dims w*WD .. w*WD + WD - 1 for every query row
+        {
+            const uint32_t ph_a = smem_u32(ph), pl_a = smem_u32(pl);
+            const int arow = (lane & 7) + ((lane >> 3) & 1) * 8, acol = (lane >> 4) * 8;
+            // V^T fragments: matrix i of the x4 load = tokens (i & 1) * 8 .., dims (i >> 1) * 8 ..
+            const int vi = lane >> 3;
+            const uint32_t v_a = smem_u32(sv) + static_cast<uint32_t>(
+                                     (((lane & 7) + (vi & 1) * 8) * HD + warp * WD + (vi >> 1) * 8) * 2);
+#pragma unroll
+            for (int kk = 0; kk < ATT_ST / 16; kk++) {
+                uint32_t bv[4];
+                if constexpr (NT == 2) {
+                    ldsm_x4_t(bv, v_a + kk * 16 * HD * 2);
+                } else {
+                    ldsm_x2_t(bv[0], bv[1], v_a + kk * 16 * HD * 2);
+                }
+#pragma unroll
+                for (int mt = 0; mt < MT; mt++) {
+                    const uint32_t off = static_cast<uint32_t>(((mt * 16 + arow) * ATT_PST + kk * 16 + acol) * 2);
+                    uint32_t a[4];
+                    ldsm_x4(a, ph_a + off);
+#pragma unroll
+                    for (int nt = 0; nt < NT; nt++) mma16816(o[mt][nt], a, bv[2 * nt], bv[2 * nt + 1]);
+                    ldsm_x4(a, pl_a + off);
+#pragma unroll
+                    for (int nt = 0; nt < NT; nt++) mma16816(o[mt][nt], a, bv[2 * nt], bv[2 * nt + 1]);
+                }
+            }
+        }
+        // this warp is done with the stage: release it to the producer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
     }
-    __syncthreads();
 
-    // ---- 4. outputs: merge the token groups (in group order), then write
-    //         directly or combine across the cluster's splits
-    float *s_o = reinterpret_cast<float *>(att_sm);   // [TG][Q][HD]: the ring is drained
+    // ---- 4. the output, or a partial for the split combine
+    const size_t pbase = (static_cast<size_t>(b) * p.nkv + kvh) * p.n_split;
 #pragma unroll
-    for (int i = 0; i < NACC; i++)
-        if (i < p.Q) s_o[(tq * QMAX + i) * HD + od] = acc[i];
-    __syncthreads();
-    for (int e = tid; e < p.Q * HD; e += ATT_THREADS) {
-        const int qi = e / HD, d = e - qi * HD;
-        float o = s_o[qi * HD + d];
+    for (int mt = 0; mt < MT; mt++) {
 #pragma unroll
-        for (int g = 1; g < TG; g++) o += s_o[(g * QMAX + qi) * HD + d];
-        if (p.n_split == 1) {
+        for (int h = 0; h < 2; h++) {
+            const int qi = mt * 16 + gid + 8 * h;
+            if (qi >= p.Q) continue;
             const int r = qi / p.G, gq = qi - r * p.G;
-            p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
-                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = o / s_l[qi];
-        } else {
-            s_o[(TG * QMAX) * HD + e] = o;   // merged partial after the group planes
+#pragma unroll
+            for (int nt = 0; nt < NT; nt++) {
+                const int d = warp * WD + nt * 8 + tig * 2;
+                const float o0 = o[mt][nt][2 * h], o1 = o[mt][nt][2 * h + 1];
+                if (p.n_split == 1) {
+                    float *dst = p.out + (static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
+                                 static_cast<size_t>(kvh * p.G + gq) * HD + d;
+                    dst[0] = o0 / l_run[mt][h];
+                    dst[1] = o1 / l_run[mt][h];
+                } else {
+                    __stcg(reinterpret_cast<float2 *>(p.part_o + ((pbase + split) * p.Q + qi) * HD + d),
+                           make_float2(o0, o1));
+                }
+            }
+            if (p.n_split > 1 && warp == 0 && tig == 0)
+                __stcg(reinterpret_cast<float2 *>(p.part_ml + ((pbase + split) * p.Q + qi) * 2),
+                       make_float2(m_run[mt][h], l_run[mt][h]));
         }
     }
     if (p.n_split == 1) return;
-    float *s_om = s_o + (TG * QMAX) * HD;
-    __syncthreads();
-    cg::cluster_group cluster = cg::this_cluster();
-    cluster.sync();
+    // the last split of this (sequence, kv head) to finish combines all of them
+    __threadfence();
+    consumers_sync();
+    uint32_t *cnt = p.cnt + static_cast<size_t>(b) * p.nkv + kvh;
+    if (tid == 0) s_last = atomicAdd(cnt, 1u) == static_cast<uint32_t>(p.n_split - 1);
+    consumers_sync();
+    if (!s_last) return;
+    __threadfence();
     const int ns = p.n_split;
-    for (int e = split * ATT_THREADS + tid; e < p.Q * HD; e += ns * ATT_THREADS) {
-        const int qi = e / HD, d = e - qi * HD;
-        float ms[ATT_MAXNS];
-        float M = -INFINITY;
-        for (int r2 = 0; r2 < ns; r2++) {
-            ms[r2] = cluster.map_shared_rank(s_m, r2)[qi];
-            M = fmaxf(M, ms[r2]);
-        }
-        float L = 0.0f, O = 0.0f;
-        for (int r2 = 0; r2 < ns; r2++) {
-            if (ms[r2] == -INFINITY) continue;
-            const float w = expf(ms[r2] - M);
-            L = fmaf(cluster.map_shared_rank(s_l, r2)[qi], w, L);
-            O = fmaf(cluster.map_shared_rank(s_om, r2)[qi * HD + d], w, O);
-        }
-        const int r = qi / p.G, g = qi - r * p.G;
-        p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
-              static_cast<size_t>(kvh * p.G + g) * HD + d] = O / L;
+    // every split's (max, sum) in one parallel pass, the weights from shared
+    // memory, then one pass of independent float4 loads of the partial outputs
+    float *s_w = reinterpret_cast<float *>(att_sm);        // [ns][Q] max, then weight (the ring is free)
+    float *s_sl = s_w + ATT_MAXNS * ATT_MAXQ;              // [ns][Q] sums
+    float *s_L = s_sl + ATT_MAXNS * ATT_MAXQ;              // [Q]
+    for (int e = tid; e < ns * p.Q; e += ATT_CT) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + (pbase * p.Q + e) * 2));
+        s_w[e] = ml.x;
+        s_sl[e] = ml.y;
     }
-    cluster.sync();   // keep this CTA's shared memory alive until every reader is done
+    consumers_sync();
+    if (tid < p.Q) {
+        const int qi = tid;
+        float M = -INFINITY;
+        for (int r2 = 0; r2 < ns; r2++) M = fmaxf(M, s_w[r2 * p.Q + qi]);
+        float L = 0.0f;
+        for (int r2 = 0; r2 < ns; r2++) {
+            const float m2 = s_w[r2 * p.Q + qi];
+            const float w = (m2 == -INFINITY) ? 0.0f : expf(m2 - M);
+            s_w[r2 * p.Q + qi] = w;
+            L = fmaf(s_sl[r2 * p.Q + qi], w, L);
+        }
+        s_L[qi] = L;
+    }
+    consumers_sync();
+    for (int e = tid; e < p.Q * (HD / 4); e += ATT_CT) {
+        const int qi = e / (HD / 4), d = (e - qi * (HD / 4)) * 4;
+        const float4 *src = reinterpret_cast<const float4 *>(p.part_o + (pbase * p.Q + qi) * HD + d);
+        const size_t stride = static_cast<size_t>(p.Q) * HD / 4;
+        float4 O = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 16
+        for (int r2 = 0; r2 < ns; r2++) {
+            const float4 v = __ldcg(src + r2 * stride);
+            const float w = s_w[r2 * p.Q + qi];
+            O.x = fmaf(v.x, w, O.x);
+            O.y = fmaf(v.y, w, O.y);
+            O.z = fmaf(v.z, w, O.z);
+            O.w = fmaf(v.w, w, O.w);
+        }
+        const int r = qi / p.G, gq = qi - r * p.G;
+        const float L = s_L[qi];
+        float *dst = p.out + (static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
+                     static_cast<size_t>(kvh * p.G + gq) * HD + d;
+        *reinterpret_cast<float4 *>(dst) = make_float4(O.x / L, O.y / L, O.z / L, O.w / L);
+    }
+    consumers_sync();
+    if (tid == 0) *cnt = 0u;
 }
 
-// Splits per (sequence, kv head) = cluster size: about one CTA per SM in
-// total, at least one stage (two pages) each, at most 16.
+// Splits per (sequence, kv head): enough CTAs for every SM to hold one or
+// two, but at least one stage (4 pages) of context per split.
 static int attn_splits(int B, int nkv, int max_pages) {
     const int groups = B * nkv;
-    int ns = (sm_count() + groups / 2) / groups;
+    int ns = (2 * sm_count() + groups - 1) / groups;
     ns = max(1, min(ns, ATT_MAXNS));
-    ns = min(ns, max(1, (max_pages + 1) / 2));
+    ns = min(ns, max(1, max_pages / 4));
     return ns;
 }
 
 size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages) {
-    (void)B; (void)R; (void)nq; (void)nkv; (void)hd; (void)max_pages;
-    return 0;
+    const int ns = attn_splits(B, nkv, max_pages);
+    if (ns == 1) return 0;
+    const size_t Q = static_cast<size_t>(nq / max(1, nkv)) * R;
+    return align_up(static_cast<size_t>(B) * nkv * ns * Q * hd * 4, BW_WS_ALIGN) +
+           align_up(static_cast<size_t>(B) * nkv * ns * Q * 2 * 4, BW_WS_ALIGN);
 }
 
-template <int HD, int QMAX>
+template <int HD, int MT>
 static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnParams &p) {
-    constexpr size_t smem = att_smem_bytes<HD, QMAX>();
-    static bool attr_set[64] = {};
+    const size_t smem = att_smem_fixed<HD, MT>() + static_cast<size_t>(p.max_pages) * 4;
+    static size_t attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
-    if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(attn_kernel<HD, QMAX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess ||
-            cudaFuncSetAttribute(attn_kernel<HD, QMAX>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-                cudaSuccess) {
+    if (attr_set[dev] < smem) {
+        if (cudaFuncSetAttribute(attn_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem)) != cudaSuccess) {
             (void)cudaGetLastError();
             return BW_ERR_CUDA;
         }
-        attr_set[dev] = true;
+        attr_set[dev] = smem;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ns, nkv, B);
-    cfg.blockDim = dim3(ATT_THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = ns;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
     AttnParams q = p;
     q.n_split = ns;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<HD, QMAX>, q);
-    if (e != cudaSuccess) {
-        (void)cudaGetLastError();
-        return BW_ERR_CUDA;
-    }
-    return BW_OK;
+    return launch_pdl(attn_kernel<HD, MT>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
 }
 
 bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
                       void *k_pool, void *v_pool, const int32_t *page_table, int max_pages,
                       int n_pages, const int32_t *pos, int B, int R, int nq, int nkv, int hd,
                       float *out, const Scratch &sc, cudaStream_t st) {
-    if (!qkv || !rope_cos || !rope_sin || !k_pool || !v_pool || !page_table || !pos || !out)
+    if (!qkv || !rope_cos || !rope_sin || !k_pool || !v_pool || !page_table || !pos || !out || !sc.cnt)
         return BW_ERR_INVALID_ARG;
     if (B <= 0 || R <= 0 || nq <= 0 || nkv <= 0 || max_pages <= 0 || n_pages <= 0 || rope_max_pos <= 0)
         return BW_ERR_INVALID_ARG;
     if ((hd != 128 && hd != 64) || nq % nkv || (nq / nkv) * R > ATT_MAXQ || R > ATT_MAXR)
         return BW_ERR_UNSUPPORTED_SHAPE;
-    if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(qkv)) return BW_ERR_INVALID_ARG;
+    if (max_pages > ATT_MAXPAGES) return BW_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(qkv) || !aligned16(out)) return BW_ERR_INVALID_ARG;
     if (nkv > 65535 || B > 65535) return BW_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<size_t>(B) * nkv > 65536 - CNT_ATTN - 16) return BW_ERR_UNSUPPORTED_SHAPE;
+    if (sc.bytes < attn_scratch_bytes(B, R, nq, nkv, hd, max_pages)) return BW_ERR_INVALID_ARG;
     AttnParams p;
     p.qkv = qkv;
     p.rope_cos = rope_cos;
@@ -457,15 +594,13 @@ bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope
     p.scale = 1.0f / sqrtf(static_cast<float>(hd));
     p.out = out;
     p.err = sc.err;
+    p.cnt = sc.cnt + CNT_ATTN;
     const int ns = attn_splits(B, nkv, max_pages);
-    if (hd == 128) {
-        if (p.Q <= 4) return attn_go<128, 4>(ns, nkv, B, st, p);
-        if (p.Q <= 8) return attn_go<128, 8>(ns, nkv, B, st, p);
-        if (p.Q <= 16) return attn_go<128, 16>(ns, nkv, B, st, p);
-        return attn_go<128, 32>(ns, nkv, B, st, p);
-    }
-    if (p.Q <= 8) return attn_go<64, 8>(ns, nkv, B, st, p);
-    return attn_go<64, 32>(ns, nkv, B, st, p);
+    Carver cv(sc.base);
+    p.part_o = ns > 1 ? cv.take<float>(static_cast<size_t>(B) * nkv * ns * p.Q * hd) : nullptr;
+    p.part_ml = ns > 1 ? cv.take<float>(static_cast<size_t>(B) * nkv * ns * p.Q * 2) : nullptr;
+    if (hd == 128) return p.Q <= 16 ? attn_go<128, 1>(ns, nkv, B, st, p) : attn_go<128, 2>(ns, nkv, B, st, p);
+    return p.Q <= 16 ? attn_go<64, 1>(ns, nkv, B, st, p) : attn_go<64, 2>(ns, nkv, B, st, p);
 }
 
 }  // namespace bw
