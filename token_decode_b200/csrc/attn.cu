@@ -11,9 +11,11 @@
 //      page table; section 5, stage 4: the draft rows of a verify pass share
 //      one cache, causally masked),
 //   3. streams its pages into a ring of shared-memory stages: a producer warp
-//      issues 1-D bulk copies (cp.async.bulk, completion on a "full"
-//      mbarrier) and refills a stage when the consumer warps have released it
-//      (an "empty" mbarrier), so the ring needs no block-wide barrier;
+//      issues TMA tile loads (cp.async.bulk.tensor, boxes of 16 tokens x 64
+//      dims with the 128-byte swizzle, completion on a "full" mbarrier) and
+//      refills a stage when the consumer warps have released it (an "empty"
+//      mbarrier), so the ring needs no block-wide barrier; the swizzle makes
+//      the 8x8 fragment loads of K and V free of bank conflicts;
 //   4. runs the scores and P.V of each 64-token stage on the tensor cores
 //      (warp-level mma.m16n8k16, fp32 accumulate): the query rows are padded
 //      to 16 (or 32); q and the probabilities are split into fp16 hi + lo
@@ -29,7 +31,10 @@
 //      deterministic and independent of the physical page order.
 // The q and P planes have padded rows, so their 8x8 fragment loads are free
 // of shared-memory bank conflicts.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <math.h>
+#include <string.h>
 
 #include "bw_common.cuh"
 
@@ -44,7 +49,6 @@ constexpr int ATT_MAXNS = 64;                   // splits per (sequence, kv head
 constexpr int ATT_MAXPAGES = 8192;              // page-table width the CTA's page list holds
 constexpr int ATT_ST = 64;                      // tokens per stage: 4 pages, 8 per consumer warp
 constexpr int ATT_PPS = ATT_ST / 16;
-constexpr int ATT_NST = 2;                      // stages in the ring (two CTAs fit an SM)
 constexpr int ATT_PST = ATT_ST + 8;             // padded row of the probability planes (halves)
 
 struct AttnParams {
@@ -62,18 +66,22 @@ struct AttnParams {
     float *part_ml;       // [B][nkv][n_split][Q][2]
     uint32_t *cnt;        // [B][nkv] arrival counters (zero between launches)
     uint32_t *err;
+    // the layer's K and V pools as 2-D tensors [n_pages*nkv*16 rows][hd],
+    // loaded in boxes of 16 rows x 64 dims with the 128-byte swizzle
+    CUtensorMap tmk, tmv;
 };
 
 // shared memory: K/V ring, q hi/lo planes, P hi/lo planes (double buffered),
 // row max / row sum exchange (double buffered), new k/v rows, barriers
-template <int HD, int MT>
+template <int HD, int MT, int NST>
 __host__ __device__ constexpr size_t att_smem_fixed() {
-    return static_cast<size_t>(ATT_NST) * 2 * ATT_ST * HD * 2            // K/V ring (fp16)
+    return static_cast<size_t>(NST) * 2 * ATT_ST * HD * 2                // K/V ring (fp16)
            + 2 * static_cast<size_t>(16 * MT) * (HD + 8) * 2              // q hi, lo
            + 2 * 2 * static_cast<size_t>(16 * MT) * ATT_PST * 2           // P hi, lo x 2 buffers
            + 2 * 2 * static_cast<size_t>(ATT_CW) * (16 * MT) * 4          // row max, row sum x 2 buffers
            + 2 * static_cast<size_t>(ATT_MAXR) * HD * 2                   // new k, v rows
-           + 2 * static_cast<size_t>(ATT_NST) * 8;                        // mbarriers
+           + 2 * static_cast<size_t>(NST) * 8                             // mbarriers
+           + 1024;                                                        // ring alignment
 }
 
 // rotate-half RoPE of one pair, rounding each product like the plain formula
@@ -83,6 +91,25 @@ __device__ __forceinline__ void rope_pair(float a, float b, float c, float s, fl
 }
 
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(ATT_CT) : "memory"); }
+
+// TMA tile load of one 2-D box (no multicast), completion on `bar`
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tmap, int x, int y, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Byte offset of (token T of a stage, dim d) in a K or V stage: page T/16 is
+// hd/64 boxes of 16 rows x 128 bytes; the 128-byte swizzle puts 16-byte chunk
+// c of box row t at chunk c ^ (t & 7).
+template <int HD>
+__device__ __forceinline__ uint32_t kv_off(int T, int d) {
+    const int t = T & 15, c = (d & 63) >> 3;
+    return static_cast<uint32_t>((((T >> 4) * (HD / 64) + (d >> 6)) << 11) + (t << 7) + ((c ^ (t & 7)) << 4) +
+                                 ((d & 7) << 1));
+}
 
 // warp-level tensor-core MMA (m16n8k16, f16 inputs, f32 accumulate) and the
 // 8x8 shared-memory matrix loads that feed it
@@ -117,8 +144,11 @@ __device__ __forceinline__ void split_f16(float v, __half &hi, __half &lo) {
     lo = __float2half_rn(v - __half2float(hi));
 }
 
-template <int HD, int MT>
-__global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
+// NST: ring stages -- 2 when two CTAs share an SM, 4 when each CTA has an SM
+// to itself (a short split then has all its pages in flight at once).
+template <int HD, int MT, int NST>
+__global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const __grid_constant__ AttnParams p) {
+    constexpr int ATT_NST = NST;
     constexpr int QM = 16 * MT;             // query rows of the MMA tiles (padded)
     constexpr int QS = HD + 8;              // padded q row (halves)
     constexpr int NKS = HD / 16;            // k-steps of the score MMA
@@ -126,7 +156,9 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
     constexpr int NT = WD / 8;              // n-tiles per warp in P.V
     constexpr int SH = ATT_ST * HD;         // halves per K (or V) stage
     constexpr uint32_t PAGE_BYTES = 16 * HD * 2;
-    extern __shared__ __align__(128) unsigned char att_sm[];
+    extern __shared__ __align__(1024) unsigned char att_sm_raw[];
+    // the swizzle pattern follows address bits, so the ring starts on 1024 bytes
+    unsigned char *att_sm = att_sm_raw + ((1024u - (smem_u32(att_sm_raw) & 1023u)) & 1023u);
     __half *ring = reinterpret_cast<__half *>(att_sm);                                  // [NST][K|V][SH]
     __half *qh = ring + static_cast<size_t>(ATT_NST) * 2 * SH;                          // [QM][QS]
     __half *ql = qh + QM * QS;
@@ -191,13 +223,17 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
                     if (lp < npl && pages[lp] >= 0) bytes += 2 * PAGE_BYTES;
                 }
                 mbar_arrive_tx(&full[st], bytes);
-                __half *sk = ring + static_cast<size_t>(st) * 2 * SH;
+                unsigned char *sk = reinterpret_cast<unsigned char *>(ring + static_cast<size_t>(st) * 2 * SH);
                 for (int j = 0; j < ATT_PPS; j++) {
                     const int lp = s * ATT_PPS + j;
                     if (lp >= npl || pages[lp] < 0) continue;
-                    const size_t off = (static_cast<size_t>(pages[lp]) * p.nkv + kvh) * 16 * HD;
-                    bulk_g2s(sk + j * 16 * HD, p.k_pool + off, PAGE_BYTES, &full[st]);
-                    bulk_g2s(sk + SH + j * 16 * HD, p.v_pool + off, PAGE_BYTES, &full[st]);
+                    const int y = (pages[lp] * p.nkv + kvh) * 16;     // first row of this page
+#pragma unroll
+                    for (int h = 0; h < HD / 64; h++) {
+                        const int box = (j * (HD / 64) + h) << 11;
+                        tma_load_2d(sk + box, &p.tmk, h * 64, y, &full[st]);
+                        tma_load_2d(sk + SH * 2 + box, &p.tmv, h * 64, y, &full[st]);
+                    }
                 }
             }
         }
@@ -292,19 +328,25 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
         if (fix_new || missing || nvalid < ATT_ST) {
             // rows written by this step replace what the copy brought; V rows the
             // copy did not fill are zeroed (their probability is 0, 0 * stale could be NaN)
+            unsigned char *skb = reinterpret_cast<unsigned char *>(sk), *svb = reinterpret_cast<unsigned char *>(sv);
             for (int r = 0; r < p.R; r++) {
                 const int slot = p0 + r - tb;
                 if (slot < 0 || slot >= nvalid || pages[s * ATT_PPS + (slot >> 4)] < 0) continue;
                 for (int d = tid; d < HD; d += ATT_CT) {
-                    sk[slot * HD + d] = newk[r * HD + d];
-                    sv[slot * HD + d] = newv[r * HD + d];
+                    *reinterpret_cast<__half *>(skb + kv_off<HD>(slot, d)) = newk[r * HD + d];
+                    *reinterpret_cast<__half *>(svb + kv_off<HD>(slot, d)) = newv[r * HD + d];
                 }
             }
-            for (int e = tid; e < ATT_ST * HD; e += ATT_CT) {
-                const int t = e / HD;
-                const bool hole = t >= nvalid || pages[s * ATT_PPS + (t >> 4)] < 0;
-                if (hole) sv[e] = __float2half_rn(0.0f);
+            // a token's 128-byte box rows hold only its own dims: zero them whole
+            for (int e = tid; e < ATT_ST * (HD / 64) * 8; e += ATT_CT) {
+                const int T = e / ((HD / 64) * 8), rem = e - T * ((HD / 64) * 8);
+                const bool hole = T >= nvalid || pages[s * ATT_PPS + (T >> 4)] < 0;
+                if (hole) {
+                    const uint32_t row = static_cast<uint32_t>((((T >> 4) * (HD / 64) + (rem >> 3)) << 11) + ((T & 15) << 7));
+                    *reinterpret_cast<uint4 *>(svb + row + ((rem & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                }
             }
+            fence_async_smem();   // the next TMA load into this stage comes after these writes
             consumers_sync();
         }
         // scores: warp w takes tokens 8w .. 8w+7 (one n-tile) for every query row
@@ -315,12 +357,13 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
 #pragma unroll
             for (int i = 0; i < 4; i++) sc[mt][i] = 0.0f;
         {
-            const uint32_t k_a = smem_u32(sk) + static_cast<uint32_t>(((t0 + (lane & 7)) * HD + ((lane >> 3) & 1) * 8) * 2);
+            const uint32_t k_a = smem_u32(sk);
+            const int ktok = t0 + (lane & 7), khalf = ((lane >> 3) & 1) * 8;
             const int arow = (lane & 7) + ((lane >> 3) & 1) * 8, acol = (lane >> 4) * 8;
 #pragma unroll
             for (int kk = 0; kk < NKS; kk++) {
                 uint32_t b0, b1;
-                ldsm_x2(b0, b1, k_a + kk * 32);
+                ldsm_x2(b0, b1, k_a + kv_off<HD>(ktok, kk * 16 + khalf));
 #pragma unroll
                 for (int mt = 0; mt < MT; mt++) {
                     const uint32_t off = static_cast<uint32_t>(((mt * 16 + arow) * QS + kk * 16 + acol) * 2);
@@ -406,15 +449,15 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
             const int arow = (lane & 7) + ((lane >> 3) & 1) * 8, acol = (lane >> 4) * 8;
             // V^T fragments: matrix i of the x4 load = tokens (i & 1) * 8 .., dims (i >> 1) * 8 ..
             const int vi = lane >> 3;
-            const uint32_t v_a = smem_u32(sv) + static_cast<uint32_t>(
-                                     (((lane & 7) + (vi & 1) * 8) * HD + warp * WD + (vi >> 1) * 8) * 2);
+            const uint32_t v_a = smem_u32(sv);
+            const int vtok = (lane & 7) + (vi & 1) * 8, vdim = warp * WD + (vi >> 1) * 8;
 #pragma unroll
             for (int kk = 0; kk < ATT_ST / 16; kk++) {
                 uint32_t bv[4];
                 if constexpr (NT == 2) {
-                    ldsm_x4_t(bv, v_a + kk * 16 * HD * 2);
+                    ldsm_x4_t(bv, v_a + kv_off<HD>(kk * 16 + vtok, vdim));
                 } else {
-                    ldsm_x2_t(bv[0], bv[1], v_a + kk * 16 * HD * 2);
+                    ldsm_x2_t(bv[0], bv[1], v_a + kv_off<HD>(kk * 16 + vtok, vdim));
                 }
 #pragma unroll
                 for (int mt = 0; mt < MT; mt++) {
@@ -521,14 +564,17 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const AttnParams p) {
     if (tid == 0) *cnt = 0u;
 }
 
-// Splits per (sequence, kv head): enough CTAs for every SM to hold one or
-// two, but at least one stage (4 pages) of context per split.
+// Splits per (sequence, kv head).  Many (sequence, kv head) groups: one
+// split, the grid already fills the GPU.  Few: about sqrt(pages) splits --
+// a split streams pages/ns pages, the merge reads ns partials -- bounded so
+// that every CTA has an SM (and a deep ring) to itself.
 static int attn_splits(int B, int nkv, int max_pages) {
     const int groups = B * nkv;
-    int ns = (2 * sm_count() + groups - 1) / groups;
-    ns = max(1, min(ns, ATT_MAXNS));
+    if (groups >= sm_count()) return 1;
+    int ns = static_cast<int>(sqrt(static_cast<double>(max_pages)) + 0.5);
+    ns = min(ns, sm_count() / groups);
     ns = min(ns, max(1, max_pages / 4));
-    return ns;
+    return max(1, min(ns, ATT_MAXNS));
 }
 
 size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages) {
@@ -539,15 +585,66 @@ size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages) 
            align_up(static_cast<size_t>(B) * nkv * ns * Q * 2 * 4, BW_WS_ALIGN);
 }
 
-template <int HD, int MT>
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// dependency on the driver library); encoded maps are cached per pool.
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            (void)cudaGetLastError();
+            return nullptr;
+        }
+        fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+static bool kv_tensor_map(CUtensorMap *out, void *pool, int n_pages, int nkv, int hd) {
+    struct Entry {
+        void *pool;
+        int rows, hd;
+        CUtensorMap map;
+    };
+    static Entry cache[512];
+    static int n_cache = 0, next = 0;
+    const int rows = n_pages * nkv * 16;
+    for (int i = 0; i < n_cache; i++)
+        if (cache[i].pool == pool && cache[i].rows == rows && cache[i].hd == hd) {
+            *out = cache[i].map;
+            return true;
+        }
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(hd), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(hd) * 2};
+    const cuuint32_t box[2] = {64, 16};
+    const cuuint32_t estr[2] = {1, 1};
+    CUtensorMap m;
+    if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pool, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+        return false;
+    Entry &e = cache[n_cache < 512 ? n_cache++ : (next++ % 512)];
+    e.pool = pool;
+    e.rows = rows;
+    e.hd = hd;
+    e.map = m;
+    *out = m;
+    return true;
+}
+
+template <int HD, int MT, int NST>
 static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnParams &p) {
-    const size_t smem = att_smem_fixed<HD, MT>() + static_cast<size_t>(p.max_pages) * 4;
+    const size_t smem = att_smem_fixed<HD, MT, NST>() + static_cast<size_t>(p.max_pages) * 4;
     static size_t attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
     if (attr_set[dev] < smem) {
-        if (cudaFuncSetAttribute(attn_kernel<HD, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  static_cast<int>(smem)) != cudaSuccess) {
             (void)cudaGetLastError();
             return BW_ERR_CUDA;
@@ -556,7 +653,14 @@ static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnPara
     }
     AttnParams q = p;
     q.n_split = ns;
-    return launch_pdl(attn_kernel<HD, MT>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
+    return launch_pdl(attn_kernel<HD, MT, NST>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
+}
+
+template <int HD, int MT>
+static bw_status attn_go_st(int ns, int nkv, int B, cudaStream_t st, const AttnParams &p) {
+    // a grid that fits one CTA per SM gets the deep ring
+    return static_cast<long>(ns) * nkv * B <= sm_count() ? attn_go<HD, MT, 4>(ns, nkv, B, st, p)
+                                                         : attn_go<HD, MT, 2>(ns, nkv, B, st, p);
 }
 
 bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
@@ -595,12 +699,15 @@ bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope
     p.out = out;
     p.err = sc.err;
     p.cnt = sc.cnt + CNT_ATTN;
+    if (static_cast<long long>(n_pages) * nkv * 16 > 0xffffffffLL) return BW_ERR_UNSUPPORTED_SHAPE;
+    if (!kv_tensor_map(&p.tmk, k_pool, n_pages, nkv, hd) || !kv_tensor_map(&p.tmv, v_pool, n_pages, nkv, hd))
+        return BW_ERR_CUDA;
     const int ns = attn_splits(B, nkv, max_pages);
     Carver cv(sc.base);
     p.part_o = ns > 1 ? cv.take<float>(static_cast<size_t>(B) * nkv * ns * p.Q * hd) : nullptr;
     p.part_ml = ns > 1 ? cv.take<float>(static_cast<size_t>(B) * nkv * ns * p.Q * 2) : nullptr;
-    if (hd == 128) return p.Q <= 16 ? attn_go<128, 1>(ns, nkv, B, st, p) : attn_go<128, 2>(ns, nkv, B, st, p);
-    return p.Q <= 16 ? attn_go<64, 1>(ns, nkv, B, st, p) : attn_go<64, 2>(ns, nkv, B, st, p);
+    if (hd == 128) return p.Q <= 16 ? attn_go_st<128, 1>(ns, nkv, B, st, p) : attn_go_st<128, 2>(ns, nkv, B, st, p);
+    return p.Q <= 16 ? attn_go_st<64, 1>(ns, nkv, B, st, p) : attn_go_st<64, 2>(ns, nkv, B, st, p);
 }
 
 }  // namespace bw

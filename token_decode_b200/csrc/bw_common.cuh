@@ -216,6 +216,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
     set_error(err, BW_DEVERR_TIMEOUT);
     return false;
 }
+// orders this thread's generic-proxy shared-memory writes before later
+// async-proxy accesses (TMA, bulk copies, tensor-core operand reads)
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 // 1-D bulk copy global -> this CTA's shared memory, completing on `bar`
 // (16-byte aligned addresses, size a multiple of 16).  No multicast.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {

@@ -24,9 +24,10 @@
 //              A slots in tensor memory with tcgen05.st, then run the
 //              epilogue from the accumulator (tcgen05.ld).
 // MMA: kind::f16, M = 128 weight rows, N = the activation rows padded to 16
-// or 32, K = 16 per instruction; A from tensor memory, B (activations,
-// staged once per CTA for its K slice) from shared memory in the canonical
-// K-major layout without swizzle; fp32 accumulators in tensor memory, double
+// or 32, K = 16 per instruction; A from tensor memory, B from shared memory
+// in the canonical K-major layout without swizzle.  The activations are
+// packed into that layout once per GEMM (act_pack_kernel, with the RMSNorm
+// fused) and each CTA fetches its K slice with one bulk copy; fp32 accumulators in tensor memory, double
 // buffered so the next row block's MMAs overlap the epilogue.
 // Work split: 128-row blocks x K slices (as the CUDA-core GEMV); slices
 // leave partial sums, the last CTA of a row block adds them in slice order.
@@ -50,9 +51,7 @@ struct MmaParams {
     const uint8_t *q, *s;
     int N, K, M, Mp;                     // Mp: rows padded to 16 or 32 (the MMA's N)
     int RB, KT, S, CT, per_slice;
-    const float *x;                      // [M][K]
-    const float *rnorm;                  // [M] or null: B = (x * rnorm) * gamma
-    const float *gamma;
+    const uint8_t *bpk;                  // activations, fp16, packed (act_pack_kernel)
     const float *residual;
     float *y;
     int32_t *argmax_out;
@@ -143,7 +142,6 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
         :
         : "memory");
 }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void dq_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, K-major canonical layout without swizzle:
@@ -203,6 +201,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
     uint64_t *full = bars, *empty = bars + MM_NST;
     uint64_t *afull = empty + MM_NST, *aempty = afull + MM_NA;
     uint64_t *dfull = aempty + MM_NA, *dempty = dfull + 2;
+    uint64_t *bfull = dempty + 2;
     __shared__ uint32_t s_tmem;
     __shared__ float s_bv[MM_DW][MM_MAXM];
     __shared__ int s_bi[MM_DW][MM_MAXM];
@@ -229,6 +228,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
             mbar_init(&dfull[i], 1);
             mbar_init(&dempty[i], MM_DW);
         }
+        mbar_init(bfull, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -242,9 +242,11 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
     pdl_trigger();
 
     if (warp == 0) {
-        // ---- producer: constant weights only, no dependency wait
+        // ---- producer: the first stages of constant weights before the
+        //      dependency wait, then this slice's packed activations (one
+        //      contiguous block), then the rest of the weights
         if (lane == 0) {
-            for (int t = 0; t < n_tiles; t++) {
+            auto issue = [&](int t) {
                 const int s = t % MM_NST;
                 if (t >= MM_NST) mbar_wait(&empty[s], static_cast<uint32_t>((t / MM_NST - 1) & 1), p.err);
                 const int item = t / T, kt = kt0 + (t - item * T);
@@ -254,22 +256,30 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
                 mbar_arrive_tx(&full[s], GV_STAGE_BYTES);
                 bulk_g2s(st, p.q + tile * GV_NIB_BYTES, GV_NIB_BYTES, &full[s]);
                 bulk_g2s(st + GV_NIB_BYTES, p.s + tile * GV_SC_BYTES, GV_SC_BYTES, &full[s]);
+            };
+            const int pre = min(MM_NST, n_tiles);
+            for (int t = 0; t < pre; t++) issue(t);
+            pdl_wait();
+            if (n_tiles > 0) {
+                const uint32_t col_bytes = static_cast<uint32_t>(GV_TC * 4 * (p.Mp / 8) * 128);   // one column tile
+                mbar_arrive_tx(bfull, static_cast<uint32_t>(T) * col_bytes);
+                bulk_g2s(bsm, p.bpk + static_cast<size_t>(kt0) * col_bytes, static_cast<uint32_t>(T) * col_bytes, bfull);
             }
+            for (int t = pre; t < n_tiles; t++) issue(t);
         }
     } else if (warp == 1) {
         // ---- MMA issuer
-        pdl_wait();
-        if (lane == 0) {
+        if (lane == 0 && n_items > 0) {
             const uint32_t idesc = mma_idesc_f16(p.Mp);
             const uint32_t b_a = smem_u32(bsm);
             const uint32_t lbo = static_cast<uint32_t>(p.Mp / 8) * 128u, sbo = 128u;
-            // B staged and visible to the tensor core (dequant warps arrive on dempty[1] once)
-            mbar_wait(&dempty[1], 0u, p.err);
+            // the slice's activations have landed in shared memory
+            mbar_wait(bfull, 0u, p.err);
             tc_fence_after();
             int g = 0;   // A-slot step
             for (int item = 0; item < n_items; item++) {
                 const int db = item & 1;
-                if (item >= 2) mbar_wait(&dempty[db], static_cast<uint32_t>(((item - 2) / 2 + (db ? 1 : 0)) & 1), p.err);
+                if (item >= 2) mbar_wait(&dempty[db], static_cast<uint32_t>(((item - 2) / 2) & 1), p.err);
                 tc_fence_after();
                 const uint32_t d_t = tmem + MM_ACC_COL + static_cast<uint32_t>(db * p.Mp);
                 for (int kt = 0; kt < T; kt++) {
@@ -298,45 +308,6 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
         const int qd = warp & 3;                  // tensor-memory lane quarter this warp may access
         const int r = qd * 32 + lane;             // tile row = tensor-memory lane
         const int dtid = dw * 32 + lane;          // 0..127
-        pdl_wait();
-        // stage this slice's activations as fp16 in the canonical K-major layout
-        {
-            const int Mp = p.Mp, G8 = Mp / 8;
-            const int units = CS * 4 * Mp;        // (core column, row) pairs, 8 elements each
-            const int kbase = kt0 * 512;
-            for (int u = dtid; u < units; u += MM_DW * 32) {
-                const int m = u % Mp, kc = u / Mp;
-                const int k = kbase + kc * 8;
-                uint32_t h[4] = {0u, 0u, 0u, 0u};
-                if (m < p.M && k < p.K) {
-                    const float *xr = p.x + static_cast<size_t>(m) * p.K + k;
-                    float v[8];
-                    const float4 a0 = *reinterpret_cast<const float4 *>(xr);
-                    const float4 a1 = *reinterpret_cast<const float4 *>(xr + 4);
-                    v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
-                    v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
-                    if (p.rnorm) {
-                        const float rn = p.rnorm[m];
-                        const float4 g0 = *reinterpret_cast<const float4 *>(p.gamma + k);
-                        const float4 g1 = *reinterpret_cast<const float4 *>(p.gamma + k + 4);
-                        const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-#pragma unroll
-                        for (int i = 0; i < 8; i++) v[i] = __fmul_rn(__fmul_rn(v[i], rn), gg[i]);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; i++) {
-                        __half2 hh = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
-                        h[i] = *reinterpret_cast<uint32_t *>(&hh);
-                    }
-                }
-                *reinterpret_cast<uint4 *>(bsm + (static_cast<size_t>(kc) * G8 + (m >> 3)) * 128 + (m & 7) * 16) =
-                    make_uint4(h[0], h[1], h[2], h[3]);
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&dempty[1]);   // "B ready" (the phase-0 completion of dempty[1])
-        }
-
         const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16);
         const float tsc = ((p.flags & BW_GEMV_SILU_GATE) && (r & 7) >= 4) ? p.ts_up : p.ts;
         float bestv[MM_MAXM];
@@ -380,7 +351,9 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
                     if (lane == 0) mbar_arrive(&afull[a]);
                 }
             }
-            // ---- accumulator of this row block
+            // ---- accumulator of this row block (the epilogue reads what earlier
+            //      kernels wrote: wait for them once)
+            if (item == 0) pdl_wait();
             const int db = item & 1;
             mbar_wait(&dfull[db], static_cast<uint32_t>((item >> 1) & 1), p.err);
             tc_fence_after();
@@ -457,6 +430,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
             }
         }
 
+        pdl_wait();   // (already done by the first epilogue when this CTA had work)
         // ---- greedy argmax: CTA partials, the last CTA reduces
         if (p.flags & BW_GEMV_ARGMAX) {
 #pragma unroll
@@ -537,23 +511,57 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
     }
 }
 
-// Per-row RMSNorm factor r[m] = 1 / sqrt(mean(x[m]^2) + eps) (the B staging
-// applies (x * r) * gamma, the order of the RMSNorm definition).
-__global__ void rownorm_kernel(const float *x, int K, float eps, float *rnorm) {
+// Activations -> fp16 B operand in the canonical K-major layout of the MMA:
+// core column kc (8 consecutive k) of row m at ((kc * Mp/8 + m/8) * 8 + m%8)
+// * 16 bytes; the column tiles of K are therefore contiguous blocks.  Rows
+// M..Mp-1 and columns K..KT*512-1 are zero.  With gamma, the row is
+// normalized first: (x * r) * gamma, r = 1 / sqrt(mean(x^2) + eps).
+__global__ void act_pack_kernel(const float *x, int M, int Mp, int K, int KT, const float *gamma, float eps,
+                                uint8_t *out) {
     pdl_trigger();
     pdl_wait();
     __shared__ float red[32];
+    __shared__ float s_rn;
     const int m = blockIdx.x;
-    const float *xr = x + static_cast<size_t>(m) * K;
-    float ss = 0.0f;
-    for (int k = threadIdx.x; k < K; k += blockDim.x) ss = fma_rn(xr[k], xr[k], ss);
-    ss = warp_sum(ss);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float t = 0.0f;
-        for (int w = 0; w < static_cast<int>(blockDim.x >> 5); w++) t += red[w];
-        rnorm[m] = 1.0f / sqrtf(t / static_cast<float>(K) + eps);
+    const bool real = m < M;
+    const float *xr = x + static_cast<size_t>(real ? m : 0) * K;
+    if (gamma && real) {
+        float ss = 0.0f;
+        for (int k = threadIdx.x; k < K; k += blockDim.x) ss = fma_rn(xr[k], xr[k], ss);
+        ss = warp_sum(ss);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float t = 0.0f;
+            for (int w = 0; w < static_cast<int>(blockDim.x >> 5); w++) t += red[w];
+            s_rn = 1.0f / sqrtf(t / static_cast<float>(K) + eps);
+        }
+        __syncthreads();
+    }
+    const float rn = (gamma && real) ? s_rn : 1.0f;
+    const int KC = KT * 64;
+    for (int kc = threadIdx.x; kc < KC; kc += blockDim.x) {
+        const int k = kc * 8;
+        uint32_t h[4] = {0u, 0u, 0u, 0u};
+        if (real && k < K) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(xr + k);
+            const float4 a1 = *reinterpret_cast<const float4 *>(xr + k + 4);
+            float v[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            if (gamma) {
+                const float4 g0 = *reinterpret_cast<const float4 *>(gamma + k);
+                const float4 g1 = *reinterpret_cast<const float4 *>(gamma + k + 4);
+                const float gg[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+                for (int i = 0; i < 8; i++) v[i] = __fmul_rn(__fmul_rn(v[i], rn), gg[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                __half2 hh = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+                h[i] = *reinterpret_cast<uint32_t *>(&hh);
+            }
+        }
+        *reinterpret_cast<uint4 *>(out + (static_cast<size_t>(kc) * (Mp / 8) + (m >> 3)) * 128 + (m & 7) * 16) =
+            make_uint4(h[0], h[1], h[2], h[3]);
     }
 }
 
@@ -570,7 +578,7 @@ static MmaPlan plan_mma(int N, int K, int Mp) {
     MmaPlan pl;
     const int RB = gv_row_blocks(N), KT = gv_col_tiles(K);
     const int G = sm_count();
-    const size_t fixed = static_cast<size_t>(MM_NST) * GV_STAGE_BYTES + 16 * 8 + 1024;
+    const size_t fixed = static_cast<size_t>(MM_NST) * GV_STAGE_BYTES + 24 * 8 + 1024;   // + mbarriers, slack
     int bestS = KT, bestCT = 1;
     double best = 1e30;
     for (int S = 1; S <= min(64, KT); S++) {
@@ -606,7 +614,7 @@ size_t mma_scratch_bytes(int N, int K, int M) {
         const MmaPlan pl = plan_mma(N, K, Mp);
         const size_t b = align_up(pl.partial_floats * 4, BW_WS_ALIGN) +
                          2 * align_up(static_cast<size_t>(pl.grid) * Mp * 4, BW_WS_ALIGN) +
-                         align_up(static_cast<size_t>(MM_MAXM) * 4, BW_WS_ALIGN);
+                         align_up(static_cast<size_t>(gv_col_tiles(K)) * 512 * Mp * 2, BW_WS_ALIGN);
         tot = max(tot, b);
     }
     return tot;
@@ -643,8 +651,6 @@ bw_status mma_gemm_launch(const void *wq, const void *ws_scales, float ts, float
         p.S = pl.S;
         p.CT = pl.CT;
         p.per_slice = pl.per_slice;
-        p.x = x + static_cast<size_t>(m0) * K;
-        p.gamma = gamma;
         p.residual = residual ? residual + static_cast<size_t>(m0) * N : nullptr;
         p.y = y ? y + static_cast<size_t>(m0) * ncols : nullptr;
         p.argmax_out = argmax_out ? argmax_out + m0 : nullptr;
@@ -654,17 +660,16 @@ bw_status mma_gemm_launch(const void *wq, const void *ws_scales, float ts, float
         p.partial = cv.take<float>(pl.partial_floats);
         p.am_val = cv.take<float>(static_cast<size_t>(pl.grid) * Mp);
         p.am_idx = cv.take<int>(static_cast<size_t>(pl.grid) * Mp);
-        float *rn = cv.take<float>(MM_MAXM);
-        p.rnorm = (flags & BW_GEMV_RMSNORM) ? rn : nullptr;
+        uint8_t *bpk = cv.take<uint8_t>(static_cast<size_t>(p.KT) * 512 * Mp * 2);
+        p.bpk = bpk;
         p.rb_cnt = sc.cnt + CNT_GEMV_RG;
         p.am_cnt = sc.cnt + CNT_ARGMAX;
         p.adv_tokens = adv_tokens ? adv_tokens + m0 : nullptr;
         p.adv_pos = adv_pos ? adv_pos + m0 : nullptr;
         p.err = sc.err;
-        if (flags & BW_GEMV_RMSNORM) {
-            const bw_status s0 = launch_pdl(rownorm_kernel, dim3(Mr), dim3(256), 0, st, p.x, K, eps, rn);
-            if (s0 != BW_OK) return s0;
-        }
+        const bw_status s0 = launch_pdl(act_pack_kernel, dim3(Mp), dim3(256), 0, st, x + static_cast<size_t>(m0) * K,
+                                        Mr, Mp, K, p.KT, (flags & BW_GEMV_RMSNORM) ? gamma : nullptr, eps, bpk);
+        if (s0 != BW_OK) return s0;
         if (attr_set[dev] < pl.smem) {
             if (cudaFuncSetAttribute(mma_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(pl.smem)) != cudaSuccess) {
