@@ -32,58 +32,51 @@ constexpr int MOE_M = 4;          // token rows per pass of the grouped GEMV
 
 // ------------------------------------------------------------------ router
 
-// logits[r][e] = sum_k Wr[e][k] y[r][k]; one warp per expert, the rows of y
-// staged in shared memory 128 columns at a time (rows rb..rb+31).
+// Partial router logits over one 512-column slice of H:
+//   part[slice][r][e] = sum_{k in slice} Wr[e][k] y[r][k]
+// CTA = (8 experts, one slice, 32 rows).  The slice of y is staged once,
+// transposed ([k][row], padded), and the 8 experts' weight slices beside it;
+// lane = row, so each thread sums its own dot product (no reductions).  The
+// top-k kernel adds the slices in slice order.
+constexpr int MOE_KS = 512;
+
 __global__ void __launch_bounds__(256) moe_router_kernel(const float *y, const float *wr, int R, int H, int E,
-                                                         float *logits) {
+                                                         float *part) {
     pdl_trigger();
-    pdl_wait();
-    __shared__ __align__(16) float ys[32][128];
+    extern __shared__ __align__(16) float rt_sm[];
+    float *ys = rt_sm;                        // [MOE_KS][33]
+    float *wsm = rt_sm + MOE_KS * 33;         // [8][MOE_KS]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int e = blockIdx.x * 8 + warp;
-    const int r0 = blockIdx.y * 32;
-    const int nr = min(32, R - r0);
-    float acc[32];
-#pragma unroll
-    for (int r = 0; r < 32; r++) acc[r] = 0.0f;
-    for (int k0 = 0; k0 < H; k0 += 128) {
-        __syncthreads();
-        for (int i = threadIdx.x; i < 32 * 128; i += 256) {
-            const int r = i >> 7, c = i & 127;
-            ys[r][c] = (r < nr && k0 + c < H) ? y[static_cast<size_t>(r0 + r) * H + k0 + c] : 0.0f;
-        }
-        __syncthreads();
-        if (e < E) {
-            const int k = k0 + lane * 4;
-            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (k < H) w = *reinterpret_cast<const float4 *>(wr + static_cast<size_t>(e) * H + k);
-#pragma unroll
-            for (int r = 0; r < 32; r++) {
-                if (r < nr) {
-                    const float4 v = *reinterpret_cast<const float4 *>(&ys[r][lane * 4]);
-                    float a = acc[r];
-                    a = fmaf(w.x, v.x, a);
-                    a = fmaf(w.y, v.y, a);
-                    a = fmaf(w.z, v.z, a);
-                    a = fmaf(w.w, v.w, a);
-                    acc[r] = a;
-                }
-            }
-        }
+    const int e0 = blockIdx.x * 8, k0 = blockIdx.y * MOE_KS, r0 = blockIdx.z * 32;
+    const int kn = min(MOE_KS, H - k0), nr = min(32, R - r0);
+    // the router weights are constant: stage them before the dependency wait
+    for (int i = threadIdx.x; i < 8 * MOE_KS; i += 256) {
+        const int w = i / MOE_KS, k = i - w * MOE_KS;
+        wsm[i] = (e0 + w < E && k < kn) ? wr[static_cast<size_t>(e0 + w) * H + k0 + k] : 0.0f;
     }
-    if (e >= E) return;
-#pragma unroll
-    for (int r = 0; r < 32; r++) {
-        if (r < nr) {
-            const float v = warp_sum(acc[r]);
-            if (lane == 0) logits[static_cast<size_t>(r0 + r) * E + e] = v;
-        }
+    pdl_wait();
+    for (int i = threadIdx.x; i < 32 * MOE_KS; i += 256) {
+        const int r = i / MOE_KS, k = i - r * MOE_KS;
+        ys[k * 33 + r] = (r < nr && k < kn) ? y[static_cast<size_t>(r0 + r) * H + k0 + k] : 0.0f;
     }
+    __syncthreads();
+    const int e = e0 + warp;
+    const float *wv = wsm + warp * MOE_KS;
+    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+    for (int k = 0; k < kn; k += 4) {
+        a0 = fmaf(wv[k], ys[k * 33 + lane], a0);
+        a1 = fmaf(wv[k + 1], ys[(k + 1) * 33 + lane], a1);
+        a2 = fmaf(wv[k + 2], ys[(k + 2) * 33 + lane], a2);
+        a3 = fmaf(wv[k + 3], ys[(k + 3) * 33 + lane], a3);
+    }
+    if (e < E && lane < nr) part[(static_cast<size_t>(blockIdx.y) * R + r0 + lane) * E + e] = (a0 + a1) + (a2 + a3);
 }
 
 // --------------------------------------------------- top-k + bucketing
 
 struct Routing {
+    int *n_items;      // [1]   work items of the grouped GEMVs (one pass over a row-block chunk)
+    int *grp_item;     // [E+2] first item of each group
     int *grp_n;        // [1]   groups = selected experts + the shared expert
     int *grp_expert;   // [E+1] expert of each group in index order; -1 = shared
     int *grp_off;      // [E+2] assignment offsets
@@ -96,28 +89,45 @@ struct Routing {
 // yet chosen; softmax over the chosen logits in selection order.  Then the
 // assignments are bucketed by expert (index order) and, within an expert, by
 // row (row order) -- deterministic.
-__global__ void __launch_bounds__(1024) moe_topk_kernel(const float *logits, int R, int E, int K, int32_t *sel_out,
-                                                        float *w_out, Routing rt) {
+constexpr int MOE_NRC = 4;   // row-block chunks per expert matrix (work items per pass)
+
+template <int LV>   // logits per lane: ceil(E / 32) <= LV
+__global__ void __launch_bounds__(1024) moe_topk_kernel(const float *part, int n_slices, int R, int E, int K,
+                                                        int32_t *sel_out, float *w_out, Routing rt) {
     pdl_trigger();
     pdl_wait();
     __shared__ int s_sel[MOE_RMAX][MOE_KMAX];
     __shared__ int s_cnt[MOE_EMAX];
     __shared__ int s_off[MOE_EMAX];
     __shared__ int s_sh_off;
+    __shared__ int s_gexp[MOE_EMAX + 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int per_lane = (E + 31) / 32;
     for (int i = threadIdx.x; i < R * K; i += blockDim.x) rt.inv[i] = -1;
     for (int r = warp; r < R; r += 32) {
-        const float *lr = logits + static_cast<size_t>(r) * E;
+        // this row's logits in registers: lane holds experts lane + 32 j, the
+        // router slices summed in slice order
+        float lv[LV];
+#pragma unroll
+        for (int j = 0; j < LV; j++) {
+            lv[j] = -INFINITY;
+            const int e = lane + 32 * j;
+            if (j < per_lane && e < E) {
+                float v = part[static_cast<size_t>(r) * E + e];
+                for (int sl = 1; sl < n_slices; sl++) v += part[(static_cast<size_t>(sl) * R + r) * E + e];
+                lv[j] = v;
+            }
+        }
         uint32_t used = 0;
         float sv[MOE_KMAX];
         for (int t = 0; t < K; t++) {
             float bv = -INFINITY;
             int be = 0x7fffffff;
-            for (int j = 0; j < per_lane; j++) {
+#pragma unroll
+            for (int j = 0; j < LV; j++) {
                 const int e = lane + 32 * j;
-                if (e < E && !(used & (1u << j))) {
-                    const float v = lr[e];
+                if (j < per_lane && e < E && !(used & (1u << j))) {
+                    const float v = lv[j];
                     if (better(v, e, bv, be)) {
                         bv = v;
                         be = e;
@@ -165,6 +175,7 @@ __global__ void __launch_bounds__(1024) moe_topk_kernel(const float *logits, int
             s_off[e] = off;
             if (s_cnt[e] > 0) {
                 rt.grp_expert[g] = e;
+                s_gexp[g] = e;
                 rt.grp_off[g] = off;
                 off += s_cnt[e];
                 g++;
@@ -175,6 +186,15 @@ __global__ void __launch_bounds__(1024) moe_topk_kernel(const float *logits, int
         rt.grp_off[g + 1] = off + R;
         *rt.grp_n = g + 1;
         s_sh_off = off;
+        // work items: MOE_NRC row-block chunks x passes of MOE_M rows per group
+        int it = 0;
+        for (int gg = 0; gg <= g; gg++) {
+            rt.grp_item[gg] = it;
+            const int cnt = (gg < g) ? s_cnt[s_gexp[gg]] : R;
+            it += MOE_NRC * ((cnt + MOE_M - 1) / MOE_M);
+        }
+        rt.grp_item[g + 1] = it;
+        *rt.n_items = it;
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
@@ -198,7 +218,8 @@ struct GroupedParams {
     const uint8_t *shq, *shs;  // shared expert (tiled layout)
     size_t q_stride, s_stride; // bytes per expert matrix
     int N, K, NC, RG, KT;      // one expert matrix: rows (GPU layout), columns
-    const int *grp_n, *grp_expert, *grp_off, *asg_row;
+    const int *grp_n, *grp_expert, *grp_off, *asg_row, *grp_item, *n_items;
+    int RB, RBC;               // row blocks of one matrix, row blocks per work item
     const float *x;            // source activations
     int gather;                // 1: row asg_row[j] of x, 0: row j of x
     float *y;                  // [assignments][N or N/2]
@@ -209,9 +230,98 @@ struct GroupedParams {
     uint32_t *err;
 };
 
-// One CTA per (128-row block, group); the group's tokens are processed MOE_M
-// rows at a time, the expert's tiles streamed for each pass (after the first
-// pass they come from L2).
+// Persistent CTAs over the work items: item = (group, pass of up to MOE_M of
+// the group's rows, chunk of RBC row blocks of the expert's matrix); CTA c
+// takes items c, c + grid, ...  The producer warp streams the same item
+// sequence (the routing comes from the previous kernel, so it waits for it
+// first) and runs ahead across items; the consumers stage each item's
+// activation rows, then consume its RBC x KT tiles, with the epilogue of each
+// 128-row block.  Items are independent: results do not depend on the grid.
+struct MoeItem {
+    int expert, off, mcnt, rb0, rb1;
+};
+
+__device__ __forceinline__ MoeItem moe_item(const GroupedParams &p, int i) {
+    // group of item i: grp_item is ascending (binary search)
+    int lo = 0, hi = *p.grp_n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.grp_item[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    const int g = lo;
+    const int local = i - p.grp_item[g];
+    const int tb = local / MOE_NRC, rc = local - tb * MOE_NRC;
+    const int cnt = p.grp_off[g + 1] - p.grp_off[g];
+    MoeItem it;
+    it.expert = p.grp_expert[g];
+    it.off = p.grp_off[g] + tb * MOE_M;
+    it.mcnt = min(MOE_M, cnt - tb * MOE_M);
+    it.rb0 = min(p.RB, rc * p.RBC);
+    it.rb1 = min(p.RB, it.rb0 + p.RBC);
+    return it;
+}
+
+// One item's row blocks with MR activation rows: the staged activations are
+// pre-scaled and swizzled, then each row block's KT tiles are consumed and
+// its outputs written.  `step` counts the ring stages (shared with the producer).
+template <int FMT, int MR>
+__device__ __forceinline__ void moe_item_rows(const GroupedParams &p, const MoeItem &it, float *xs, float *ct, int CS,
+                                              int nc, int warp, int lane, uint32_t stages_a, uint32_t xs_a,
+                                              uint32_t ct_a, uint64_t *full, uint64_t *empty, int &step, float ts,
+                                              float ts_up) {
+    const int nst = p.nst, T = p.KT;
+    stage_pass2<FMT, MR>(xs, ct, nullptr, nullptr, CS, nc, warp, lane);
+    consumer_sync();
+    for (int rb = it.rb0; rb < it.rb1; rb++) {
+        const int rg = rb * (GV_TR / 8) + 2 * warp + (lane >> 4);
+        float acc[8][MR];
+#pragma unroll
+        for (int r = 0; r < 8; r++)
+#pragma unroll
+            for (int m = 0; m < MR; m++) acc[r][m] = 0.0f;
+        for (int kt = 0; kt < T; kt++, step++) {
+            const int s = step % nst;
+            mbar_wait(&full[s], static_cast<uint32_t>((step / nst) & 1), p.err);
+            const int cl = kt * GV_TC + (lane & 15);
+            if (cl < nc)
+                stage_chunk<FMT, MR>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, warp, lane, xs_a, ct_a, cl,
+                                     CS, acc);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_relaxed(&empty[s]);
+        }
+        float tot[MR];
+        reduce_rows16<MR>(acc, lane, tot);
+        const int r = (lane >> 1) & 7;
+        float val[MR];
+#pragma unroll
+        for (int m = 0; m < MR; m++) {
+            float v = tot[m];
+            if constexpr (FMT == BW_FMT_Q4_0) {
+                v *= 281474976710656.0f;   // 2^48
+            } else {
+                v *= (p.silu && r >= 4) ? ts_up : ts;
+            }
+            val[m] = v;
+        }
+        const bool act = (lane & 1) == 0 && rg < p.RG;
+        if (p.silu) {
+#pragma unroll
+            for (int m = 0; m < MR; m++) {
+                const float up = __shfl_down_sync(0xffffffffu, val[m], 8);
+                if (act && r < 4 && m < it.mcnt) {
+                    const float gt = val[m];
+                    const size_t j = static_cast<size_t>(it.off + m);
+                    p.y[j * (p.N / 2) + rg * 4 + r] = (gt / (1.0f + expf(-gt))) * up;
+                }
+            }
+        } else if (act) {
+#pragma unroll
+            for (int m = 0; m < MR; m++)
+                if (m < it.mcnt) p.y[static_cast<size_t>(it.off + m) * p.N + rg * 8 + r] = val[m];
+        }
+    }
+}
+
 template <int FMT>
 __global__ void __launch_bounds__(GV_THREADS, 1) moe_grouped_gemv_kernel(const GroupedParams p) {
     constexpr int M = MOE_M;
@@ -236,55 +346,52 @@ __global__ void __launch_bounds__(GV_THREADS, 1) moe_grouped_gemv_kernel(const G
     __syncthreads();
     pdl_trigger();
     pdl_wait();   // the routing tables come from the previous kernel
-    const int g = blockIdx.y;
-    if (g >= *p.grp_n) return;
-    const int expert = p.grp_expert[g];
-    const int off = p.grp_off[g];
-    const int cnt = p.grp_off[g + 1] - off;
-    const int rb = blockIdx.x;
-    const int ntb = (cnt + M - 1) / M;
+    const int n_items = *p.n_items;
     const int T = p.KT;
-    const int n_steps = ntb * T;
-    const uint8_t *bq = expert >= 0 ? p.eq + static_cast<size_t>(expert) * p.q_stride : p.shq;
-    const uint8_t *bs = expert >= 0 ? p.es + static_cast<size_t>(expert) * p.s_stride : p.shs;
 
     if (warp == GV_CW) {
         if (lane == 0) {
-            for (int step = 0; step < n_steps; step++) {
-                const int s = step % nst;
-                if (step >= nst) mbar_wait(&empty[s], static_cast<uint32_t>((step / nst - 1) & 1), p.err);
-                const size_t tile = static_cast<size_t>(rb) * p.KT + step % T;
-                unsigned char *st = stages + static_cast<size_t>(s) * GV_STAGE_BYTES;
-                mbar_arrive_tx_relaxed(&full[s], GV_STAGE_BYTES);
-                bulk_g2s(st, bq + tile * GV_NIB_BYTES, GV_NIB_BYTES, &full[s]);
-                bulk_g2s(st + GV_NIB_BYTES, bs + tile * GV_SC_BYTES, GV_SC_BYTES, &full[s]);
+            int step = 0;
+            for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
+                const MoeItem it = moe_item(p, i);
+                const uint8_t *bq = it.expert >= 0 ? p.eq + static_cast<size_t>(it.expert) * p.q_stride : p.shq;
+                const uint8_t *bs = it.expert >= 0 ? p.es + static_cast<size_t>(it.expert) * p.s_stride : p.shs;
+                for (int rb = it.rb0; rb < it.rb1; rb++)
+                    for (int kt = 0; kt < T; kt++, step++) {
+                        const int s = step % nst;
+                        if (step >= nst) mbar_wait(&empty[s], static_cast<uint32_t>((step / nst - 1) & 1), p.err);
+                        const size_t tile = static_cast<size_t>(rb) * p.KT + kt;
+                        unsigned char *st = stages + static_cast<size_t>(s) * GV_STAGE_BYTES;
+                        mbar_arrive_tx_relaxed(&full[s], GV_STAGE_BYTES);
+                        bulk_g2s(st, bq + tile * GV_NIB_BYTES, GV_NIB_BYTES, &full[s]);
+                        bulk_g2s(st + GV_NIB_BYTES, bs + tile * GV_SC_BYTES, GV_SC_BYTES, &full[s]);
+                    }
             }
         }
         return;
     }
 
-    float ts = 1.0f, ts_up = 1.0f;
-    if constexpr (FMT == BW_FMT_NVFP4) {
-        if (expert >= 0) {
-            ts = p.silu ? p.ts_tab[2 * expert] : p.ts_tab[expert];
-            ts_up = p.silu ? p.ts_tab[2 * expert + 1] : ts;
-        } else {
-            ts = p.ts_sh;
-            ts_up = p.ts_sh_up;
-        }
-    }
-    const int rg = rb * (GV_TR / 8) + 2 * warp + (lane >> 4);
     const int nc = p.NC;
     int step = 0;
-    for (int tb = 0; tb < ntb; tb++) {
-        const int mcnt = min(M, cnt - tb * M);
-        consumer_sync();   // the previous pass is done with the staged activations
-        // pass 1: the tokens' activation rows in natural order, loads back to back
+    for (int i = blockIdx.x; i < n_items; i += gridDim.x) {
+        const MoeItem it = moe_item(p, i);
+        float ts = 1.0f, ts_up = 1.0f;
+        if constexpr (FMT == BW_FMT_NVFP4) {
+            if (it.expert >= 0) {
+                ts = p.silu ? p.ts_tab[2 * it.expert] : p.ts_tab[it.expert];
+                ts_up = p.silu ? p.ts_tab[2 * it.expert + 1] : ts;
+            } else {
+                ts = p.ts_sh;
+                ts_up = p.ts_sh_up;
+            }
+        }
+        consumer_sync();   // the previous item is done with the staged activations
+        // the item's activation rows in natural order, loads back to back
 #pragma unroll
         for (int m = 0; m < M; m++) {
             const float *xr = nullptr;
-            if (m < mcnt) {
-                const int j = off + tb * M + m;
+            if (m < it.mcnt) {
+                const int j = it.off + m;
                 xr = p.x + static_cast<size_t>(p.gather ? p.asg_row[j] : j) * p.K;
             }
 #pragma unroll 4
@@ -292,53 +399,13 @@ __global__ void __launch_bounds__(GV_THREADS, 1) moe_grouped_gemv_kernel(const G
                 xs[static_cast<size_t>(m) * CS * 32 + e] = xr ? xr[e] : 0.0f;
         }
         consumer_sync();
-        stage_pass2<FMT, M>(xs, ct, nullptr, nullptr, CS, nc, warp, lane);
-        consumer_sync();
-        float acc[8][M];
-#pragma unroll
-        for (int r = 0; r < 8; r++)
-#pragma unroll
-            for (int m = 0; m < M; m++) acc[r][m] = 0.0f;
-        for (int kt = 0; kt < T; kt++, step++) {
-            const int s = step % nst;
-            mbar_wait(&full[s], static_cast<uint32_t>((step / nst) & 1), p.err);
-            const int cl = kt * GV_TC + (lane & 15);
-            if (cl < nc)
-                stage_chunk<FMT, M>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, warp, lane, xs_a, ct_a, cl,
-                                    CS, acc);
-            __syncwarp();
-            if (lane == 0) mbar_arrive_relaxed(&empty[s]);
-        }
-        float tot[M];
-        reduce_rows16<M>(acc, lane, tot);
-        const int r = (lane >> 1) & 7;
-        float val[M];
-#pragma unroll
-        for (int m = 0; m < M; m++) {
-            float v = tot[m];
-            if constexpr (FMT == BW_FMT_Q4_0) {
-                v *= 281474976710656.0f;   // 2^48
-            } else {
-                v *= (p.silu && r >= 4) ? ts_up : ts;
-            }
-            val[m] = v;
-        }
-        const bool act = (lane & 1) == 0 && rg < p.RG;
-        if (p.silu) {
-#pragma unroll
-            for (int m = 0; m < M; m++) {
-                const float up = __shfl_down_sync(0xffffffffu, val[m], 8);
-                if (act && r < 4 && m < mcnt) {
-                    const float gt = val[m];
-                    const size_t j = static_cast<size_t>(off + tb * M + m);
-                    p.y[j * (p.N / 2) + rg * 4 + r] = (gt / (1.0f + expf(-gt))) * up;
-                }
-            }
-        } else if (act) {
-#pragma unroll
-            for (int m = 0; m < M; m++)
-                if (m < mcnt) p.y[static_cast<size_t>(off + tb * M + m) * p.N + rg * 8 + r] = val[m];
-        }
+        // the inner loop for the item's actual row count (1, 2 or up to 4)
+        if (it.mcnt == 1)
+            moe_item_rows<FMT, 1>(p, it, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
+        else if (it.mcnt == 2)
+            moe_item_rows<FMT, 2>(p, it, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
+        else
+            moe_item_rows<FMT, M>(p, it, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
     }
 }
 
@@ -379,9 +446,11 @@ static size_t moe_carve(const bw_model *m, int R, char *base, MoeScratch *ms) {
     Carver cv(base);
     MoeScratch s;
     s.y = cv.take<float>(static_cast<size_t>(R) * H);
-    s.logits = cv.take<float>(static_cast<size_t>(R) * E);
+    s.logits = cv.take<float>(static_cast<size_t>((H + MOE_KS - 1) / MOE_KS) * R * E);   // router slice partials
     s.wts = cv.take<float>(static_cast<size_t>(R) * K);
     s.sel = cv.take<int32_t>(static_cast<size_t>(R) * K);
+    s.rt.n_items = cv.take<int>(1);
+    s.rt.grp_item = cv.take<int>(E + 2);
     s.rt.grp_n = cv.take<int>(1);
     s.rt.grp_expert = cv.take<int>(E + 1);
     s.rt.grp_off = cv.take<int>(E + 2);
@@ -396,7 +465,7 @@ static size_t moe_carve(const bw_model *m, int R, char *base, MoeScratch *ms) {
 size_t moe_scratch_bytes(const bw_model *m, int R) { return moe_carve(m, R, nullptr, nullptr); }
 
 template <int FMT>
-static bw_status grouped_go(const GroupedParams &p, int RB, int groups, cudaStream_t st) {
+static bw_status grouped_go(const GroupedParams &p, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(p.nst) * GV_STAGE_BYTES +
                         static_cast<size_t>(MOE_M) * p.KT * GV_TC * 33 * 4 + 16 + 2 * static_cast<size_t>(p.nst) * 8;
     static size_t attr_set[64] = {};
@@ -411,7 +480,8 @@ static bw_status grouped_go(const GroupedParams &p, int RB, int groups, cudaStre
         }
         attr_set[dev] = smem;
     }
-    return launch_pdl(moe_grouped_gemv_kernel<FMT>, dim3(RB, groups), dim3(GV_THREADS), smem, st, p);
+    // persistent: one CTA per SM, items assigned round robin
+    return launch_pdl(moe_grouped_gemv_kernel<FMT>, dim3(sm_count()), dim3(GV_THREADS), smem, st, p);
 }
 
 bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R, const Scratch &sc, char *moe_base,
@@ -440,20 +510,40 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
     moe_carve(m, R, moe_base, &ms);
     bw_status s = rmsnorm_launch(x, nullptr, ly->ffn_norm, R, H, m->eps, ms.y, 0, st);
     if (s != BW_OK) return s;
-    s = launch_pdl(moe_router_kernel, dim3((E + 7) / 8, (R + 31) / 32), dim3(256), 0, st,
-                   static_cast<const float *>(ms.y), ly->router, R, H, E, ms.logits);
+    const int n_slices = (H + MOE_KS - 1) / MOE_KS;
+    {
+        const size_t rsm = (static_cast<size_t>(MOE_KS) * 33 + 8 * MOE_KS) * 4;
+        static bool attr_set[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(moe_router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(rsm)) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return BW_ERR_CUDA;
+            }
+            attr_set[dev] = true;
+        }
+        s = launch_pdl(moe_router_kernel, dim3((E + 7) / 8, n_slices, (R + 31) / 32), dim3(256), rsm, st,
+                       static_cast<const float *>(ms.y), ly->router, R, H, E, ms.logits);
+    }
     if (s != BW_OK) return s;
     int32_t *sel = topk_idx ? topk_idx : ms.sel;
     float *wts = topk_w ? topk_w : ms.wts;
-    s = launch_pdl(moe_topk_kernel, dim3(1), dim3(1024), 0, st, static_cast<const float *>(ms.logits), R, E, K, sel,
-                   wts, ms.rt);
+    s = E <= 256 ? launch_pdl(moe_topk_kernel<8>, dim3(1), dim3(1024), 0, st, static_cast<const float *>(ms.logits),
+                              n_slices, R, E, K, sel, wts, ms.rt)
+                 : launch_pdl(moe_topk_kernel<MOE_EMAX / 32>, dim3(1), dim3(1024), 0, st,
+                              static_cast<const float *>(ms.logits), n_slices, R, E, K, sel, wts, ms.rt);
     if (s != BW_OK) return s;
     GroupedParams gp;
     gp.grp_n = ms.rt.grp_n;
     gp.grp_expert = ms.rt.grp_expert;
     gp.grp_off = ms.rt.grp_off;
     gp.asg_row = ms.rt.asg_row;
-    gp.nst = 3;
+    gp.grp_item = ms.rt.grp_item;
+    gp.n_items = ms.rt.n_items;
+    gp.nst = 4;
     gp.err = sc.err;
     size_t qb = 0, sb = 0;
     // gate/up: rows of y gathered per assignment -> act[assignment][Fe]
@@ -469,6 +559,8 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
     gp.NC = H / 32;
     gp.RG = gp.N / 8;
     gp.KT = gv_col_tiles(H);
+    gp.RB = gv_row_blocks(gp.N);
+    gp.RBC = (gp.RB + MOE_NRC - 1) / MOE_NRC;
     gp.x = ms.y;
     gp.gather = 1;
     gp.y = ms.act;
@@ -476,8 +568,7 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
     gp.ts_tab = ly->egu_ts;
     gp.ts_sh = ly->sgu.ts;
     gp.ts_sh_up = ly->sgu.ts_up;
-    s = fmt == BW_FMT_Q4_0 ? grouped_go<BW_FMT_Q4_0>(gp, gv_row_blocks(gp.N), E + 1, st)
-                           : grouped_go<BW_FMT_NVFP4>(gp, gv_row_blocks(gp.N), E + 1, st);
+    s = fmt == BW_FMT_Q4_0 ? grouped_go<BW_FMT_Q4_0>(gp, st) : grouped_go<BW_FMT_NVFP4>(gp, st);
     if (s != BW_OK) return s;
     // down: act[assignment] -> dout[assignment][H]
     bw_repack_bytes(H, Fe, &qb, &sb);
@@ -492,6 +583,8 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
     gp.NC = Fe / 32;
     gp.RG = H / 8;
     gp.KT = gv_col_tiles(Fe);
+    gp.RB = gv_row_blocks(H);
+    gp.RBC = (gp.RB + MOE_NRC - 1) / MOE_NRC;
     gp.x = ms.act;
     gp.gather = 0;
     gp.y = ms.dout;
@@ -499,8 +592,7 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
     gp.ts_tab = ly->ed_ts;
     gp.ts_sh = ly->sd.ts;
     gp.ts_sh_up = ly->sd.ts;
-    s = fmt == BW_FMT_Q4_0 ? grouped_go<BW_FMT_Q4_0>(gp, gv_row_blocks(H), E + 1, st)
-                           : grouped_go<BW_FMT_NVFP4>(gp, gv_row_blocks(H), E + 1, st);
+    s = fmt == BW_FMT_Q4_0 ? grouped_go<BW_FMT_Q4_0>(gp, st) : grouped_go<BW_FMT_NVFP4>(gp, st);
     if (s != BW_OK) return s;
     const size_t nblk = (static_cast<size_t>(R) * H + 255) / 256;
     const int blocks = static_cast<int>(nblk < 4096 ? nblk : 4096);
