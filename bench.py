@@ -146,6 +146,24 @@ def _ncu_traffic(kind, cfg_name):
         return None
 
 
+def step_launches(cfg):
+    """libbw kernel launches of one decode step: embedding; per layer QKV,
+    attention, O and the FFN (dense gate/up + down, or the MoE block's
+    RMSNorm, router, top-k, two grouped GEMVs and combine); LM head.  A
+    projection is ceil(rows/4) CUDA-core GEMV launches, or (NVFP4 with more
+    than 4 rows) an activation pack plus a tensor-core GEMM per 32 rows."""
+    from token_decode_b200 import synth
+
+    def proj(rows):
+        if cfg.fmt == synth.FMT_NVFP4 and rows > 4:
+            return 2 * ((rows + 31) // 32)
+        return (rows + 3) // 4
+
+    R = cfg.B
+    per_layer = proj(R) + 1 + proj(R) + (6 if cfg.n_experts else 2 * proj(R))
+    return 1 + cfg.L * per_layer + proj(R)
+
+
 def run_ours(args):
     from token_decode_b200 import build, bw, runtime, synth
     ws_, rank, local = dist_env()
@@ -295,8 +313,7 @@ def run_ours(args):
     avg_ctx = cfg.ctx + (cfg.steps + 1) / 2
     sb = step_bytes(cfg, model, avg_ctx)
     step_gbs = sb / (ms_step / 1000.0) / 1e9
-    launches_per_step = 1 + 5 * cfg.L + 1
-    launches_per_step += (cfg.B - 1) // 4 * (4 * cfg.L + 1)
+    launches_per_step = step_launches(cfg)
 
     line = {
         "metric": METRIC,
