@@ -308,7 +308,7 @@ def run_ours(args):
     dom = "gu" if "gu" in kern else "moe"
     peak, peak_kind = _peaks()
     achieved = kern[dom]["GBps"]
-    traffic = _ncu_traffic(dom, cfg.name)
+    traffic = _ncu_traffic(dom, args.config)
 
     avg_ctx = cfg.ctx + (cfg.steps + 1) / 2
     sb = step_bytes(cfg, model, avg_ctx)

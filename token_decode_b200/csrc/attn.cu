@@ -31,12 +31,15 @@
 //      deterministic and independent of the physical page order.
 // The q and P planes have padded rows, so their 8x8 fragment loads are free
 // of shared-memory bank conflicts.
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
 #include <string.h>
 
 #include "bw_common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace bw {
 
@@ -46,6 +49,7 @@ constexpr int ATT_CT = ATT_CW * 32;             // consumer threads
 constexpr int ATT_MAXQ = 32;                    // query vectors per CTA (G * n_rows)
 constexpr int ATT_MAXR = 8;                     // query rows per sequence (1 + draft tokens)
 constexpr int ATT_MAXNS = 64;                   // splits per (sequence, kv head)
+constexpr int ATT_MAXCL = 16;                   // splits merged inside one thread-block cluster
 constexpr int ATT_MAXPAGES = 8192;              // page-table width the CTA's page list holds
 constexpr int ATT_ST = 64;                      // tokens per stage: 4 pages, 8 per consumer warp
 constexpr int ATT_PPS = ATT_ST / 16;
@@ -60,6 +64,7 @@ struct AttnParams {
     int max_pages, n_pages;
     const int32_t *pos;
     int B, R, nq, nkv, G, Q, n_split;
+    int cluster;          // 1: the splits of a (sequence, kv head) are one cluster and merge through DSMEM
     float scale;
     float *out;
     float *part_o;        // [B][nkv][n_split][Q][HD]
@@ -147,7 +152,7 @@ __device__ __forceinline__ void split_f16(float v, __half &hi, __half &lo) {
 // NST: ring stages -- 2 when two CTAs share an SM, 4 when each CTA has an SM
 // to itself (a short split then has all its pages in flight at once).
 template <int HD, int MT, int NST>
-__global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(const __grid_constant__ AttnParams p) {
     constexpr int ATT_NST = NST;
     constexpr int QM = 16 * MT;             // query rows of the MMA tiles (padded)
     constexpr int QS = HD + 8;              // padded q row (halves)
@@ -478,6 +483,54 @@ __global__ void __launch_bounds__(ATT_THREADS) attn_kernel(const __grid_constant
     }
 
     // ---- 4. the output, or a partial for the split combine
+    if (p.cluster) {
+        // the splits form one thread-block cluster: partials stay in shared
+        // memory (the drained ring), each CTA merges a slice of the outputs
+        // from every split's shared memory, in split order
+        float *s_o = reinterpret_cast<float *>(att_sm);           // [Q][HD] unnormalized output
+        float *s_m = s_o + ATT_MAXQ * HD;                           // [Q]
+        float *s_l = s_m + ATT_MAXQ;                                // [Q]
+#pragma unroll
+        for (int mt = 0; mt < MT; mt++) {
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const int qi = mt * 16 + gid + 8 * h;
+                if (qi >= p.Q) continue;
+#pragma unroll
+                for (int nt = 0; nt < NT; nt++) {
+                    const int d = warp * WD + nt * 8 + tig * 2;
+                    s_o[qi * HD + d] = o[mt][nt][2 * h];
+                    s_o[qi * HD + d + 1] = o[mt][nt][2 * h + 1];
+                }
+                if (warp == 0 && tig == 0) {
+                    s_m[qi] = m_run[mt][h];
+                    s_l[qi] = l_run[mt][h];
+                }
+            }
+        }
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        const int ns = p.n_split;
+        const int per = (p.Q * HD + ns - 1) / ns;
+        for (int e = split * per + tid; e < min(p.Q * HD, (split + 1) * per); e += ATT_CT) {
+            const int qi = e / HD, d = e - qi * HD;
+            float M = -INFINITY;
+            for (int r2 = 0; r2 < ns; r2++) M = fmaxf(M, cluster.map_shared_rank(s_m, r2)[qi]);
+            float L = 0.0f, O = 0.0f;
+            for (int r2 = 0; r2 < ns; r2++) {
+                const float m2 = cluster.map_shared_rank(s_m, r2)[qi];
+                if (m2 == -INFINITY) continue;
+                const float w = expf(m2 - M);
+                L = fmaf(cluster.map_shared_rank(s_l, r2)[qi], w, L);
+                O = fmaf(cluster.map_shared_rank(s_o, r2)[qi * HD + d], w, O);
+            }
+            const int r = qi / p.G, gq = qi - r * p.G;
+            p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
+                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = O / L;
+        }
+        cluster.sync();   // keep this CTA's shared memory alive until every reader is done
+        return;
+    }
     const size_t pbase = (static_cast<size_t>(b) * p.nkv + kvh) * p.n_split;
 #pragma unroll
     for (int mt = 0; mt < MT; mt++) {
@@ -653,7 +706,36 @@ static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnPara
     }
     AttnParams q = p;
     q.n_split = ns;
-    return launch_pdl(attn_kernel<HD, MT, NST>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
+    q.cluster = (ns > 1 && ns <= ATT_MAXCL && NST == 4) ? 1 : 0;
+    if (!q.cluster) return launch_pdl(attn_kernel<HD, MT, NST>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
+    static bool cl_set[64] = {};
+    if (!cl_set[dev]) {
+        if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            cudaSuccess) {
+            (void)cudaGetLastError();
+            return BW_ERR_CUDA;
+        }
+        cl_set[dev] = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ns, nkv, B);
+    cfg.blockDim = dim3(ATT_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = ns;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, attn_kernel<HD, MT, NST>, q) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BW_ERR_CUDA;
+    }
+    return BW_OK;
 }
 
 template <int HD, int MT>

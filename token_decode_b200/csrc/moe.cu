@@ -110,13 +110,19 @@ __global__ void __launch_bounds__(1024) moe_topk_kernel(const float *part, int n
         float lv[LV];
 #pragma unroll
         for (int j = 0; j < LV; j++) {
-            lv[j] = -INFINITY;
             const int e = lane + 32 * j;
-            if (j < per_lane && e < E) {
-                float v = part[static_cast<size_t>(r) * E + e];
-                for (int sl = 1; sl < n_slices; sl++) v += part[(static_cast<size_t>(sl) * R + r) * E + e];
-                lv[j] = v;
+            lv[j] = (j < per_lane && e < E) ? part[static_cast<size_t>(r) * E + e] : -INFINITY;
+        }
+        // slice by slice (in slice order), each slice's loads issued together
+        for (int sl = 1; sl < n_slices; sl++) {
+            float t[LV];
+#pragma unroll
+            for (int j = 0; j < LV; j++) {
+                const int e = lane + 32 * j;
+                t[j] = (j < per_lane && e < E) ? part[(static_cast<size_t>(sl) * R + r) * E + e] : 0.0f;
             }
+#pragma unroll
+            for (int j = 0; j < LV; j++) lv[j] += t[j];
         }
         uint32_t used = 0;
         float sv[MOE_KMAX];
