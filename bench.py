@@ -101,6 +101,27 @@ def dist_env():
     return ws, rank, local
 
 
+def job_throughput(ms_local, tokens_per_rank, world_size, device="cuda"):
+    """Whole-job rate of N independent replicas: the slowest rank's time (max
+    over ranks, on the device clock each rank measured) and every rank's
+    tokens.  Returns (ms, tokens per second)."""
+    ms = float(ms_local)
+    if world_size > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, tokens_per_rank * world_size / (ms / 1000.0)
+
+
+def workload_config(cfg, world_size):
+    """The `config` object of the JSON line: the workload, identical for both arms."""
+    return {"workload": cfg.name, "batch": cfg.B, "context": cfg.ctx,
+            "decode_tokens_per_generation": cfg.steps, "layers": cfg.L, "hidden": cfg.H,
+            "heads": f"{cfg.nq}/{cfg.nkv}x{cfg.hd}", "ffn": cfg.F, "vocab": cfg.V,
+            "parallelism": f"replicas x{world_size}"}
+
+
 def step_bytes(cfg, model, avg_ctx):
     """Algorithmic bytes of one decode step: every weight matrix streamed once
     (4.5-bit blocks + fp32 norm gains), the KV read over the context, the new
@@ -259,15 +280,11 @@ def run_ours(args):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     err = bw.read_error(dec.ws, stream)
+    ms, value = job_throughput(ms, args.steps * cfg.B, ws_)
     if ws_ > 1:
         import torch.distributed as dist
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     ms_step = ms / args.steps
-    tokens = args.steps * cfg.B * ws_
-    value = tokens / (ms / 1000.0)
 
     # ---- end to end through the C ABI: host tokens in, host token out, every step
     pin_in = torch.empty(cfg.B, dtype=torch.int32).pin_memory()
@@ -298,8 +315,7 @@ def run_ours(args):
         pin_in.copy_(pin_out)
     f1.record(stream)
     f1.synchronize()
-    e2e_ms = f0.elapsed_time(f1)
-    e2e_value = n_e2e * cfg.B / (e2e_ms / 1000.0) * ws_
+    e2e_ms, e2e_value = job_throughput(f0.elapsed_time(f1), n_e2e * cfg.B, ws_)
 
     # ---- per kernel: every launch kind of the step over all layers, graph-replayed;
     # the dominant one (gate/up GEMV, or the MoE FFN) gives the roofline figure
@@ -329,12 +345,10 @@ def run_ours(args):
         "dtype": "q4_0 weights, fp32 accumulate, fp16 KV" if cfg.fmt == synth.FMT_Q4_0 else
                  "nvfp4 weights, fp32 accumulate, fp16 KV",
         "data": "synthetic (seeded random-init weights N(0,0.02) quantized; N(0,1) fp16 KV context)",
-        "config": {"workload": cfg.name, "batch": cfg.B, "context": cfg.ctx,
-                   "decode_tokens_per_generation": cfg.steps, "layers": cfg.L, "hidden": cfg.H,
-                   "heads": f"{cfg.nq}/{cfg.nkv}x{cfg.hd}", "ffn": cfg.F, "vocab": cfg.V,
-                   "parallelism": f"replicas x{ws_}",
-                   "l2": "inputs larger than L2 (each step streams ~%.2f GB)" % (sb / 1e9),
-                   "timing": "CUDA graphs of %d steps, on-device token/position advance" % G},
+        "config": dict(workload_config(cfg, ws_),
+                       l2="inputs larger than L2 (each step streams ~%.2f GB)" % (sb / 1e9)),
+        "timing": "CUDA graphs of %d steps, on-device token/position advance; CUDA events on the launching "
+                  "stream" % G,
         "hbm_gbs_step": round(step_gbs, 1),
         "roofline_step_frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4),
         "roofline_step_frac_of_measured": round(step_gbs / peak, 4),
@@ -430,7 +444,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * wall / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32 (CPU oracle)",
             "data": "synthetic (seeded random-init weights)", "impl": "reference",
-            "config": {"workload": cfg.name, "batch": cfg.B, "context": cfg.ctx},
+            "config": workload_config(cfg, ws_),
             "cpu_baseline": {"value": round(value, 5), "unit": "tok/s", "cores": 1, "kind": "oracle",
                              "sample": f"each step = one of the {cfg.L} layers of one decode token "
                                        f"(+ embedding/LM head timed once, {t_head:.2f} s), scaled "

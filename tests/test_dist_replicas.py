@@ -1,0 +1,68 @@
+"""The multi-GPU path of bench.py is N independent replicas (no data-path
+collective): whole-job throughput = every rank's tokens / the slowest rank's
+device time.  Checked here with two gloo ranks on the CPU."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+_WORKER = r"""
+import importlib.util, json, os, sys
+from datetime import timedelta
+import torch.distributed as dist
+spec = importlib.util.spec_from_file_location("bench", os.path.join(sys.argv[1], "bench.py"))
+bench = importlib.util.module_from_spec(spec)
+spec.loader.exec_module(bench)
+ws, rank, local = bench.dist_env()
+dist.init_process_group("gloo", timeout=timedelta(seconds=60))
+ms, value = bench.job_throughput(10.0 + 5.0 * rank, 100, ws, device="cpu")
+dist.barrier()
+dist.destroy_process_group()
+print(json.dumps({"rank": rank, "ms": ms, "value": value}))
+"""
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_two_replicas_take_the_slowest_rank_and_all_tokens():
+    port = _free_port()
+    procs = []
+    for rank in range(2):
+        env = dict(os.environ, MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                   LOCAL_RANK=str(rank), WORLD_SIZE="2", CUDA_VISIBLE_DEVICES="")
+        procs.append(subprocess.Popen([sys.executable, "-c", _WORKER, ROOT], env=env, stdout=subprocess.PIPE,
+                                      stderr=subprocess.PIPE, text=True))
+    outs = []
+    for p in procs:
+        out, err = p.communicate(timeout=120)
+        assert p.returncode == 0, err[-2000:]
+        outs.append(json.loads(out.strip().splitlines()[-1]))
+    for o in outs:
+        assert o["ms"] == 15.0                          # max over ranks
+        assert abs(o["value"] - 200 / 0.015) < 1e-6     # both ranks' tokens / the slowest time
+
+
+def test_single_rank_needs_no_process_group():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    ms, value = bench.job_throughput(20.0, 64, 1, device="cpu")
+    assert ms == 20.0 and abs(value - 3200.0) < 1e-9
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun the other ranks of the reference arm exit without work."""
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1", CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--config", "tiny", "--steps", "3", "--warmup", "3"], env=env, capture_output=True,
+                       text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
