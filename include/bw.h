@@ -45,10 +45,16 @@
  *    error word at the start of the workspace; read it with bw_read_error
  *    after the stream has drained.  No exception crosses the ABI.
  *  - Workspace: scratch device memory of at least the queried size, 256-byte
- *    aligned, zero-filled ONCE before first use (bw_workspace_init).  Kernels
+ *    aligned (any other address returns BW_ERR_INVALID_ARG), zero-filled
+ *    ONCE before first use (bw_workspace_init).  Kernels
  *    leave their counters at zero on return, so the same workspace serves
  *    any number of later calls and CUDA-graph replays on one stream.  Calls
  *    sharing a workspace must not run concurrently.
+ *  - Kernels start early (programmatic dependent launch): they may read
+ *    model data -- weights, scales, norm gains, router, RoPE table -- while
+ *    the previous kernel on the stream is still running, and wait for it
+ *    only before reading activations, KV or token inputs.  Model data must
+ *    therefore not be written by work still in flight on the stream.
  *  - Weights live in the tiled GPU layout written by bw_repack_q4_0 /
  *    bw_repack_nvfp4 from the canonical (file) layout.  W[N][K] is cut into
  *    tiles of 128 rows x 512 columns (N padded to a multiple of 128 rows and

@@ -74,11 +74,22 @@ def test_host_validation_rejects_bad_arguments(lib):
     # unaligned weights
     assert lib.bw_gemv_q4_0(p(4097), fake, 64, 64, fake, 1, None, 1e-6, None, fake, None, 0, fake,
                             1 << 20, None) == 1
+    # RMSNORM with unaligned gains; a workspace off its 256-byte alignment
+    assert lib.bw_gemv_q4_0(fake, fake, 64, 64, fake, 1, p(4100), 1e-6, None, fake, None, 1, fake,
+                            1 << 20, None) == 1
+    assert lib.bw_gemv_q4_0(fake, fake, 64, 64, fake, 1, None, 1e-6, None, fake, None, 0, p(4096 + 16),
+                            1 << 20, None) == 1
+    assert lib.bw_gemv_nvfp4(fake, fake, 1.0, 1.0, 64, 64, fake, 1, None, 1e-6, None, fake, None,
+                             0, p(4096 + 128), 1 << 20, None) == 1
+    assert lib.bw_workspace_init(p(4096 + 64), 1 << 20, None) == 1
+    assert lib.bw_moe_route_gemv(fake, fake, fake, 32, None, None, p(4096 + 16), 1 << 30, None) == 1
     # attention: unsupported head dim, too many query rows per kv head
     args = [fake, fake, fake, 128, fake, fake, fake, 8, 8, fake, 1, 1, 8, 2, 96, fake, fake, 1 << 24, None]
     assert lib.bw_paged_attn_decode(*args) == 2
     args[11], args[12], args[13], args[14] = 4, 64, 2, 128    # G * n_rows = 128 > 32
     assert lib.bw_paged_attn_decode(*args) == 2
+    args[16] = p(4096 + 32)                                   # unaligned workspace
+    assert lib.bw_paged_attn_decode(*args) == 1
     # repack: rows not a multiple of 8
     assert lib.bw_repack_q4_0(fake, None, 12, 64, fake, fake, None) == 2
     assert lib.bw_rope_table(C.c_float(-1.0), 64, 16, fake, fake, None) == 1

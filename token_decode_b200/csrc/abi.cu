@@ -42,7 +42,7 @@ const char *bw_status_string(bw_status s) {
 int bw_abi_version(void) { return BW_ABI_VERSION; }
 
 bw_status bw_workspace_init(void *ws, size_t bytes, void *stream) {
-    if (!ws || bytes < BW_WS_HDR_BYTES) return BW_ERR_INVALID_ARG;
+    if (!bw::ws_ok(ws) || bytes < BW_WS_HDR_BYTES) return BW_ERR_INVALID_ARG;
     if (cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
         (void)cudaGetLastError();
         return BW_ERR_CUDA;

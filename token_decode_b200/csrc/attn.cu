@@ -801,7 +801,7 @@ bw_status bw_paged_attn_decode(const float *qkv, const float *rope_cos, const fl
                                const int32_t *page_table, int max_pages, int n_pages,
                                const int32_t *pos, int B, int n_rows, int nq, int nkv, int hd,
                                float *out, void *ws, size_t ws_bytes, void *stream) {
-    if (!ws) return BW_ERR_INVALID_ARG;
+    if (!bw::ws_ok(ws)) return BW_ERR_INVALID_ARG;
     return bw::attn_launch(qkv, rope_cos, rope_sin, rope_max_pos, k_pool, v_pool, page_table,
                            max_pages, n_pages, pos, B, n_rows, nq, nkv, hd, out,
                            bw::scratch_of(ws, ws_bytes), static_cast<cudaStream_t>(stream));

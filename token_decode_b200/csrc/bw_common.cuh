@@ -21,6 +21,9 @@ bw_status launch_status();              // BW_OK or BW_ERR_CUDA after a launch
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// A workspace as the ABI requires it: non-null and BW_WS_ALIGN-byte aligned
+// (the kernels' scratch regions inherit that alignment).
+inline bool ws_ok(const void *ws) { return ws && (reinterpret_cast<uintptr_t>(ws) & (BW_WS_ALIGN - 1)) == 0; }
 
 inline uint32_t *ws_error_word(void *ws) { return static_cast<uint32_t *>(ws); }
 inline uint32_t *ws_counters(void *ws) { return static_cast<uint32_t *>(ws) + 16; }

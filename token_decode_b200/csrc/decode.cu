@@ -84,7 +84,7 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
                          int n_rows, int32_t *tokens_out, float *logits, unsigned flags, void *ws,
                          size_t ws_bytes, void *stream) {
     using namespace bw;
-    if (!m || !kv || !tokens_in || !pos || !tokens_out || !ws || B <= 0 || n_rows <= 0)
+    if (!m || !kv || !tokens_in || !pos || !tokens_out || !ws_ok(ws) || B <= 0 || n_rows <= 0)
         return BW_ERR_INVALID_ARG;
     if (!m->layers || !kv->k || !kv->v || !kv->page_table || !m->rope_cos || !m->rope_sin ||
         !m->final_norm)

@@ -73,12 +73,26 @@ struct GemvParams {
     uint32_t *err;
 };
 
+// The residual values of row group rg that this lane's epilogue adds
+// (zeros where it adds none), loaded early so the load overlaps other work.
+template <int M>
+__device__ __forceinline__ void load_residual(const GemvParams &p, int rg, int lane, float (&res)[M]) {
+#pragma unroll
+    for (int m = 0; m < M; m++) res[m] = 0.0f;
+    if (!(p.flags & BW_GEMV_RESIDUAL) || (lane & 1) != 0 || rg >= p.RG) return;
+    const int n = rg * 8 + ((lane >> 1) & 7);
+#pragma unroll
+    for (int m = 0; m < M; m++)
+        if (m < p.M) res[m] = p.residual[static_cast<size_t>(m) * p.N + n];
+}
+
 // Final values of row group rg (lanes with (lane & 1) == 0 hold row
-// (lane >> 1) & 7): scale, epilogue, outputs, argmax tracking.
-// All lanes must call it (it shuffles); `act` gates the stores.
+// (lane >> 1) & 7): scale, epilogue (res: the residual to add), outputs,
+// argmax tracking.  All lanes must call it (it shuffles); `act` gates the
+// stores.
 template <int FMT, int M>
 __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, const float (&tot)[M],
-                                         float (&bestv)[M], int (&besti)[M], bool act) {
+                                         const float (&res)[M], float (&bestv)[M], int (&besti)[M], bool act) {
     const int r = (lane >> 1) & 7;
     const bool gu = p.flags & BW_GEMV_SILU_GATE;
     float val[M];
@@ -112,7 +126,7 @@ __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, 
         if (m >= p.M) break;
         float v = val[m];
         const size_t o = static_cast<size_t>(m) * p.N + n;
-        if (p.flags & BW_GEMV_RESIDUAL) v = p.residual[o] + v;
+        if (p.flags & BW_GEMV_RESIDUAL) v = res[m] + v;
         if (p.y) p.y[o] = v;
         if (better(v, n, bestv[m], besti[m])) {
             bestv[m] = v;
@@ -178,44 +192,34 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
     }
 
     // ---- consumers
-    pdl_wait();
     const int ctid = threadIdx.x;   // 0 .. 255
     const bool norm = p.flags & BW_GEMV_RMSNORM;
-    // pass 1: the slice's activations (and gains) in natural order, all loads
-    // issued back to back; the RMSNorm sum of squares on the way
     const int ne = nc * 32;
+    // the slice's RMSNorm gains are model data like the weights: staged
+    // before the dependency wait
+    if (norm)
+        (void)stage_row4(reinterpret_cast<const float4 *>(p.gamma + c0 * 32), ne / 4, reinterpret_cast<float4 *>(gt),
+                         0, ne / 4, ctid);
+    pdl_wait();
+    // pass 1: the slice's activations in natural order, one batch of
+    // independent 16-byte loads per thread; with RMSNorm over a K slice the
+    // whole row is read in the same batch, for the sum of squares
     float ss[M];
 #pragma unroll
     for (int m = 0; m < M; m++) {
-        ss[m] = 0.0f;
+        float4 *xs4 = reinterpret_cast<float4 *>(xs + static_cast<size_t>(m) * CS * 32);
         if (m >= p.M) {
-            for (int e = ctid; e < ne; e += GV_CW * 32) xs[static_cast<size_t>(m) * CS * 32 + e] = 0.0f;
+            for (int e = ctid; e < ne / 4; e += GV_CW * 32) xs4[e] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            ss[m] = 0.0f;
             continue;
         }
-        const float *xr = p.x + static_cast<size_t>(m) * p.K + c0 * 32;
-#pragma unroll 4
-        for (int e = ctid; e < ne; e += GV_CW * 32) {
-            const float v = xr[e];
-            xs[static_cast<size_t>(m) * CS * 32 + e] = v;
-            ss[m] = fma_rn(v, v, ss[m]);
-        }
+        const float4 *xr4 = reinterpret_cast<const float4 *>(p.x + static_cast<size_t>(m) * p.K);
+        if (norm && p.S > 1)
+            ss[m] = stage_row4(xr4, p.K / 4, xs4, c0 * 8, ne / 4, ctid);
+        else
+            ss[m] = stage_row4(xr4 + c0 * 8, ne / 4, xs4, 0, ne / 4, ctid);
     }
     if (norm) {
-#pragma unroll 4
-        for (int e = ctid; e < ne; e += GV_CW * 32) gt[e] = p.gamma[c0 * 32 + e];
-        if (p.S > 1) {
-            // the norm needs the whole row, not just this slice
-#pragma unroll
-            for (int m = 0; m < M; m++) {
-                ss[m] = 0.0f;
-                if (m < p.M)
-#pragma unroll 4
-                    for (int k = ctid; k < p.K; k += GV_CW * 32) {
-                        const float v = p.x[static_cast<size_t>(m) * p.K + k];
-                        ss[m] = fma_rn(v, v, ss[m]);
-                    }
-            }
-        }
 #pragma unroll
         for (int m = 0; m < M; m++) {
             ss[m] = warp_sum(ss[m]);
@@ -260,6 +264,8 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
             __syncwarp();
             if (lane == 0) mbar_arrive_relaxed(&empty[s]);
         }
+        float res[M];
+        load_residual<M>(p, rg, lane, res);
         float tot[M];
         reduce_rows16<M>(acc, lane, tot);
 #pragma unroll
@@ -267,7 +273,7 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
 #pragma unroll
             for (int m = 0; m < M; m++) acc[r][m] = 0.0f;
         if (p.S == 1) {
-            epilogue<FMT, M>(p, rg, lane, tot, bestv, besti, true);
+            epilogue<FMT, M>(p, rg, lane, tot, res, bestv, besti, true);
         } else {
             // split K: leave the partial sums; the last slice to finish a row
             // group (per half-warp) adds them in slice order and runs the epilogue
@@ -290,13 +296,23 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
             if (last) {
                 __threadfence();
                 if ((lane & 1) == 0)
-                    for (int s2 = 0; s2 < p.S; s2++) {
-                        const float *src = p.partial + ((static_cast<size_t>(s2) * p.RG + rg) * 8 + r) * M;
+                    // batches of 8 slices' loads in flight, added in slice order
+                    for (int s0 = 0; s0 < p.S; s0 += 8) {
+                        float v[8][M];
 #pragma unroll
-                        for (int m = 0; m < M; m++) sum[m] += ld_cg(src + m);
+                        for (int u = 0; u < 8; u++) {
+                            const float *src = p.partial + ((static_cast<size_t>(s0 + u) * p.RG + rg) * 8 + r) * M;
+#pragma unroll
+                            for (int m = 0; m < M; m++) v[u][m] = s0 + u < p.S ? ld_cg(src + m) : 0.0f;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 8; u++)
+                            if (s0 + u < p.S)
+#pragma unroll
+                                for (int m = 0; m < M; m++) sum[m] += v[u][m];
                     }
             }
-            epilogue<FMT, M>(p, rg, lane, sum, bestv, besti, last);
+            epilogue<FMT, M>(p, rg, lane, sum, res, bestv, besti, last);
             if (last && (lane & 15) == 0) p.rg_cnt[rg] = 0u;
         }
     }
@@ -461,7 +477,7 @@ bw_status gemv_launch(int fmt, const void *wq, const void *ws_scales, float ts, 
     if (!wq || !ws_scales || !x || !sc.cnt || N <= 0 || K <= 0 || M <= 0) return BW_ERR_INVALID_ARG;
     if (N % 8 || K % 32) return BW_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(wq) || !aligned16(ws_scales) || !aligned16(x)) return BW_ERR_INVALID_ARG;
-    if ((flags & BW_GEMV_RMSNORM) && !gamma) return BW_ERR_INVALID_ARG;
+    if ((flags & BW_GEMV_RMSNORM) && (!gamma || !aligned16(gamma))) return BW_ERR_INVALID_ARG;
     if ((flags & BW_GEMV_RESIDUAL) && !residual) return BW_ERR_INVALID_ARG;
     if ((flags & BW_GEMV_ARGMAX) && !argmax_out) return BW_ERR_INVALID_ARG;
     if ((flags & BW_GEMV_SILU_GATE) && (flags & (BW_GEMV_RESIDUAL | BW_GEMV_ARGMAX)))
@@ -532,7 +548,7 @@ bw_status bw_gemv_q4_0(const void *w_q, const void *w_d, int N, int K, const flo
                        const float *gamma, float eps, const float *residual, float *y,
                        int32_t *argmax_out, unsigned flags, void *ws, size_t ws_bytes,
                        void *stream) {
-    if (!ws) return BW_ERR_INVALID_ARG;
+    if (!bw::ws_ok(ws)) return BW_ERR_INVALID_ARG;
     return bw::gemv_launch(BW_FMT_Q4_0, w_q, w_d, 1.0f, 1.0f, N, K, x, M, gamma, eps, residual, y,
                            argmax_out, flags, bw::scratch_of(ws, ws_bytes),
                            static_cast<cudaStream_t>(stream));
@@ -542,7 +558,7 @@ bw_status bw_gemv_nvfp4(const void *w_q, const void *w_s, float ts, float ts_up,
                         const float *x, int M, const float *gamma, float eps,
                         const float *residual, float *y, int32_t *argmax_out, unsigned flags,
                         void *ws, size_t ws_bytes, void *stream) {
-    if (!ws) return BW_ERR_INVALID_ARG;
+    if (!bw::ws_ok(ws)) return BW_ERR_INVALID_ARG;
     return bw::gemv_launch(BW_FMT_NVFP4, w_q, w_s, ts, ts_up, N, K, x, M, gamma, eps, residual, y,
                            argmax_out, flags, bw::scratch_of(ws, ws_bytes),
                            static_cast<cudaStream_t>(stream));

@@ -88,6 +88,33 @@ __device__ __forceinline__ float lds_f(uint32_t a) {
     return v;
 }
 
+// Loads the 16-byte elements [0, n4) of a row, a batch of 8 independent
+// loads per thread in flight before the first is used; elements
+// [lo, lo + n_keep) are also stored to dst[e - lo].  Returns this thread's
+// sum of squares over every element it loaded.
+__device__ __forceinline__ float stage_row4(const float4 *src, int n4, float4 *dst, int lo, int n_keep, int tid) {
+    constexpr int U = 8, STEP = GV_CW * 32;
+    float ss = 0.0f;
+    for (int b = 0; b < n4; b += U * STEP) {
+        float4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int e = b + u * STEP + tid;
+            v[u] = e < n4 ? src[e] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int d = b + u * STEP + tid - lo;
+            if (d >= 0 && d < n_keep) dst[d] = v[u];
+            ss = fma_rn(v[u].x, v[u].x, ss);
+            ss = fma_rn(v[u].y, v[u].y, ss);
+            ss = fma_rn(v[u].z, v[u].z, ss);
+            ss = fma_rn(v[u].w, v[u].w, ss);
+        }
+    }
+    return ss;
+}
+
 // Staged activations: chunk c of row m at (m*chunk_stride + c)*128 bytes; its
 // 16-byte granule g is stored at granule (g ^ (c & 7)), so 8 lanes reading
 // granule g of 8 consecutive chunks hit 8 different bank groups.
@@ -115,15 +142,25 @@ __device__ __forceinline__ void stage_x(float *xs, float *ct, int chunk_stride, 
 // start of each chunk's slot (first pass: one wide burst of independent
 // global loads); each warp turns its chunks into the swizzled, pre-scaled
 // form in place, applying the RMSNorm (x * rnorm) * gamma when gt != null.
+// Two chunks per iteration, so that their loads and lane sums overlap.
 template <int FMT, int M>
 __device__ __forceinline__ void stage_pass2(float *xs, float *ct, const float *gt, const float *rnorm, int CS,
                                             int nc, int warp, int lane) {
-    for (int pair = warp; pair < M * nc; pair += GV_CW) {
+    const int np = M * nc;
+    for (int pair = warp; pair < np; pair += 2 * GV_CW) {
+        const int pair2 = pair + GV_CW;
+        const bool two = pair2 < np;
         const int m = pair / nc, cl = pair - m * nc;
+        const int m2 = two ? pair2 / nc : m, cl2 = two ? pair2 - m2 * nc : cl;
         float v = xs[static_cast<size_t>(m * CS + cl) * 32 + lane];
-        if (gt) v = (v * rnorm[m]) * gt[cl * 32 + lane];
+        float v2 = xs[static_cast<size_t>(m2 * CS + cl2) * 32 + lane];
+        if (gt) {
+            v = (v * rnorm[m]) * gt[cl * 32 + lane];
+            v2 = (v2 * rnorm[m2]) * gt[cl2 * 32 + lane];
+        }
         __syncwarp();
         stage_x<FMT>(xs, ct, CS, m, cl, lane, v);
+        if (two) stage_x<FMT>(xs, ct, CS, m2, cl2, lane, v2);
     }
 }
 

@@ -392,17 +392,38 @@ __global__ void __launch_bounds__(GV_THREADS, 1) moe_grouped_gemv_kernel(const G
             }
         }
         consumer_sync();   // the previous item is done with the staged activations
-        // the item's activation rows in natural order, loads back to back
+        // the item's activation rows in natural order: the 16-byte loads of
+        // all its rows in flight together (rows past its count are zeros)
+        {
+            const float *xr[M];
 #pragma unroll
-        for (int m = 0; m < M; m++) {
-            const float *xr = nullptr;
-            if (m < it.mcnt) {
-                const int j = it.off + m;
-                xr = p.x + static_cast<size_t>(p.gather ? p.asg_row[j] : j) * p.K;
+            for (int m = 0; m < M; m++) {
+                xr[m] = p.x;
+                if (m < it.mcnt) {
+                    const int j = it.off + m;
+                    xr[m] = p.x + static_cast<size_t>(p.gather ? p.asg_row[j] : j) * p.K;
+                }
             }
-#pragma unroll 4
-            for (int e = threadIdx.x; e < nc * 32; e += GV_CW * 32)
-                xs[static_cast<size_t>(m) * CS * 32 + e] = xr ? xr[e] : 0.0f;
+            const int n4 = nc * 8, tot = M * n4;
+            for (int b = 0; b < tot; b += 8 * GV_CW * 32) {
+                float4 v[8];
+                int at[8];
+#pragma unroll
+                for (int u = 0; u < 8; u++) {
+                    const int i = b + u * GV_CW * 32 + static_cast<int>(threadIdx.x);
+                    const int m = i / n4, e = i - m * n4;
+                    const float *row = xr[0];
+#pragma unroll
+                    for (int mm = 1; mm < M; mm++)
+                        if (m == mm) row = xr[mm];
+                    v[u] = (i < tot && m < it.mcnt) ? reinterpret_cast<const float4 *>(row)[e]
+                                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    at[u] = i < tot ? m * CS * 8 + e : -1;
+                }
+#pragma unroll
+                for (int u = 0; u < 8; u++)
+                    if (at[u] >= 0) reinterpret_cast<float4 *>(xs)[at[u]] = v[u];
+            }
         }
         consumer_sync();
         // the inner loop for the item's actual row count (1, 2 or up to 4)
@@ -613,7 +634,7 @@ extern "C" {
 
 bw_status bw_moe_route_gemv(const bw_model *m, const bw_layer *ly, float *x, int R, int32_t *topk_idx,
                             float *topk_w, void *ws, size_t ws_bytes, void *stream) {
-    if (!m || !ly || !ws) return BW_ERR_INVALID_ARG;
+    if (!m || !ly || !bw::ws_ok(ws)) return BW_ERR_INVALID_ARG;
     if (ws_bytes < bw_moe_workspace_bytes(m, R)) return BW_ERR_INVALID_ARG;
     bw::Scratch sc = bw::scratch_of(ws, ws_bytes);
     return bw::moe_ffn_launch(m, ly, x, R, sc, sc.base, static_cast<cudaStream_t>(stream), topk_idx, topk_w);
