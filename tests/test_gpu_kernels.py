@@ -322,6 +322,8 @@ def _attn_oracle(kp, vp, table, qkv, pos, B, R, nq, nkv, hd, n_pages, theta=1e6)
     dict(B=1, R=1, nq=4, nkv=2, hd=64, ctxs=[8000]),          # long splits: the 4-stage ring wraps
     dict(B=40, R=1, nq=8, nkv=4, hd=64,                       # >= one group per SM: one split, 2-stage ring
          ctxs=[17 + 7 * i for i in range(40)]),
+    dict(B=3, R=1, nq=8, nkv=4, hd=64, ctxs=[9300, 40, 5000]),  # page-table rows too wide to load with the
+                                                               # position; cluster merge of ragged lengths
 ])
 def test_paged_attention_matches_oracle(case):
     B, R, nq, nkv, hd, ctxs = case["B"], case["R"], case["nq"], case["nkv"], case["hd"], case["ctxs"]

@@ -54,6 +54,7 @@ constexpr int ATT_MAXPAGES = 8192;              // page-table width the CTA's pa
 constexpr int ATT_ST = 64;                      // tokens per stage: 4 pages, 8 per consumer warp
 constexpr int ATT_PPS = ATT_ST / 16;
 constexpr int ATT_PST = ATT_ST + 8;             // padded row of the probability planes (halves)
+constexpr int ATT_PT_U = 2;                     // page-table entries per thread loaded with the position
 
 struct AttnParams {
     const float *qkv;
@@ -161,6 +162,10 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
     constexpr int NT = WD / 8;              // n-tiles per warp in P.V
     constexpr int SH = ATT_ST * HD;         // halves per K (or V) stage
     constexpr uint32_t PAGE_BYTES = 16 * HD * 2;
+    // the cluster merge's partials and weights live in the drained ring
+    static_assert(NST != 4 || (static_cast<size_t>(ATT_MAXQ) * HD + 3 * ATT_MAXQ + 2 * ATT_MAXCL * ATT_MAXQ) * 4 <=
+                                  static_cast<size_t>(NST) * 2 * SH * 2,
+                  "cluster merge scratch exceeds the ring");
     extern __shared__ __align__(1024) unsigned char att_sm_raw[];
     // the swizzle pattern follows address bits, so the ring starts on 1024 bytes
     unsigned char *att_sm = att_sm_raw + ((1024u - (smem_u32(att_sm_raw) & 1023u)) & 1023u);
@@ -190,6 +195,17 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
     pdl_trigger();
     pdl_wait();
 
+    // a page-table row of up to ATT_PT_U * ATT_THREADS entries is loaded
+    // together with the position, so the split's page list does not cost a
+    // second dependent round trip
+    const int32_t *pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
+    const bool pt_pre = p.max_pages <= ATT_PT_U * ATT_THREADS;
+    int pte[ATT_PT_U];
+#pragma unroll
+    for (int u = 0; u < ATT_PT_U; u++) {
+        const int i = tid + u * ATT_THREADS;
+        pte[u] = (pt_pre && i < p.max_pages) ? pt[i] : -1;
+    }
     const int p0 = p.pos[b];
     int len = p0 + p.R;
     if (p0 < 0 || len > p.max_pages * 16 || len > p.rope_max_pos) {
@@ -202,17 +218,31 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
     const int npl = pg1 - pg0;                          // pages of this split
     const int t1 = min(len, pg1 * 16);
     const int n_stages = (npl + ATT_PPS - 1) / ATT_PPS;
-    const int32_t *pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
     const size_t row_stride = static_cast<size_t>(p.nq + 2 * p.nkv) * HD;
 
     // the split's physical pages, validated once, in parallel
-    for (int i = tid; i < npl; i += ATT_THREADS) {
-        int page = pt[pg0 + i];
-        if (page < 0 || page >= p.n_pages) {
-            set_error(p.err, BW_DEVERR_BAD_PAGE);
-            page = -1;
+    if (pt_pre) {
+#pragma unroll
+        for (int u = 0; u < ATT_PT_U; u++) {
+            const int i = tid + u * ATT_THREADS;
+            if (i >= pg0 && i < pg1) {
+                int page = pte[u];
+                if (page < 0 || page >= p.n_pages) {
+                    set_error(p.err, BW_DEVERR_BAD_PAGE);
+                    page = -1;
+                }
+                pages[i - pg0] = page;
+            }
         }
-        pages[i] = page;
+    } else {
+        for (int i = tid; i < npl; i += ATT_THREADS) {
+            int page = pt[pg0 + i];
+            if (page < 0 || page >= p.n_pages) {
+                set_error(p.err, BW_DEVERR_BAD_PAGE);
+                page = -1;
+            }
+            pages[i] = page;
+        }
     }
     __syncthreads();
 
@@ -511,22 +541,46 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
         cg::cluster_group cluster = cg::this_cluster();
         cluster.sync();
         const int ns = p.n_split;
+        // every split's (max, sum) in one parallel pass of remote loads, the
+        // merge weights once per query row, then one pass of independent
+        // remote loads of the partial outputs, summed in split order
+        float *s_w = s_l + ATT_MAXQ;                  // [ns][Q] max, then weight (local only)
+        float *s_sl = s_w + ATT_MAXCL * ATT_MAXQ;     // [ns][Q] sums
+        float *s_L = s_sl + ATT_MAXCL * ATT_MAXQ;     // [Q]
+        for (int e = tid; e < ns * p.Q; e += ATT_CT) {
+            const int r2 = e / p.Q, qi = e - r2 * p.Q;
+            s_w[e] = cluster.map_shared_rank(s_m, r2)[qi];
+            s_sl[e] = cluster.map_shared_rank(s_l, r2)[qi];
+        }
+        consumers_sync();
+        if (tid < p.Q) {
+            const int qi = tid;
+            float M = -INFINITY;
+            for (int r2 = 0; r2 < ns; r2++) M = fmaxf(M, s_w[r2 * p.Q + qi]);
+            float L = 0.0f;
+            for (int r2 = 0; r2 < ns; r2++) {
+                const float m2 = s_w[r2 * p.Q + qi];
+                const float w = (m2 == -INFINITY) ? 0.0f : expf(m2 - M);
+                s_w[r2 * p.Q + qi] = w;
+                L = fmaf(s_sl[r2 * p.Q + qi], w, L);
+            }
+            s_L[qi] = L;
+        }
+        consumers_sync();
         const int per = (p.Q * HD + ns - 1) / ns;
         for (int e = split * per + tid; e < min(p.Q * HD, (split + 1) * per); e += ATT_CT) {
             const int qi = e / HD, d = e - qi * HD;
-            float M = -INFINITY;
-            for (int r2 = 0; r2 < ns; r2++) M = fmaxf(M, cluster.map_shared_rank(s_m, r2)[qi]);
-            float L = 0.0f, O = 0.0f;
-            for (int r2 = 0; r2 < ns; r2++) {
-                const float m2 = cluster.map_shared_rank(s_m, r2)[qi];
-                if (m2 == -INFINITY) continue;
-                const float w = expf(m2 - M);
-                L = fmaf(cluster.map_shared_rank(s_l, r2)[qi], w, L);
-                O = fmaf(cluster.map_shared_rank(s_o, r2)[qi * HD + d], w, O);
-            }
+            float ov[ATT_MAXCL];
+#pragma unroll
+            for (int r2 = 0; r2 < ATT_MAXCL; r2++)
+                ov[r2] = r2 < ns ? cluster.map_shared_rank(s_o, min(r2, ns - 1))[qi * HD + d] : 0.0f;
+            float O = 0.0f;
+#pragma unroll
+            for (int r2 = 0; r2 < ATT_MAXCL; r2++)
+                if (r2 < ns) O = fmaf(ov[r2], s_w[r2 * p.Q + qi], O);
             const int r = qi / p.G, gq = qi - r * p.G;
             p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
-                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = O / L;
+                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = O / s_L[qi];
         }
         cluster.sync();   // keep this CTA's shared memory alive until every reader is done
         return;
