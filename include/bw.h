@@ -38,6 +38,9 @@
  *    paths (bw_read_error is the one call that synchronizes).
  *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
  *    kernel call is asynchronous on it.
+ *  - Host threads may call the entry points concurrently (each with its own
+ *    workspace): the library's host-side caches (SM counts, kernel
+ *    attributes, tensor maps) are guarded by locks.
  *  - Arguments are validated on the host before any launch; a failed check
  *    returns BW_ERR_INVALID_ARG or BW_ERR_UNSUPPORTED_SHAPE and launches
  *    nothing.  A launch failure returns BW_ERR_CUDA.  Conditions only the

@@ -696,6 +696,8 @@ size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages) 
 // dependency on the driver library); encoded maps are cached per pool.
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::mutex mu;   // host threads may call the library concurrently
+    std::lock_guard<std::mutex> lk(mu);
     if (!fn) {
         void *f = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -717,6 +719,8 @@ static bool kv_tensor_map(CUtensorMap *out, void *pool, int n_pages, int nkv, in
     };
     static Entry cache[512];
     static int n_cache = 0, next = 0;
+    static std::mutex mu;   // host threads may call the library concurrently
+    std::lock_guard<std::mutex> lk(mu);
     const int rows = n_pages * nkv * 16;
     for (int i = 0; i < n_cache; i++)
         if (cache[i].pool == pool && cache[i].rows == rows && cache[i].hd == hd) {
@@ -750,27 +754,31 @@ static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnPara
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
-    if (attr_set[dev] < smem) {
-        if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess) {
-            (void)cudaGetLastError();
-            return BW_ERR_CUDA;
-        }
-        attr_set[dev] = smem;
-    }
     AttnParams q = p;
     q.n_split = ns;
     q.cluster = (ns > 1 && ns <= ATT_MAXCL && NST == 4) ? 1 : 0;
-    if (!q.cluster) return launch_pdl(attn_kernel<HD, MT, NST>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
-    static bool cl_set[64] = {};
-    if (!cl_set[dev]) {
-        if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-            cudaSuccess) {
-            (void)cudaGetLastError();
-            return BW_ERR_CUDA;
+    {
+        static bool cl_set[64] = {};
+        static std::mutex mu;   // host threads may call the library concurrently
+        std::lock_guard<std::mutex> lk(mu);
+        if (attr_set[dev] < smem) {
+            if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return BW_ERR_CUDA;
+            }
+            attr_set[dev] = smem;
         }
-        cl_set[dev] = true;
+        if (q.cluster && !cl_set[dev]) {
+            if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+                cudaSuccess) {
+                (void)cudaGetLastError();
+                return BW_ERR_CUDA;
+            }
+            cl_set[dev] = true;
+        }
     }
+    if (!q.cluster) return launch_pdl(attn_kernel<HD, MT, NST>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ns, nkv, B);
     cfg.blockDim = dim3(ATT_THREADS);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/bw.h"
 
 #define BW_WS_HDR_BYTES (1u << 18)     // error word + counters at the start of a workspace

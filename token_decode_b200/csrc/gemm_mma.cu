@@ -670,13 +670,17 @@ bw_status mma_gemm_launch(const void *wq, const void *ws_scales, float ts, float
         const bw_status s0 = launch_pdl(act_pack_kernel, dim3(Mp), dim3(256), 0, st, x + static_cast<size_t>(m0) * K,
                                         Mr, Mp, K, p.KT, (flags & BW_GEMV_RMSNORM) ? gamma : nullptr, eps, bpk);
         if (s0 != BW_OK) return s0;
-        if (attr_set[dev] < pl.smem) {
-            if (cudaFuncSetAttribute(mma_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(pl.smem)) != cudaSuccess) {
-                (void)cudaGetLastError();
-                return BW_ERR_CUDA;
+        {
+            static std::mutex mu;   // host threads may call the library concurrently
+            std::lock_guard<std::mutex> lk(mu);
+            if (attr_set[dev] < pl.smem) {
+                if (cudaFuncSetAttribute(mma_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(pl.smem)) != cudaSuccess) {
+                    (void)cudaGetLastError();
+                    return BW_ERR_CUDA;
+                }
+                attr_set[dev] = pl.smem;
             }
-            attr_set[dev] = pl.smem;
         }
         const bw_status s1 = launch_pdl(mma_gemm_kernel, dim3(pl.grid), dim3(MM_THREADS), pl.smem, st, p);
         if (s1 != BW_OK) return s1;

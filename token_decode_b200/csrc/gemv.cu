@@ -459,13 +459,17 @@ static bw_status launch_gemv_m(const GemvParams &p0, const GemvPlan &pl, cudaStr
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
-    if (attr_set[dev] < pl.smem) {
-        if (cudaFuncSetAttribute(gemv_kernel<FMT, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(pl.smem)) != cudaSuccess) {
-            (void)cudaGetLastError();
-            return BW_ERR_CUDA;
+    {
+        static std::mutex mu;   // host threads may call the library concurrently
+        std::lock_guard<std::mutex> lk(mu);
+        if (attr_set[dev] < pl.smem) {
+            if (cudaFuncSetAttribute(gemv_kernel<FMT, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(pl.smem)) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return BW_ERR_CUDA;
+            }
+            attr_set[dev] = pl.smem;
         }
-        attr_set[dev] = pl.smem;
     }
     return launch_pdl(gemv_kernel<FMT, M>, dim3(pl.grid), dim3(GV_THREADS), pl.smem, st, p0);
 }

@@ -499,13 +499,17 @@ static bw_status grouped_go(const GroupedParams &p, cudaStream_t st) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
-    if (attr_set[dev] < smem) {
-        if (cudaFuncSetAttribute(moe_grouped_gemv_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem)) != cudaSuccess) {
-            (void)cudaGetLastError();
-            return BW_ERR_CUDA;
+    {
+        static std::mutex mu;   // host threads may call the library concurrently
+        std::lock_guard<std::mutex> lk(mu);
+        if (attr_set[dev] < smem) {
+            if (cudaFuncSetAttribute(moe_grouped_gemv_kernel<FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return BW_ERR_CUDA;
+            }
+            attr_set[dev] = smem;
         }
-        attr_set[dev] = smem;
     }
     // persistent: one CTA per SM, items assigned round robin
     return launch_pdl(moe_grouped_gemv_kernel<FMT>, dim3(sm_count()), dim3(GV_THREADS), smem, st, p);
@@ -544,6 +548,8 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
         int dev = 0;
         cudaGetDevice(&dev);
         if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
+        static std::mutex mu;   // host threads may call the library concurrently
+        std::unique_lock<std::mutex> lk(mu);
         if (!attr_set[dev]) {
             if (cudaFuncSetAttribute(moe_router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(rsm)) != cudaSuccess) {
@@ -552,6 +558,7 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
             }
             attr_set[dev] = true;
         }
+        lk.unlock();
         s = launch_pdl(moe_router_kernel, dim3((E + 7) / 8, n_slices, (R + 31) / 32), dim3(256), rsm, st,
                        static_cast<const float *>(ms.y), ly->router, R, H, E, ms.logits);
     }
