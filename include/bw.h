@@ -110,6 +110,7 @@ typedef int bw_status;
 
 /* decode-step flags */
 #define BW_STEP_ADVANCE 1u    /* after the step: tokens_in <- tokens_out, pos += n_rows */
+#define BW_STEP_VALIDATE_ONLY 2u  /* validate descriptors and arguments on the host; launch nothing */
 #define BW_MAX_VERIFY_ROWS 8  /* n_rows limit of a verify pass (the last token + up to 7 drafts) */
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -300,7 +301,11 @@ size_t bw_moe_workspace_bytes(const struct bw_model *m, int R);
  *   tokens_in: int32 [B*n_rows]; pos: int32 [B] (position of each sequence's
  *   first row); tokens_out: int32 [B*n_rows] (argmax after each row);
  *   logits: fp32 [B*n_rows][V] or NULL.
- * flags: BW_STEP_ADVANCE (n_rows == 1 only).
+ * flags: BW_STEP_ADVANCE (n_rows == 1 only); BW_STEP_VALIDATE_ONLY runs every
+ *   host-side check of the step (descriptor shapes and alignment, every
+ *   launch's limits) and returns without touching the device -- the same
+ *   checks a normal call makes before its first launch, so a rejected call
+ *   never leaves a partial step queued.
  * ws must hold bw_decode_workspace_bytes(m, kv, B, n_rows). */
 bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in, int32_t *pos,
                          int B, int n_rows, int32_t *tokens_out, float *logits, unsigned flags,

@@ -20,6 +20,7 @@ DEVERR_BAD_PAGE, DEVERR_TIMEOUT, DEVERR_BAD_TOKEN, DEVERR_BAD_POS = 1, 2, 4, 8
 FMT_Q4_0, FMT_NVFP4 = 0, 1
 GEMV_RMSNORM, GEMV_RESIDUAL, GEMV_SILU_GATE, GEMV_ARGMAX = 1, 2, 4, 8
 STEP_ADVANCE = 1
+STEP_VALIDATE_ONLY = 2
 MAX_VERIFY_ROWS = 8
 
 # every symbol include/bw.h declares (checked by the CPU test-suite)

@@ -807,10 +807,9 @@ static bw_status attn_go_st(int ns, int nkv, int B, cudaStream_t st, const AttnP
                                                          : attn_go<HD, MT, 2>(ns, nkv, B, st, p);
 }
 
-bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
-                      void *k_pool, void *v_pool, const int32_t *page_table, int max_pages,
-                      int n_pages, const int32_t *pos, int B, int R, int nq, int nkv, int hd,
-                      float *out, const Scratch &sc, cudaStream_t st) {
+bw_status attn_check(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
+                     const void *k_pool, const void *v_pool, const int32_t *page_table, int max_pages, int n_pages,
+                     const int32_t *pos, int B, int R, int nq, int nkv, int hd, const float *out, const Scratch &sc) {
     if (!qkv || !rope_cos || !rope_sin || !k_pool || !v_pool || !page_table || !pos || !out || !sc.cnt)
         return BW_ERR_INVALID_ARG;
     if (B <= 0 || R <= 0 || nq <= 0 || nkv <= 0 || max_pages <= 0 || n_pages <= 0 || rope_max_pos <= 0)
@@ -821,7 +820,18 @@ bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope
     if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(qkv) || !aligned16(out)) return BW_ERR_INVALID_ARG;
     if (nkv > 65535 || B > 65535) return BW_ERR_UNSUPPORTED_SHAPE;
     if (static_cast<size_t>(B) * nkv > 65536 - CNT_ATTN - 16) return BW_ERR_UNSUPPORTED_SHAPE;
+    if (static_cast<long long>(n_pages) * nkv * 16 > 0xffffffffLL) return BW_ERR_UNSUPPORTED_SHAPE;
     if (sc.bytes < attn_scratch_bytes(B, R, nq, nkv, hd, max_pages)) return BW_ERR_INVALID_ARG;
+    return BW_OK;
+}
+
+bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
+                      void *k_pool, void *v_pool, const int32_t *page_table, int max_pages,
+                      int n_pages, const int32_t *pos, int B, int R, int nq, int nkv, int hd,
+                      float *out, const Scratch &sc, cudaStream_t st) {
+    const bw_status chk = attn_check(qkv, rope_cos, rope_sin, rope_max_pos, k_pool, v_pool, page_table, max_pages,
+                                     n_pages, pos, B, R, nq, nkv, hd, out, sc);
+    if (chk != BW_OK) return chk;
     AttnParams p;
     p.qkv = qkv;
     p.rope_cos = rope_cos;
@@ -843,7 +853,6 @@ bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope
     p.out = out;
     p.err = sc.err;
     p.cnt = sc.cnt + CNT_ATTN;
-    if (static_cast<long long>(n_pages) * nkv * 16 > 0xffffffffLL) return BW_ERR_UNSUPPORTED_SHAPE;
     if (!kv_tensor_map(&p.tmk, k_pool, n_pages, nkv, hd) || !kv_tensor_map(&p.tmv, v_pool, n_pages, nkv, hd))
         return BW_ERR_CUDA;
     const int ns = attn_splits(B, nkv, max_pages);

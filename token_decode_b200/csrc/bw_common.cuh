@@ -66,8 +66,20 @@ constexpr unsigned CNT_ARGMAX = 1;
 constexpr unsigned CNT_GEMV_RG = 64;
 constexpr unsigned CNT_ATTN = 32768;
 
-// internal launchers (host), shared by the single-op entry points and the step
+// internal launchers (host), shared by the single-op entry points and the step.
+// Each *_check validates exactly what its launcher would reject, without
+// launching, so that a caller composing several launches (the decode step)
+// can reject bad arguments before the first one is queued.
 size_t gemv_scratch_bytes(int N, int K, int M);
+bw_status gemv_check(int fmt, const void *wq, const void *wscales, int N, int K, const float *x, int M,
+                     const float *gamma, const float *residual, const float *y, const int32_t *argmax_out,
+                     unsigned flags, const Scratch &sc);
+bw_status mma_check(int N, int K, int M);
+bw_status attn_check(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
+                     const void *k_pool, const void *v_pool, const int32_t *page_table, int max_pages, int n_pages,
+                     const int32_t *pos, int B, int R, int nq, int nkv, int hd, const float *out, const Scratch &sc);
+bw_status embed_check(int fmt, const void *e_q, const void *e_s, int V, int H, const int32_t *tokens, int M,
+                      const float *x);
 bw_status gemv_launch(int fmt, const void *wq, const void *wscales, float ts, float ts_up, int N, int K,
                       const float *x, int M, const float *gamma, float eps, const float *residual,
                       float *y, int32_t *argmax_out, unsigned flags, const Scratch &sc,

@@ -19,6 +19,7 @@ namespace bw {
 
 bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R, const Scratch &sc,
                          char *moe_base, cudaStream_t st);
+bw_status moe_check(const bw_model *m, const bw_layer *ly, int R);
 size_t moe_scratch_bytes(const bw_model *m, int R);
 
 struct StepBuffers {
@@ -71,6 +72,42 @@ static bool qw_ok(const bw_qweight &w, int N, int K, int fmt) {
     return w.q && w.s && w.N == N && w.K == K && w.fmt == fmt;
 }
 
+// Every launch of the step validated before the first is queued, with the
+// arguments the launches below pass (same order, same buffers).
+static bw_status step_check(const bw_model *m, const bw_kv *kv, const int32_t *tokens_in, const int32_t *pos, int B,
+                            int n_rows, const int32_t *tokens_out, const float *logits, const StepBuffers &bf) {
+    const int fmt = m->embed.fmt;
+    const int R = B * n_rows;
+    const int nqkv = (m->nq + 2 * m->nkv) * m->hd;
+    bw_status s = embed_check(fmt, m->embed.q, m->embed.s, m->V, m->H, tokens_in, R, bf.x);
+    for (int l = 0; l < m->L && s == BW_OK; l++) {
+        const bw_layer &ly = m->layers[l];
+        s = gemv_check(fmt, ly.wqkv.q, ly.wqkv.s, nqkv, m->H, bf.x, R, ly.attn_norm, nullptr, bf.qkv, nullptr,
+                       BW_GEMV_RMSNORM, bf.kern);
+        if (s == BW_OK)
+            s = attn_check(bf.qkv, m->rope_cos, m->rope_sin, m->rope_max_pos, kv->k[l], kv->v[l], kv->page_table,
+                           kv->max_pages, kv->n_pages, pos, B, n_rows, m->nq, m->nkv, m->hd, bf.attn, bf.kern);
+        if (s == BW_OK)
+            s = gemv_check(fmt, ly.wo.q, ly.wo.s, m->H, m->nq * m->hd, bf.attn, R, nullptr, bf.x, bf.x, nullptr,
+                           BW_GEMV_RESIDUAL, bf.kern);
+        if (s != BW_OK) break;
+        if (m->n_experts == 0) {
+            s = gemv_check(fmt, ly.wgu.q, ly.wgu.s, 2 * m->F, m->H, bf.x, R, ly.ffn_norm, nullptr, bf.act, nullptr,
+                           BW_GEMV_RMSNORM | BW_GEMV_SILU_GATE, bf.kern);
+            if (s == BW_OK)
+                s = gemv_check(fmt, ly.wd.q, ly.wd.s, m->H, m->F, bf.act, R, nullptr, bf.x, bf.x, nullptr,
+                               BW_GEMV_RESIDUAL, bf.kern);
+        } else {
+            s = moe_check(m, &ly, R);
+            if (s == BW_OK && ly.sgu.fmt != fmt) s = BW_ERR_INVALID_ARG;
+        }
+    }
+    if (s == BW_OK)
+        s = gemv_check(fmt, m->lm_head.q, m->lm_head.s, m->V, m->H, bf.x, R, m->final_norm, nullptr, logits,
+                       tokens_out, BW_GEMV_RMSNORM | BW_GEMV_ARGMAX, bf.kern);
+    return s;
+}
+
 }  // namespace bw
 
 extern "C" {
@@ -105,9 +142,10 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
     }
     StepBuffers bf;
     if (ws_bytes < step_bytes(m, kv, B, n_rows, &bf, ws)) return BW_ERR_INVALID_ARG;
+    bw_status s = step_check(m, kv, tokens_in, pos, B, n_rows, tokens_out, logits, bf);
+    if (s != BW_OK || (flags & BW_STEP_VALIDATE_ONLY)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int R = B * n_rows;
-    bw_status s;
 
     s = embed_launch(fmt, m->embed.q, m->embed.s, m->embed.ts, m->V, m->H, tokens_in, R, bf.x,
                      bf.kern.err, st);

@@ -620,13 +620,25 @@ size_t mma_scratch_bytes(int N, int K, int M) {
     return tot;
 }
 
+bw_status mma_check(int N, int K, int M) {
+    if (N <= 0 || K <= 0 || M <= 0) return BW_ERR_INVALID_ARG;
+    if (K % 8) return BW_ERR_UNSUPPORTED_SHAPE;
+    for (int m0 = 0; m0 < M; m0 += MM_MAXM) {
+        const MmaPlan pl = plan_mma(N, K, mma_rows_padded(min(MM_MAXM, M - m0)));
+        if (pl.smem > MM_SMEM_LIMIT) return BW_ERR_UNSUPPORTED_SHAPE;
+        if (pl.S > 1 && gv_row_blocks(N) + CNT_GEMV_RG > CNT_ATTN) return BW_ERR_UNSUPPORTED_SHAPE;
+    }
+    return BW_OK;
+}
+
 bw_status mma_gemm_launch(const void *wq, const void *ws_scales, float ts, float ts_up, int N, int K,
                           const float *x, int M, const float *gamma, float eps, const float *residual, float *y,
                           int32_t *argmax_out, unsigned flags, const Scratch &sc, cudaStream_t st,
                           int32_t *adv_tokens, int32_t *adv_pos) {
     if (sc.bytes < mma_scratch_bytes(N, K, M)) return BW_ERR_INVALID_ARG;
     if (!aligned16(gamma) && (flags & BW_GEMV_RMSNORM)) return BW_ERR_INVALID_ARG;
-    if (K % 8) return BW_ERR_UNSUPPORTED_SHAPE;
+    const bw_status chk = mma_check(N, K, M);
+    if (chk != BW_OK) return chk;
     const int ncols = (flags & BW_GEMV_SILU_GATE) ? N / 2 : N;
     static size_t attr_set[64] = {};
     int dev = 0;

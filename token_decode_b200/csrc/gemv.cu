@@ -38,6 +38,9 @@
 
 namespace bw {
 
+// Largest dynamic shared memory a CTA may request (the static arrays take the rest).
+constexpr size_t GV_SMEM_LIMIT = 227 * 1024 - 2048;
+
 // One activation row: a CTA is half an SM (2 stages, <= 32 KB of staged
 // activations, <= 113 registers), so two CTAs share an SM -- two of this
 // kernel, or this one and the next kernel on the stream starting early.
@@ -474,11 +477,11 @@ static bw_status launch_gemv_m(const GemvParams &p0, const GemvPlan &pl, cudaStr
     return launch_pdl(gemv_kernel<FMT, M>, dim3(pl.grid), dim3(GV_THREADS), pl.smem, st, p0);
 }
 
-bw_status gemv_launch(int fmt, const void *wq, const void *ws_scales, float ts, float ts_up, int N,
-                      int K, const float *x, int M, const float *gamma, float eps,
-                      const float *residual, float *y, int32_t *argmax_out, unsigned flags,
-                      const Scratch &sc, cudaStream_t st, int32_t *adv_tokens, int32_t *adv_pos) {
+bw_status gemv_check(int fmt, const void *wq, const void *ws_scales, int N, int K, const float *x, int M,
+                     const float *gamma, const float *residual, const float *y, const int32_t *argmax_out,
+                     unsigned flags, const Scratch &sc) {
     if (!wq || !ws_scales || !x || !sc.cnt || N <= 0 || K <= 0 || M <= 0) return BW_ERR_INVALID_ARG;
+    if (fmt != BW_FMT_Q4_0 && fmt != BW_FMT_NVFP4) return BW_ERR_INVALID_ARG;
     if (N % 8 || K % 32) return BW_ERR_UNSUPPORTED_SHAPE;
     if (!aligned16(wq) || !aligned16(ws_scales) || !aligned16(x)) return BW_ERR_INVALID_ARG;
     if ((flags & BW_GEMV_RMSNORM) && (!gamma || !aligned16(gamma))) return BW_ERR_INVALID_ARG;
@@ -488,6 +491,21 @@ bw_status gemv_launch(int fmt, const void *wq, const void *ws_scales, float ts, 
         return BW_ERR_INVALID_ARG;
     if (!(flags & BW_GEMV_ARGMAX) && !y) return BW_ERR_INVALID_ARG;
     if (sc.bytes < gemv_scratch_bytes(N, K, M)) return BW_ERR_INVALID_ARG;
+    if (use_mma(fmt, M)) return mma_check(N, K, M);
+    for (int m0 = 0; m0 < M; m0 += GV_MAX_M) {
+        const GemvPlan pl = plan_gemv(N, K, kernel_m(min(GV_MAX_M, M - m0)), (flags & BW_GEMV_RMSNORM) != 0);
+        if (pl.smem > GV_SMEM_LIMIT) return BW_ERR_UNSUPPORTED_SHAPE;
+        if (pl.S > 1 && N / 8 + CNT_GEMV_RG > CNT_ATTN) return BW_ERR_UNSUPPORTED_SHAPE;
+    }
+    return BW_OK;
+}
+
+bw_status gemv_launch(int fmt, const void *wq, const void *ws_scales, float ts, float ts_up, int N,
+                      int K, const float *x, int M, const float *gamma, float eps,
+                      const float *residual, float *y, int32_t *argmax_out, unsigned flags,
+                      const Scratch &sc, cudaStream_t st, int32_t *adv_tokens, int32_t *adv_pos) {
+    const bw_status chk = gemv_check(fmt, wq, ws_scales, N, K, x, M, gamma, residual, y, argmax_out, flags, sc);
+    if (chk != BW_OK) return chk;
     if (use_mma(fmt, M))
         return mma_gemm_launch(wq, ws_scales, ts, ts_up, N, K, x, M, gamma, eps, residual, y, argmax_out, flags, sc,
                                st, adv_tokens, adv_pos);

@@ -200,11 +200,18 @@ __global__ void rmsnorm_kernel(float *x, const float *add, const float *gamma, i
     }
 }
 
-bw_status embed_launch(int fmt, const void *e_q, const void *e_s, float ts, int V, int H,
-                       const int32_t *tokens, int M, float *x, uint32_t *err, cudaStream_t st) {
+bw_status embed_check(int fmt, const void *e_q, const void *e_s, int V, int H, const int32_t *tokens, int M,
+                      const float *x) {
     if (!e_q || !e_s || !tokens || !x || V <= 0 || H <= 0 || M <= 0) return BW_ERR_INVALID_ARG;
     if (H % 32) return BW_ERR_UNSUPPORTED_SHAPE;
     if (fmt != BW_FMT_Q4_0 && fmt != BW_FMT_NVFP4) return BW_ERR_INVALID_ARG;
+    return BW_OK;
+}
+
+bw_status embed_launch(int fmt, const void *e_q, const void *e_s, float ts, int V, int H,
+                       const int32_t *tokens, int M, float *x, uint32_t *err, cudaStream_t st) {
+    const bw_status chk = embed_check(fmt, e_q, e_s, V, H, tokens, M, x);
+    if (chk != BW_OK) return chk;
     return launch_pdl(embed_kernel, dim3(M), dim3(256), 0, st, fmt, static_cast<const uint8_t *>(e_q),
                       static_cast<const uint8_t *>(e_s), ts, V, H, tokens, x, err);
 }

@@ -523,20 +523,35 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
     return moe_ffn_launch(m, ly, x, R, sc, moe_base, st, nullptr, nullptr);
 }
 
-bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R, const Scratch &sc, char *moe_base,
-                         cudaStream_t st, int32_t *topk_idx, float *topk_w) {
+bw_status moe_check(const bw_model *m, const bw_layer *ly, int R) {
+    if (!m || !ly) return BW_ERR_INVALID_ARG;
     const int E = m->n_experts, K = m->topk, H = m->H, Fe = m->F_exp;
     const int fmt = ly->sgu.fmt;
     if (E <= 0 || E > MOE_EMAX || K <= 0 || K > MOE_KMAX || K > E || R <= 0 || R > MOE_RMAX)
         return BW_ERR_UNSUPPORTED_SHAPE;
-    if (H % 32 || Fe % 32 || H % 4) return BW_ERR_UNSUPPORTED_SHAPE;
+    if (H <= 0 || Fe <= 0 || H % 32 || Fe % 32) return BW_ERR_UNSUPPORTED_SHAPE;
     if (static_cast<size_t>(MOE_M) * gv_col_tiles(H) * GV_TC * 33 * 4 > 66 * 1024) return BW_ERR_UNSUPPORTED_SHAPE;
     if (!ly->router || !ly->egu_q || !ly->egu_s || !ly->ed_q || !ly->ed_s || !ly->ffn_norm || !ly->sgu.q ||
-        !ly->sgu.s || !ly->sd.q || !ly->sd.s || !x || !moe_base)
+        !ly->sgu.s || !ly->sd.q || !ly->sd.s)
         return BW_ERR_INVALID_ARG;
+    if (fmt != BW_FMT_Q4_0 && fmt != BW_FMT_NVFP4) return BW_ERR_INVALID_ARG;
     if (fmt == BW_FMT_NVFP4 && (!ly->egu_ts || !ly->ed_ts)) return BW_ERR_INVALID_ARG;
     if (ly->sgu.N != 2 * Fe || ly->sgu.K != H || ly->sd.N != H || ly->sd.K != Fe || ly->sd.fmt != fmt)
         return BW_ERR_INVALID_ARG;
+    // the grouped GEMVs stream every expert matrix with bulk copies
+    if (!aligned16(ly->egu_q) || !aligned16(ly->egu_s) || !aligned16(ly->ed_q) || !aligned16(ly->ed_s) ||
+        !aligned16(ly->sgu.q) || !aligned16(ly->sgu.s) || !aligned16(ly->sd.q) || !aligned16(ly->sd.s))
+        return BW_ERR_INVALID_ARG;
+    return BW_OK;
+}
+
+bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R, const Scratch &sc, char *moe_base,
+                         cudaStream_t st, int32_t *topk_idx, float *topk_w) {
+    const bw_status chk = moe_check(m, ly, R);
+    if (chk != BW_OK) return chk;
+    if (!x || !moe_base) return BW_ERR_INVALID_ARG;
+    const int E = m->n_experts, K = m->topk, H = m->H, Fe = m->F_exp;
+    const int fmt = ly->sgu.fmt;
     MoeScratch ms;
     moe_carve(m, R, moe_base, &ms);
     bw_status s = rmsnorm_launch(x, nullptr, ly->ffn_norm, R, H, m->eps, ms.y, 0, st);
