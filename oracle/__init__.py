@@ -6,7 +6,8 @@ imports nothing from the GPU package; it takes any objects with the attribute
 names of the seeded inputs (fmt, N, K, q, s, ts for a matrix; the layer and
 model fields listed in oracle.h).
 
-Every function here marshals arguments; the arithmetic is in oracle.c.
+Every function here marshals arguments or sequences oracle calls (the
+generation loops); the arithmetic is in oracle.c.
 """
 from __future__ import annotations
 
@@ -82,6 +83,7 @@ def lib():
             "or_topk_softmax": (None, [p, i, i, p, p]),
             "or_argmax": (C.c_int32, [p, i, p]),
             "or_spec_accept": (C.c_int32, [p, p, i, p]),
+            "or_draft_token": (C.c_int32, [p, p, p, f, p, C.c_int32, p, p]),
             "or_decode_token": (C.c_int32, [p, p, i, C.c_int32, i, i, p, p, p, p]),
         }
         for name, (res, args) in sig.items():
@@ -222,6 +224,28 @@ def spec_accept(rows, greedy):
     return int(n), int(nxt[0])
 
 
+class DraftHead:
+    """Host copy of a speculative draft head (norm gains [H], W_draft [V_draft][H])
+    next to the main model's embedding, which it shares."""
+
+    def __init__(self, head, embed, eps: float):
+        self.norm = _np(head.norm).astype(np.float32)
+        self.w = QMat(head.w)
+        self.embed = embed if isinstance(embed, QMat) else QMat(embed)
+        self.eps = float(eps)
+
+
+def draft_token(dh: DraftHead, h, tok: int):
+    """One draft: (token, g, z) with g = rmsnorm(h + deq(E)[tok]) * norm, the
+    hidden the next draft starts from, and z the draft logits [V_draft]."""
+    h = _np(h).astype(np.float32)
+    g = np.empty(dh.embed.K, np.float32)
+    z = np.empty(dh.w.N, np.float32)
+    d = lib().or_draft_token(C.byref(dh.embed.c), C.byref(dh.w.c), _ptr(dh.norm), dh.eps, _ptr(h), int(tok),
+                             _ptr(g), _ptr(z))
+    return int(d), g, z
+
+
 # --------------------------------------------------------------- the model
 
 class Model:
@@ -299,3 +323,51 @@ def decode_token(model: Model, kv: KV, b: int, token: int, pos: int, moe_dense: 
                                 None if moe_idx is None else _ptr(moe_idx), _ptr(margin))
     return {"token": int(tok), "margin": float(margin[0]), "logits": logits, "hidden": hidden,
             "moe_idx": moe_idx}
+
+
+# ------------------------------------------------------ generation loops
+
+def greedy_generate(model: Model, kv: KV, b: int, token: int, pos: int, n_tokens: int):
+    """Plain greedy decoding: the n_tokens tokens after `token` at `pos`."""
+    out = []
+    for i in range(n_tokens):
+        token = decode_token(model, kv, b, token, pos + i)["token"]
+        out.append(token)
+    return out
+
+
+def mtp_generate(model: Model, kv: KV, dh: DraftHead, b: int, token: int, pos: int, n_tokens: int, k: int,
+                 drafter=None):
+    """Speculative decoding with K drafts per verify pass (the deep-dive page,
+    section 5, stage 4, and section 1): one plain step gives the first token
+    and the main model's last hidden state; then each pass drafts d1..dK with
+    the draft head (or `drafter(t0, pos, h, k)` when given), runs the verify
+    rows t0, d1..dK at positions p..p+K over the shared cache, accepts drafts
+    while each equals the greedy token of the row before it, and emits the
+    accepted drafts plus the greedy token after the last accepted row.  The
+    next pass starts from that token and from the hidden state of that row.
+    Returns dict(tokens, accepted per pass, passes)."""
+    L = model.c.L
+    res = decode_token(model, kv, b, token, pos, want_logits=False, want_hidden=True)
+    out = [res["token"]]
+    t0, p, h = res["token"], pos + 1, res["hidden"][L]
+    accepted = []
+    while len(out) < n_tokens:
+        if drafter is None:
+            drafts, g, t = [], h, t0
+            for _ in range(k):
+                t, g, _ = draft_token(dh, g, t)
+                drafts.append(t)
+        else:
+            drafts = list(drafter(t0, p, h, k))
+        rows = [t0] + drafts
+        greedy, hid = [], []
+        for r, tr in enumerate(rows):
+            rr = decode_token(model, kv, b, tr, p + r, want_logits=False, want_hidden=True)
+            greedy.append(rr["token"])
+            hid.append(rr["hidden"][L])
+        n, nxt = spec_accept(rows, greedy)
+        accepted.append(n)
+        out.extend(drafts[:n] + [nxt])
+        t0, h, p = nxt, hid[n], p + n + 1
+    return {"tokens": out[:n_tokens], "accepted": accepted, "passes": len(accepted)}

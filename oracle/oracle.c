@@ -270,6 +270,26 @@ int32_t or_spec_accept(const int32_t *rows, const int32_t *greedy, int n_rows, i
     return n;
 }
 
+/* ------------------------------------------------------------ draft head */
+
+int32_t or_draft_token(const or_qmat *embed, const or_qmat *w_draft, const float *gamma, float eps,
+                       const float *h, int32_t tok, float *g_out, float *z_out)
+{
+    const int H = embed->K;
+    float *x = (float *)malloc(sizeof(float) * (size_t)H);
+    float *z = z_out ? z_out : (float *)malloc(sizeof(float) * (size_t)w_draft->N);
+    or_dequant_row(embed, tok, x);
+    for (int i = 0; i < H; i++)
+        x[i] = h[i] + x[i];
+    or_rmsnorm(x, gamma, H, eps, g_out);
+    or_matvec(w_draft, g_out, z);
+    int32_t d = or_argmax(z, w_draft->N, NULL);
+    free(x);
+    if (!z_out)
+        free(z);
+    return d;
+}
+
 /* ------------------------------------------------------------- decode step */
 
 /* SwiGLU feed-forward: Wd (silu(Wg y) * (Wu y)) */

@@ -128,6 +128,19 @@ int32_t or_argmax(const float *v, int n, float *margin);
  * token of the row before it.  *next = greedy[n]. */
 int32_t or_spec_accept(const int32_t *rows, const int32_t *greedy, int n_rows, int32_t *next);
 
+/* Speculative draft head (the deep-dive page, section 7: a light draft head
+ * that shares the main model's embedding, with its output vocabulary pruned
+ * to a fraction of the full one).  The pages fix no further detail; the
+ * reading taken here:
+ *   g = rmsnorm(h + deq(E)[tok]) * gamma     (h: the main model's residual
+ *                                             stream after its last layer)
+ *   z = deq(W_draft) g                       (W_draft: V_draft x H, the first
+ *                                             V_draft token ids)
+ *   draft = lowest index of max z; g_out[H] <- g, the h of the next draft.
+ * z_out [V_draft] may be NULL. */
+int32_t or_draft_token(const or_qmat *embed, const or_qmat *w_draft, const float *gamma, float eps,
+                       const float *h, int32_t tok, float *g_out, float *z_out);
+
 /* One greedy decode token of sequence b at position pos (writes its K/V into
  * the cache, attends over positions 0..pos).  logits [V] may be NULL;
  * hidden [(L+1)*H] (residual stream after the embedding and after each layer)

@@ -527,3 +527,81 @@ def test_spec_accept_reproduces_greedy_sequence():
         # maximal: the next draft, if any, was wrong
         if n < K:
             assert drafts[n] != truth[n]
+
+
+# ------------------------------------------------------- speculative drafting
+
+@pytest.mark.parametrize("fmt", [synth.FMT_Q4_0, synth.FMT_NVFP4])
+def test_draft_head_matches_fp64_brute_force(fmt):
+    """The draft head, g = rmsnorm(h + E[tok]) * norm and z = W_draft g over the
+    pruned vocabulary, against an fp64 evaluation with the test's own
+    dequantizers."""
+    cfg = synth.CONFIGS["tiny"].with_(fmt=fmt)
+    model = synth.make_model(cfg, "cpu", seed=4)
+    head = synth.make_draft_head(cfg, "cpu", seed=4)
+    dh = oracle.DraftHead(head, model.embed, cfg.eps)
+    deq = _np_deq_q4_0 if fmt == synth.FMT_Q4_0 else _np_deq_nvfp4
+    E, W = deq(model.embed), deq(head.w)
+    assert W.shape == (cfg.draft_vocab, cfg.H) and cfg.draft_vocab < cfg.V
+    gam = head.norm.numpy().astype(np.float64)
+    rng = np.random.default_rng(4)
+    for tok in (0, 17, cfg.V - 1):
+        h = rng.standard_normal(cfg.H).astype(np.float32) * 3
+        d, g, z = oracle.draft_token(dh, h, tok)
+        x = h.astype(np.float64) + E[tok]
+        want_g = x / np.sqrt(np.mean(x * x) + cfg.eps) * gam
+        want_z = W @ want_g
+        assert np.max(np.abs(g - want_g)) < 2e-6 * np.max(np.abs(want_g))
+        assert np.max(np.abs(z - want_z)) < 2e-5 * np.max(np.abs(want_z))
+        assert 0 <= d < cfg.draft_vocab and z[d] == z.max() and d == int(np.argmax(z))
+        top2 = np.sort(want_z)[-2:]
+        if top2[1] - top2[0] > 1e-3:
+            assert d == int(np.argmax(want_z))
+
+
+def _mtp_setup(seed):
+    cfg = synth.CONFIGS["tiny"].with_(steps=32)
+    model = synth.make_model(cfg, "cpu", seed=seed)
+    kv = synth.make_kv(cfg, "cpu", seed=seed)
+    head = synth.make_draft_head(cfg, "cpu", seed=seed)
+    om = oracle.Model(model)
+    return cfg, model, kv, om, oracle.DraftHead(head, model.embed, cfg.eps)
+
+
+@pytest.mark.parametrize("k", [1, 3, 5])
+def test_mtp_output_is_the_greedy_output(k):
+    """The section-1 gate on the oracle's own model: speculative decoding with
+    the draft head emits exactly the tokens of plain greedy decoding."""
+    cfg, model, kv, om, dh = _mtp_setup(5)
+    tok, n = int(synth.start_tokens(cfg, 5)[0]), 12
+    want = oracle.greedy_generate(om, oracle.KV(kv), 0, tok, cfg.ctx, n)
+    got = oracle.mtp_generate(om, oracle.KV(kv), dh, 0, tok, cfg.ctx, n, k)
+    assert got["tokens"] == want
+    assert all(0 <= a <= k for a in got["accepted"])
+    assert 1 + sum(a + 1 for a in got["accepted"]) >= n
+
+
+def test_mtp_pass_counts_for_perfect_and_hopeless_drafts():
+    """Drafts that are the true continuation are all accepted (K + 1 tokens per
+    pass); drafts that are all wrong are all rejected (one token per pass); the
+    output is the greedy output either way."""
+    cfg, model, kv, om, dh = _mtp_setup(6)
+    tok, n, k = int(synth.start_tokens(cfg, 6)[0]), 13, 3
+    truth = oracle.greedy_generate(om, oracle.KV(kv), 0, tok, cfg.ctx, n + k + 1)
+    first = cfg.ctx + 1          # position of the token the first verify pass starts from
+
+    def perfect(t0, p, h, kk):
+        i = p - first            # truth[i] is the token at position p
+        assert truth[i] == t0
+        return truth[i + 1: i + 1 + kk]
+
+    def hopeless(t0, p, h, kk):
+        i = p - first
+        return [(t + 1) % cfg.V for t in truth[i + 1: i + 1 + kk]]
+
+    got = oracle.mtp_generate(om, oracle.KV(kv), dh, 0, tok, cfg.ctx, n, k, drafter=perfect)
+    assert got["tokens"] == truth[:n]
+    assert got["accepted"] == [k] * got["passes"] and got["passes"] == math.ceil((n - 1) / (k + 1))
+    got = oracle.mtp_generate(om, oracle.KV(kv), dh, 0, tok, cfg.ctx, n, k, drafter=hopeless)
+    assert got["tokens"] == truth[:n]
+    assert got["accepted"] == [0] * (n - 1)

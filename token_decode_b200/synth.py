@@ -58,6 +58,7 @@ class Config:
     theta: float = 1.0e6
     eps: float = 1.0e-6
     verify_k: int = 0   # draft tokens checked by one speculative-verify pass
+    draft_vocab: int = 32768   # output ids of the speculative draft head (the first ids)
 
     @property
     def nqkv(self) -> int:
@@ -77,7 +78,7 @@ class Config:
 
 CONFIGS = {
     "tiny": Config("tiny-1L-h256-q4_0", L=1, H=256, nq=4, nkv=2, hd=64, F=704, V=1024,
-                   fmt=FMT_Q4_0, ctx=128, steps=8),
+                   fmt=FMT_Q4_0, ctx=128, steps=8, draft_vocab=256),
     "7b": Config("7b-dense-q4_0", L=28, H=3584, nq=28, nkv=4, hd=128, F=18944, V=152064,
                  fmt=FMT_Q4_0, ctx=2000, steps=512),
     "9b": Config("9b-dense-nvfp4", L=36, H=4096, nq=32, nkv=8, hd=128, F=12288, V=151936,
@@ -285,6 +286,21 @@ def make_model(cfg: Config, device="cpu", seed: int = 0, n_layers: Optional[int]
         final_norm=1.0 + randn((cfg.H,), 0.02, device, seed, "final_norm"),
         layers=layers,
     )
+
+
+@dataclasses.dataclass
+class DraftHead:
+    """Weights of a speculative draft head: RMSNorm gains [H] and an output
+    matrix over the first draft_vocab token ids, in the model's format (the
+    draft head shares the model's embedding)."""
+    norm: torch.Tensor
+    w: QMat
+
+
+def make_draft_head(cfg: Config, device="cpu", seed: int = 0) -> DraftHead:
+    vd = min(cfg.draft_vocab, cfg.V)
+    return DraftHead(norm=1.0 + randn((cfg.H,), 0.02, device, seed, "draft.norm"),
+                     w=_qmat((vd, cfg.H), cfg, device, seed, "draft.w"))
 
 
 # -------------------------------------------------------------- KV context
