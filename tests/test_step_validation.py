@@ -70,10 +70,16 @@ class _Step:
                                   self.ptr() if ws is None else ws, need if ws_bytes is None else ws_bytes, None)
 
 
-@pytest.mark.parametrize("name,n_rows", [("tiny", 1), ("tiny", 4), ("7b", 1), ("9b", 1), ("9b_b32", 1),
-                                         ("9b", 8), ("27b", 4), ("moe", 1)])
-def test_workload_descriptors_pass(bw, name, n_rows):
-    cfg = synth.CONFIGS[name]
+_NV = synth.FMT_NVFP4
+
+
+@pytest.mark.parametrize("name,over,n_rows", [
+    ("tiny", {}, 1), ("tiny", dict(B=2), 4), ("tiny", dict(fmt=_NV, B=1), 8), ("tiny", dict(fmt=_NV, B=8), 1),
+    ("tiny", dict(B=5), 1), ("tiny", dict(fmt=_NV, F=0, n_experts=16, topk=4, F_exp=64, B=4), 1),
+    ("7b", {}, 1), ("9b", {}, 1), ("9b_b32", {}, 1), ("9b", {}, 8), ("27b", {}, 4), ("moe", {}, 1)])
+def test_workload_descriptors_pass(bw, name, over, n_rows):
+    """Every shape the GPU tests and the benchmark run passes the step's checks."""
+    cfg = synth.CONFIGS[name].with_(**over)
     if n_rows > 1:
         cfg = cfg.with_(verify_k=n_rows - 1)
     assert _Step(bw, cfg).validate(n_rows=n_rows) == OK
