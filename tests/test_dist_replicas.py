@@ -95,3 +95,30 @@ def test_reference_arm_prints_the_contract_line():
     spec.loader.exec_module(bench)
     from token_decode_b200 import synth
     assert d["config"] == bench.workload_config(synth.CONFIGS["tiny"], 1)
+
+
+def test_clock_summary_keeps_the_timed_region():
+    """Clock samples are summarised over the ones inside the timed region (by
+    their nvidia-smi timestamps), or over all of them when none falls inside."""
+    import datetime
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    c = bench.ClockSampler(0)
+    c.t0 = datetime.datetime(2026, 1, 2, 3, 4, 5, 100000)
+    c.t1 = datetime.datetime(2026, 1, 2, 3, 4, 5, 400000)
+    idle = "2026/01/02 03:04:05.050, 1100, 1965, 120.0, Not Active, Not Active, Not Active, Not Active"
+    busy1 = "2026/01/02 03:04:05.150, 1965, 1965, 700.5, Not Active, Not Active, Not Active, Active"
+    busy2 = "2026/01/02 03:04:05.350, 1950, 1965, 720.0, Not Active, Not Active, Not Active, Not Active"
+    after = "2026/01/02 03:04:05.450, 1000, 1965, 90.0, Active, Not Active, Not Active, Not Active"
+    c.out = "\n".join([idle, busy1, busy2, after])
+    s = c.summary()
+    assert s["sm_mhz"] == 1957.5 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["samples_in_timed_region"] == 2
+    c.t0 = c.t1 = datetime.datetime(2025, 1, 1)        # no sample inside: all of them
+    s = c.summary()
+    assert s["samples"] == 4 and s["samples_in_timed_region"] == 0
+    assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    c.out = "not a sample\n"
+    assert c.summary()["reasons"] == ["unavailable"]
