@@ -168,6 +168,8 @@ float or_silu(float z)
 static const uint16_t *kv_row(const uint16_t *pool, const or_kv *kv, int b, int nkv,
                               int kvh, int hd, int pos)
 {
+    if (pos < 0 || pos / kv->page_tokens >= kv->max_pages)
+        return NULL;        /* outside the page table: no row */
     int32_t page = kv->page_table[(size_t)b * (size_t)kv->max_pages + (size_t)(pos / kv->page_tokens)];
     if (page < 0 || page >= kv->n_pages)
         return NULL;
