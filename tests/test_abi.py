@@ -104,3 +104,15 @@ def test_workspace_queries_are_host_only(lib):
     z = lib.bw_gemv_workspace_bytes(4608, 3584, 1, 0)
     assert z >= 1 << 18
     assert lib.bw_attn_workspace_bytes(1, 1, 28, 4, 128, 160) >= 1 << 18
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """The binding hands the library device addresses only: a host tensor (or
+    a strided view) raises before any call instead of reaching a kernel."""
+    import torch
+    from token_decode_b200 import bw
+    assert bw._ptr(None) is None and bw._ptr(4096) == 4096
+    with pytest.raises(ValueError, match="device memory"):
+        bw._ptr(torch.zeros(4))
+    with pytest.raises(ValueError):
+        bw.gemv_q4_0(torch.zeros(16, dtype=torch.uint8), 4096, 8, 32, 4096, 1, 4096, torch.zeros(1))

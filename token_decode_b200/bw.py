@@ -118,10 +118,17 @@ def _check(status: int, what: str) -> None:
 
 
 def _ptr(t) -> int | None:
+    """Device address of a tensor argument (None stays NULL, an int is taken
+    as an address).  The library reads every pointer as dense device memory,
+    so a host or strided tensor is refused here instead of reaching a kernel."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError(f"libbw takes device memory; got a tensor on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError("libbw takes dense (contiguous) tensors")
     return t.data_ptr()
 
 

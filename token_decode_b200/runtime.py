@@ -27,7 +27,7 @@ def _gpu_layout(m, up=None):
     else:
         bw.repack_nvfp4(m.q, m.s, m.N, m.K, q, s, q_up=None if up is None else up.q,
                         s_up=None if up is None else up.s)
-    qw = bw.QWeight(m.fmt, rows, m.K, q.data_ptr(), s.data_ptr(), m.ts,
+    qw = bw.QWeight(m.fmt, rows, m.K, bw._ptr(q), bw._ptr(s), m.ts,
                     up.ts if up is not None else m.ts)
     return qw, [q, s]
 
@@ -49,8 +49,8 @@ class DeviceModel:
         self.layers = (bw.Layer * L)()
         for l, ly in enumerate(model.layers):
             c = self.layers[l]
-            c.attn_norm = ly.attn_norm.data_ptr()
-            c.ffn_norm = ly.ffn_norm.data_ptr()
+            c.attn_norm = bw._ptr(ly.attn_norm)
+            c.ffn_norm = bw._ptr(ly.ffn_norm)
             keep += [ly.attn_norm, ly.ffn_norm]
             c.wqkv = qw(ly.wqkv)
             c.wo = qw(ly.wo)
@@ -65,7 +65,7 @@ class DeviceModel:
         keep += [model.final_norm]
         self.c = bw.Model(L, cfg.H, cfg.nq, cfg.nkv, cfg.hd, cfg.F, cfg.V, cfg.n_experts, cfg.topk,
                           cfg.F_exp, cfg.eps, qw(model.embed), qw(model.lm_head),
-                          model.final_norm.data_ptr(), self.cos.data_ptr(), self.sin.data_ptr(),
+                          bw._ptr(model.final_norm), bw._ptr(self.cos), bw._ptr(self.sin),
                           max_pos, C.cast(self.layers, C.c_void_p).value)
         self._keep = keep
         self.weight_bytes = sum(t.numel() * t.element_size() for t in keep)
@@ -88,9 +88,9 @@ class DeviceModel:
                 bw.repack_nvfp4(d.q, d.s, H, Fe, dq[e], ds[e])
         gts = torch.stack([ly.eg.ts, ly.eu.ts], dim=1).contiguous().to("cuda")
         dts = ly.ed.ts.contiguous().to("cuda")
-        c.router = ly.router.data_ptr()
-        c.egu_q, c.egu_s, c.ed_q, c.ed_s = gq.data_ptr(), gs.data_ptr(), dq.data_ptr(), ds.data_ptr()
-        c.egu_ts, c.ed_ts = gts.data_ptr(), dts.data_ptr()
+        c.router = bw._ptr(ly.router)
+        c.egu_q, c.egu_s, c.ed_q, c.ed_s = bw._ptr(gq), bw._ptr(gs), bw._ptr(dq), bw._ptr(ds)
+        c.egu_ts, c.ed_ts = bw._ptr(gts), bw._ptr(dts)
         keep += [ly.router, gq, gs, dq, ds, gts, dts]
         w, t = _gpu_layout(ly.sg, ly.su)
         c.sgu = w
@@ -108,10 +108,10 @@ class DeviceKV:
         self.v = kv.v
         self.page_table = kv.page_table.to(torch.int32).contiguous()
         L = len(kv.k)
-        self._kp = (C.c_void_p * L)(*[t.data_ptr() for t in kv.k])
-        self._vp = (C.c_void_p * L)(*[t.data_ptr() for t in kv.v])
+        self._kp = (C.c_void_p * L)(*[bw._ptr(t) for t in kv.k])
+        self._vp = (C.c_void_p * L)(*[bw._ptr(t) for t in kv.v])
         self.c = bw.KV(C.cast(self._kp, C.c_void_p).value, C.cast(self._vp, C.c_void_p).value,
-                       int(kv.n_pages), int(self.page_table.shape[1]), self.page_table.data_ptr())
+                       int(kv.n_pages), int(self.page_table.shape[1]), bw._ptr(self.page_table))
 
 
 class Decoder:
