@@ -222,7 +222,9 @@ bw_status bw_argmax(const float *logits, int M, int V, int32_t *idx_out, float *
  *   out: fp32 [B*n_rows][nq hd]; row r of sequence b attends over positions
  *        0 .. pos[b] + r (causal within the rows); query head h reads kv head
  *        h / (nq / nkv); scale 1/sqrt(hd); fp32 softmax.
- * Requires hd == 128 or 64, nq % nkv == 0, (nq/nkv) * n_rows <= 32.
+ * Requires hd == 128 or 64, nq % nkv == 0, (nq/nkv) * n_rows <= 32,
+ * n_rows <= 8, max_pages <= 8192 (else BW_ERR_UNSUPPORTED_SHAPE); qkv, out,
+ * k_pool and v_pool 16-byte aligned (else BW_ERR_INVALID_ARG).
  * A page-table entry outside [0, n_pages) sets BW_DEVERR_BAD_PAGE; the page
  * is neither read nor written. */
 bw_status bw_paged_attn_decode(const float *qkv, const float *rope_cos, const float *rope_sin,
@@ -291,7 +293,9 @@ typedef struct bw_kv {
  *   x: fp32 [R][H]; topk_idx: int32 [R][topk] and topk_w: fp32 [R][topk]
  *   (optional outputs, in selection order).
  * Expert weights: m->layers-style bw_layer fields egu_* / ed_* (E matrices
- * back to back in the GPU layout) and sgu / sd (shared expert).
+ * back to back in the GPU layout) and sgu / sd (shared expert), all 16-byte
+ * aligned and in one format.  Limits: E <= 1024, topk <= 16, R <= 256,
+ * H % 32 == 0, F_exp % 32 == 0 (else BW_ERR_UNSUPPORTED_SHAPE).
  * ws must hold bw_moe_workspace_bytes(m, R). */
 bw_status bw_moe_route_gemv(const struct bw_model *m, const struct bw_layer *ly, float *x, int R,
                             int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes, void *stream);
