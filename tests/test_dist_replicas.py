@@ -122,3 +122,25 @@ def test_clock_summary_keeps_the_timed_region():
     assert s["reasons"] == ["hw_slowdown", "sw_power_cap"]
     c.out = "not a sample\n"
     assert c.summary()["reasons"] == ["unavailable"]
+
+
+def test_launch_count_claim_matches_the_committed_launch_lists():
+    """bench.py's gpu_launches per step agrees with the ncu launch lists under
+    profiles/: 142 launches for one 7B Q4_0 step at B = 1, and six launches per
+    MoE block."""
+    import importlib.util
+    import re
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    from token_decode_b200 import synth
+    text = open(os.path.join(ROOT, "profiles", "launches_decode_step_7b_q4_0.md")).read()
+    n_listed = int(re.search(r"^(\d+) launches", text, flags=re.M).group(1))
+    assert bench.step_launches(synth.CONFIGS["7b"]) == n_listed == 142
+    moe = synth.CONFIGS["moe"]
+    # a MoE layer replaces the dense FFN's two projections (each an activation
+    # pack + a tensor-core GEMM at 32 rows) with the six launches of the block
+    dense = moe.with_(n_experts=0, F=512)
+    assert bench.step_launches(moe) - bench.step_launches(dense) == moe.L * (6 - 2 * 2)
+    text = open(os.path.join(ROOT, "profiles", "launches_moe_layer_b32.md")).read()
+    assert re.search(r"^12 launches", text, flags=re.M)
