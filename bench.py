@@ -135,13 +135,16 @@ def workload_config(cfg, world_size):
             "parallelism": f"replicas x{world_size}"}
 
 
-def step_bytes(cfg, model, avg_ctx):
+def step_bytes(cfg, model, avg_ctx, moe_layer_bytes=0):
     """Algorithmic bytes of one decode step: every weight matrix streamed once
     (4.5-bit blocks + fp32 norm gains), the KV read over the context, the new
-    K/V written (the embedding row is not counted)."""
+    K/V written (the embedding row is not counted).  A MoE layer adds
+    moe_layer_bytes: its fp32 router, its shared expert and the experts the
+    router selected (counted from the library's own routing of the batch)."""
     kv_read = 2 * cfg.L * cfg.nkv * cfg.hd * 2 * avg_ctx * cfg.B
     kv_write = 2 * cfg.L * cfg.nkv * cfg.hd * 2 * cfg.B
-    return model.weight_bytes_dense() + kv_read + kv_write
+    moe = cfg.L * moe_layer_bytes if cfg.n_experts else 0
+    return model.weight_bytes_dense() + kv_read + kv_write + moe
 
 
 # ncu summaries of the dominant kernel: DRAM traffic per launch, valid while the
@@ -340,7 +343,7 @@ def run_ours(args):
     traffic = _ncu_traffic(dom, args.config)
 
     avg_ctx = cfg.ctx + (cfg.steps + 1) / 2
-    sb = step_bytes(cfg, model, avg_ctx)
+    sb = step_bytes(cfg, model, avg_ctx, kern["moe"]["bytes_per_launch"] if cfg.n_experts else 0)
     step_gbs = sb / (ms_step / 1000.0) / 1e9
     launches_per_step = step_launches(cfg)
 

@@ -144,3 +144,24 @@ def test_launch_count_claim_matches_the_committed_launch_lists():
     assert bench.step_launches(moe) - bench.step_launches(dense) == moe.L * (6 - 2 * 2)
     text = open(os.path.join(ROOT, "profiles", "launches_moe_layer_b32.md")).read()
     assert re.search(r"^12 launches", text, flags=re.M)
+
+
+def test_step_bytes_counts_weights_kv_and_routed_experts():
+    """The roofline's algorithmic bytes per step: every dense weight matrix and
+    norm once, K + V over the context and the new rows, and per MoE layer the
+    bytes its launch touches (router, shared expert, selected experts)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    from token_decode_b200 import synth
+    cfg = synth.CONFIGS["tiny"]
+    model = synth.make_model(cfg, "cpu", seed=0)
+    H, F, V, L = cfg.H, cfg.F, cfg.V, cfg.L
+    w = (cfg.nqkv * H + H * cfg.nq * cfg.hd + 3 * F * H + V * H) * 9 // 16 + (2 * L + 1) * H * 4
+    kv = 2 * L * cfg.nkv * cfg.hd * 2 * cfg.B
+    assert bench.step_bytes(cfg, model, 100.0) == w + kv * 100 + kv
+    moe = cfg.with_(fmt=synth.FMT_NVFP4, F=0, n_experts=8, topk=2, F_exp=64, B=2)
+    mm = synth.make_model(moe, "cpu", seed=0)
+    dense = bench.step_bytes(moe, mm, 10.0)
+    assert bench.step_bytes(moe, mm, 10.0, moe_layer_bytes=12345) == dense + moe.L * 12345
