@@ -131,3 +131,18 @@ def test_planted_defects_are_rejected_before_any_launch(bw):
     s.layers[0].sgu.fmt = synth.FMT_Q4_0
     s.layers[0].sd.fmt = synth.FMT_Q4_0
     assert s.validate() == INVALID
+
+
+def test_empty_inputs_are_rejected(bw):
+    """Zero sequences, zero rows per sequence or zero layers of work are argument
+    errors, reported before anything is queued."""
+    s = _Step(bw, synth.CONFIGS["tiny"])
+    assert s.validate(B=0) == INVALID
+    assert s.validate(n_rows=0) == INVALID
+    lib, p = bw.lib(), C.c_void_p
+    fake = p(1 << 32)
+    assert lib.bw_gemv_q4_0(fake, fake, 64, 64, fake, 0, None, 1e-6, None, fake, None, 0, fake, 1 << 20,
+                            None) == INVALID
+    assert lib.bw_gemv_nvfp4(fake, fake, 1.0, 1.0, 0, 64, fake, 1, None, 1e-6, None, fake, None, 0, fake,
+                             1 << 20, None) == INVALID
+    assert lib.bw_spec_accept(fake, fake, 0, 1, fake, None, 1, None, None) == INVALID
