@@ -150,7 +150,10 @@ bw_status bw_repack_nvfp4(const void *q, const void *s, const void *q_up, const 
  *   x: fp32 [M][K]; y: fp32 [M][N] ([M][N/2] with SILU_GATE; may be NULL
  *   with ARGMAX); residual: fp32 [M][N] or NULL; argmax_out: int32 [M] or NULL;
  *   gamma: fp32 [K] or NULL.
- * Shapes: N % 8 == 0, K % 32 == 0, 1 <= M <= 8.  Pointers 16-byte aligned.
+ * Shapes: N % 8 == 0, K % 32 == 0, M >= 1 (Q4_0 runs in passes of up to 4
+ * rows on the CUDA cores; NVFP4 with M > 4 runs on the tensor cores in passes
+ * of up to 32 rows, with fp16-rounded activations).  Pointers 16-byte
+ * aligned; fmt-specific shape limits return BW_ERR_UNSUPPORTED_SHAPE.
  * ws must hold bw_gemv_workspace_bytes(N, K, M, flags). */
 bw_status bw_gemv_q4_0(const void *w_q, const void *w_d, int N, int K,
                        const float *x, int M, const float *gamma, float eps,
