@@ -197,8 +197,10 @@ bw_status bw_gemv_q4_0_noalloc(const void *w_q, const void *w_d, int N, int K,
 bw_status bw_rmsnorm_fused(float *x, const float *add, const float *gamma, int M, int H,
                            float eps, void *y, int y_fp16, void *stream);
 
-/* x[m][:] = dequantized row tokens[m] of the embedding matrix (tiled GPU layout).
- * A token outside [0, V) sets BW_DEVERR_BAD_TOKEN and writes zeros. */
+/* x[m][:] = dequantized row tokens[m] of the embedding matrix (tiled GPU layout,
+ * e_q / e_s 16-byte aligned).  A token outside [0, V) sets BW_DEVERR_BAD_TOKEN
+ * in ws's error word (ws optional; when given, a workspace as above) and
+ * writes zeros. */
 bw_status bw_embed(int fmt, const void *e_q, const void *e_s, float ts, int V, int H,
                    const int32_t *tokens, int M, float *x, void *ws, void *stream);
 

@@ -146,3 +146,14 @@ def test_empty_inputs_are_rejected(bw):
     assert lib.bw_gemv_nvfp4(fake, fake, 1.0, 1.0, 0, 64, fake, 1, None, 1e-6, None, fake, None, 0, fake,
                              1 << 20, None) == INVALID
     assert lib.bw_spec_accept(fake, fake, 0, 1, fake, None, 1, None, None) == INVALID
+
+
+def test_embedding_pointers_are_checked(bw):
+    lib, p = bw.lib(), C.c_void_p
+    fake = p(1 << 32)
+    # scales off the tiled layout's alignment; a workspace off its 256-byte alignment
+    assert lib.bw_embed(0, fake, p((1 << 32) + 2), 1.0, 64, 64, fake, 1, fake, None, None) == INVALID
+    assert lib.bw_embed(0, fake, fake, 1.0, 64, 64, fake, 1, fake, p((1 << 32) + 4), None) == INVALID
+    s = _Step(bw, synth.CONFIGS["tiny"])
+    s.m.embed.s += 2
+    assert s.validate() == INVALID

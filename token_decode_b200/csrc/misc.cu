@@ -205,6 +205,7 @@ bw_status embed_check(int fmt, const void *e_q, const void *e_s, int V, int H, c
     if (!e_q || !e_s || !tokens || !x || V <= 0 || H <= 0 || M <= 0) return BW_ERR_INVALID_ARG;
     if (H % 32) return BW_ERR_UNSUPPORTED_SHAPE;
     if (fmt != BW_FMT_Q4_0 && fmt != BW_FMT_NVFP4) return BW_ERR_INVALID_ARG;
+    if (!aligned16(e_q) || !aligned16(e_s)) return BW_ERR_INVALID_ARG;   // the tiled layout's alignment
     return BW_OK;
 }
 
@@ -281,6 +282,7 @@ bw_status bw_repack_nvfp4(const void *q, const void *s, const void *q_up, const 
 
 bw_status bw_embed(int fmt, const void *e_q, const void *e_s, float ts, int V, int H, const int32_t *tokens,
                    int M, float *x, void *ws, void *stream) {
+    if (ws && !bw::ws_ok(ws)) return BW_ERR_INVALID_ARG;
     return bw::embed_launch(fmt, e_q, e_s, ts, V, H, tokens, M, x, ws ? bw::ws_error_word(ws) : nullptr,
                             static_cast<cudaStream_t>(stream));
 }
