@@ -320,6 +320,12 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
                          int B, int n_rows, int32_t *tokens_out, float *logits, unsigned flags,
                          void *ws, size_t ws_bytes, void *stream);
 size_t bw_decode_workspace_bytes(const bw_model *m, const bw_kv *kv, int B, int n_rows);
+/* Device address, inside ws, of the step's residual stream: fp32
+ * [B*n_rows][H].  After bw_decode_step it holds each row's hidden state after
+ * the last layer (the LM head's input before its RMSNorm) until the next call
+ * on ws -- what a speculative draft head starts from.  Host arithmetic only;
+ * NULL for arguments bw_decode_workspace_bytes would not size. */
+const float *bw_decode_hidden(const bw_model *m, const bw_kv *kv, int B, int n_rows, const void *ws);
 
 /* Acceptance after a speculative verify pass.  "bw24" deep-dive page
  * (10100.com), section 5, stage 4 (the verify kernel unrolls the drafts as

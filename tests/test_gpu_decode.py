@@ -129,6 +129,23 @@ def test_tiny_moe_decode_and_router_topk():
     assert torch.isfinite(x).all() and not torch.equal(x, x0)
 
 
+def test_step_hidden_state_matches_oracle():
+    """The residual stream bw_decode_hidden exposes after a step is each row's
+    hidden state after the last layer, as the oracle computes it."""
+    cfg = synth.CONFIGS["tiny"].with_(B=2, L=2)
+    model, kv, om, okv, dm, dkv = _setup(cfg, seed=9)
+    dec = runtime.Decoder(dm, dkv, cfg.B)
+    toks = synth.start_tokens(cfg, 9)[: cfg.B]
+    dec.tokens_in.copy_(toks)
+    dec.pos.fill_(cfg.ctx)
+    dec.step()
+    assert bw.read_error(dec.ws) == 0
+    hid = bw.decode_hidden(dm.c, dkv.c, cfg.B, 1, dec.ws).cpu().numpy()
+    for b in range(cfg.B):
+        res = oracle.decode_token(om, okv, b, int(toks[b]), cfg.ctx, want_logits=False, want_hidden=True)
+        assert rel_err(hid[b], res["hidden"][cfg.L]) < TOL
+
+
 def test_graph_replay_with_device_advance_matches_eager():
     cfg = synth.CONFIGS["tiny"].with_(B=2)
     model, kv, om, okv, dm, dkv = _setup(cfg, seed=5)

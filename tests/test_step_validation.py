@@ -157,3 +157,19 @@ def test_embedding_pointers_are_checked(bw):
     s = _Step(bw, synth.CONFIGS["tiny"])
     s.m.embed.s += 2
     assert s.validate() == INVALID
+
+
+def test_decode_hidden_points_at_the_step_residual_stream(bw):
+    """bw_decode_hidden is host arithmetic: the residual stream is the first
+    region after the workspace header, sized B*n_rows x H floats, and the same
+    address for every call with the same shapes."""
+    s = _Step(bw, synth.CONFIGS["9b_b32"])
+    lib = bw.lib()
+    ws = 1 << 40
+    a = lib.bw_decode_hidden(C.byref(s.m), C.byref(s.kv), 32, 1, ws)
+    assert a == ws + (1 << 18)
+    assert lib.bw_decode_hidden(C.byref(s.m), C.byref(s.kv), 32, 1, ws) == a
+    assert lib.bw_decode_hidden(C.byref(s.m), C.byref(s.kv), 0, 1, ws) is None
+    assert lib.bw_decode_hidden(None, C.byref(s.kv), 32, 1, ws) is None
+    need = lib.bw_decode_workspace_bytes(C.byref(s.m), C.byref(s.kv), 32, 1)
+    assert (a - ws) + 32 * s.cfg.H * 4 <= need

@@ -29,7 +29,7 @@ EXPORTS = (
     "bw_repack_bytes", "bw_repack_q4_0", "bw_repack_nvfp4", "bw_gemv_q4_0", "bw_gemv_nvfp4",
     "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
     "bw_paged_attn_decode", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
-    "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes", "bw_spec_accept",
+    "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes", "bw_decode_hidden", "bw_spec_accept",
 )
 
 
@@ -98,6 +98,7 @@ def lib() -> C.CDLL:
             "bw_moe_workspace_bytes": (z, [p, i]),
             "bw_decode_step": (i, [p, p, p, p, i, i, p, p, u, p, z, p]),
             "bw_decode_workspace_bytes": (z, [p, p, i, i]),
+            "bw_decode_hidden": (p, [p, p, i, i, p]),
             "bw_spec_accept": (i, [p, p, i, i, p, p, i, p, p]),
         }
         for name, (res, args) in sig.items():
@@ -244,6 +245,17 @@ def moe_route_gemv(model: Model, layer: Layer, x, R, ws, topk_idx=None, topk_w=N
 
 def decode_workspace_bytes(model: Model, kv: KV, B: int, n_rows: int) -> int:
     return lib().bw_decode_workspace_bytes(C.byref(model), C.byref(kv), B, n_rows)
+
+
+def decode_hidden(model: Model, kv: KV, B, n_rows, ws) -> torch.Tensor:
+    """The step's residual stream inside ws as an fp32 [B*n_rows][H] view: each
+    row's hidden state after the last layer, valid until the next step on ws."""
+    addr = lib().bw_decode_hidden(C.byref(model), C.byref(kv), B, n_rows, _ptr(ws))
+    if not addr:
+        raise BWError(ERR_INVALID_ARG, "bw_decode_hidden")
+    off = addr - ws.data_ptr()
+    n = B * n_rows * model.H
+    return ws[off: off + 4 * n].view(torch.float32).view(B * n_rows, model.H)
 
 
 def decode_step(model: Model, kv: KV, tokens_in, pos, B, n_rows, tokens_out, ws, logits=None,

@@ -112,6 +112,13 @@ static bw_status step_check(const bw_model *m, const bw_kv *kv, const int32_t *t
 
 extern "C" {
 
+const float *bw_decode_hidden(const bw_model *m, const bw_kv *kv, int B, int n_rows, const void *ws) {
+    if (!m || !kv || !ws || B <= 0 || n_rows <= 0) return nullptr;
+    bw::StepBuffers bf;
+    bw::step_bytes(m, kv, B, n_rows, &bf, const_cast<void *>(ws));
+    return bf.x;
+}
+
 size_t bw_decode_workspace_bytes(const bw_model *m, const bw_kv *kv, int B, int n_rows) {
     if (!m || !kv || B <= 0 || n_rows <= 0) return BW_WS_HDR_BYTES;
     return bw::step_bytes(m, kv, B, n_rows, nullptr, nullptr);
