@@ -74,6 +74,8 @@ def lib():
             "or_f32_to_fp16": (C.c_uint16, [f]),
             "or_e4m3_to_f32": (f, [C.c_uint8]),
             "or_e2m1_to_f32": (f, [C.c_uint8]),
+            "or_f32_to_e4m3": (C.c_uint8, [f]),
+            "or_attend_head_e4m3": (None, [p, p, p, f, f, p, i, i, i, i, i, p]),
             "or_dequant_row": (None, [p, i, p]),
             "or_matvec": (None, [p, p, p]),
             "or_rmsnorm": (None, [p, p, i, f, p]),
@@ -138,6 +140,10 @@ def e2m1_to_f32(c: int) -> float:
     return lib().or_e2m1_to_f32(c)
 
 
+def f32_to_e4m3(x: float) -> int:
+    return int(lib().or_f32_to_e4m3(x))
+
+
 def dequant(m, rows=None) -> np.ndarray:
     """Dequantized rows of m (all rows by default) as float32 [len(rows), K]."""
     qm = m if isinstance(m, QMat) else QMat(m)
@@ -195,6 +201,19 @@ def attend_head(q, kv: KV, layer: int, b: int, nkv: int, kvh: int, length: int) 
     out = np.empty_like(q)
     lib().or_attend_head(_ptr(q), _ptr(kv.k[layer]), _ptr(kv.v[layer]), C.byref(kv.c), b, nkv,
                          kvh, q.size, length, _ptr(out))
+    return out
+
+
+def attend_head_e4m3(q, kpool, vpool, k_scale: float, v_scale: float, kv: KV, b: int, nkv: int, kvh: int,
+                     length: int) -> np.ndarray:
+    """One query head over an E4M3 cache (byte pools [n_pages][nkv][16][hd] laid
+    out like the fp16 ones, behind kv's page table)."""
+    q = _np(q).astype(np.float32)
+    kp = _np(kpool, np.uint8)
+    vp = _np(vpool, np.uint8)
+    out = np.empty_like(q)
+    lib().or_attend_head_e4m3(_ptr(q), _ptr(kp), _ptr(vp), float(k_scale), float(v_scale), C.byref(kv.c), b, nkv,
+                              kvh, q.size, length, _ptr(out))
     return out
 
 

@@ -77,6 +77,32 @@ float or_e4m3_to_f32(uint8_t c)
     return s ? -v : v;
 }
 
+/* binary32 -> E4M3 "fn": the representable magnitudes are k * 2^-9 for
+ * k < 8 (subnormals) and (8 + m) * 2^(e-10) for e = 1..15, m = 0..7 (except
+ * e = 15, m = 7, which is NaN); 448 is the largest.  Round to nearest, ties to
+ * the even code; a magnitude that rounds past 448 saturates to 448. */
+uint8_t or_f32_to_e4m3(float f)
+{
+    if (f != f)
+        return 0x7Fu;
+    uint8_t sign = signbit(f) ? 0x80u : 0u;
+    double a = fabs((double)f);
+    if (a >= 464.0)                          /* halfway to the next step (480): saturate */
+        return (uint8_t)(sign | 0x7Eu);
+    /* scan the 127 non-negative finite codes in order for the nearest value */
+    uint8_t best = 0;
+    double bestd = a;                        /* code 0 stands for 0 */
+    for (int c = 1; c <= 0x7E; c++) {
+        double v = (double)or_e4m3_to_f32((uint8_t)c);
+        double d = fabs(v - a);
+        if (d < bestd || (d == bestd && (c & 1) == 0)) {
+            best = (uint8_t)c;
+            bestd = d;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
 /* OCP 4-bit E2M1: s | 2-bit exponent (bias 1) | 1-bit mantissa;
  * magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
 float or_e2m1_to_f32(uint8_t c)
@@ -211,6 +237,58 @@ void or_attend_head(const float *q, const uint16_t *kpool, const uint16_t *vpool
         for (int j = 0; j < len; j++) {
             const uint16_t *vr = kv_row(vpool, kv, b, nkv, kvh, hd, j);
             acc += s[j] * or_fp16_to_f32(vr[d]);
+        }
+        out[d] = acc / l;
+    }
+    free(s);
+}
+
+/* Element offset of the row of (b, kvh, pos) in a layer pool, or -1 when its
+ * page-table entry is outside the pool or pos is outside the table. */
+static long kv_row_off(const or_kv *kv, int b, int nkv, int kvh, int hd, int pos)
+{
+    if (pos < 0 || pos / kv->page_tokens >= kv->max_pages)
+        return -1;
+    int32_t page = kv->page_table[(size_t)b * (size_t)kv->max_pages + (size_t)(pos / kv->page_tokens)];
+    if (page < 0 || page >= kv->n_pages)
+        return -1;
+    return (long)((((size_t)page * (size_t)nkv + (size_t)kvh) * (size_t)kv->page_tokens +
+                   (size_t)(pos % kv->page_tokens)) * (size_t)hd);
+}
+
+void or_attend_head_e4m3(const float *q, const uint8_t *kpool, const uint8_t *vpool, float k_scale,
+                         float v_scale, const or_kv *kv, int b, int nkv, int kvh, int hd, int len,
+                         float *out)
+{
+    float scale = 1.0f / sqrtf((float)hd);
+    float *s = (float *)malloc(sizeof(float) * (size_t)len);
+    for (int j = 0; j < len; j++) {
+        long off = kv_row_off(kv, b, nkv, kvh, hd, j);
+        if (off < 0) {
+            for (int d = 0; d < hd; d++)
+                out[d] = NAN;
+            free(s);
+            return;
+        }
+        float dot = 0.0f;
+        for (int d = 0; d < hd; d++)
+            dot += q[d] * (or_e4m3_to_f32(kpool[off + d]) * k_scale);
+        s[j] = dot * scale;
+    }
+    float m = s[0];
+    for (int j = 1; j < len; j++)
+        if (s[j] > m)
+            m = s[j];
+    float l = 0.0f;
+    for (int j = 0; j < len; j++) {
+        s[j] = expf(s[j] - m);
+        l += s[j];
+    }
+    for (int d = 0; d < hd; d++) {
+        float acc = 0.0f;
+        for (int j = 0; j < len; j++) {
+            long off = kv_row_off(kv, b, nkv, kvh, hd, j);
+            acc += s[j] * (or_e4m3_to_f32(vpool[off + d]) * v_scale);
         }
         out[d] = acc / l;
     }

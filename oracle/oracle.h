@@ -101,6 +101,9 @@ float or_fp16_to_f32(uint16_t h);
 uint16_t or_f32_to_fp16(float f);          /* round to nearest even */
 float or_e4m3_to_f32(uint8_t c);
 float or_e2m1_to_f32(uint8_t c);
+/* binary32 -> E4M3 "fn", round to nearest, ties to even; magnitudes that
+ * round above 448 saturate to 448 (a KV cache never stores NaN); NaN -> 0x7F. */
+uint8_t or_f32_to_e4m3(float f);
 
 /* dequantize row n of W into out[K] */
 void or_dequant_row(const or_qmat *w, int n, float *out);
@@ -115,6 +118,14 @@ float or_silu(float z);
  * kv head kvh of layer pool (kpool, vpool); out[hd] */
 void or_attend_head(const float *q, const uint16_t *kpool, const uint16_t *vpool,
                     const or_kv *kv, int b, int nkv, int kvh, int hd, int len, float *out);
+/* The same head over an E4M3 cache (the FP8 KV variant; one fp32 scale per
+ * layer for K and one for V): a stored code c stands for e4m3(c) * scale,
+ * the scale applied to each decoded element; pools are bytes
+ * [n_pages][nkv][page_tokens][hd] behind kv's page table.  Otherwise
+ * identical to or_attend_head. */
+void or_attend_head_e4m3(const float *q, const uint8_t *kpool, const uint8_t *vpool, float k_scale,
+                         float v_scale, const or_kv *kv, int b, int nkv, int kvh, int hd, int len,
+                         float *out);
 /* top-k of r[E]: value descending, lower index first on ties; softmax weights
  * over the selected values */
 void or_topk_softmax(const float *r, int E, int k, int32_t *idx, float *w);

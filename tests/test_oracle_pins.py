@@ -605,3 +605,60 @@ def test_mtp_pass_counts_for_perfect_and_hopeless_drafts():
     got = oracle.mtp_generate(om, oracle.KV(kv), dh, 0, tok, cfg.ctx, n, k, drafter=hopeless)
     assert got["tokens"] == truth[:n]
     assert got["accepted"] == [0] * (n - 1)
+
+
+# ------------------------------------------------------- FP8 (E4M3) KV cache
+
+def test_e4m3_encoder_matches_torch_and_saturates():
+    """The E4M3 encoder against torch's float8_e4m3fn conversion (round to
+    nearest even) below the overflow midpoint 464; every code round-trips;
+    magnitudes from 464 up saturate to 448 where torch gives NaN; NaN stays NaN."""
+    codes = [c for c in range(256) if c & 0x7F != 0x7F]
+    for c in codes:
+        assert oracle.f32_to_e4m3(oracle.e4m3_to_f32(c)) == c, c
+    vals = np.array([oracle.e4m3_to_f32(c) for c in range(0x7F)], np.float64)   # ascending magnitudes
+    mids = (vals[:-1] + vals[1:]) / 2                                           # exact ties
+    rng = np.random.default_rng(8)
+    xs = np.concatenate([mids, -mids, rng.standard_normal(4000) * 30, rng.standard_normal(2000) * 0.01,
+                         rng.uniform(-463.9, 463.9, 2000), [0.0, 2.0 ** -10, 3 * 2.0 ** -11, 447.9, 463.99]])
+    xs = xs.astype(np.float32)
+    want = torch.from_numpy(xs).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.f32_to_e4m3(float(x)) for x in xs], np.uint8)
+    assert np.array_equal(got, want)
+    for x, c in ((464.0, 0x7E), (1e6, 0x7E), (float("inf"), 0x7E), (-500.0, 0xFE)):
+        assert oracle.f32_to_e4m3(x) == c
+    assert oracle.f32_to_e4m3(float("nan")) & 0x7F == 0x7F
+
+
+def test_attention_over_e4m3_cache_matches_fp64_brute_force():
+    """A query head over an FP8 cache with per-layer K and V scales, through a
+    permuted page table, against fp64 softmax attention over torch's decoding
+    of the same codes times the scales."""
+    rng = np.random.default_rng(9)
+    n_pages, nkv, P, hd, max_pages = 12, 2, 16, 64, 6
+    kq = rng.integers(0, 256, size=(n_pages, nkv, P, hd), dtype=np.uint8)
+    vq = rng.integers(0, 256, size=(n_pages, nkv, P, hd), dtype=np.uint8)
+    kq[(kq & 0x7F) == 0x7F] = 0x30        # no NaN codes in a cache
+    vq[(vq & 0x7F) == 0x7F] = 0x31
+    table = rng.permutation(n_pages)[: 2 * max_pages].reshape(2, max_pages).astype(np.int32)
+
+    class _KV:
+        pass
+    kv = _KV()
+    kv.k = [torch.zeros((n_pages, nkv, P, hd), dtype=torch.int16)]
+    kv.v = [torch.zeros((n_pages, nkv, P, hd), dtype=torch.int16)]
+    kv.page_table = torch.from_numpy(table)
+    kv.n_pages, kv.page_tokens = n_pages, P
+    okv = oracle.KV(kv)
+    dec = lambda a: torch.from_numpy(a.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    kf, vf = dec(kq), dec(vq)
+    ks, vs = 0.0625, 0.03
+    for b, kvh, length in ((0, 0, 1), (1, 1, 37), (1, 0, 90)):
+        q = rng.standard_normal(hd).astype(np.float32)
+        got = oracle.attend_head_e4m3(q, kq, vq, ks, vs, okv, b, nkv, kvh, length)
+        K = np.stack([kf[table[b, j // P], kvh, j % P] for j in range(length)]) * ks
+        V = np.stack([vf[table[b, j // P], kvh, j % P] for j in range(length)]) * vs
+        s = K @ q.astype(np.float64) / math.sqrt(hd)
+        p = np.exp(s - s.max())
+        want = (p / p.sum()) @ V
+        assert np.max(np.abs(got - want)) < 1e-5 * max(1.0, np.max(np.abs(want))), (b, kvh, length)
