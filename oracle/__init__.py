@@ -56,7 +56,8 @@ class ModelC(C.Structure):
 
 class KVC(C.Structure):
     _fields_ = [("k", C.c_void_p), ("v", C.c_void_p), ("n_pages", C.c_int),
-                ("page_tokens", C.c_int), ("page_table", C.c_void_p), ("max_pages", C.c_int)]
+                ("page_tokens", C.c_int), ("page_table", C.c_void_p), ("max_pages", C.c_int),
+                ("kv_fmt", C.c_int), ("k_scale", C.c_void_p), ("v_scale", C.c_void_p)]
 
 
 _lib = None
@@ -181,19 +182,27 @@ def silu(z: float) -> float:
 
 
 class KV:
-    """Host copy of the paged KV cache (fp16 bits per layer) + page table."""
+    """Host copy of the paged KV cache (fp16 bits per layer, or E4M3 bytes with
+    per-layer scales when the input carries k_scale / v_scale) + page table."""
 
     def __init__(self, kv, layers=None):
         L = len(kv.k) if layers is None else layers
-        self.k = [_np(kv.k[l], np.uint16).copy() for l in range(L)]
-        self.v = [_np(kv.v[l], np.uint16).copy() for l in range(L)]
+        self.fp8 = getattr(kv, "k_scale", None) is not None
+        elem = np.uint8 if self.fp8 else np.uint16
+        self.k = [_np(kv.k[l], elem).copy() for l in range(L)]
+        self.v = [_np(kv.v[l], elem).copy() for l in range(L)]
         self.page_table = _np(kv.page_table, np.int32).copy()
         self.n_pages = int(kv.n_pages)
         self.page_tokens = int(kv.page_tokens)
         self._kp = (C.c_void_p * L)(*[_ptr(a).value for a in self.k])
         self._vp = (C.c_void_p * L)(*[_ptr(a).value for a in self.v])
+        self.k_scale = _np(kv.k_scale).astype(np.float32)[:L].copy() if self.fp8 else None
+        self.v_scale = _np(kv.v_scale).astype(np.float32)[:L].copy() if self.fp8 else None
         self.c = KVC(C.cast(self._kp, C.c_void_p), C.cast(self._vp, C.c_void_p), self.n_pages,
-                     self.page_tokens, _ptr(self.page_table).value, self.page_table.shape[1])
+                     self.page_tokens, _ptr(self.page_table).value, self.page_table.shape[1],
+                     1 if self.fp8 else 0,
+                     _ptr(self.k_scale).value if self.fp8 else None,
+                     _ptr(self.v_scale).value if self.fp8 else None)
 
 
 def attend_head(q, kv: KV, layer: int, b: int, nkv: int, kvh: int, length: int) -> np.ndarray:
@@ -330,6 +339,9 @@ def decode_token(model: Model, kv: KV, b: int, token: int, pos: int, moe_dense: 
         kc = KVC.from_buffer_copy(kv.c)
         kc.k = kv.c.k + layers[0] * C.sizeof(C.c_void_p)
         kc.v = kv.c.v + layers[0] * C.sizeof(C.c_void_p)
+        if kv.fp8:
+            kc.k_scale = kv.c.k_scale + layers[0] * 4
+            kc.v_scale = kv.c.v_scale + layers[0] * 4
     L = mc.L
     logits = np.empty(cfg.V, np.float32) if want_logits else None
     hidden = np.empty((L + 1, cfg.H), np.float32) if want_hidden else None

@@ -415,6 +415,17 @@ int32_t or_decode_token(const or_model *m, or_kv *kv, int b, int32_t token, int 
         for (int h = 0; h < nkv; h++)
             or_rope(k + h * hd, hd, pos, m->theta);
         for (int h = 0; h < nkv; h++) {
+            if (kv->kv_fmt == 1) {
+                long off = kv_row_off(kv, b, nkv, h, hd, pos);
+                if (off < 0)
+                    continue;   /* bad page: the attention below reports NaN */
+                uint8_t *kr = (uint8_t *)kv->k[l] + off, *vr = (uint8_t *)kv->v[l] + off;
+                for (int d = 0; d < hd; d++) {
+                    kr[d] = or_f32_to_e4m3(k[h * hd + d] / kv->k_scale[l]);
+                    vr[d] = or_f32_to_e4m3(v[h * hd + d] / kv->v_scale[l]);
+                }
+                continue;
+            }
             uint16_t *kr = (uint16_t *)kv_row(kv->k[l], kv, b, nkv, h, hd, pos);
             uint16_t *vr = (uint16_t *)kv_row(kv->v[l], kv, b, nkv, h, hd, pos);
             if (!kr || !vr)
@@ -426,7 +437,11 @@ int32_t or_decode_token(const or_model *m, or_kv *kv, int b, int32_t token, int 
         }
         for (int h = 0; h < nq; h++) {
             int kvh = h / (nq / nkv);
-            or_attend_head(q + h * hd, kv->k[l], kv->v[l], kv, b, nkv, kvh, hd, pos + 1, o + h * hd);
+            if (kv->kv_fmt == 1)
+                or_attend_head_e4m3(q + h * hd, (const uint8_t *)kv->k[l], (const uint8_t *)kv->v[l],
+                                    kv->k_scale[l], kv->v_scale[l], kv, b, nkv, kvh, hd, pos + 1, o + h * hd);
+            else
+                or_attend_head(q + h * hd, kv->k[l], kv->v[l], kv, b, nkv, kvh, hd, pos + 1, o + h * hd);
         }
         or_matvec(&ly->wo, o, t);
         for (int i = 0; i < H; i++)

@@ -83,10 +83,14 @@ typedef struct {
     const or_layer *layers;       /* L entries */
 } or_model;
 
-/* Paged fp16 KV cache: k[l] and v[l] point at the pool of layer l, laid out
- * [n_pages][nkv][page_tokens][hd] (fp16 bit patterns).  The page table maps
- * logical page j of sequence b to physical page page_table[b*max_pages + j];
- * all layers use the same physical page index. */
+/* Paged KV cache: k[l] and v[l] point at the pool of layer l, laid out
+ * [n_pages][nkv][page_tokens][hd].  The page table maps logical page j of
+ * sequence b to physical page page_table[b*max_pages + j]; all layers use the
+ * same physical page index.
+ *  kv_fmt 0: fp16 bit patterns (the workload's cache format);
+ *  kv_fmt 1: E4M3 bytes with per-layer fp32 scales k_scale[l], v_scale[l]
+ *            (the FP8 variant: a value x is written as e4m3(x / scale) and
+ *            read as e4m3(code) * scale). */
 typedef struct {
     uint16_t **k;
     uint16_t **v;
@@ -94,6 +98,9 @@ typedef struct {
     int page_tokens;
     const int32_t *page_table;
     int max_pages;
+    int kv_fmt;
+    const float *k_scale;
+    const float *v_scale;
 } or_kv;
 
 /* scalar decoders (IEEE-754 binary16; OCP 8-bit E4M3 "fn"; OCP 4-bit E2M1) */

@@ -346,9 +346,11 @@ def test_quantizers_round_trip_within_format_bounds():
 
 # ------------------------------------------------------- whole decode step
 
-def _np_forward(model, kv_np, b, token, pos):
+def _np_forward(model, kv_np, b, token, pos, write=True, rows_out=None):
     """fp64 numpy brute force of one decode token on a tiny model (contiguous
-    per-position K/V gathered through the page table)."""
+    per-position K/V gathered through the page table).  write=False reads the
+    new position's K/V from kv_np as given instead of storing it (rounded to
+    fp16) first; rows_out, when given, receives each layer's fp64 (k, v)."""
     cfg = model.cfg
     deq = (lambda m: _np_deq_q4_0(m)) if cfg.fmt == synth.FMT_Q4_0 else (lambda m: _np_deq_nvfp4(m))
 
@@ -374,8 +376,11 @@ def _np_forward(model, kv_np, b, token, pos):
         v = qkv[(cfg.nq + cfg.nkv) * cfg.hd:].reshape(cfg.nkv, cfg.hd)
         q, k = rope(q, pos), rope(k, pos)
         kp, vp = kv_np["k"][l], kv_np["v"][l]
-        kp[table[pos // P], :, pos % P] = k.astype(np.float16)
-        vp[table[pos // P], :, pos % P] = v.astype(np.float16)
+        if rows_out is not None:
+            rows_out[l] = (k.copy(), v.copy())
+        if write:
+            kp[table[pos // P], :, pos % P] = k.astype(np.float16)
+            vp[table[pos // P], :, pos % P] = v.astype(np.float16)
         K = np.stack([kp[table[j // P], :, j % P] for j in range(pos + 1)]).astype(np.float64)
         Vv = np.stack([vp[table[j // P], :, j % P] for j in range(pos + 1)]).astype(np.float64)
         o = np.empty((cfg.nq, cfg.hd))
@@ -662,3 +667,43 @@ def test_attention_over_e4m3_cache_matches_fp64_brute_force():
         p = np.exp(s - s.max())
         want = (p / p.sum()) @ V
         assert np.max(np.abs(got - want)) < 1e-5 * max(1.0, np.max(np.abs(want))), (b, kvh, length)
+
+
+def test_decode_step_over_fp8_cache_matches_fp64_brute_force():
+    """Whole decode steps over the FP8 cache: the row each step writes is the
+    E4M3 rounding (torch float8) of k / scale and v / scale, and the logits
+    and hidden state match the fp64 forward over the same stored values."""
+    cfg = synth.CONFIGS["tiny"].with_(L=2)
+    model = synth.make_model(cfg, "cpu", seed=7)
+    kv = synth.make_kv_fp8(cfg, "cpu", seed=7)
+    om, okv = oracle.Model(model), oracle.KV(kv)
+    ks, vs = kv.k_scale.numpy().astype(np.float64), kv.v_scale.numpy().astype(np.float64)
+
+    def dec8(a, s):
+        return torch.from_numpy(np.ascontiguousarray(a)).view(torch.float8_e4m3fn).to(torch.float64).numpy() * s
+
+    def enc8(x, s):
+        t = torch.from_numpy((x / s).astype(np.float32)).clamp(-448.0, 448.0)
+        return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+    table = kv.page_table.numpy()
+    tok = int(synth.start_tokens(cfg, 7)[0])
+    for step in range(3):
+        pos = cfg.ctx + step
+        res = oracle.decode_token(om, okv, 0, tok, pos, want_hidden=True)
+        kv_np = {"k": [dec8(okv.k[l], ks[l]) for l in range(cfg.L)],
+                 "v": [dec8(okv.v[l], vs[l]) for l in range(cfg.L)], "table": table}
+        rows = {}
+        want_logits, want_x = _np_forward(model, kv_np, 0, tok, pos, write=False, rows_out=rows)
+        assert np.max(np.abs(res["logits"] - want_logits)) < 2e-5 * np.max(np.abs(want_logits))
+        assert np.max(np.abs(res["hidden"][-1] - want_x)) < 2e-5 * np.max(np.abs(want_x))
+        page, slot = table[0, pos // 16], pos % 16
+        mism = 0
+        for l in range(cfg.L):
+            k, v = rows[l]
+            for got, want in ((okv.k[l][page, :, slot], enc8(k, ks[l])), (okv.v[l][page, :, slot], enc8(v, vs[l]))):
+                mism += int(np.sum(got != want))
+                # a value within fp32 rounding of a tie may land on the neighbouring code
+                assert np.all(np.abs(got.astype(np.int32) - want.astype(np.int32)) <= 1)
+        assert mism <= 1
+        tok = res["token"]

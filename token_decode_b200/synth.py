@@ -315,14 +315,21 @@ class KVCache:
     page_table: torch.Tensor
     n_pages: int
     page_tokens: int = PAGE_TOKENS
+    # FP8 variant: k[l], v[l] hold E4M3 codes (uint8) and these hold one fp32
+    # scale per layer (a code c stands for e4m3(c) * scale); None for fp16
+    k_scale: Optional[torch.Tensor] = None
+    v_scale: Optional[torch.Tensor] = None
 
     def clone(self) -> "KVCache":
         return KVCache([t.clone() for t in self.k], [t.clone() for t in self.v],
-                       self.page_table.clone(), self.n_pages, self.page_tokens)
+                       self.page_table.clone(), self.n_pages, self.page_tokens,
+                       None if self.k_scale is None else self.k_scale.clone(),
+                       None if self.v_scale is None else self.v_scale.clone())
 
     def to(self, device) -> "KVCache":
         return KVCache([t.to(device) for t in self.k], [t.to(device) for t in self.v],
-                       self.page_table.to(device), self.n_pages, self.page_tokens)
+                       self.page_table.to(device), self.n_pages, self.page_tokens,
+                       self.k_scale, self.v_scale)
 
 
 def page_table(cfg: Config, device="cpu", seed: int = 0, permute: bool = True) -> torch.Tensor:
@@ -346,6 +353,24 @@ def make_kv(cfg: Config, device="cpu", seed: int = 0, permute: bool = True,
         ks.append(randn(shape, 1.0, device, seed, f"kv.k{l}").to(torch.float16).view(torch.int16))
         vs.append(randn(shape, 1.0, device, seed, f"kv.v{l}").to(torch.float16).view(torch.int16))
     return KVCache(ks, vs, page_table(cfg, device, seed, permute), cfg.n_pages)
+
+
+def make_kv_fp8(cfg: Config, device="cpu", seed: int = 0, permute: bool = True,
+                n_layers: Optional[int] = None) -> KVCache:
+    """The FP8 (E4M3) variant of make_kv: the same N(0, 1) context stored as
+    E4M3 codes of x / scale with per-layer scales 1/16 + l/256 (K) and
+    1/20 + l/256 (V), rounded by torch's float8 conversion after clamping to
+    the format's +-448."""
+    L = cfg.L if n_layers is None else n_layers
+    shape = (cfg.n_pages, cfg.nkv, PAGE_TOKENS, cfg.hd)
+    k_scale = torch.tensor([1 / 16 + l / 256 for l in range(L)], dtype=torch.float32)
+    v_scale = torch.tensor([1 / 20 + l / 256 for l in range(L)], dtype=torch.float32)
+    ks, vs = [], []
+    for l in range(L):
+        for name, sc, out in (("k", k_scale[l], ks), ("v", v_scale[l], vs)):
+            x = randn(shape, 1.0, device, seed, f"kv.{name}{l}") / sc.to(device)
+            out.append(x.clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8))
+    return KVCache(ks, vs, page_table(cfg, device, seed, permute), cfg.n_pages, PAGE_TOKENS, k_scale, v_scale)
 
 
 def start_tokens(cfg: Config, seed: int = 0, n: Optional[int] = None) -> torch.Tensor:
