@@ -131,14 +131,21 @@ void or_dequant_row(const or_qmat *w, int n, float *out)
             }
         }
     } else {
-        /* w = (e2m1(q) * e4m3(s)) * ts */
+        /* w = (e2m1(q) * e4m3(s)) * ts.  The 16 E2M1 values are the decoder's
+         * own outputs, looked up; each block's E4M3 scale is decoded once. */
+        float e2m1[16];
+        for (int c = 0; c < 16; c++)
+            e2m1[c] = or_e2m1_to_f32((uint8_t)c);
         const uint8_t *row = w->q + (size_t)n * (size_t)(K / 2);
         const uint8_t *sc = w->s + (size_t)n * (size_t)(K / 16);
-        for (int k = 0; k < K; k++) {
-            uint8_t byte = row[k / 2];
-            uint8_t code = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
-            float blk_scale = or_e4m3_to_f32(sc[k / 16]);
-            out[k] = (or_e2m1_to_f32(code) * blk_scale) * w->ts;
+        for (int b = 0; b < K / 16; b++) {
+            float blk_scale = or_e4m3_to_f32(sc[b]);
+            for (int j = 0; j < 16; j++) {
+                int k = b * 16 + j;
+                uint8_t byte = row[k / 2];
+                uint8_t code = (k & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 15);
+                out[k] = (e2m1[code] * blk_scale) * w->ts;
+            }
         }
     }
 }
