@@ -123,7 +123,8 @@ int bw_abi_version(void);
 /* Zero-fill `bytes` of workspace on `stream` (once, before first use). */
 bw_status bw_workspace_init(void *ws, size_t bytes, void *stream);
 /* Synchronize `stream`, then copy the device error word of `ws` into
- * *err_out (host) and clear it on the device. */
+ * *err_out (host) and clear it on the device.  ws == NULL reads the error word
+ * of bw_gemv_q4_0_noalloc's fixed scratch on the current device instead. */
 bw_status bw_read_error(void *ws, uint32_t *err_out, void *stream);
 
 /* ---------------------------------------------------------------- layout */
@@ -174,10 +175,15 @@ size_t bw_gemv_workspace_bytes(int N, int K, int M, unsigned flags);
  * library only inputs and outputs, or a path where cudaMalloc's implicit
  * synchronization is not acceptable).  No counterpart in the pages: a
  * library-interface addition.
- *   Same arguments, layout and results as bw_gemv_q4_0.  The scratch is a
+ *   Same arguments, layout and results as bw_gemv_q4_0 (the same kernel and
+ *   split plan, so the outputs are bit-identical).  The scratch is a
  *   file-scope __device__ array of BW_GEMV_NOALLOC_SCRATCH_BYTES that every
  *   GPU loading the library holds until process exit; nothing is allocated
- *   or freed (it issues one cudaMemsetAsync to clear its counters).
+ *   or freed (it issues one cudaMemsetAsync to clear its counters, after
+ *   every argument check has passed).
+ *   Device-side conditions (a bounded wait that ran out) set bits in the
+ *   array's error word, which calls do not clear: read and clear it with
+ *   bw_read_error(NULL, &err, stream).
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.
@@ -326,6 +332,14 @@ size_t bw_decode_workspace_bytes(const bw_model *m, const bw_kv *kv, int B, int 
  * on ws -- what a speculative draft head starts from.  Host arithmetic only;
  * NULL for arguments bw_decode_workspace_bytes would not size. */
 const float *bw_decode_hidden(const bw_model *m, const bw_kv *kv, int B, int n_rows, const void *ws);
+/* Device addresses, inside ws, of the expert choice of the last MoE layer the
+ * latest bw_decode_step on ws ran: *idx = int32 [B*n_rows][topk] expert ids in
+ * selection order (logit descending, ties to the lower id), *w = fp32
+ * [B*n_rows][topk] their softmax weights.  Deep-dive page, section 7 (the
+ * router's ordering of expert choices).  Host arithmetic only; valid until
+ * the next call on ws.  BW_ERR_UNSUPPORTED_SHAPE for a dense model. */
+bw_status bw_decode_moe_route(const bw_model *m, const bw_kv *kv, int B, int n_rows, const void *ws,
+                              const int32_t **idx, const float **w);
 
 /* Acceptance after a speculative verify pass.  "bw24" deep-dive page
  * (10100.com), section 5, stage 4 (the verify kernel unrolls the drafts as

@@ -87,7 +87,7 @@ def lib():
             "or_argmax": (C.c_int32, [p, i, p]),
             "or_spec_accept": (C.c_int32, [p, p, i, p]),
             "or_draft_token": (C.c_int32, [p, p, p, f, p, C.c_int32, p, p]),
-            "or_decode_token": (C.c_int32, [p, p, i, C.c_int32, i, i, p, p, p, p]),
+            "or_decode_token": (C.c_int32, [p, p, i, C.c_int32, i, i, p, p, p, p, p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(_lib, name)
@@ -331,7 +331,7 @@ def decode_token(model: Model, kv: KV, b: int, token: int, pos: int, moe_dense: 
                  want_logits: bool = True, want_hidden: bool = False, layers=None):
     """One greedy token of sequence b at position pos.  Writes K/V of pos into kv.
     layers=(l0, l1) runs only those layers (a bounded sample of the step).
-    Returns dict(token, margin, logits, hidden, moe_idx)."""
+    Returns dict(token, margin, logits, hidden, moe_idx, moe_logits)."""
     cfg = model.cfg
     mc, kc = model.c, kv.c
     if layers is not None:
@@ -346,14 +346,16 @@ def decode_token(model: Model, kv: KV, b: int, token: int, pos: int, moe_dense: 
     logits = np.empty(cfg.V, np.float32) if want_logits else None
     hidden = np.empty((L + 1, cfg.H), np.float32) if want_hidden else None
     moe_idx = np.empty((L, cfg.topk), np.int32) if cfg.n_experts else None
+    moe_logits = np.empty((L, cfg.n_experts), np.float32) if cfg.n_experts else None
     margin = np.zeros(1, np.float32)
     tok = lib().or_decode_token(C.byref(mc), C.byref(kc), b, int(token), int(pos),
                                 int(moe_dense),
                                 None if logits is None else _ptr(logits),
                                 None if hidden is None else _ptr(hidden),
-                                None if moe_idx is None else _ptr(moe_idx), _ptr(margin))
+                                None if moe_idx is None else _ptr(moe_idx), _ptr(margin),
+                                None if moe_logits is None else _ptr(moe_logits))
     return {"token": int(tok), "margin": float(margin[0]), "logits": logits, "hidden": hidden,
-            "moe_idx": moe_idx}
+            "moe_idx": moe_idx, "moe_logits": moe_logits}
 
 
 # ------------------------------------------------------ generation loops

@@ -396,7 +396,7 @@ static void ffn(const or_qmat *wg, const or_qmat *wu, const or_qmat *wd, const f
 
 int32_t or_decode_token(const or_model *m, or_kv *kv, int b, int32_t token, int pos,
                         int moe_dense, float *logits, float *hidden, int32_t *moe_idx,
-                        float *margin)
+                        float *margin, float *moe_logits)
 {
     const int H = m->H, hd = m->hd, nq = m->nq, nkv = m->nkv;
     const int nqkv = (nq + 2 * nkv) * hd;
@@ -473,6 +473,8 @@ int32_t or_decode_token(const or_model *m, or_kv *kv, int b, int32_t token, int 
                     a += ly->router[(size_t)e * (size_t)H + (size_t)i] * y[i];
                 r[e] = a;
             }
+            if (moe_logits)
+                memcpy(moe_logits + (size_t)l * (size_t)E, r, sizeof(float) * (size_t)E);
             or_topk_softmax(r, E, K, sel, w);
             if (moe_idx)
                 memcpy(moe_idx + (size_t)l * (size_t)K, sel, sizeof(int32_t) * (size_t)K);

@@ -162,13 +162,14 @@ int32_t or_draft_token(const or_qmat *embed, const or_qmat *w_draft, const float
 /* One greedy decode token of sequence b at position pos (writes its K/V into
  * the cache, attends over positions 0..pos).  logits [V] may be NULL;
  * hidden [(L+1)*H] (residual stream after the embedding and after each layer)
- * may be NULL; moe_idx [L*topk] (selected experts) may be NULL.
+ * may be NULL; moe_idx [L*topk] (selected experts) and moe_logits [L*E]
+ * (each layer's router logits) may be NULL.
  * moe_dense != 0 evaluates every expert and then combines the selected ones
  * (identical result; a self-check of the sparse path).  Returns the argmax
  * token; *margin receives the top-2 logit margin when non-NULL. */
 int32_t or_decode_token(const or_model *m, or_kv *kv, int b, int32_t token, int pos,
                         int moe_dense, float *logits, float *hidden, int32_t *moe_idx,
-                        float *margin);
+                        float *margin, float *moe_logits);
 
 #ifdef __cplusplus
 }

@@ -46,3 +46,15 @@ def check_kv(gpu_pools, ora_pools, page_table, B, first_pos, n_new, page_tokens=
         gw = g[written].view(np.float16).astype(np.float64)
         ow = o[written].view(np.float16).astype(np.float64)
         assert rel_err(gw, ow) < TOL
+
+
+def parallel_rows(fn, items):
+    """fn(item) for every item, on host threads (the oracle's C calls release the
+    interpreter lock; rows of different sequences touch disjoint KV pages)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    items = list(items)
+    if len(items) <= 1:
+        return [fn(i) for i in items]
+    with ThreadPoolExecutor(max_workers=min(len(items), os.cpu_count() or 1)) as ex:
+        return list(ex.map(fn, items))

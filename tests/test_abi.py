@@ -116,3 +116,19 @@ def test_binding_refuses_host_and_strided_tensors():
         bw._ptr(torch.zeros(4))
     with pytest.raises(ValueError):
         bw.gemv_q4_0(torch.zeros(16, dtype=torch.uint8), 4096, 8, 32, 4096, 1, 4096, torch.zeros(1))
+
+
+def test_noalloc_gemv_refuses_shapes_beyond_its_fixed_scratch(lib):
+    """bw_gemv_q4_0_noalloc refuses, before touching any device, a shape whose
+    split-K partial sums would not fit the fixed scratch array, and one with
+    more row groups than its counters cover."""
+    p = C.c_void_p
+    fake = p(4096)   # never dereferenced: the shape check comes first
+    # K = 131072 splits K into >= 37 slices: 37 x 4096 rows x 4 rows x 4 B > 768 KiB
+    assert lib.bw_gemv_q4_0_noalloc(fake, fake, 4096, 131072, fake, 4, None, C.c_float(1e-6), None, fake,
+                                    None, 0, None) == 2
+    assert lib.bw_gemv_q4_0_noalloc(fake, fake, 262144, 512, fake, 1, None, C.c_float(1e-6), None, fake,
+                                    None, 0, None) == 2
+    assert lib.bw_gemv_q4_0_noalloc(fake, fake, 0, 512, fake, 1, None, C.c_float(1e-6), None, fake,
+                                    None, 0, None) == 1
+    assert lib.bw_read_error(fake, None, None) == 1

@@ -8,8 +8,11 @@ import torch
 
 import oracle
 from token_decode_b200 import bw, runtime, synth
-from gpu_util import MARGIN, TOL, rel_err
+from gpu_util import MARGIN, TOL, parallel_rows, rel_err
 from gpu_util import check_kv as check_kv_pools
+
+# router top-k must agree with the oracle when the k-th / (k+1)-th logit gap exceeds this
+ROUTER_GAP = 1e-3
 
 pytestmark = pytest.mark.gpu
 
@@ -32,9 +35,11 @@ def _setup(cfg, seed=0, n_layers=None, permute=True):
     return model, kv, om, okv, dm, dkv
 
 
-def _run_steps(cfg, steps, seed=0, n_layers=None, B=None, check_kv=True):
+def _run_steps(cfg, steps, seed=0, n_layers=None, B=None, check_kv=True, check_route=False):
     """Greedy decode on the GPU with the oracle teacher-forced on the GPU's
-    tokens; returns the worst normwise logit error."""
+    tokens (the oracle's rows run on host threads); returns the worst normwise
+    logit error.  check_route: after every step, the last MoE layer's expert
+    choice (bw_decode_moe_route) against the oracle's, under the gap rule."""
     B = cfg.B if B is None else B
     model, kv, om, okv, dm, dkv = _setup(cfg, seed, n_layers)
     dec = runtime.Decoder(dm, dkv, B)
@@ -50,20 +55,44 @@ def _run_steps(cfg, steps, seed=0, n_layers=None, B=None, check_kv=True):
         assert bw.read_error(dec.ws) == 0
         got_tok = dec.tokens_out.cpu().tolist()
         got_lg = logits.cpu().numpy()
-        for b in range(B):
-            res = oracle.decode_token(om, okv, b, cur[b], cfg.ctx + step)
+        ress = parallel_rows(lambda b: oracle.decode_token(om, okv, b, cur[b], cfg.ctx + step), range(B))
+        for b, res in enumerate(ress):
             err = rel_err(got_lg[b], res["logits"])
             worst = max(worst, err)
             assert err < TOL, (step, b, err)
             assert got_tok[b] == int(np.argmax(got_lg[b]))
             if res["margin"] > MARGIN:
                 assert got_tok[b] == res["token"], (step, b, res["margin"])
+        if check_route:
+            idx, w = bw.decode_moe_route(dm.c, dkv.c, B, 1, dec.ws)
+            _check_route(idx.cpu().numpy(), w.cpu().numpy(), [r["moe_idx"][-1] for r in ress],
+                         [r["moe_logits"][-1] for r in ress], cfg.topk)
         cur = got_tok
         dec.pos += 1
     if check_kv:
         check_kv_pools(list(dkv.k) + list(dkv.v), list(okv.k) + list(okv.v), dkv.page_table, B,
                        cfg.ctx, steps)
     return worst
+
+
+def _check_route(g_idx, g_w, o_idx, o_logits, k):
+    """GPU expert choice per row vs the oracle's: the same set whenever the
+    oracle's k-th / (k+1)-th router-logit gap exceeds ROUTER_GAP, the same
+    order when every gap among its top k+1 does, weights within the
+    tolerance."""
+    for b in range(len(o_idx)):
+        r = np.asarray(o_logits[b], np.float64)
+        top = np.sort(r)[::-1][: k + 1]
+        gaps = top[:-1] - top[1:]
+        if gaps[k - 1] > ROUTER_GAP:
+            assert sorted(g_idx[b].tolist()) == sorted(o_idx[b].tolist()), (b, g_idx[b], o_idx[b])
+            ow = np.exp(r[o_idx[b]] - r[o_idx[b]].max())
+            ow /= ow.sum()
+            want = dict(zip(o_idx[b].tolist(), ow))
+            got = dict(zip(g_idx[b].tolist(), g_w[b].tolist()))
+            assert max(abs(got[e] - want[e]) for e in want) < TOL, (b, got, want)
+        if np.all(gaps > ROUTER_GAP):
+            assert g_idx[b].tolist() == o_idx[b].tolist(), (b, g_idx[b], o_idx[b])
 
 
 def test_tiny_decode_8_steps():
@@ -88,45 +117,81 @@ def test_tiny_batch5_rows_above_gemv_block():
 
 
 def _tiny_moe(**kw):
-    return synth.CONFIGS["tiny"].with_(name="tiny-moe", fmt=synth.FMT_NVFP4, F=0, n_experts=16,
-                                       topk=4, F_exp=64, B=4, L=2, **kw)
+    args = dict(name="tiny-moe", fmt=synth.FMT_NVFP4, F=0, n_experts=16, topk=4, F_exp=64, B=4, L=2)
+    args.update(kw)
+    return synth.CONFIGS["tiny"].with_(**args)
 
 
 def test_tiny_moe_decode_and_router_topk():
-    """MoE decode vs the oracle: logits, tokens and the selected experts."""
+    """MoE decode vs the oracle: logits, tokens, and every layer's expert
+    choice (the step over layers 0..l, read through bw_decode_moe_route)."""
     cfg = _tiny_moe()
+    _run_steps(cfg, 2, seed=3, check_route=True)
     model, kv, om, okv, dm, dkv = _setup(cfg, seed=3)
-    dec = runtime.Decoder(dm, dkv, cfg.B)
     toks = synth.start_tokens(cfg, 3)[: cfg.B]
-    dec.tokens_in.copy_(toks)
-    dec.pos.fill_(cfg.ctx)
-    logits = torch.empty((cfg.B, cfg.V), device="cuda")
-    dec.step(logits=logits)
-    assert bw.read_error(dec.ws) == 0
-    for b in range(cfg.B):
-        res = oracle.decode_token(om, okv, b, int(toks[b]), cfg.ctx)
-        assert rel_err(logits[b].cpu().numpy(), res["logits"]) < TOL
-        if res["margin"] > MARGIN:
-            assert int(dec.tokens_out[b]) == res["token"]
-    # the routing kernel alone: same inputs -> same expert choice as the oracle's
-    x = torch.randn((cfg.B, cfg.H), device="cuda")
-    ly = dm.layers[0]
-    idx = torch.empty((cfg.B, cfg.topk), dtype=torch.int32, device="cuda")
-    wts = torch.empty((cfg.B, cfg.topk), device="cuda")
-    ws = bw.workspace(bw.moe_workspace_bytes(dm.c, cfg.B))
-    x0 = x.clone()
-    bw.moe_route_gemv(dm.c, ly, x, cfg.B, ws, topk_idx=idx, topk_w=wts)
-    torch.cuda.synchronize()
-    g = model.layers[0]
-    for b in range(cfg.B):
-        y = oracle.rmsnorm(x0[b].cpu().numpy(), g.ffn_norm.cpu().numpy(), cfg.eps)
-        r = (g.router.cpu().numpy().astype(np.float64) @ y.astype(np.float64))
-        order = np.lexsort((np.arange(cfg.n_experts), -r))
-        gap = r[order[cfg.topk - 1]] - r[order[cfg.topk]]
-        if gap > 1e-3:
-            assert sorted(idx[b].tolist()) == sorted(order[: cfg.topk].tolist())
-        assert abs(float(wts[b].sum()) - 1.0) < 1e-5
-    assert torch.isfinite(x).all() and not torch.equal(x, x0)
+    kv0 = kv.clone()
+    for l in range(cfg.L):
+        sub = bw.Model.from_buffer_copy(dm.c)
+        sub.L = l + 1
+        dkv_l = runtime.DeviceKV(kv0.clone())
+        dec = runtime.Decoder(dm, dkv_l, cfg.B)
+        dec.tokens_in.copy_(toks)
+        dec.pos.fill_(cfg.ctx)
+        bw.decode_step(sub, dkv_l.c, dec.tokens_in, dec.pos, cfg.B, 1, dec.tokens_out, dec.ws)
+        assert bw.read_error(dec.ws) == 0
+        idx, w = bw.decode_moe_route(sub, dkv_l.c, cfg.B, 1, dec.ws)
+        ress = [oracle.decode_token(om, oracle.KV(kv0), b, int(toks[b]), cfg.ctx, want_logits=False)
+                for b in range(cfg.B)]
+        _check_route(idx.cpu().numpy(), w.cpu().numpy(), [r["moe_idx"][l] for r in ress],
+                     [r["moe_logits"][l] for r in ress], cfg.topk)
+
+
+@pytest.mark.parametrize("E,k", [(16, 4), (256, 8)])
+def test_router_topk_bit_exact_on_identical_logits(E, k):
+    """bw_moe_route_gemv's selection fed logits the oracle computes identically
+    (x = 16 e_c, unit gains, eps = 0: every row's logits are exactly 16 * Wr[:, c])
+    equals oracle.topk_softmax's, in order, with planted ties (lower id first),
+    one-ulp neighbours, signed zeros and repeated values; weights within 1e-6."""
+    B = 32
+    cfg = _tiny_moe(n_experts=E, topk=k, eps=0.0).with_(B=B, L=1)
+    model = synth.make_model(cfg, "cuda", seed=4)
+    ly = model.layers[0]
+    ly.ffn_norm.fill_(1.0)
+    rng = np.random.default_rng(E)
+    wr = ly.router.cpu().numpy()
+    for b in range(B):
+        if b == 0:
+            col = np.full(E, 0.25, np.float32)                         # all equal
+        elif b == 1:
+            col = np.zeros(E, np.float32)
+            col[::2] = -0.0                                            # +0 / -0 ties
+        elif b == 2:
+            col = rng.normal(size=E).astype(np.float32)
+            order = np.argsort(-col)
+            col[order[k]] = col[order[k - 1]]                          # tie across the k-th boundary
+        elif b == 3:
+            col = rng.normal(size=E).astype(np.float32)
+            order = np.argsort(-col)
+            col[order[k]] = np.nextafter(col[order[k - 1]], np.float32(-np.inf))   # one ulp below
+        else:
+            col = rng.choice(np.array([-1.5, -0.5, 0.0, 0.5, 0.75, 1.0], np.float32), size=E)
+            col[rng.integers(0, E)] = np.float32(rng.normal())
+        wr[:, b] = col
+    ly.router.copy_(torch.from_numpy(wr))
+    dm = runtime.DeviceModel(model, cfg.max_pages * synth.PAGE_TOKENS)
+    x = torch.zeros((B, cfg.H), device="cuda")
+    x[torch.arange(B), torch.arange(B)] = 16.0
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    wts = torch.empty((B, k), device="cuda")
+    ws = bw.workspace(bw.moe_workspace_bytes(dm.c, B))
+    bw.moe_route_gemv(dm.c, dm.layers[0], x, B, ws, topk_idx=idx, topk_w=wts)
+    assert bw.read_error(ws) == 0
+    g_idx, g_w = idx.cpu().numpy(), wts.cpu().numpy()
+    for b in range(B):
+        logits = (wr[:, b] * np.float32(16.0)).astype(np.float32)
+        o_idx, o_w = oracle.topk_softmax(logits, k)
+        assert g_idx[b].tolist() == o_idx.tolist(), (b, g_idx[b], o_idx)
+        assert np.max(np.abs(g_w[b] - o_w) / o_w) < 1e-6, (b, g_w[b], o_w)
 
 
 def test_step_hidden_state_matches_oracle():
@@ -256,7 +321,7 @@ def test_7b_full_model_two_steps():
 def test_moe_full_size_layers_batch32():
     """35B-A3B-class shapes (256 experts, top-8, shared expert), B = 32, two layers."""
     cfg = synth.CONFIGS["moe"].with_(L=2)
-    _run_steps(cfg, 1, n_layers=2, check_kv=False)
+    _run_steps(cfg, 1, n_layers=2, check_kv=False, check_route=True)
 
 
 @pytest.mark.slow

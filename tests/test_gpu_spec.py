@@ -12,7 +12,7 @@ import torch
 
 import oracle
 from token_decode_b200 import bw, runtime, synth
-from gpu_util import MARGIN, TOL, check_kv, rel_err
+from gpu_util import MARGIN, TOL, check_kv, parallel_rows, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -51,10 +51,13 @@ def _verify_vs_oracle(cfg, K, seed, n_layers=None, drafts=None):
     assert bw.read_error(dec.ws) == 0
     lg = logits.cpu().numpy()
     got = dec.tokens_out.cpu().tolist()
+    def seq_rows(b):
+        # the rows of one sequence run in order: row r reads the K/V rows 0..r-1 wrote
+        return [oracle.decode_token(om, okv, b, rows[b][r], cfg.ctx + r) for r in range(R)]
+
     margins = []
-    for b in range(B):
-        for r in range(R):
-            res = oracle.decode_token(om, okv, b, rows[b][r], cfg.ctx + r)
+    for b, ress in enumerate(parallel_rows(seq_rows, range(B))):
+        for r, res in enumerate(ress):
             err = rel_err(lg[b * R + r], res["logits"])
             assert err < TOL, (b, r, err)
             assert got[b * R + r] == int(np.argmax(lg[b * R + r]))

@@ -30,6 +30,7 @@ EXPORTS = (
     "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
     "bw_paged_attn_decode", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
     "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes", "bw_decode_hidden", "bw_spec_accept",
+    "bw_decode_moe_route",
 )
 
 
@@ -99,6 +100,7 @@ def lib() -> C.CDLL:
             "bw_decode_step": (i, [p, p, p, p, i, i, p, p, u, p, z, p]),
             "bw_decode_workspace_bytes": (z, [p, p, i, i]),
             "bw_decode_hidden": (p, [p, p, i, i, p]),
+            "bw_decode_moe_route": (i, [p, p, i, i, p, p, p]),
             "bw_spec_accept": (i, [p, p, i, i, p, p, i, p, p]),
         }
         for name, (res, args) in sig.items():
@@ -256,6 +258,18 @@ def decode_hidden(model: Model, kv: KV, B, n_rows, ws) -> torch.Tensor:
     off = addr - ws.data_ptr()
     n = B * n_rows * model.H
     return ws[off: off + 4 * n].view(torch.float32).view(B * n_rows, model.H)
+
+
+def decode_moe_route(model: Model, kv: KV, B, n_rows, ws):
+    """(expert ids int32 [B*n_rows][topk], weights fp32 [B*n_rows][topk]): views
+    into ws of the last MoE layer's expert choice in the latest step on ws."""
+    ia, wa = C.c_void_p(0), C.c_void_p(0)
+    _check(lib().bw_decode_moe_route(C.byref(model), C.byref(kv), B, n_rows, _ptr(ws), C.byref(ia),
+                                     C.byref(wa)), "bw_decode_moe_route")
+    n = B * n_rows * model.topk
+    oi, ow = ia.value - ws.data_ptr(), wa.value - ws.data_ptr()
+    return (ws[oi: oi + 4 * n].view(torch.int32).view(B * n_rows, model.topk),
+            ws[ow: ow + 4 * n].view(torch.float32).view(B * n_rows, model.topk))
 
 
 def decode_step(model: Model, kv: KV, tokens_in, pos, B, n_rows, tokens_out, ws, logits=None,

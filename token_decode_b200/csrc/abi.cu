@@ -5,6 +5,8 @@
 
 namespace bw {
 
+bw_status noalloc_scratch(void **out);   // gemv_noalloc.cu
+
 int sm_count() {
     static int cached[64] = {};
     static std::mutex mu;   // host threads may call the library concurrently
@@ -53,7 +55,12 @@ bw_status bw_workspace_init(void *ws, size_t bytes, void *stream) {
 }
 
 bw_status bw_read_error(void *ws, uint32_t *err_out, void *stream) {
-    if (!ws || !err_out) return BW_ERR_INVALID_ARG;
+    if (!err_out) return BW_ERR_INVALID_ARG;
+    if (!ws) {
+        // the error word of bw_gemv_q4_0_noalloc's fixed scratch on this device
+        const bw_status s = bw::noalloc_scratch(&ws);
+        if (s != BW_OK) return s;
+    }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) {
         (void)cudaGetLastError();

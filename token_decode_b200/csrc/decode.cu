@@ -21,6 +21,7 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
                          char *moe_base, cudaStream_t st);
 bw_status moe_check(const bw_model *m, const bw_layer *ly, int R);
 size_t moe_scratch_bytes(const bw_model *m, int R);
+void moe_route_buffers(const bw_model *m, int R, char *base, int32_t **sel, float **wts);
 
 struct StepBuffers {
     float *x, *qkv, *attn, *act;
@@ -117,6 +118,20 @@ const float *bw_decode_hidden(const bw_model *m, const bw_kv *kv, int B, int n_r
     bw::StepBuffers bf;
     bw::step_bytes(m, kv, B, n_rows, &bf, const_cast<void *>(ws));
     return bf.x;
+}
+
+bw_status bw_decode_moe_route(const bw_model *m, const bw_kv *kv, int B, int n_rows, const void *ws,
+                              const int32_t **idx, const float **w) {
+    if (!m || !kv || !ws || B <= 0 || n_rows <= 0 || !idx || !w) return BW_ERR_INVALID_ARG;
+    if (m->n_experts <= 0) return BW_ERR_UNSUPPORTED_SHAPE;
+    bw::StepBuffers bf;
+    bw::step_bytes(m, kv, B, n_rows, &bf, const_cast<void *>(ws));
+    int32_t *sel = nullptr;
+    float *wts = nullptr;
+    bw::moe_route_buffers(m, B * n_rows, bf.moe, &sel, &wts);
+    *idx = sel;
+    *w = wts;
+    return BW_OK;
 }
 
 size_t bw_decode_workspace_bytes(const bw_model *m, const bw_kv *kv, int B, int n_rows) {

@@ -21,13 +21,20 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[BW_GEMV_NOALLOC
 // code the array's name is only a host-side stand-in, so the address must
 // come from cudaGetSymbolAddress with that device current.
 void *g_noalloc_ptr[64] = {};
+std::mutex g_noalloc_mu;   // host threads may call the library concurrently
 
+}  // namespace
+
+// The scratch array's device address on the current device (looked up on
+// first use).  Also used by bw_read_error(NULL, ...), which reads and clears
+// the array's error word.
 bw_status noalloc_scratch(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         (void)cudaGetLastError();
         return BW_ERR_CUDA;
     }
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
     if (!g_noalloc_ptr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
@@ -40,7 +47,6 @@ bw_status noalloc_scratch(void **out) {
     return BW_OK;
 }
 
-}  // namespace
 }  // namespace bw
 
 extern "C" bw_status bw_gemv_q4_0_noalloc(const void *w_q, const void *w_d, int N, int K, const float *x,
@@ -55,14 +61,21 @@ extern "C" bw_status bw_gemv_q4_0_noalloc(const void *w_q, const void *w_d, int 
     void *ws = nullptr;
     bw_status s = bw::noalloc_scratch(&ws);
     if (s != BW_OK) return s;
+    const bw::Scratch sc = bw::scratch_of(ws, BW_GEMV_NOALLOC_SCRATCH_BYTES);
+    // every argument check runs before anything is queued
+    s = bw::gemv_check(BW_FMT_Q4_0, w_q, w_d, N, K, x, M, gamma, residual, y, argmax_out, flags, sc);
+    if (s != BW_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // The array keeps whatever the previous call left: clear the error word
-    // and the counters this launch can use, which must start at zero.
+    // The array keeps whatever the previous call left.  The counters this
+    // launch can use must start at zero: clear them (a call cut short by a
+    // device-side timeout may have left some behind).  The error word before
+    // them is left alone, so a timeout stays visible to bw_read_error(NULL).
     const size_t clear = (16u + bw::CNT_GEMV_RG + static_cast<size_t>(N / 8)) * sizeof(uint32_t);
-    if (cudaMemsetAsync(ws, 0, clear, st) != cudaSuccess) {
+    if (cudaMemsetAsync(static_cast<char *>(ws) + sizeof(uint32_t), 0, clear - sizeof(uint32_t), st) !=
+        cudaSuccess) {
         (void)cudaGetLastError();
         return BW_ERR_CUDA;
     }
-    return bw::gemv_launch(BW_FMT_Q4_0, w_q, w_d, 1.0f, 1.0f, N, K, x, M, gamma, eps, residual, y,
-                           argmax_out, flags, bw::scratch_of(ws, BW_GEMV_NOALLOC_SCRATCH_BYTES), st);
+    return bw::gemv_launch(BW_FMT_Q4_0, w_q, w_d, 1.0f, 1.0f, N, K, x, M, gamma, eps, residual, y, argmax_out,
+                           flags, sc, st);
 }

@@ -491,6 +491,15 @@ static size_t moe_carve(const bw_model *m, int R, char *base, MoeScratch *ms) {
 
 size_t moe_scratch_bytes(const bw_model *m, int R) { return moe_carve(m, R, nullptr, nullptr); }
 
+// Where, inside a MoE scratch region at `base`, the top-k kernel leaves the
+// selected experts and their weights (when the caller passes no outputs).
+void moe_route_buffers(const bw_model *m, int R, char *base, int32_t **sel, float **wts) {
+    MoeScratch ms;
+    moe_carve(m, R, base, &ms);
+    *sel = ms.sel;
+    *wts = ms.wts;
+}
+
 template <int FMT>
 static bw_status grouped_go(const GroupedParams &p, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(p.nst) * GV_STAGE_BYTES +
