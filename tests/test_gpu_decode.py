@@ -330,3 +330,112 @@ def test_full_size_layers_nvfp4(name, layers):
     """Full-size layer shapes of the NVFP4 models (a few layers, one step)."""
     cfg = synth.CONFIGS[name].with_(L=layers)
     _run_steps(cfg, 1, n_layers=layers, check_kv=False)
+
+
+# ------------------------------------------- persistent batch-1 step
+
+def _step_once(dm, kv, tok, pos, flags=0, L=None):
+    """One step of a fresh copy of kv; returns (logits, token, pools, hidden)."""
+    cfg = dm.cfg
+    dkv = runtime.DeviceKV(kv.clone())
+    dec = runtime.Decoder(dm, dkv, 1)
+    dec.tokens_in.fill_(int(tok))
+    dec.pos.fill_(int(pos))
+    lg = torch.empty((1, cfg.V), device="cuda")
+    model_c = dm.c
+    if L is not None:
+        model_c = bw.Model.from_buffer_copy(dm.c)
+        model_c.L = L
+    bw.decode_step(model_c, dkv.c, dec.tokens_in, dec.pos, 1, 1, dec.tokens_out, dec.ws, logits=lg, flags=flags)
+    assert bw.read_error(dec.ws) == 0
+    hid = bw.decode_hidden(model_c, dkv.c, 1, 1, dec.ws).clone()
+    return lg[0].cpu().numpy(), int(dec.tokens_out[0]), dkv, hid.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,fmt,layers", [
+    ("tiny", synth.FMT_Q4_0, 1), ("tiny", synth.FMT_NVFP4, 2),
+    ("7b", synth.FMT_Q4_0, 2), ("9b", synth.FMT_NVFP4, 2), ("27b", synth.FMT_NVFP4, 2)])
+def test_persistent_step_matches_layerwise_chain_and_oracle(name, fmt, layers):
+    """The one-kernel batch-1 step against the per-layer kernel chain on the same
+    inputs (logits, token, hidden state, the KV rows written) and against the oracle."""
+    cfg = synth.CONFIGS[name].with_(fmt=fmt, L=layers)
+    model, kv, om, okv, dm, dkv = _setup(cfg, seed=31, n_layers=layers)
+    tok = int(synth.start_tokens(cfg, 31)[0])
+    lg_p, tok_p, kv_p, hid_p = _step_once(dm, kv, tok, cfg.ctx)
+    lg_c, tok_c, kv_c, hid_c = _step_once(dm, kv, tok, cfg.ctx, flags=bw.STEP_LAYERWISE)
+    assert rel_err(lg_p, lg_c) < 1e-4
+    assert rel_err(hid_p, hid_c) < 1e-4
+    res = oracle.decode_token(om, okv, 0, tok, cfg.ctx, want_hidden=True)
+    assert rel_err(lg_p, res["logits"]) < TOL
+    assert rel_err(hid_p[0], res["hidden"][layers]) < TOL
+    assert tok_p == int(np.argmax(lg_p))
+    if res["margin"] > MARGIN:
+        assert tok_p == res["token"] == tok_c
+    check_kv_pools(list(kv_p.k) + list(kv_p.v), list(okv.k) + list(okv.v), kv_p.page_table, 1, cfg.ctx, 1)
+
+
+def test_persistent_step_graph_replay_and_determinism():
+    """Six batch-1 steps with on-device advance: eager, host-driven steps and
+    one CUDA graph of six steps give the same tokens; two runs of the same step
+    give bit-identical logits."""
+    cfg = synth.CONFIGS["tiny"].with_(L=2)
+    model, kv, om, okv, dm, dkv = _setup(cfg, seed=12)
+    kv0 = kv.clone()
+    tok = int(synth.start_tokens(cfg, 12)[0])
+    a = _step_once(dm, kv0, tok, cfg.ctx)
+    b = _step_once(dm, kv0, tok, cfg.ctx)
+    assert np.array_equal(a[0], b[0]) and a[1] == b[1]
+    dec = runtime.Decoder(dm, dkv, 1)
+    dec.tokens_in.fill_(tok)
+    dec.pos.fill_(cfg.ctx)
+    eager = []
+    for _ in range(6):
+        dec.step(advance=True)
+        eager.append(int(dec.tokens_out[0]))
+    assert bw.read_error(dec.ws) == 0
+    dkv2 = runtime.DeviceKV(kv0.clone())
+    dec2 = runtime.Decoder(dm, dkv2, 1)
+    dec2.tokens_in.fill_(tok)
+    dec2.pos.fill_(cfg.ctx)
+    outs = torch.empty(6, dtype=torch.int32, device="cuda")
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(6):
+                dec2.step(advance=True, stream=s)
+                outs[i].copy_(dec2.tokens_out[0])
+    torch.cuda.current_stream().wait_stream(s)
+    g.replay()
+    torch.cuda.synchronize()
+    assert outs.tolist() == eager
+    assert int(dec2.pos[0]) == cfg.ctx + 6
+    assert bw.read_error(dec2.ws) == 0
+    # the oracle, teacher-forced on the GPU tokens
+    cur = tok
+    for i in range(6):
+        res = oracle.decode_token(om, okv, 0, cur, cfg.ctx + i)
+        if res["margin"] > MARGIN:
+            assert eager[i] == res["token"]
+        cur = eager[i]
+
+
+def test_persistent_step_bad_page_sets_error():
+    """A page-table entry outside the pool inside the context: the step reports
+    BW_DEVERR_BAD_PAGE, neither reads nor writes that page, and finishes."""
+    cfg = synth.CONFIGS["tiny"]
+    model, kv, om, okv, dm, dkv = _setup(cfg, seed=13)
+    kv.page_table[0, 3] = cfg.n_pages + 7
+    dkv = runtime.DeviceKV(kv)
+    dec = runtime.Decoder(dm, dkv, 1)
+    dec.tokens_in.fill_(1)
+    dec.pos.fill_(cfg.ctx)
+    lg = torch.empty((1, cfg.V), device="cuda")
+    dec.step(logits=lg)
+    assert bw.read_error(dec.ws) & bw.DEVERR_BAD_PAGE
+    assert torch.isfinite(lg).all()
+    # the workspace is usable again: a clean step after restoring the entry
+    dkv.page_table[0, 3] = int(synth.page_table(cfg, "cuda", 13)[0, 3])
+    dec.step(logits=lg)
+    assert bw.read_error(dec.ws) == 0

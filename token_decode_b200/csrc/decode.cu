@@ -11,6 +11,9 @@
 // feeds the next step (token in, position + 1), so a graph of many steps
 // decodes autoregressively without the host.
 //
+// A batch-1 step of a dense model runs instead as one persistent kernel
+// (step_persistent.cu) unless BW_STEP_LAYERWISE asks for the chain.
+//
 // The deep-dive page (10100.com), section 4, describes the engine facade that
 // exposes prefill and decode; this is its decode call on device memory.
 #include "bw_common.cuh"
@@ -22,10 +25,16 @@ bw_status moe_ffn_launch(const bw_model *m, const bw_layer *ly, float *x, int R,
 bw_status moe_check(const bw_model *m, const bw_layer *ly, int R);
 size_t moe_scratch_bytes(const bw_model *m, int R);
 void moe_route_buffers(const bw_model *m, int R, char *base, int32_t **sel, float **wts);
+bool persistent_step_applies(const bw_model *m, int B, int n_rows);
+size_t persistent_scratch_bytes(const bw_model *m);
+bw_status persistent_step_launch(const bw_model *m, const bw_kv *kv, int32_t *tokens_in, int32_t *pos,
+                                 int32_t *tokens_out, float *logits, bool advance, float *x, float *qkv, float *attn,
+                                 float *act, char *scratch, const Scratch &sc, cudaStream_t st);
 
 struct StepBuffers {
     float *x, *qkv, *attn, *act;
     char *moe;
+    char *pk;       // scratch of the persistent batch-1 step (when it applies)
     Scratch kern;   // scratch shared by the kernels of the step
 };
 
@@ -53,6 +62,7 @@ static size_t step_bytes(const bw_model *m, const bw_kv *kv, int B, int n_rows, 
     float *attn = cv.take<float>(static_cast<size_t>(R) * m->nq * m->hd);
     float *act = cv.take<float>(static_cast<size_t>(R) * max(m->F, 1));
     char *moe = m->n_experts ? cv.take<char>(moe_scratch_bytes(m, R)) : nullptr;
+    char *pk = persistent_step_applies(m, B, n_rows) ? cv.take<char>(persistent_scratch_bytes(m)) : nullptr;
     const size_t kb = kernel_scratch_bytes(m, kv, B, n_rows);
     char *kbase = cv.take<char>(kb);
     if (bufs) {
@@ -61,6 +71,7 @@ static size_t step_bytes(const bw_model *m, const bw_kv *kv, int B, int n_rows, 
         bufs->attn = attn;
         bufs->act = act;
         bufs->moe = moe;
+        bufs->pk = pk;
         bufs->kern.err = ws ? ws_error_word(ws) : nullptr;
         bufs->kern.cnt = ws ? ws_counters(ws) : nullptr;
         bufs->kern.base = kbase;
@@ -168,6 +179,9 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
     if (s != BW_OK || (flags & BW_STEP_VALIDATE_ONLY)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int R = B * n_rows;
+    if (bf.pk && !(flags & BW_STEP_LAYERWISE))
+        return persistent_step_launch(m, kv, tokens_in, pos, tokens_out, logits, (flags & BW_STEP_ADVANCE) != 0,
+                                      bf.x, bf.qkv, bf.attn, bf.act, bf.pk, bf.kern, st);
 
     s = embed_launch(fmt, m->embed.q, m->embed.s, m->embed.ts, m->V, m->H, tokens_in, R, bf.x,
                      bf.kern.err, st);
