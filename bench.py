@@ -149,8 +149,10 @@ def step_bytes(cfg, model, avg_ctx, moe_layer_bytes=0):
 
 # ncu summaries of the dominant kernel: DRAM traffic per launch, valid while the
 # kernel's sources hash to the recorded value
-_PROFILE_FILES = {("gu", "7b"): "gemv_gate_up_7b.md"}
-_KERNEL_SOURCES = {"gu": ("gemv.cu", "gemv_core.cuh", "bw_common.cuh")}
+_PROFILE_FILES = {("gu", "7b-dense-q4_0"): "gemv_gate_up_7b.md",
+                  ("step", "7b-dense-q4_0"): "step_persistent_7b.md"}
+_KERNEL_SOURCES = {"gu": ("gemv.cu", "gemv_core.cuh", "bw_common.cuh"),
+                   "step": ("step_persistent.cu", "gemv_core.cuh", "bw_common.cuh")}
 
 
 def kernel_sources_sha(kind):
@@ -165,6 +167,8 @@ def kernel_sources_sha(kind):
 
 def _ncu_traffic(kind, cfg_name):
     name = _PROFILE_FILES.get((kind, cfg_name))
+    if kind not in _KERNEL_SOURCES:
+        return None
     if name is None:
         return None
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", name)
@@ -201,31 +205,32 @@ def step_launches(cfg):
     return 1 + cfg.L * per_layer + proj(R)
 
 
-def run_ours(args):
-    from token_decode_b200 import build, bw, runtime, synth
-    ws_, rank, local = dist_env()
-    if ws_ > 1:
-        import torch.distributed as dist
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    torch.cuda.set_device(local)
-    build.build()
-    bw.lib()
-    cfg = synth.CONFIGS[args.config]
-    total = args.warmup + args.steps
-    # one generation = `cfg.steps` tokens from position ctx; longer runs start new generations
-    model = synth.make_model(cfg, "cuda", seed=rank)
-    kv = synth.make_kv(cfg, "cuda", seed=rank)
-    dm = runtime.DeviceModel(model, cfg.max_pages * synth.PAGE_TOKENS)
+HEADLINE = "7b"                                   # the workload the metric is quoted on
+SECONDARY = ("9b", "9b_b32", "27b", "moe")         # the other decode workloads, one line
+
+
+PERSISTENT = False   # --persistent: batch-1 dense steps as one persistent kernel (BW_STEP_PERSISTENT)
+
+
+def uses_persistent_step(cfg) -> bool:
+    """Whether the timed steps run as bw_decode_step's one-kernel persistent step."""
+    return PERSISTENT and cfg.B == 1 and cfg.n_experts == 0
+
+
+def measure(cfg, model, kv, dm, rank, world, local, steps, warmup, cpu_budget, stream, with_kernels=True):
+    """Timed decode of one workload: device-timed graph replays, the end-to-end
+    C-ABI loop with host tokens, the dominant kernel's roofline, and (rank 0,
+    one GPU) the CPU oracle on a bounded sample."""
+    from token_decode_b200 import bw, runtime, synth
     dkv = runtime.DeviceKV(kv)
     dec = runtime.Decoder(dm, dkv, cfg.B)
-    toks = synth.start_tokens(cfg, rank)
-    stream = torch.cuda.Stream()
+    toks = synth.start_tokens(cfg, rank)[: cfg.B]
 
     def reset():
         dec.tokens_in.copy_(toks)
         dec.pos.fill_(cfg.ctx)
 
+    pers = uses_persistent_step(cfg)
     G = 16  # steps per captured graph
     graphs = {}
 
@@ -233,10 +238,10 @@ def run_ours(args):
         if n not in graphs:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.stream(stream):
-                dec.step(advance=True, stream=stream)   # warm the launch path outside capture
+                dec.step(advance=True, stream=stream, persistent=pers)   # warm the launch path outside capture
                 with torch.cuda.graph(g, stream=stream):
                     for _ in range(n):
-                        dec.step(advance=True, stream=stream)
+                        dec.step(advance=True, stream=stream, persistent=pers)
             graphs[n] = g
         return graphs[n]
 
@@ -264,26 +269,17 @@ def run_ours(args):
                     graph_for(op).replay()
 
     torch.cuda.synchronize()
-    reset()
-    torch.cuda.synchronize()
-    warm_ops, p_after = plan(args.warmup, 0)
-    for op in warm_ops:
+    warm_ops, p_after = plan(warmup, 0)
+    timed_ops, _ = plan(steps, p_after)
+    for op in warm_ops + timed_ops:
         if op != "reset":
             graph_for(op)
-    # graph capture ran extra steps: restart the generation before warm-up
-    with torch.cuda.stream(stream):
-        reset()
-    run(warm_ops)
-    timed_ops, _ = plan(args.steps, p_after)
-    for op in timed_ops:
-        if op != "reset":
-            graph_for(op)
-    # the captures above advanced the state; rebuild the exact start of the timed region
+    # graph capture ran extra steps: rebuild the exact start, then warm up
     with torch.cuda.stream(stream):
         reset()
     run(warm_ops)
     stream.synchronize()
-    if ws_ > 1:
+    if world > 1:
         import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
@@ -294,114 +290,207 @@ def run_ours(args):
         e1.record(stream)
         e1.synchronize()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    ms_local = e0.elapsed_time(e1)
     err = bw.read_error(dec.ws, stream)
-    ms, value = job_throughput(ms, args.steps * cfg.B, ws_)
-    if ws_ > 1:
+    ms, value = job_throughput(ms_local, steps * cfg.B, world)
+    if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    ms_step = ms / args.steps
+    ms_step = ms / steps
+    graphs.clear()
 
-    # ---- end to end through the C ABI: host tokens in, host token out, every step
+    # ---- end to end through the C ABI: host tokens in, host tokens out, every step
     pin_in = torch.empty(cfg.B, dtype=torch.int32).pin_memory()
     pin_out = torch.empty(cfg.B, dtype=torch.int32).pin_memory()
     pin_in.copy_(toks)
-    n_e2e = min(args.steps, 64)
+    n_e2e = min(steps, 32)
     with torch.cuda.stream(stream):
         reset()
     stream.synchronize()
-    for _ in range(3):
+
+    def e2e_step():
         with torch.cuda.stream(stream):
             dec.tokens_in.copy_(pin_in, non_blocking=True)
-            dec.step(stream=stream)
+            dec.step(stream=stream, persistent=pers)
             dec.pos += 1
             pin_out.copy_(dec.tokens_out, non_blocking=True)
         stream.synchronize()
         pin_in.copy_(pin_out)
-    t0 = time.perf_counter()
+
+    for _ in range(3):
+        e2e_step()
     f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     f0.record(stream)
     for _ in range(n_e2e):
-        with torch.cuda.stream(stream):
-            dec.tokens_in.copy_(pin_in, non_blocking=True)
-            dec.step(stream=stream)
-            dec.pos += 1
-            pin_out.copy_(dec.tokens_out, non_blocking=True)
-        stream.synchronize()
-        pin_in.copy_(pin_out)
+        e2e_step()
     f1.record(stream)
     f1.synchronize()
-    e2e_ms, e2e_value = job_throughput(f0.elapsed_time(f1), n_e2e * cfg.B, ws_)
-
-    # ---- per kernel: every launch kind of the step over all layers, graph-replayed;
-    # the dominant one (gate/up GEMV, or the MoE FFN) gives the roofline figure
-    from token_decode_b200 import kernel_bench
-    kern = kernel_bench.run_all(dm, dkv, cfg.B, stream, cfg.ctx + cfg.steps // 2, reps=5)
-    dom = "gu" if "gu" in kern else "moe"
-    peak, peak_kind = _peaks()
-    achieved = kern[dom]["GBps"]
-    traffic = _ncu_traffic(dom, args.config)
+    _, e2e_value = job_throughput(f0.elapsed_time(f1), n_e2e * cfg.B, world)
 
     avg_ctx = cfg.ctx + (cfg.steps + 1) / 2
-    sb = step_bytes(cfg, model, avg_ctx, kern["moe"]["bytes_per_launch"] if cfg.n_experts else 0)
+    peak, peak_kind = _peaks()
+    kern, moe_bytes = {}, 0
+    if with_kernels and (cfg.n_experts or not uses_persistent_step(cfg)):
+        from token_decode_b200 import kernel_bench
+        kern = kernel_bench.run_all(dm, dkv, cfg.B, stream, cfg.ctx + cfg.steps // 2, reps=5)
+        moe_bytes = kern["moe"]["bytes_per_launch"] if cfg.n_experts else 0
+    sb = step_bytes(cfg, model, avg_ctx, moe_bytes)
     step_gbs = sb / (ms_step / 1000.0) / 1e9
-    launches_per_step = step_launches(cfg)
-
-    line = {
-        "metric": METRIC,
-        "value": round(value, 3),
-        "unit": "tok/s",
-        "n_gpus": ws_,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": round(ms_step, 5),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
+    if uses_persistent_step(cfg):
+        # one kernel per step: its algorithmic bytes are the step's
+        roof = {"bound": "hbm", "kernel": "step_persistent_kernel (the whole batch-1 step)",
+                "achieved": round(step_gbs, 1), "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": round(step_gbs / peak, 4), "traffic": _ncu_traffic("step", cfg.name),
+                "bytes_per_launch": int(sb), "avg_launch_us": round(ms_step * 1000.0, 2)}
+        launches = 1
+    else:
+        dom = max(kern, key=lambda k: kern[k]["us_per_launch"] * kern[k]["launches"])
+        roof = {"bound": "hbm", "kernel": KERNEL_NAMES.get(dom, dom), "achieved": kern[dom]["GBps"],
+                "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": round(kern[dom]["GBps"] / peak, 4),
+                "traffic": _ncu_traffic(dom, cfg.name), "bytes_per_launch": kern[dom]["bytes_per_launch"],
+                "avg_launch_us": kern[dom]["us_per_launch"]}
+        launches = step_launches(cfg)
+    entry = {
+        "workload": cfg.name, "value": round(value, 3), "unit": "tok/s", "batch": cfg.B,
+        "ms_per_step": round(ms_step, 5), "steps": steps,
+        "path": "persistent kernel (1 launch per step)" if uses_persistent_step(cfg)
+                else "kernel chain (%d launches per step)" % step_launches(cfg),
         "dtype": "q4_0 weights, fp32 accumulate, fp16 KV" if cfg.fmt == synth.FMT_Q4_0 else
                  "nvfp4 weights, fp32 accumulate, fp16 KV",
-        "data": "synthetic (seeded random-init weights N(0,0.02) quantized; N(0,1) fp16 KV context)",
-        "config": dict(workload_config(cfg, ws_),
-                       l2="inputs larger than L2 (each step streams ~%.2f GB)" % (sb / 1e9)),
-        "timing": "CUDA graphs of %d steps, on-device token/position advance; CUDA events on the launching "
-                  "stream" % G,
         "hbm_gbs_step": round(step_gbs, 1),
         "roofline_step_frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4),
         "roofline_step_frac_of_measured": round(step_gbs / peak, 4),
         "bytes_per_step": int(sb),
-        "roofline": {"bound": "hbm",
-                     "kernel": "gemv_kernel (fused RMSNorm + gate/up + SiLU gate)" if dom == "gu"
-                               else "MoE FFN (route + grouped expert GEMVs + combine)",
-                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "bytes_per_launch": kern[dom]["bytes_per_launch"],
-                     "avg_launch_us": kern[dom]["us_per_launch"]},
-        "kernels": kern,
+        "roofline": roof,
         "e2e": {"value": round(e2e_value, 3), "unit": "tok/s", "steps": n_e2e,
                 "h2d_bytes_per_step": 4 * cfg.B, "d2h_bytes_per_step": 4 * cfg.B,
-                "path": "bw_decode_step via the C ABI, pinned host token in/out, sync each step"},
-        "gpu_launches": launches_per_step * args.steps,
+                "path": "bw_decode_step via the C ABI, pinned host tokens in/out, sync each step"},
+        "gpu_launches": launches * steps,
         "device_error_word": err,
         "clocks": clk.summary(),
     }
-    if rank == 0 and ws_ == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(cfg, model, kv, toks, budget_s=args.cpu_budget)
+    if kern:
+        entry["kernels"] = kern
+    if cfg.verify_k:
+        entry["verify_pass"] = verify_pass(cfg, dm, kv, stream, ms_step)
+    if rank == 0 and world == 1 and cpu_budget > 0:
+        entry["cpu_baseline"] = cpu_baseline(cfg, model, kv, toks, budget_s=cpu_budget)
+    del dec, dkv
+    return entry
+
+
+def verify_pass(cfg, dm, kv, stream, ms_plain):
+    """Device time of one speculative-verify pass (the last token plus K drafts
+    as K+1 rows of one step, bw_decode_step with n_rows = K+1) against a plain step."""
+    from token_decode_b200 import bw, runtime, synth
+    R = cfg.verify_k + 1
+    dkv = runtime.DeviceKV(kv.clone())
+    dec = runtime.Decoder(dm, dkv, 1, n_rows=R)
+    t0 = synth.start_tokens(cfg, 0)[:1].tolist()
+    rows = t0 + synth.draft_tokens(cfg, cfg.verify_k, 0)[0].tolist()
+    dec.tokens_in.copy_(torch.tensor(rows, dtype=torch.int32))
+    dec.pos.fill_(cfg.ctx)
+    n = 8
+    with torch.cuda.stream(stream):
+        dec.step(stream=stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(n):
+                dec.step(stream=stream)
+        g.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / n
+    err = bw.read_error(dec.ws, stream)
+    del g
+    return {"rows": R, "drafts": cfg.verify_k, "ms_per_pass": round(ms, 4),
+            "vs_plain_step": round(ms / ms_plain, 3), "device_error_word": err,
+            "path": "kernel chain, %d rows per projection" % R}
+
+
+KERNEL_NAMES = {"gu": "gemv_kernel (fused RMSNorm + gate/up + SiLU gate)", "down": "gemv_kernel (down + residual)",
+                "attn": "attn_kernel (paged GQA decode attention)", "qkv": "gemv_kernel (RMSNorm + QKV)",
+                "o": "gemv_kernel (O + residual)", "lm_head": "gemv_kernel (LM head + argmax)",
+                "moe": "MoE FFN (route + grouped expert GEMVs + combine)"}
+
+
+def run_ours(args):
+    from token_decode_b200 import build, bw, runtime, synth
+    ws_, rank, local = dist_env()
+    if ws_ > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    build.build()
+    bw.lib()
+    stream = torch.cuda.Stream()
+    names = [args.config] + ([] if args.only else [n for n in SECONDARY if n != args.config])
+    entries = {}
+    cache = {}
+    for i, name in enumerate(names):
+        cfg = synth.CONFIGS[name]
+        key = (cfg.L, cfg.H, cfg.nq, cfg.nkv, cfg.hd, cfg.F, cfg.V, cfg.fmt, cfg.n_experts)
+        if key not in cache:
+            cache.clear()
+            torch.cuda.empty_cache()
+            model = synth.make_model(cfg, "cuda", seed=rank)
+            cache[key] = (model, runtime.DeviceModel(model, cfg.max_pages * synth.PAGE_TOKENS))
+        model, dm = cache[key]
+        if dm.c.rope_max_pos < cfg.max_pages * synth.PAGE_TOKENS:
+            dm = runtime.DeviceModel(model, cfg.max_pages * synth.PAGE_TOKENS)
+            cache[key] = (model, dm)
+        kv = synth.make_kv(cfg, "cuda", seed=rank)
+        head = i == 0
+        steps = args.steps if head else max(4, min(args.steps, 16))
+        entries[name] = measure(cfg, model, kv, dm, rank, ws_, local, steps, args.warmup,
+                                0 if args.no_cpu_baseline else (args.cpu_budget if head else args.cpu_budget / 3),
+                                stream)
+        del kv
+    h = entries[names[0]]
+    hcfg = synth.CONFIGS[names[0]]
+    line = {
+        "metric": METRIC,
+        "value": h["value"],
+        "unit": "tok/s",
+        "n_gpus": ws_,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": h["ms_per_step"],
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": h["dtype"],
+        "data": "synthetic (seeded random-init weights N(0,0.02) quantized; N(0,1) fp16 KV context)",
+        "config": workload_config(hcfg, ws_),
+        "l2": "inputs larger than L2: every step streams the whole model (%.2f GB for %s)" % (
+            h["bytes_per_step"] / 1e9, hcfg.name),
+        "timing": "CUDA graphs of 16 steps, on-device token/position advance; CUDA events on the launching stream",
+    }
+    for k in ("path", "hbm_gbs_step", "roofline_step_frac_of_8tbs", "roofline_step_frac_of_measured",
+              "bytes_per_step", "roofline", "kernels", "e2e", "gpu_launches", "device_error_word", "clocks",
+              "cpu_baseline"):
+        if k in h:
+            line[k] = h[k]
+    line["configs"] = {n: e for n, e in entries.items() if n != names[0]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_ > 1:
         import torch.distributed as dist
-        graphs.clear()
         dist.barrier()
         dist.destroy_process_group()
 
 
-def _oracle_setup(cfg, model, kv):
+def _oracle_setup(cfg, model, kv, n_layers=None):
     import oracle
     oracle.build()
-    return oracle, oracle.Model(model), oracle.KV(kv)
+    return oracle, oracle.Model(model, n_layers=n_layers), oracle.KV(kv, layers=n_layers)
 
 
-def _oracle_token_seconds(oracle, om, okv, cfg, tok, n_layer_samples, t_budget):
+def _oracle_token_seconds(oracle, om, okv, cfg, tok, n_layer_samples, t_budget, n_host_layers):
     """Seconds of one full oracle decode token, estimated from a bounded sample:
     the head alone (embedding + final norm + LM head) and single layers."""
     t = time.perf_counter()
@@ -409,7 +498,7 @@ def _oracle_token_seconds(oracle, om, okv, cfg, tok, n_layer_samples, t_budget):
     t_head = time.perf_counter() - t
     per_layer = []
     for i in range(n_layer_samples):
-        l = (i * 7) % cfg.L
+        l = (i * 7) % n_host_layers
         t = time.perf_counter()
         oracle.decode_token(om, okv, 0, tok, cfg.ctx, layers=(l, l + 1))
         per_layer.append(max(0.0, time.perf_counter() - t - t_head))
@@ -418,13 +507,17 @@ def _oracle_token_seconds(oracle, om, okv, cfg, tok, n_layer_samples, t_budget):
     return t_head + cfg.L * statistics.mean(per_layer), t_head, per_layer
 
 
-def cpu_baseline(cfg, model, kv, toks, budget_s=20.0):
-    oracle, om, okv = _oracle_setup(cfg, model, kv)
-    tok_s, t_head, per_layer = _oracle_token_seconds(oracle, om, okv, cfg, int(toks[0]), 64, budget_s)
-    return {"value": round(cfg.B / tok_s, 5), "unit": "tok/s", "cores": 1, "kind": "oracle",
+def cpu_baseline(cfg, model, kv, toks, budget_s=20.0, host_layers=4):
+    """The oracle as it stands, one host thread, on a bounded sample of one
+    sequence's decode token (its first host_layers layers are copied to the host)."""
+    nl = min(cfg.L, host_layers)
+    oracle, om, okv = _oracle_setup(cfg, model, kv, nl)
+    tok_s, t_head, per_layer = _oracle_token_seconds(oracle, om, okv, cfg, int(toks[0]), 64, budget_s, nl)
+    return {"value": round(1.0 / tok_s, 5), "unit": "tok/s", "cores": 1, "kind": "oracle",
             "sample": f"embedding + LM head once ({t_head:.2f} s) and {len(per_layer)} single "
-                      f"layers of the {cfg.name} step at ctx {cfg.ctx}, scaled to {cfg.L} layers "
-                      f"(one token = {tok_s:.1f} s), single-threaded fp32 C",
+                      f"layers of one {cfg.name} sequence at ctx {cfg.ctx}, scaled to {cfg.L} layers "
+                      f"(one token = {tok_s:.1f} s; the sequences of a batch run one after another), "
+                      f"single-threaded fp32 C",
             "host_cores_total": os.cpu_count()}
 
 
@@ -479,9 +572,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--only", action="store_true", help="measure only --config (no other workloads)")
+    ap.add_argument("--persistent", action="store_true",
+                    help="batch-1 dense steps as one persistent kernel (BW_STEP_PERSISTENT)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    global PERSISTENT
+    PERSISTENT = args.persistent
     if args.impl == "reference":
         run_reference(args)
     else:

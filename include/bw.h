@@ -111,7 +111,7 @@ typedef int bw_status;
 /* decode-step flags */
 #define BW_STEP_ADVANCE 1u    /* after the step: tokens_in <- tokens_out, pos += n_rows */
 #define BW_STEP_VALIDATE_ONLY 2u  /* validate descriptors and arguments on the host; launch nothing */
-#define BW_STEP_LAYERWISE 4u  /* run the chain of per-layer kernels even where the persistent step applies */
+#define BW_STEP_PERSISTENT 4u /* batch-1 dense step as one persistent kernel (else: the per-layer chain) */
 #define BW_MAX_VERIFY_ROWS 8  /* n_rows limit of a verify pass (the last token + up to 7 drafts) */
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -314,12 +314,12 @@ bw_status bw_moe_route_gemv(const struct bw_model *m, const struct bw_layer *ly,
 size_t bw_moe_workspace_bytes(const struct bw_model *m, int R);
 
 /* One greedy decode step for B sequences of n_rows tokens each.
- * A batch-1 step (B == 1, n_rows == 1) of a dense model runs as ONE persistent
- * cooperative kernel with a CTA per SM (streaming every layer's weights and KV
- * pages through a shared-memory ring, phases ordered by device-side counters);
- * other steps, and any step with BW_STEP_LAYERWISE, run as a chain of kernels
- * (about five per layer).  Both give the same results within the tolerance of
- * fp32 summation order.
+ * The step runs as a chain of kernels (about five per layer).  With
+ * BW_STEP_PERSISTENT a batch-1 step (B == 1, n_rows == 1) of a dense model runs
+ * instead as ONE persistent cooperative kernel with a CTA per SM (streaming
+ * every layer's weights and KV pages through a shared-memory ring, phases
+ * ordered by device-side counters); both give the same results within the
+ * tolerance of fp32 summation order.
  *   tokens_in: int32 [B*n_rows]; pos: int32 [B] (position of each sequence's
  *   first row); tokens_out: int32 [B*n_rows] (argmax after each row);
  *   logits: fp32 [B*n_rows][V] or NULL.

@@ -361,8 +361,8 @@ def test_persistent_step_matches_layerwise_chain_and_oracle(name, fmt, layers):
     cfg = synth.CONFIGS[name].with_(fmt=fmt, L=layers)
     model, kv, om, okv, dm, dkv = _setup(cfg, seed=31, n_layers=layers)
     tok = int(synth.start_tokens(cfg, 31)[0])
-    lg_p, tok_p, kv_p, hid_p = _step_once(dm, kv, tok, cfg.ctx)
-    lg_c, tok_c, kv_c, hid_c = _step_once(dm, kv, tok, cfg.ctx, flags=bw.STEP_LAYERWISE)
+    lg_p, tok_p, kv_p, hid_p = _step_once(dm, kv, tok, cfg.ctx, flags=bw.STEP_PERSISTENT)
+    lg_c, tok_c, kv_c, hid_c = _step_once(dm, kv, tok, cfg.ctx)
     assert rel_err(lg_p, lg_c) < 1e-4
     assert rel_err(hid_p, hid_c) < 1e-4
     res = oracle.decode_token(om, okv, 0, tok, cfg.ctx, want_hidden=True)
@@ -382,15 +382,15 @@ def test_persistent_step_graph_replay_and_determinism():
     model, kv, om, okv, dm, dkv = _setup(cfg, seed=12)
     kv0 = kv.clone()
     tok = int(synth.start_tokens(cfg, 12)[0])
-    a = _step_once(dm, kv0, tok, cfg.ctx)
-    b = _step_once(dm, kv0, tok, cfg.ctx)
+    a = _step_once(dm, kv0, tok, cfg.ctx, flags=bw.STEP_PERSISTENT)
+    b = _step_once(dm, kv0, tok, cfg.ctx, flags=bw.STEP_PERSISTENT)
     assert np.array_equal(a[0], b[0]) and a[1] == b[1]
     dec = runtime.Decoder(dm, dkv, 1)
     dec.tokens_in.fill_(tok)
     dec.pos.fill_(cfg.ctx)
     eager = []
     for _ in range(6):
-        dec.step(advance=True)
+        dec.step(advance=True, persistent=True)
         eager.append(int(dec.tokens_out[0]))
     assert bw.read_error(dec.ws) == 0
     dkv2 = runtime.DeviceKV(kv0.clone())
@@ -404,7 +404,7 @@ def test_persistent_step_graph_replay_and_determinism():
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
             for i in range(6):
-                dec2.step(advance=True, stream=s)
+                dec2.step(advance=True, stream=s, persistent=True)
                 outs[i].copy_(dec2.tokens_out[0])
     torch.cuda.current_stream().wait_stream(s)
     g.replay()
@@ -432,10 +432,10 @@ def test_persistent_step_bad_page_sets_error():
     dec.tokens_in.fill_(1)
     dec.pos.fill_(cfg.ctx)
     lg = torch.empty((1, cfg.V), device="cuda")
-    dec.step(logits=lg)
+    dec.step(logits=lg, persistent=True)
     assert bw.read_error(dec.ws) & bw.DEVERR_BAD_PAGE
     assert torch.isfinite(lg).all()
     # the workspace is usable again: a clean step after restoring the entry
     dkv.page_table[0, 3] = int(synth.page_table(cfg, "cuda", 13)[0, 3])
-    dec.step(logits=lg)
+    dec.step(logits=lg, persistent=True)
     assert bw.read_error(dec.ws) == 0

@@ -21,7 +21,7 @@ FMT_Q4_0, FMT_NVFP4 = 0, 1
 GEMV_RMSNORM, GEMV_RESIDUAL, GEMV_SILU_GATE, GEMV_ARGMAX = 1, 2, 4, 8
 STEP_ADVANCE = 1
 STEP_VALIDATE_ONLY = 2
-STEP_LAYERWISE = 4
+STEP_PERSISTENT = 4
 MAX_VERIFY_ROWS = 8
 
 # every symbol include/bw.h declares (checked by the CPU test-suite)

@@ -11,8 +11,8 @@
 // feeds the next step (token in, position + 1), so a graph of many steps
 // decodes autoregressively without the host.
 //
-// A batch-1 step of a dense model runs instead as one persistent kernel
-// (step_persistent.cu) unless BW_STEP_LAYERWISE asks for the chain.
+// With BW_STEP_PERSISTENT, a batch-1 step of a dense model runs instead as one
+// persistent kernel (step_persistent.cu).
 //
 // The deep-dive page (10100.com), section 4, describes the engine facade that
 // exposes prefill and decode; this is its decode call on device memory.
@@ -179,7 +179,7 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
     if (s != BW_OK || (flags & BW_STEP_VALIDATE_ONLY)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int R = B * n_rows;
-    if (bf.pk && !(flags & BW_STEP_LAYERWISE))
+    if (bf.pk && (flags & BW_STEP_PERSISTENT))
         return persistent_step_launch(m, kv, tokens_in, pos, tokens_out, logits, (flags & BW_STEP_ADVANCE) != 0,
                                       bf.x, bf.qkv, bf.attn, bf.act, bf.pk, bf.kern, st);
 

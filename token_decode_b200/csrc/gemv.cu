@@ -140,7 +140,7 @@ __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, 
 
 template <int FMT, int M>
 __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(const GemvParams p) {
-    extern __shared__ __align__(128) unsigned char gv_smem[];
+    extern __shared__ __align__(1024) unsigned char gv_smem[];
     const int nst = p.nst;
     unsigned char *stages = gv_smem;                                                     // nst x 36 KB
     float *xs = reinterpret_cast<float *>(gv_smem + static_cast<size_t>(nst) * GV_STAGE_BYTES);  // [M][CS][32]
@@ -179,9 +179,10 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
     if (warp == GV_CW) {
         // ---- producer: constant weights only, so no dependency wait
         if (lane == 0) {
-            for (int step = 0; step < n_steps; step++) {
-                const int s = step % nst;
-                if (step >= nst) mbar_wait(&empty[s], static_cast<uint32_t>((step / nst - 1) & 1), p.err);
+            RingPos rp = {0, 0u};
+            for (int step = 0; step < n_steps; step++, ring_next(rp, nst)) {
+                const int s = rp.s;
+                if (step >= nst) mbar_wait(&empty[s], rp.ph ^ 1u, p.err);
                 const int item = step / T, kt = kt0 + (step - item * T);
                 const int rb = j0 + item * p.per_slice;
                 const size_t tile = static_cast<size_t>(rb) * p.KT + kt;
@@ -253,17 +254,17 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
         besti[m] = 0x7fffffff;
     }
 
-    int step = 0;
+    const ChunkLane cn = chunk_lane(warp, lane);
+    RingPos rp = {0, 0u};
     for (int item = 0; item < n_items; item++) {
         const int rb = j0 + item * p.per_slice;
         const int rg = rb * (GV_TR / 8) + 2 * warp + (lane >> 4);
-        for (int kt = 0; kt < T; kt++, step++) {
-            const int s = step % nst;
-            mbar_wait(&full[s], static_cast<uint32_t>((step / nst) & 1), p.err);
+        for (int kt = 0; kt < T; kt++, ring_next(rp, nst)) {
+            const int s = rp.s;
+            mbar_wait(&full[s], rp.ph, p.err);
             const int cl = kt * GV_TC + (lane & 15);
             if (cl < nc)
-                stage_chunk<FMT, M>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, warp, lane, xs_a, ct_a,
-                                    cl, CS, acc);
+                stage_chunk<FMT, M>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, cn, xs_a, ct_a, cl, CS, acc);
             __syncwarp();
             if (lane == 0) mbar_arrive_relaxed(&empty[s]);
         }

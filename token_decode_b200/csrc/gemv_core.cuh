@@ -168,84 +168,129 @@ __device__ __forceinline__ uint32_t u4_get(const uint4 &v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
+// 64-bit helpers: the f32x2 FMA takes register pairs; building every operand
+// pair in one 64-bit register (masks applied to {v, v}, activations loaded as
+// 64-bit words, accumulators kept as pairs) leaves nothing to re-pair.
+__device__ __forceinline__ uint64_t and_pair(uint32_t v, uint64_t mask) {
+    uint64_t r;
+    asm("{\n\t.reg .b64 vv;\n\tmov.b64 vv, {%1, %1};\n\tand.b64 %0, vv, %2;\n\t}" : "=l"(r) : "r"(v), "l"(mask));
+    return r;
+}
+__device__ __forceinline__ uint64_t ffma2_64(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ void lds_2x64(uint32_t a, uint64_t &lo, uint64_t &hi) {
+    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];" : "=l"(lo), "=l"(hi) : "r"(a));
+}
+__device__ __forceinline__ uint64_t pair_f(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float pair_sum(uint64_t p) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+    return lo + hi;
+}
+// E2M1 codes of one byte (low nibble -> low half) as an fp32 pair (exact)
+__device__ __forceinline__ uint64_t e2m1x2_pair(uint32_t byte) {
+    uint64_t r;
+    asm("{\n\t.reg .b8 b;\n\t.reg .b32 p;\n\t.reg .b16 h0, h1;\n\t.reg .f32 f0, f1;\n\t"
+        "cvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 p, b;\n\tmov.b32 {h0, h1}, p;\n\t"
+        "cvt.f32.f16 f0, h0;\n\tcvt.f32.f16 f1, h1;\n\tmov.b64 %0, {f0, f1};\n\t}"
+        : "=l"(r) : "r"(byte));
+    return r;
+}
+
 // acc[r][m] += dot(row r of this chunk, x'[m] of this chunk).
 //   w: 8 rows x 16 bytes of codes + 16 bytes of scales (this lane's chunk)
 //   xs_a: shared address of the staged activations [M][chunk_stride][32]
+//         (128-byte aligned); x7 = 16 * (cl & 7), the chunk's granule swizzle,
+//         so granule g of a chunk sits at (chunk address + x7) ^ (16 g)
 //   ctv[m]: the chunk's -8 * 2^-48 * sum(x) term (Q4_0)
 template <int FMT, int M>
-__device__ __forceinline__ void compute_chunk(const uint4 (&w)[9], uint32_t xs_a, const float (&ctv)[M], int cl,
-                                              int chunk_stride, float (&acc)[8][M]) {
+__device__ __forceinline__ void compute_chunk(const uint4 (&w)[9], uint32_t xs_a, uint32_t x7, const float (&ctv)[M],
+                                              int cl, int chunk_stride, float (&acc)[8][M]) {
     if constexpr (FMT == BW_FMT_Q4_0) {
-        float2 bd[8][M];
+        uint64_t bd[8][M];
 #pragma unroll
-        for (int r = 0; r < 8; r++)
+        for (int m = 0; m < M; m++) {
+            const uint64_t init = pair_f(ctv[m], 0.0f);
 #pragma unroll
-            for (int m = 0; m < M; m++) bd[r][m] = make_float2(ctv[m], 0.0f);
+            for (int r = 0; r < 8; r++) bd[r][m] = init;
+        }
 #pragma unroll
         for (int wd = 0; wd < 4; wd++) {
-            float4 xa[M], xb[M];
+            uint64_t x01[M], x23[M], x45[M], x67[M];
 #pragma unroll
             for (int m = 0; m < M; m++) {
-                const uint32_t xc = xs_a + 128u * static_cast<uint32_t>(m * chunk_stride + cl);
-                xa[m] = lds_f4(gran_addr(xc, 2 * wd, cl));
-                xb[m] = lds_f4(gran_addr(xc, 2 * wd + 1, cl));
+                const uint32_t xc = xs_a + 128u * static_cast<uint32_t>(m * chunk_stride + cl) + x7;
+                lds_2x64(xc ^ (32u * wd), x01[m], x23[m]);
+                lds_2x64(xc ^ (32u * wd + 16u), x45[m], x67[m]);
             }
 #pragma unroll
             for (int r = 0; r < 8; r++) {
                 const uint32_t v = u4_get(w[r], wd);
                 const uint32_t h = v >> 16;
-                const float2 f01 = make_float2(__uint_as_float(v & 0xfu), __uint_as_float(v & 0xf0u));
-                const float2 f23 = make_float2(__uint_as_float(v & 0xf00u), __uint_as_float(v & 0xf000u));
-                const float2 f45 = make_float2(__uint_as_float(h & 0xfu), __uint_as_float(h & 0xf0u));
-                const float2 f67 = make_float2(__uint_as_float(h & 0xf00u), __uint_as_float(h & 0xf000u));
+                // nibble slots 0..3 of each 16-bit half, masked in place: (slot 0, slot 1), (slot 2, slot 3)
+                const uint64_t f01 = and_pair(v, 0x000000F00000000Full);
+                const uint64_t f23 = and_pair(v, 0x0000F00000000F00ull);
+                const uint64_t f45 = and_pair(h, 0x000000F00000000Full);
+                const uint64_t f67 = and_pair(h, 0x0000F00000000F00ull);
 #pragma unroll
                 for (int m = 0; m < M; m++) {
-                    float2 b = bd[r][m];
-                    b = ffma2(f01, make_float2(xa[m].x, xa[m].y), b);
-                    b = ffma2(f23, make_float2(xa[m].z, xa[m].w), b);
-                    b = ffma2(f45, make_float2(xb[m].x, xb[m].y), b);
-                    b = ffma2(f67, make_float2(xb[m].z, xb[m].w), b);
+                    uint64_t b = bd[r][m];
+                    b = ffma2_64(f01, x01[m], b);
+                    b = ffma2_64(f23, x23[m], b);
+                    b = ffma2_64(f45, x45[m], b);
+                    b = ffma2_64(f67, x67[m], b);
                     bd[r][m] = b;
                 }
             }
         }
 #pragma unroll
-        for (int r = 0; r < 8; r++) {
-            const float d = half_bits_to_f((u4_get(w[8], r >> 1) >> (16 * (r & 1))) & 0xffffu);
+        for (int r2 = 0; r2 < 4; r2++) {
+            const float2 d = __half22float2(*reinterpret_cast<const __half2 *>(&(r2 == 0 ? w[8].x : r2 == 1 ? w[8].y
+                                                                                  : r2 == 2 ? w[8].z : w[8].w)));
 #pragma unroll
-            for (int m = 0; m < M; m++) acc[r][m] = fma_rn(d, bd[r][m].x + bd[r][m].y, acc[r][m]);
+            for (int m = 0; m < M; m++) {
+                acc[2 * r2][m] = fma_rn(d.x, pair_sum(bd[2 * r2][m]), acc[2 * r2][m]);
+                acc[2 * r2 + 1][m] = fma_rn(d.y, pair_sum(bd[2 * r2 + 1][m]), acc[2 * r2 + 1][m]);
+            }
         }
     } else {
 #pragma unroll
         for (int half = 0; half < 2; half++) {
-            float2 bd[8][M];
+            uint64_t bd[8][M];
 #pragma unroll
             for (int r = 0; r < 8; r++)
 #pragma unroll
-                for (int m = 0; m < M; m++) bd[r][m] = make_float2(0.0f, 0.0f);
+                for (int m = 0; m < M; m++) bd[r][m] = 0ull;
 #pragma unroll
             for (int wd = 2 * half; wd < 2 * half + 2; wd++) {
-                float4 xa[M], xb[M];
+                uint64_t x01[M], x23[M], x45[M], x67[M];
 #pragma unroll
                 for (int m = 0; m < M; m++) {
-                    const uint32_t xc = xs_a + 128u * static_cast<uint32_t>(m * chunk_stride + cl);
-                    xa[m] = lds_f4(gran_addr(xc, 2 * wd, cl));
-                    xb[m] = lds_f4(gran_addr(xc, 2 * wd + 1, cl));
+                    const uint32_t xc = xs_a + 128u * static_cast<uint32_t>(m * chunk_stride + cl) + x7;
+                    lds_2x64(xc ^ (32u * wd), x01[m], x23[m]);
+                    lds_2x64(xc ^ (32u * wd + 16u), x45[m], x67[m]);
                 }
 #pragma unroll
                 for (int r = 0; r < 8; r++) {
                     const uint32_t v = u4_get(w[r], wd);
-                    const float2 e0 = e2m1x2_to_f2(v & 0xffu);
-                    const float2 e1 = e2m1x2_to_f2((v >> 8) & 0xffu);
-                    const float2 e2 = e2m1x2_to_f2((v >> 16) & 0xffu);
-                    const float2 e3 = e2m1x2_to_f2(v >> 24);
+                    const uint64_t e0 = e2m1x2_pair(v);
+                    const uint64_t e1 = e2m1x2_pair(v >> 8);
+                    const uint64_t e2 = e2m1x2_pair(v >> 16);
+                    const uint64_t e3 = e2m1x2_pair(v >> 24);
 #pragma unroll
                     for (int m = 0; m < M; m++) {
-                        float2 b = bd[r][m];
-                        b = ffma2(e0, make_float2(xa[m].x, xa[m].y), b);
-                        b = ffma2(e1, make_float2(xa[m].z, xa[m].w), b);
-                        b = ffma2(e2, make_float2(xb[m].x, xb[m].y), b);
-                        b = ffma2(e3, make_float2(xb[m].z, xb[m].w), b);
+                        uint64_t b = bd[r][m];
+                        b = ffma2_64(e0, x01[m], b);
+                        b = ffma2_64(e1, x23[m], b);
+                        b = ffma2_64(e2, x45[m], b);
+                        b = ffma2_64(e3, x67[m], b);
                         bd[r][m] = b;
                     }
                 }
@@ -256,27 +301,52 @@ __device__ __forceinline__ void compute_chunk(const uint4 (&w)[9], uint32_t xs_a
                 const float2 sc = e4m3x2_to_f2(two);
                 const float s = half ? sc.y : sc.x;
 #pragma unroll
-                for (int m = 0; m < M; m++) acc[r][m] = fma_rn(s, bd[r][m].x + bd[r][m].y, acc[r][m]);
+                for (int m = 0; m < M; m++) acc[r][m] = fma_rn(s, pair_sum(bd[r][m]), acc[r][m]);
             }
         }
     }
 }
 
-// One lane's chunk of one stage.  Warp w owns row groups 2w (lanes 0..15)
-// and 2w+1 (lanes 16..31) of the 128-row tile; lane & 15 is the chunk.
+// The lane-constant part of a stage's shared-memory addresses (callers hoist
+// it out of their stage loops).  Warp w owns row groups 2w (lanes 0..15) and
+// 2w+1 (lanes 16..31) of the 128-row tile; lane & 15 is the chunk.
+struct ChunkLane {
+    uint32_t w;    // row 8g's chunk c before the XOR swizzle: g * 2048 + c * 16
+    uint32_t s;    // the chunk's scales: 32 KB + g * 256 + c * 16
+    uint32_t x7;   // 16 * (c & 7), the activation granule swizzle
+};
+__device__ __forceinline__ ChunkLane chunk_lane(int warp, int lane) {
+    const uint32_t g = 2 * warp + (lane >> 4), c = lane & 15;
+    return {g * (8u * GV_TC * 16u) + c * 16u, GV_NIB_BYTES + g * (GV_TC * 16u) + c * 16u, 16u * (c & 7u)};
+}
+
+// Ring position of a stage stream: slot and the parity of its full barrier.
+struct RingPos {
+    int s;
+    uint32_t ph;
+};
+__device__ __forceinline__ void ring_next(RingPos &r, int nst) {
+    if (++r.s == nst) {
+        r.s = 0;
+        r.ph ^= 1u;
+    }
+}
+
+// One lane's chunk of one stage (stage_a 256-byte aligned, so row r's slot
+// c ^ r of row group g sits at (stage_a + g*2048 + c*16) ^ (16 r), + 256 r).
 template <int FMT, int M>
-__device__ __forceinline__ void stage_chunk(uint32_t stage_a, int warp, int lane, uint32_t xs_a, uint32_t ct_a,
+__device__ __forceinline__ void stage_chunk(uint32_t stage_a, const ChunkLane &cn, uint32_t xs_a, uint32_t ct_a,
                                             int cl, int chunk_stride, float (&acc)[8][M]) {
-    const int g = 2 * warp + (lane >> 4), c = lane & 15;
+    const uint32_t wb = stage_a + cn.w;
     uint4 w[9];
 #pragma unroll
-    for (int r = 0; r < 8; r++) w[r] = lds_u4(stage_a + (g * 8 + r) * (GV_TC * 16) + ((c ^ r) * 16));
-    w[8] = lds_u4(stage_a + GV_NIB_BYTES + g * (GV_TC * 16) + c * 16);
+    for (int r = 0; r < 8; r++) w[r] = lds_u4((wb ^ (16u * r)) + 256u * r);
+    w[8] = lds_u4(stage_a + cn.s);
     float ctv[M];
 #pragma unroll
     for (int m = 0; m < M; m++)
         ctv[m] = (FMT == BW_FMT_Q4_0) ? lds_f(ct_a + 4u * static_cast<uint32_t>(m * chunk_stride + cl)) : 0.0f;
-    compute_chunk<FMT, M>(w, xs_a, ctv, cl, chunk_stride, acc);
+    compute_chunk<FMT, M>(w, xs_a, cn.x7, ctv, cl, chunk_stride, acc);
 }
 
 // Reduce acc[8][M] over each half-warp (16 lanes, one row group each).

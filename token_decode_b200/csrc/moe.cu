@@ -285,13 +285,14 @@ __device__ __forceinline__ void moe_item_rows(const GroupedParams &p, const MoeI
         for (int r = 0; r < 8; r++)
 #pragma unroll
             for (int m = 0; m < MR; m++) acc[r][m] = 0.0f;
+        const ChunkLane cn = chunk_lane(warp, lane);
         for (int kt = 0; kt < T; kt++, step++) {
             const int s = step % nst;
             mbar_wait(&full[s], static_cast<uint32_t>((step / nst) & 1), p.err);
             const int cl = kt * GV_TC + (lane & 15);
             if (cl < nc)
-                stage_chunk<FMT, MR>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, warp, lane, xs_a, ct_a, cl,
-                                     CS, acc);
+                stage_chunk<FMT, MR>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, cn, xs_a, ct_a, cl, CS,
+                                     acc);
             __syncwarp();
             if (lane == 0) mbar_arrive_relaxed(&empty[s]);
         }
@@ -331,7 +332,7 @@ __device__ __forceinline__ void moe_item_rows(const GroupedParams &p, const MoeI
 template <int FMT>
 __global__ void __launch_bounds__(GV_THREADS, 1) moe_grouped_gemv_kernel(const GroupedParams p) {
     constexpr int M = MOE_M;
-    extern __shared__ __align__(128) unsigned char gg_smem[];
+    extern __shared__ __align__(1024) unsigned char gg_smem[];
     const int nst = p.nst;
     const int CS = p.KT * GV_TC;
     unsigned char *stages = gg_smem;

@@ -212,20 +212,35 @@ __device__ __forceinline__ void pk_signal(const PkParams &p, unsigned which, uin
 
 // ------------------------------------------------------------- producer
 
+// Position in the CTA's stage stream: index, ring slot, parity of the slot's
+// full barrier (advanced incrementally: no division by the ring depth).
+struct PkStream {
+    uint32_t i;
+    int s;
+    uint32_t ph;
+    __device__ __forceinline__ void adv(int nst) {
+        i++;
+        if (++s == nst) {
+            s = 0;
+            ph ^= 1u;
+        }
+    }
+    __device__ __forceinline__ void skip(int n, int nst) {
+        for (int k = 0; k < n; k++) adv(nst);
+    }
+};
+
 struct PkRing {
     unsigned char *stages;
     uint64_t *full, *empty;
     int nst;
 };
 
-__device__ __forceinline__ bool pk_slot(const PkParams &p, const PkRing &r, uint32_t i, unsigned char *&dst,
+__device__ __forceinline__ bool pk_slot(const PkParams &p, const PkRing &r, const PkStream &st, unsigned char *&dst,
                                         uint64_t *&bar) {
-    const int s = static_cast<int>(i % r.nst);
-    if (i >= static_cast<uint32_t>(r.nst) &&
-        !pk_mbar_wait(p, &r.empty[s], static_cast<uint32_t>((i / r.nst - 1) & 1)))
-        return false;
-    dst = r.stages + static_cast<size_t>(s) * GV_STAGE_BYTES;
-    bar = &r.full[s];
+    if (st.i >= static_cast<uint32_t>(r.nst) && !pk_mbar_wait(p, &r.empty[st.s], st.ph ^ 1u)) return false;
+    dst = r.stages + static_cast<size_t>(st.s) * GV_STAGE_BYTES;
+    bar = &r.full[st.s];
     return true;
 }
 
@@ -245,7 +260,7 @@ __device__ __forceinline__ bool pk_att_range(const PkParams &p, int c, int pos, 
 __device__ __forceinline__ int pk_pages_per_stage(int hd) { return static_cast<int>(32768 / (2 * 16 * hd * 2)); }
 
 __device__ void pk_producer(const PkParams &p, const PkRing &r, int c, int G, int lane, int pos) {
-    uint32_t stream = 0;
+    PkStream stream = {0u, 0, 0u};
     bool live = true;
     const int PB = 16 * p.hd * 2;
     const int PPS = pk_pages_per_stage(p.hd);
@@ -273,19 +288,19 @@ __device__ void pk_producer(const PkParams &p, const PkRing &r, int c, int G, in
                     // every lane with a page issues its two copies (after the expect-tx above)
                     if (live && okp) {
                         const size_t off = (static_cast<size_t>(pg) * p.nkv + kvh) * 16 * p.hd;
-                        unsigned char *dst = r.stages + static_cast<size_t>(stream % r.nst) * GV_STAGE_BYTES +
+                        unsigned char *dst = r.stages + static_cast<size_t>(stream.s) * GV_STAGE_BYTES +
                                              static_cast<size_t>(lane) * 2 * PB;
-                        bulk_g2s(dst, kp + off, PB, &r.full[stream % r.nst]);
-                        bulk_g2s(dst + PB, vp + off, PB, &r.full[stream % r.nst]);
+                        bulk_g2s(dst, kp + off, PB, &r.full[stream.s]);
+                        bulk_g2s(dst + PB, vp + off, PB, &r.full[stream.s]);
                     }
-                    if (live) stream++;
+                    if (live) stream.adv(r.nst);
                 }
                 continue;
             }
             const PkMat m = pk_mat(p, kind, l);
             const int a = pk_start(m.T, c, G), b = pk_start(m.T, c + 1, G);
             if (lane == 0) {
-                for (int t = a; t < b && live; t++, stream++) {
+                for (int t = a; t < b && live; t++, stream.adv(r.nst)) {
                     unsigned char *dst;
                     uint64_t *bar;
                     live = pk_slot(p, r, stream, dst, bar);
@@ -295,14 +310,16 @@ __device__ void pk_producer(const PkParams &p, const PkRing &r, int c, int G, in
                     bulk_g2s(dst + GV_NIB_BYTES, m.s + static_cast<size_t>(t) * GV_SC_BYTES, GV_SC_BYTES, bar);
                 }
             }
-            stream = __shfl_sync(0xffffffffu, stream, 0);
+            stream.i = __shfl_sync(0xffffffffu, stream.i, 0);
+            stream.s = __shfl_sync(0xffffffffu, stream.s, 0);
+            stream.ph = __shfl_sync(0xffffffffu, stream.ph, 0);
             live = __shfl_sync(0xffffffffu, live, 0);
         }
     }
     // no copy may still be landing in shared memory when the CTA exits
     if (lane == 0) {
-        const uint32_t first = stream > static_cast<uint32_t>(r.nst) ? stream - r.nst : 0u;
-        for (uint32_t i = first; i < stream; i++)
+        const uint32_t first = stream.i > static_cast<uint32_t>(r.nst) ? stream.i - r.nst : 0u;
+        for (uint32_t i = first; i < stream.i; i++)
             (void)mbar_wait(&r.full[i % r.nst], static_cast<uint32_t>((i / r.nst) & 1), p.err);
     }
 }
@@ -450,7 +467,7 @@ __device__ __forceinline__ void pk_epilogue(const PkParams &p, int kind, const P
 
 template <int FMT>
 __device__ void pk_gemv_phase(const PkParams &p, int kind, int l, const PkRing &rg_ring, const PkSmem &sm,
-                              uint32_t &stream, int &par, int c, int G, int ctid, int warp, int lane,
+                              PkStream &stream, int &par, int c, int G, int ctid, int warp, int lane,
                               float &bestv, int &besti) {
     const PkMat m = pk_mat(p, kind, l);
     const int a = pk_start(m.T, c, G), b = pk_start(m.T, c + 1, G);
@@ -473,7 +490,7 @@ __device__ void pk_gemv_phase(const PkParams &p, int kind, int l, const PkRing &
         wc = PKC_X; target = p.H / 32 + p.L * (p.H / 8); xin = p.x; gamma = p.final_norm;
     }
     if (!pk_wait(p, wc, target, ctid, sm.misc)) {
-        stream += b - a;
+        stream.skip(b - a, rg_ring.nst);
         return;
     }
     const int kt_a = a % m.KT;
@@ -487,13 +504,14 @@ __device__ void pk_gemv_phase(const PkParams &p, int kind, int l, const PkRing &
     for (int r = 0; r < 8; r++) acc[r][0] = 0.0f;
     const int RG = m.N / 8;
     const int rb_first = a / m.KT;
-    for (int t = a; t < b; t++, stream++) {
+    const ChunkLane cn = chunk_lane(wig, lane);
+    for (int t = a; t < b; t++, stream.adv(rg_ring.nst)) {
         const int rb = t / m.KT, kt = t - rb * m.KT;
-        if (static_cast<int>(stream & 1) == gid) {
-            const int s = static_cast<int>(stream % rg_ring.nst);
-            (void)pk_mbar_wait(p, &rg_ring.full[s], static_cast<uint32_t>((stream / rg_ring.nst) & 1));
+        if (static_cast<int>(stream.i & 1) == gid) {
+            const int s = stream.s;
+            (void)pk_mbar_wait(p, &rg_ring.full[s], stream.ph);
             const int slot = (kt - kt_a + m.KT) % m.KT;
-            stage_chunk<FMT, 1>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, wig, lane, xs_a, ct_a,
+            stage_chunk<FMT, 1>(stages_a + static_cast<uint32_t>(s) * GV_STAGE_BYTES, cn, xs_a, ct_a,
                                 slot * GV_TC + (lane & 15), CS, acc);
             __syncwarp();
             if (lane == 0) mbar_arrive_relaxed(&rg_ring.empty[s]);
@@ -643,7 +661,7 @@ __device__ __forceinline__ void pk_rope(const PkParams &p, const float *h, int p
 }
 
 template <int DPL>
-__device__ void pk_att_phase(const PkParams &p, int l, const PkRing &ring, const PkSmem &sm, uint32_t &stream, int c,
+__device__ void pk_att_phase(const PkParams &p, int l, const PkRing &ring, const PkSmem &sm, PkStream &stream, int c,
                              int ctid, int warp, int lane, int pos) {
     const int natt = p.S * p.nkv;
     if (c >= natt) return;
@@ -656,7 +674,7 @@ __device__ void pk_att_phase(const PkParams &p, int l, const PkRing &ring, const
     const int nstg = (p1 - p0 + PPS - 1) / PPS;
     const int gid = warp >> 3, wig = warp & 7;
     if (!pk_wait(p, PKC_QKV, (l + 1) * ((p.nq + 2 * p.nkv) * hd / 8), ctid, sm.misc)) {
-        stream += nstg;
+        stream.skip(nstg, ring.nst);
         return;
     }
     if (!pos_ok && ctid == 0) set_error(p.err, BW_DEVERR_BAD_POS);
@@ -670,10 +688,10 @@ __device__ void pk_att_phase(const PkParams &p, int l, const PkRing &ring, const
     float q[DPL];
     if (head && pos_ok) pk_rope<DPL>(p, p.qkv + static_cast<size_t>(kvh * G + g) * hd, pos, lane, q);
     const int last_slot = pos % 16;   // slot of the new token in the last page (not yet in the pool)
-    for (int i = 0; i < nstg; i++, stream++) {
-        if (static_cast<int>(stream & 1) != gid) continue;
-        const int sidx = static_cast<int>(stream % ring.nst);
-        (void)pk_mbar_wait(p, &ring.full[sidx], static_cast<uint32_t>((stream / ring.nst) & 1));
+    for (int i = 0; i < nstg; i++, stream.adv(ring.nst)) {
+        if (static_cast<int>(stream.i & 1) != gid) continue;
+        const int sidx = stream.s;
+        (void)pk_mbar_wait(p, &ring.full[sidx], stream.ph);
         if (head && pos_ok) {
             const unsigned char *stg = ring.stages + static_cast<size_t>(sidx) * GV_STAGE_BYTES;
             const int j0 = p0 + i * PPS, n = min(PPS, p1 - j0);
@@ -830,7 +848,7 @@ __device__ void pk_att_phase(const PkParams &p, int l, const PkRing &ring, const
 
 template <int FMT, int DPL>
 __global__ void __launch_bounds__(PK_THREADS, 1) step_persistent_kernel(const __grid_constant__ PkParams p) {
-    extern __shared__ __align__(128) unsigned char pk_smem[];
+    extern __shared__ __align__(1024) unsigned char pk_smem[];
     const int c = blockIdx.x, G = gridDim.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     PkRing ring;
@@ -874,7 +892,7 @@ __global__ void __launch_bounds__(PK_THREADS, 1) step_persistent_kernel(const __
         pk_producer(p, ring, c, G, lane, pos);
     } else {
         const int ctid = threadIdx.x;
-        uint32_t stream = 0;
+        PkStream stream = {0u, 0, 0u};
         int par = 0;
         // embedding: x = dequantized row tokens_in[0], 32 columns per CTA and round
         {

@@ -4,6 +4,9 @@ every layer of a model from a CUDA graph, timed with CUDA events on the
 launching stream, reported as microseconds per launch and algorithmic GB/s
 (the bytes of weights and KV that launch must touch, divided by its time).
 
+"step" (batch 1, dense models) is the whole decode step run as one persistent
+kernel (bw_decode_step with BW_STEP_PERSISTENT).
+
 Also the small, self-contained target for `ncu` captures:
 
     python -m token_decode_b200.kernel_bench --config 7b --layers 2 --only gu --reps 2 --eager
@@ -96,6 +99,21 @@ class KernelBench:
             # by the caller from the router output (see moe_touched_bytes)
             out["moe"] = (moe, lambda l: 4 * cfg.n_experts * cfg.H + exp_bytes
                           + self.moe_expert_bytes, L)
+        if self.with_step and self.B == 1 and cfg.n_experts == 0:
+            # the whole batch-1 step: one persistent kernel (bw_decode_step); its
+            # bytes are every matrix plus the KV read and written
+            tin = torch.zeros(1, dtype=torch.int32, device="cuda")
+            tout = torch.zeros(1, dtype=torch.int32, device="cuda")
+            wsz = bw.decode_workspace_bytes(dm.c, dkv.c, 1, 1)
+            self._sws = bw.workspace(wsz)
+            step_b = sum(_wbytes(w) for ly in dm.layers for w in (ly.wqkv, ly.wo, ly.wgu, ly.wd)) + \
+                _wbytes(dm.c.lm_head) + L * kv_layer * (self.avg_len + 1)
+
+            def step(l):
+                # no advance: every launch decodes the same position
+                bw.decode_step(dm.c, dkv.c, tin, self.pos, 1, 1, tout, self._sws, flags=bw.STEP_PERSISTENT,
+                               stream=self.st)
+            out["step"] = (step, lambda l: step_b, 1)
         lm = dm.c.lm_head
         out["lm_head"] = (lambda l: self._gemv(lm, self.x, self.logits, bw.GEMV_RMSNORM | bw.GEMV_ARGMAX,
                                                gamma=self.gamma, argmax_out=self.am),
@@ -103,6 +121,7 @@ class KernelBench:
         return out
 
     moe_expert_bytes = 0
+    with_step = False   # also the persistent whole-step kernel (only when asked for by name)
 
     def time(self, name, reps=10):
         """Graph of the kind over all its layers, replayed `reps` times."""
@@ -149,6 +168,7 @@ def moe_touched_bytes(dm, B, kb: KernelBench) -> int:
 
 def run_all(dm, dkv, B, stream, pos, reps=10, only=None):
     kb = KernelBench(dm, dkv, B, stream, pos)
+    kb.with_step = only == "step"
     if dm.cfg.n_experts:
         kb.moe_expert_bytes = moe_touched_bytes(dm, B, kb)
     res = {}
@@ -186,6 +206,7 @@ def main():
     pos = cfg.ctx + cfg.steps // 2
     if a.eager:
         kb = KernelBench(dm, dkv, cfg.B, st, pos)
+        kb.with_step = a.only == "step"
         if cfg.n_experts:
             kb.moe_expert_bytes = moe_touched_bytes(dm, cfg.B, kb)
         for name, (fn, _, n) in kb.kinds().items():

@@ -124,7 +124,7 @@ class Decoder:
         self.tokens_out = torch.zeros(B * n_rows, dtype=torch.int32, device="cuda")
         self.pos = torch.zeros(B, dtype=torch.int32, device="cuda")
 
-    def step(self, logits=None, advance=False, stream=None):
+    def step(self, logits=None, advance=False, stream=None, persistent=False):
+        flags = (bw.STEP_ADVANCE if advance else 0) | (bw.STEP_PERSISTENT if persistent else 0)
         bw.decode_step(self.dm.c, self.dkv.c, self.tokens_in, self.pos, self.B, self.n_rows,
-                       self.tokens_out, self.ws, logits=logits,
-                       flags=bw.STEP_ADVANCE if advance else 0, stream=stream)
+                       self.tokens_out, self.ws, logits=logits, flags=flags, stream=stream)
