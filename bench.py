@@ -373,6 +373,7 @@ def measure(cfg, model, kv, dm, rank, world, local, steps, warmup, cpu_budget, s
         entry["kernels"] = kern
     if cfg.verify_k:
         entry["verify_pass"] = verify_pass(cfg, dm, kv, stream, ms_step)
+        entry["speculative"] = speculative(cfg, dm, kv, stream, ms_step)
     if rank == 0 and world == 1 and cpu_budget > 0:
         entry["cpu_baseline"] = cpu_baseline(cfg, model, kv, toks, budget_s=cpu_budget)
     del dec, dkv
@@ -409,6 +410,48 @@ def verify_pass(cfg, dm, kv, stream, ms_plain):
     return {"rows": R, "drafts": cfg.verify_k, "ms_per_pass": round(ms, 4),
             "vs_plain_step": round(ms / ms_plain, 3), "device_error_word": err,
             "path": "kernel chain, %d rows per projection" % R}
+
+
+def speculative(cfg, dm, kv, stream, ms_plain, passes=8):
+    """Speculative decoding with the (synthetic, random-init) MTP draft head, K =
+    cfg.verify_k drafts per pass: device time of CUDA-graph replays of whole
+    passes (draft, verify, accept) and the tokens they emitted, counted on the
+    device.  A random draft head rarely guesses the main model's greedy token,
+    so the measured acceptance is low; the rate at full acceptance ((K + 1)
+    tokens per pass at the same pass time) is reported beside it."""
+    from token_decode_b200 import bw, runtime, synth
+    K = cfg.verify_k
+    head = synth.make_draft_head(cfg, "cuda", seed=0)
+    ddh = runtime.DeviceDraftHead(head)
+    sd = runtime.SpecDecoder(dm, runtime.DeviceKV(kv.clone()), ddh, K)
+    tok = int(synth.start_tokens(cfg, 0)[0])
+    total = torch.zeros(1, dtype=torch.int32, device="cuda")
+    with torch.cuda.stream(stream):
+        sd.start(tok, cfg.ctx, stream=stream)
+        sd.step_pass(stream=stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for _ in range(passes):
+                sd.step_pass(stream=stream)
+                total.add_(sd.n_acc + 1)
+        g.replay()
+        total.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    n = int(total.item())
+    err = bw.read_error(sd.ver.ws, stream) | bw.read_error(sd.mws, stream)
+    del g
+    ms_pass = ms / passes
+    return {"drafts_per_pass": K, "draft_head": "synthetic random-init (N(0,0.02)), vocabulary %d" % head.w.N,
+            "passes": passes, "tokens": n, "accepted_per_pass": round(n / passes - 1, 3),
+            "ms_per_pass": round(ms_pass, 4), "effective_tok_s": round(n / (ms / 1000.0), 3),
+            "tok_s_if_all_accepted": round((K + 1) / (ms_pass / 1000.0), 3),
+            "plain_step_tok_s": round(1000.0 / ms_plain, 3), "device_error_word": err,
+            "path": "bw_mtp_draft (2K launches) + bw_decode_step (K+1 rows) + bw_spec_accept, one graph"}
 
 
 KERNEL_NAMES = {"gu": "gemv_kernel (fused RMSNorm + gate/up + SiLU gate)", "down": "gemv_kernel (down + residual)",
@@ -472,7 +515,7 @@ def run_ours(args):
     }
     for k in ("path", "hbm_gbs_step", "roofline_step_frac_of_8tbs", "roofline_step_frac_of_measured",
               "bytes_per_step", "roofline", "kernels", "e2e", "gpu_launches", "device_error_word", "clocks",
-              "cpu_baseline"):
+              "cpu_baseline", "verify_pass", "speculative"):
         if k in h:
             line[k] = h[k]
     line["configs"] = {n: e for n, e in entries.items() if n != names[0]}

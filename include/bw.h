@@ -348,6 +348,32 @@ const float *bw_decode_hidden(const bw_model *m, const bw_kv *kv, int B, int n_r
 bw_status bw_decode_moe_route(const bw_model *m, const bw_kv *kv, int B, int n_rows, const void *ws,
                               const int32_t **idx, const float **w);
 
+/* Speculative draft head: K draft tokens for the next verify pass.  "bw24"
+ * deep-dive page (10100.com), section 7 (a light MTP draft head sharing the
+ * main model's embedding, its output vocabulary pruned to the first ids) and
+ * section 5, stage 4 (the drafts become the rows of one verify pass).  The
+ * page gives no formula; draft i = 1..K is
+ *     x = h + E[t];  g = rmsnorm(x) * norm;  d_i = lowest index of max (w g)
+ * with h <- g and t <- d_i for the next draft.  The first draft starts from
+ * row *row (row == NULL: row 0) of `hidden` and t = tokens[0].
+ *   hidden: fp32 [n_rows][H], the residual stream of the last step
+ *           (bw_decode_hidden: a verify pass's rows, or a plain step's row);
+ *   row:    optional int32 [1] on the device -- e.g. bw_spec_accept's n_accept
+ *           of the pass that produced `hidden`, the row whose greedy token is
+ *           tokens[0];
+ *   tokens: int32 [K + 1]: tokens[0] in (the last emitted token); tokens[1..K]
+ *           out (the drafts) -- the token row of the next verify pass.
+ * B = 1; 1 <= K <= BW_MAX_VERIFY_ROWS - 1; H <= 12288.  A token or row outside
+ * its range sets BW_DEVERR_BAD_TOKEN.  2K launches; graph capturable.
+ * ws must hold bw_mtp_workspace_bytes(m, dh). */
+typedef struct bw_draft_head {
+    const float *norm;           /* gamma [H] */
+    bw_qweight w;                /* [V_draft][H] over token ids 0 .. V_draft-1, in the model's format */
+} bw_draft_head;
+bw_status bw_mtp_draft(const bw_model *m, const bw_draft_head *dh, const float *hidden, int n_rows,
+                       const int32_t *row, int32_t *tokens, int K, void *ws, size_t ws_bytes, void *stream);
+size_t bw_mtp_workspace_bytes(const bw_model *m, const bw_draft_head *dh);
+
 /* Acceptance after a speculative verify pass.  "bw24" deep-dive page
  * (10100.com), section 5, stage 4 (the verify kernel unrolls the drafts as
  * sequence rows and masks every row after the first mismatch) and section 1

@@ -31,7 +31,7 @@ EXPORTS = (
     "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
     "bw_paged_attn_decode", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
     "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes", "bw_decode_hidden", "bw_spec_accept",
-    "bw_decode_moe_route",
+    "bw_decode_moe_route", "bw_mtp_draft", "bw_mtp_workspace_bytes",
 )
 
 
@@ -60,6 +60,10 @@ class Model(C.Structure):
                 ("F_exp", C.c_int), ("eps", C.c_float), ("embed", QWeight), ("lm_head", QWeight),
                 ("final_norm", C.c_void_p), ("rope_cos", C.c_void_p), ("rope_sin", C.c_void_p),
                 ("rope_max_pos", C.c_int), ("layers", C.c_void_p)]
+
+
+class DraftHead(C.Structure):
+    _fields_ = [("norm", C.c_void_p), ("w", QWeight)]
 
 
 class KV(C.Structure):
@@ -102,6 +106,8 @@ def lib() -> C.CDLL:
             "bw_decode_workspace_bytes": (z, [p, p, i, i]),
             "bw_decode_hidden": (p, [p, p, i, i, p]),
             "bw_decode_moe_route": (i, [p, p, i, i, p, p, p]),
+            "bw_mtp_draft": (i, [p, p, p, i, p, p, i, p, z, p]),
+            "bw_mtp_workspace_bytes": (z, [p, p]),
             "bw_spec_accept": (i, [p, p, i, i, p, p, i, p, p]),
         }
         for name, (res, args) in sig.items():
@@ -278,6 +284,16 @@ def decode_step(model: Model, kv: KV, tokens_in, pos, B, n_rows, tokens_out, ws,
     _check(lib().bw_decode_step(C.byref(model), C.byref(kv), _ptr(tokens_in), _ptr(pos), B, n_rows,
                                 _ptr(tokens_out), _ptr(logits), flags, _ptr(ws), ws.numel(),
                                 _stream(stream)), "bw_decode_step")
+
+
+def mtp_workspace_bytes(model: Model, dh: DraftHead) -> int:
+    return lib().bw_mtp_workspace_bytes(C.byref(model), C.byref(dh))
+
+
+def mtp_draft(model: Model, dh: DraftHead, hidden, n_rows, tokens, K, ws, row=None, stream=None):
+    """K draft tokens into tokens[1..K] from tokens[0] and hidden row *row (see bw.h)."""
+    _check(lib().bw_mtp_draft(C.byref(model), C.byref(dh), _ptr(hidden), n_rows, _ptr(row), _ptr(tokens), K,
+                              _ptr(ws), ws.numel(), _stream(stream)), "bw_mtp_draft")
 
 
 def spec_accept(tokens_in, tokens_out, B, n_rows, n_accept, next_out=None, next_stride=1, pos=None,

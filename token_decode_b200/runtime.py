@@ -128,3 +128,59 @@ class Decoder:
         flags = (bw.STEP_ADVANCE if advance else 0) | (bw.STEP_PERSISTENT if persistent else 0)
         bw.decode_step(self.dm.c, self.dkv.c, self.tokens_in, self.pos, self.B, self.n_rows,
                        self.tokens_out, self.ws, logits=logits, flags=flags, stream=stream)
+
+
+class DeviceDraftHead:
+    """GPU-layout draft head (norm gains + W_draft) as a bw_draft_head."""
+
+    def __init__(self, head):
+        qw, keep = _gpu_layout(head.w)
+        self.c = bw.DraftHead(bw._ptr(head.norm), qw)
+        self._keep = keep + [head.norm]
+
+
+class SpecDecoder:
+    """Speculative decoding of one sequence with K drafts per pass: a plain step
+    gives the first token and the hidden state the draft head starts from; each
+    pass then drafts (bw_mtp_draft), verifies the last token and the K drafts as
+    K + 1 rows of one step (bw_decode_step) and accepts (bw_spec_accept), which
+    also writes the next pass's first token and advances the position.  The
+    plain and the verify steps share the model's KV cache."""
+
+    def __init__(self, dm: DeviceModel, dkv: DeviceKV, ddh: DeviceDraftHead, K: int):
+        self.dm, self.ddh, self.K = dm, ddh, K
+        self.plain = Decoder(dm, dkv, 1)
+        self.ver = Decoder(dm, dkv, 1, n_rows=K + 1)
+        self.mws = bw.workspace(bw.mtp_workspace_bytes(dm.c, ddh.c))
+        self.n_acc = torch.zeros(1, dtype=torch.int32, device="cuda")
+        self.first = True
+
+    def start(self, token: int, pos: int, stream=None):
+        """Plain step on `token` at `pos`: its greedy token is the first output."""
+        self.plain.tokens_in.fill_(int(token))
+        self.plain.pos.fill_(int(pos))
+        self.plain.step(stream=stream)
+        self.ver.tokens_in[:1].copy_(self.plain.tokens_out)
+        self.ver.pos.fill_(int(pos) + 1)
+        self.first = True
+
+    def draft(self, stream=None):
+        if self.first:
+            hid = bw.decode_hidden(self.dm.c, self.plain.dkv.c, 1, 1, self.plain.ws)
+            bw.mtp_draft(self.dm.c, self.ddh.c, hid, 1, self.ver.tokens_in, self.K, self.mws, stream=stream)
+        else:
+            hid = bw.decode_hidden(self.dm.c, self.ver.dkv.c, 1, self.K + 1, self.ver.ws)
+            bw.mtp_draft(self.dm.c, self.ddh.c, hid, self.K + 1, self.ver.tokens_in, self.K, self.mws,
+                         row=self.n_acc, stream=stream)
+
+    def verify_accept(self, stream=None):
+        self.ver.step(stream=stream)
+        bw.spec_accept(self.ver.tokens_in, self.ver.tokens_out, 1, self.K + 1, self.n_acc,
+                       next_out=self.ver.tokens_in, next_stride=self.K + 1, pos=self.ver.pos, stream=stream)
+        self.first = False
+
+    def step_pass(self, stream=None):
+        """One pass; afterwards tokens_in[1..n_acc] (the accepted drafts) and
+        tokens_in[0] (the greedy token after them) are its output."""
+        self.draft(stream)
+        self.verify_accept(stream)
