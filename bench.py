@@ -141,8 +141,9 @@ def step_bytes(cfg, model, avg_ctx, moe_layer_bytes=0):
     K/V written (the embedding row is not counted).  A MoE layer adds
     moe_layer_bytes: its fp32 router, its shared expert and the experts the
     router selected (counted from the library's own routing of the batch)."""
-    kv_read = 2 * cfg.L * cfg.nkv * cfg.hd * 2 * avg_ctx * cfg.B
-    kv_write = 2 * cfg.L * cfg.nkv * cfg.hd * 2 * cfg.B
+    eb = 1 if cfg.kv_fp8 else 2          # bytes per cached element (E4M3 or fp16)
+    kv_read = 2 * cfg.L * cfg.nkv * cfg.hd * eb * avg_ctx * cfg.B
+    kv_write = 2 * cfg.L * cfg.nkv * cfg.hd * eb * cfg.B
     moe = cfg.L * moe_layer_bytes if cfg.n_experts else 0
     return model.weight_bytes_dense() + kv_read + kv_write + moe
 
@@ -206,7 +207,7 @@ def step_launches(cfg):
 
 
 HEADLINE = "7b"                                   # the workload the metric is quoted on
-SECONDARY = ("9b", "9b_b32", "27b", "moe")         # the other decode workloads, one line
+SECONDARY = ("9b", "9b_b32", "9b_b32_fp8", "27b", "moe")   # the other decode workloads, one line
 
 
 PERSISTENT = False   # --persistent: batch-1 dense steps as one persistent kernel (BW_STEP_PERSISTENT)
@@ -355,8 +356,8 @@ def measure(cfg, model, kv, dm, rank, world, local, steps, warmup, cpu_budget, s
         "ms_per_step": round(ms_step, 5), "steps": steps,
         "path": "persistent kernel (1 launch per step)" if uses_persistent_step(cfg)
                 else "kernel chain (%d launches per step)" % step_launches(cfg),
-        "dtype": "q4_0 weights, fp32 accumulate, fp16 KV" if cfg.fmt == synth.FMT_Q4_0 else
-                 "nvfp4 weights, fp32 accumulate, fp16 KV",
+        "dtype": ("q4_0 weights, fp32 accumulate" if cfg.fmt == synth.FMT_Q4_0 else
+                  "nvfp4 weights, fp32 accumulate") + (", e4m3 KV (per-layer scales)" if cfg.kv_fp8 else ", fp16 KV"),
         "hbm_gbs_step": round(step_gbs, 1),
         "roofline_step_frac_of_8tbs": round(step_gbs / NOMINAL_HBM_GBS, 4),
         "roofline_step_frac_of_measured": round(step_gbs / peak, 4),
@@ -486,7 +487,7 @@ def run_ours(args):
         if dm.c.rope_max_pos < cfg.max_pages * synth.PAGE_TOKENS:
             dm = runtime.DeviceModel(model, cfg.max_pages * synth.PAGE_TOKENS)
             cache[key] = (model, dm)
-        kv = synth.make_kv(cfg, "cuda", seed=rank)
+        kv = (synth.make_kv_fp8 if cfg.kv_fp8 else synth.make_kv)(cfg, "cuda", seed=rank)
         head = i == 0
         steps = args.steps if head else max(4, min(args.steps, 16))
         entries[name] = measure(cfg, model, kv, dm, rank, ws_, local, steps, args.warmup,

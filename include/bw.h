@@ -102,6 +102,9 @@ typedef int bw_status;
 #define BW_FMT_Q4_0 0
 #define BW_FMT_NVFP4 1
 
+#define BW_KV_FP16 0
+#define BW_KV_E4M3 1
+
 /* GEMV flags */
 #define BW_GEMV_RMSNORM 1u    /* prologue: each row of x -> rmsnorm(x) * gamma */
 #define BW_GEMV_RESIDUAL 2u   /* epilogue: y = residual + W x (residual may alias y) */
@@ -244,6 +247,14 @@ bw_status bw_paged_attn_decode(const float *qkv, const float *rope_cos, const fl
                                const int32_t *page_table, int max_pages, int n_pages,
                                const int32_t *pos, int B, int n_rows, int nq, int nkv, int hd,
                                float *out, void *ws, size_t ws_bytes, void *stream);
+/* The same over an E4M3 cache (bw_kv, kv_fmt BW_KV_E4M3): k_pool / v_pool are
+ * byte pools in the fp16 pools' layout; k_scale, v_scale > 0 the layer's
+ * scales.  The new rows are written as E4M3 codes of value / scale. */
+bw_status bw_paged_attn_decode_fp8(const float *qkv, const float *rope_cos, const float *rope_sin,
+                                   int rope_max_pos, void *k_pool, void *v_pool, float k_scale, float v_scale,
+                                   const int32_t *page_table, int max_pages, int n_pages,
+                                   const int32_t *pos, int B, int n_rows, int nq, int nkv, int hd,
+                                   float *out, void *ws, size_t ws_bytes, void *stream);
 size_t bw_attn_workspace_bytes(int B, int n_rows, int nq, int nkv, int hd, int max_pages);
 
 /* ------------------------------------------------------------ whole step */
@@ -295,6 +306,15 @@ typedef struct bw_kv {
     int n_pages;
     int max_pages;
     const int32_t *page_table;   /* device int32 [B][max_pages] */
+    /* BW_KV_FP16 (0), or BW_KV_E4M3 (1): the pools hold one byte per element in
+     * the same layout, an OCP E4M3 code c standing for e4m3(c) * scale with one
+     * fp32 scale per layer for K and one for V; a new row x is stored as the
+     * E4M3 code of x / scale, rounded to nearest even and saturated to +-448.
+     * The pages name FP8 on Blackwell (deep-dive page, section 7) without a
+     * scheme; this per-layer scaling is the plainest one. */
+    int kv_fmt;
+    const float *k_scale;        /* HOST array of L fp32 scales (kv_fmt 1), each > 0 */
+    const float *v_scale;
 } bw_kv;
 
 /* Mixture-of-experts feed-forward block of one layer for R token rows, in place:

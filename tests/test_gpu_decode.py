@@ -439,3 +439,50 @@ def test_persistent_step_bad_page_sets_error():
     dkv.page_table[0, 3] = int(synth.page_table(cfg, "cuda", 13)[0, 3])
     dec.step(logits=lg, persistent=True)
     assert bw.read_error(dec.ws) == 0
+
+
+# ---------------------------------------------------------- FP8 KV cache
+
+@pytest.mark.parametrize("name,fmt,layers,B", [("tiny", synth.FMT_Q4_0, 2, 2), ("9b", synth.FMT_NVFP4, 2, 2),
+                                               ("tiny", synth.FMT_NVFP4, 1, 8)])
+def test_fp8_kv_decode_matches_oracle(name, fmt, layers, B):
+    """Decode steps over an E4M3 cache (per-layer scales) against the oracle's
+    FP8-cache step: logits within the tolerance, tokens under the margin rule,
+    untouched cache bytes unchanged and the written rows the oracle's codes
+    (within one code step)."""
+    cfg = synth.CONFIGS[name].with_(fmt=fmt, L=layers, B=B)
+    model = synth.make_model(cfg, "cuda", seed=51, n_layers=layers)
+    kv = synth.make_kv_fp8(cfg, "cuda", seed=51, n_layers=layers)
+    om, okv = oracle.Model(model), oracle.KV(kv)
+    dm = runtime.DeviceModel(model, cfg.max_pages * synth.PAGE_TOKENS)
+    dkv = runtime.DeviceKV(kv)
+    assert dkv.fp8
+    dec = runtime.Decoder(dm, dkv, B)
+    cur = synth.start_tokens(cfg, 51)[:B].tolist()
+    lg = torch.empty((B, cfg.V), device="cuda")
+    steps = 2
+    for step in range(steps):
+        dec.tokens_in.copy_(torch.tensor(cur, dtype=torch.int32))
+        dec.pos.fill_(cfg.ctx + step)
+        dec.step(logits=lg)
+        assert bw.read_error(dec.ws) == 0
+        got = dec.tokens_out.cpu().tolist()
+        gl = lg.cpu().numpy()
+        ress = parallel_rows(lambda b: oracle.decode_token(om, okv, b, cur[b], cfg.ctx + step), range(B))
+        for b, res in enumerate(ress):
+            assert rel_err(gl[b], res["logits"]) < TOL, (step, b)
+            if res["margin"] > MARGIN:
+                assert got[b] == res["token"]
+        cur = got
+    pt = dkv.page_table.cpu().numpy()
+    for gp, op in zip(list(dkv.k) + list(dkv.v), list(okv.k) + list(okv.v)):
+        g = gp.cpu().numpy().transpose(0, 2, 1, 3)
+        o = np.asarray(op).transpose(0, 2, 1, 3)
+        written = np.zeros(g.shape[:2], dtype=bool)
+        for b in range(B):
+            for p in range(cfg.ctx, cfg.ctx + steps):
+                written[pt[b, p // 16], p % 16] = True
+        assert np.array_equal(g[~written], o[~written])
+        a, c = g[written].astype(np.int64), o[written].astype(np.int64)
+        oa, oc = np.where(a & 0x80, -(a & 0x7F), a), np.where(c & 0x80, -(c & 0x7F), c)
+        assert np.max(np.abs(oa - oc)) <= 1

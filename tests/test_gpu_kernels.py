@@ -402,3 +402,93 @@ def test_paged_attention_bad_page_sets_error_and_skips():
     pos2 = torch.tensor([max_pages * 16 + 3], dtype=torch.int32, device="cuda")
     bw.paged_attn_decode(qkv, cos, sin, maxpos, kp, vp, table, max_pages, n_pages, pos2, B, R, nq, nkv, hd, out, ws)
     assert bw.read_error(ws) & bw.DEVERR_BAD_POS
+
+
+# ------------------------------------------------------ FP8 (E4M3) attention
+
+def _attn_fp8_oracle(kp8, vp8, ks, vs, table, qkv, pos, B, R, nq, nkv, hd, n_pages, theta=1e6):
+    """The oracle over an E4M3 cache: the new rows encoded as E4M3 of value /
+    scale, then each query head attends (oracle.attend_head_e4m3)."""
+    class _KV:
+        pass
+    kv = _KV()
+    kv.k = [kp8.cpu()]
+    kv.v = [vp8.cpu()]
+    kv.page_table = table.cpu()
+    kv.n_pages = n_pages
+    kv.page_tokens = 16
+    okv = oracle.KV(kv)      # byte pools read as uint16 pairs are not used: attend_head_e4m3 takes the bytes
+    kb = kp8.cpu().numpy().copy()
+    vb = vp8.cpu().numpy().copy()
+    q_all = qkv.cpu().numpy()
+    out = np.zeros((B * R, nq * hd), np.float32)
+    for b in range(B):
+        for r in range(R):
+            p = int(pos[b]) + r
+            row = q_all[b * R + r]
+            q = row[: nq * hd].reshape(nq, hd)
+            k = row[nq * hd:(nq + nkv) * hd].reshape(nkv, hd)
+            v = row[(nq + nkv) * hd:].reshape(nkv, hd)
+            page = int(okv.page_table[b, p // 16])
+            for h in range(nkv):
+                kr = oracle.rope(k[h], p, theta)
+                kb[page, h, p % 16] = [oracle.f32_to_e4m3(float(np.float32(t) / np.float32(ks))) for t in kr]
+                vb[page, h, p % 16] = [oracle.f32_to_e4m3(float(np.float32(t) / np.float32(vs))) for t in v[h]]
+            for h in range(nq):
+                qr = oracle.rope(q[h], p, theta)
+                out[b * R + r, h * hd:(h + 1) * hd] = oracle.attend_head_e4m3(qr, kb, vb, ks, vs, okv, b, nkv,
+                                                                              h // (nq // nkv), p + 1)
+    return out, kb, vb
+
+
+@pytest.mark.parametrize("case", [
+    dict(B=1, R=1, nq=4, nkv=2, hd=64, ctxs=[128]),
+    dict(B=1, R=1, nq=28, nkv=4, hd=128, ctxs=[2000]),
+    dict(B=1, R=4, nq=64, nkv=8, hd=128, ctxs=[8190]),        # verify rows across a page boundary
+    dict(B=3, R=1, nq=32, nkv=8, hd=128, ctxs=[15, 16, 333]),
+    dict(B=40, R=1, nq=8, nkv=4, hd=64, ctxs=[17 + 7 * i for i in range(40)]),
+])
+def test_paged_attention_fp8_matches_oracle(case):
+    """Attention over an E4M3 cache with per-layer scales against the oracle's
+    E4M3 attention: outputs within 2e-5; the written codes are the oracle's
+    (V exactly; RoPE'd K within one code), every other byte untouched."""
+    B, R, nq, nkv, hd, ctxs = case["B"], case["R"], case["nq"], case["nkv"], case["hd"], case["ctxs"]
+    kp, vp, table, qkv, pos, max_pages, n_pages = _attn_case(B, R, nq, nkv, hd, ctxs, seed=7)
+    ks, vs = 1.0 / 16 + 3.0 / 256, 1.0 / 20 + 3.0 / 256
+    kp8 = (kp.float() / ks).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    vp8 = (vp.float() / vs).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).contiguous()
+    maxpos = max_pages * 16
+    cos = torch.empty((maxpos, hd // 2), device="cuda")
+    sin = torch.empty_like(cos)
+    bw.rope_table(1e6, hd, maxpos, cos, sin)
+    out = torch.empty((B * R, nq * hd), device="cuda")
+    ws = _ws(bw.attn_workspace_bytes(B, R, nq, nkv, hd, max_pages))
+    kg, vg = kp8.clone(), vp8.clone()
+    bw.paged_attn_decode_fp8(qkv, cos, sin, maxpos, kg, vg, ks, vs, table, max_pages, n_pages, pos, B, R,
+                             nq, nkv, hd, out, ws)
+    assert bw.read_error(ws) == 0
+    want, kb, vb = _attn_fp8_oracle(kp8, vp8, ks, vs, table, qkv, pos, B, R, nq, nkv, hd, n_pages)
+    assert rel_err(out.cpu().numpy(), want) < 2e-5, rel_err(out.cpu().numpy(), want)
+    assert np.array_equal(vg.cpu().numpy(), vb)
+    kgn = kg.cpu().numpy()
+    diff = kgn != kb
+    if diff.any():
+        # a RoPE'd k may land one code away (its cos/sin come from a table rounded once from fp64)
+        a = kgn[diff].astype(np.int64)
+        o = kb[diff].astype(np.int64)
+        oa = np.where(a & 0x80, -(a & 0x7F), a)
+        oo = np.where(o & 0x80, -(o & 0x7F), o)
+        assert np.max(np.abs(oa - oo)) <= 1
+        assert diff.sum() <= B * R * nkv * hd // 8
+
+
+def test_paged_attention_fp8_rejects_bad_scales():
+    kp, vp, table, qkv, pos, max_pages, n_pages = _attn_case(1, 1, 4, 2, 64, [40], seed=8)
+    kp8 = torch.zeros_like(kp, dtype=torch.uint8)
+    cos = torch.zeros((max_pages * 16, 32), device="cuda")
+    out = torch.empty((1, 4 * 64), device="cuda")
+    ws = _ws(bw.attn_workspace_bytes(1, 1, 4, 2, 64, max_pages))
+    for ks in (0.0, -1.0, float("inf")):
+        with pytest.raises(bw.BWError):
+            bw.paged_attn_decode_fp8(qkv, cos, cos, max_pages * 16, kp8, kp8.clone(), ks, 0.05, table, max_pages,
+                                     n_pages, pos, 1, 1, 4, 2, 64, out, ws)

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libbw.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED_SHAPE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_BAD_PAGE_INDEX = range(6)
 DEVERR_BAD_PAGE, DEVERR_TIMEOUT, DEVERR_BAD_TOKEN, DEVERR_BAD_POS = 1, 2, 4, 8
 FMT_Q4_0, FMT_NVFP4 = 0, 1
+KV_FP16, KV_E4M3 = 0, 1
 GEMV_RMSNORM, GEMV_RESIDUAL, GEMV_SILU_GATE, GEMV_ARGMAX = 1, 2, 4, 8
 STEP_ADVANCE = 1
 STEP_VALIDATE_ONLY = 2
@@ -29,7 +30,7 @@ EXPORTS = (
     "bw_status_string", "bw_abi_version", "bw_workspace_init", "bw_read_error",
     "bw_repack_bytes", "bw_repack_q4_0", "bw_repack_nvfp4", "bw_gemv_q4_0", "bw_gemv_nvfp4",
     "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
-    "bw_paged_attn_decode", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
+    "bw_paged_attn_decode", "bw_paged_attn_decode_fp8", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
     "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes", "bw_decode_hidden", "bw_spec_accept",
     "bw_decode_moe_route", "bw_mtp_draft", "bw_mtp_workspace_bytes",
 )
@@ -68,7 +69,7 @@ class DraftHead(C.Structure):
 
 class KV(C.Structure):
     _fields_ = [("k", C.c_void_p), ("v", C.c_void_p), ("n_pages", C.c_int), ("max_pages", C.c_int),
-                ("page_table", C.c_void_p)]
+                ("page_table", C.c_void_p), ("kv_fmt", C.c_int), ("k_scale", C.c_void_p), ("v_scale", C.c_void_p)]
 
 
 _lib = None
@@ -99,6 +100,7 @@ def lib() -> C.CDLL:
             "bw_rope_table": (i, [f, i, i, p, p, p]),
             "bw_argmax": (i, [p, i, i, p, p, p]),
             "bw_paged_attn_decode": (i, [p, p, p, i, p, p, p, i, i, p, i, i, i, i, i, p, p, z, p]),
+            "bw_paged_attn_decode_fp8": (i, [p, p, p, i, p, p, f, f, p, i, i, p, i, i, i, i, i, p, p, z, p]),
             "bw_attn_workspace_bytes": (z, [i, i, i, i, i, i]),
             "bw_moe_route_gemv": (i, [p, p, p, i, p, p, p, z, p]),
             "bw_moe_workspace_bytes": (z, [p, i]),
@@ -240,6 +242,16 @@ def paged_attn_decode(qkv, rope_cos, rope_sin, rope_max_pos, k_pool, v_pool, pag
                                       _ptr(k_pool), _ptr(v_pool), _ptr(page_table), max_pages,
                                       n_pages, _ptr(pos), B, n_rows, nq, nkv, hd, _ptr(out),
                                       _ptr(ws), ws.numel(), _stream(stream)), "bw_paged_attn_decode")
+
+
+def paged_attn_decode_fp8(qkv, rope_cos, rope_sin, rope_max_pos, k_pool, v_pool, k_scale, v_scale, page_table,
+                          max_pages, n_pages, pos, B, n_rows, nq, nkv, hd, out, ws, stream=None):
+    """bw_paged_attn_decode over an E4M3 cache (byte pools, per-layer scales)."""
+    _check(lib().bw_paged_attn_decode_fp8(_ptr(qkv), _ptr(rope_cos), _ptr(rope_sin), rope_max_pos,
+                                          _ptr(k_pool), _ptr(v_pool), float(k_scale), float(v_scale),
+                                          _ptr(page_table), max_pages, n_pages, _ptr(pos), B, n_rows, nq, nkv,
+                                          hd, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "bw_paged_attn_decode_fp8")
 
 
 def moe_workspace_bytes(model: Model, R: int) -> int:

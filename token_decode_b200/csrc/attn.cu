@@ -37,6 +37,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <cuda_fp8.h>
+
 #include "bw_common.cuh"
 
 namespace cg = cooperative_groups;
@@ -60,13 +62,14 @@ struct AttnParams {
     const float *qkv;
     const float *rope_cos, *rope_sin;
     int rope_max_pos;
-    __half *k_pool, *v_pool;
+    __half *k_pool, *v_pool;  // fp16 pools, or E4M3 byte pools (same layout) with FP8 KV
     const int32_t *page_table;
     int max_pages, n_pages;
     const int32_t *pos;
     int B, R, nq, nkv, G, Q, n_split;
     int cluster;          // 1: the splits of a (sequence, kv head) are one cluster and merge through DSMEM
-    float scale;
+    float scale;          // 1/sqrt(hd), times the K scale with FP8 KV
+    float kscale, vscale; // FP8 KV: a stored code c stands for e4m3(c) * scale (1 for fp16)
     float *out;
     float *part_o;        // [B][nkv][n_split][Q][HD]
     float *part_ml;       // [B][nkv][n_split][Q][2]
@@ -78,10 +81,12 @@ struct AttnParams {
 };
 
 // shared memory: K/V ring, q hi/lo planes, P hi/lo planes (double buffered),
-// row max / row sum exchange (double buffered), new k/v rows, barriers
-template <int HD, int MT, int NST>
+// row max / row sum exchange (double buffered), new k/v rows, barriers, and
+// with FP8 KV the E4M3 landing ring the copies fill
+template <int HD, int MT, int NST, int F8 = 0>
 __host__ __device__ constexpr size_t att_smem_fixed() {
     return static_cast<size_t>(NST) * 2 * ATT_ST * HD * 2                // K/V ring (fp16)
+           + static_cast<size_t>(F8) * NST * 2 * ATT_ST * HD              // E4M3 landing ring
            + 2 * static_cast<size_t>(16 * MT) * (HD + 8) * 2              // q hi, lo
            + 2 * 2 * static_cast<size_t>(16 * MT) * ATT_PST * 2           // P hi, lo x 2 buffers
            + 2 * 2 * static_cast<size_t>(ATT_CW) * (16 * MT) * 4          // row max, row sum x 2 buffers
@@ -152,7 +157,14 @@ __device__ __forceinline__ void split_f16(float v, __half &hi, __half &lo) {
 
 // NST: ring stages -- 2 when two CTAs share an SM, 4 when each CTA has an SM
 // to itself (a short split then has all its pages in flight at once).
-template <int HD, int MT, int NST>
+//
+// F8 = 1: the pools hold E4M3 codes with per-layer K and V scales (the FP8 KV
+// cache).  The copies bring a stage's codes into a landing ring; the consumers
+// turn them into fp16 (exact: every E4M3 value is an fp16 value) in the fp16
+// ring's layout and release the landing slot at once, so the tensor-core code
+// below runs unchanged on the codes' values; the K scale is folded into the
+// score scale and the V scale multiplies the output.
+template <int HD, int MT, int NST, int F8>
 __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(const __grid_constant__ AttnParams p) {
     constexpr int ATT_NST = NST;
     constexpr int QM = 16 * MT;             // query rows of the MMA tiles (padded)
@@ -170,7 +182,10 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
     // the swizzle pattern follows address bits, so the ring starts on 1024 bytes
     unsigned char *att_sm = att_sm_raw + ((1024u - (smem_u32(att_sm_raw) & 1023u)) & 1023u);
     __half *ring = reinterpret_cast<__half *>(att_sm);                                  // [NST][K|V][SH]
-    __half *qh = ring + static_cast<size_t>(ATT_NST) * 2 * SH;                          // [QM][QS]
+    // E4M3 landing ring [NST][K|V][ATT_ST][HD] (FP8 KV only): 1024-byte aligned,
+    // right after the fp16 ring, as tensor copies need
+    unsigned char *land = reinterpret_cast<unsigned char *>(ring + static_cast<size_t>(ATT_NST) * 2 * SH);
+    __half *qh = reinterpret_cast<__half *>(land + static_cast<size_t>(F8) * ATT_NST * 2 * ATT_ST * HD);  // [QM][QS]
     __half *ql = qh + QM * QS;
     __half *Ph = ql + QM * QS;                                                        // [2][QM][PST]
     __half *Pl = Ph + 2 * QM * ATT_PST;
@@ -252,22 +267,30 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
             for (int s = 0; s < n_stages; s++) {
                 const int st = s % ATT_NST;
                 if (s >= ATT_NST) mbar_wait(&empty[st], static_cast<uint32_t>((s / ATT_NST - 1) & 1), p.err);
+                constexpr uint32_t PB = F8 ? 16 * HD : PAGE_BYTES;   // bytes of one page of K (or V)
                 uint32_t bytes = 0;
                 for (int j = 0; j < ATT_PPS; j++) {
                     const int lp = s * ATT_PPS + j;
-                    if (lp < npl && pages[lp] >= 0) bytes += 2 * PAGE_BYTES;
+                    if (lp < npl && pages[lp] >= 0) bytes += 2 * PB;
                 }
                 mbar_arrive_tx(&full[st], bytes);
-                unsigned char *sk = reinterpret_cast<unsigned char *>(ring + static_cast<size_t>(st) * 2 * SH);
+                unsigned char *sk = F8 ? land + static_cast<size_t>(st) * 2 * ATT_ST * HD
+                                       : reinterpret_cast<unsigned char *>(ring + static_cast<size_t>(st) * 2 * SH);
                 for (int j = 0; j < ATT_PPS; j++) {
                     const int lp = s * ATT_PPS + j;
                     if (lp >= npl || pages[lp] < 0) continue;
                     const int y = (pages[lp] * p.nkv + kvh) * 16;     // first row of this page
+                    if constexpr (F8) {
+                        // one box of 16 rows x HD bytes per page, tokens back to back
+                        tma_load_2d(sk + j * PB, &p.tmk, 0, y, &full[st]);
+                        tma_load_2d(sk + ATT_ST * HD + j * PB, &p.tmv, 0, y, &full[st]);
+                    } else {
 #pragma unroll
-                    for (int h = 0; h < HD / 64; h++) {
-                        const int box = (j * (HD / 64) + h) << 11;
-                        tma_load_2d(sk + box, &p.tmk, h * 64, y, &full[st]);
-                        tma_load_2d(sk + SH * 2 + box, &p.tmv, h * 64, y, &full[st]);
+                        for (int h = 0; h < HD / 64; h++) {
+                            const int box = (j * (HD / 64) + h) << 11;
+                            tma_load_2d(sk + box, &p.tmk, h * 64, y, &full[st]);
+                            tma_load_2d(sk + SH * 2 + box, &p.tmv, h * 64, y, &full[st]);
+                        }
                     }
                 }
             }
@@ -313,18 +336,36 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
             const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
             float ra, rb;
             rope_pair(krow[d], krow[d + HD / 2], c, s, ra, rb);
-            const __half ha = __float2half_rn(ra), hb = __float2half_rn(rb);
-            newk[r * HD + d] = ha;
-            newk[r * HD + d + HD / 2] = hb;
-            if (ok) {
-                p.k_pool[off + d] = ha;
-                p.k_pool[off + d + HD / 2] = hb;
+            if constexpr (F8) {
+                // E4M3 of value / scale, round to nearest even, saturating to +-448
+                const __nv_fp8_storage_t ca = __nv_cvt_float_to_fp8(__fdiv_rn(ra, p.kscale), __NV_SATFINITE, __NV_E4M3);
+                const __nv_fp8_storage_t cb = __nv_cvt_float_to_fp8(__fdiv_rn(rb, p.kscale), __NV_SATFINITE, __NV_E4M3);
+                newk[r * HD + d] = __float2half_rn(e4m3_to_f(ca));
+                newk[r * HD + d + HD / 2] = __float2half_rn(e4m3_to_f(cb));
+                if (ok) {
+                    reinterpret_cast<uint8_t *>(p.k_pool)[off + d] = ca;
+                    reinterpret_cast<uint8_t *>(p.k_pool)[off + d + HD / 2] = cb;
+                }
+            } else {
+                const __half ha = __float2half_rn(ra), hb = __float2half_rn(rb);
+                newk[r * HD + d] = ha;
+                newk[r * HD + d + HD / 2] = hb;
+                if (ok) {
+                    p.k_pool[off + d] = ha;
+                    p.k_pool[off + d + HD / 2] = hb;
+                }
             }
         }
         for (int d = tid; d < HD; d += ATT_CT) {
-            const __half hv = __float2half_rn(vrow[d]);
-            newv[r * HD + d] = hv;
-            if (ok) p.v_pool[off + d] = hv;
+            if constexpr (F8) {
+                const __nv_fp8_storage_t cv = __nv_cvt_float_to_fp8(__fdiv_rn(vrow[d], p.vscale), __NV_SATFINITE, __NV_E4M3);
+                newv[r * HD + d] = __float2half_rn(e4m3_to_f(cv));
+                if (ok) reinterpret_cast<uint8_t *>(p.v_pool)[off + d] = cv;
+            } else {
+                const __half hv = __float2half_rn(vrow[d]);
+                newv[r * HD + d] = hv;
+                if (ok) p.v_pool[off + d] = hv;
+            }
         }
     }
     consumers_sync();
@@ -352,6 +393,32 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
         mbar_wait(&full[st], static_cast<uint32_t>((s / ATT_NST) & 1), p.err);
         __half *sk = ring + static_cast<size_t>(st) * 2 * SH;
         __half *sv = sk + SH;
+        if constexpr (F8) {
+            // E4M3 codes -> fp16 values in the ring's layout (16 codes per item),
+            // then the landing slot goes back to the producer
+            const unsigned char *lk = land + static_cast<size_t>(st) * 2 * ATT_ST * HD;
+            for (int e = tid; e < 2 * ATT_ST * (HD / 16); e += ATT_CT) {
+                const int kv = e / (ATT_ST * (HD / 16)), rem = e - kv * (ATT_ST * (HD / 16));
+                const int T = rem / (HD / 16), d0 = (rem - T * (HD / 16)) * 16;
+                const uint4 c = *reinterpret_cast<const uint4 *>(lk + static_cast<size_t>(kv) * ATT_ST * HD +
+                                                                 static_cast<size_t>(T) * HD + d0);
+                uint32_t h[8];
+                const uint32_t w4[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const float2 lo = e4m3x2_to_f2(w4[i] & 0xffffu), hi = e4m3x2_to_f2(w4[i] >> 16);
+                    const __half2 a = __floats2half2_rn(lo.x, lo.y), b2 = __floats2half2_rn(hi.x, hi.y);
+                    h[2 * i] = *reinterpret_cast<const uint32_t *>(&a);
+                    h[2 * i + 1] = *reinterpret_cast<const uint32_t *>(&b2);
+                }
+                unsigned char *dst = reinterpret_cast<unsigned char *>(kv ? sv : sk);
+                *reinterpret_cast<uint4 *>(dst + kv_off<HD>(T, d0)) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4 *>(dst + kv_off<HD>(T, d0 + 8)) = make_uint4(h[4], h[5], h[6], h[7]);
+            }
+            consumers_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
         const int tb = (pg0 + s * ATT_PPS) * 16;       // position of the stage's first token
         const int nvalid = min(ATT_ST, t1 - tb);
         bool missing = false;
@@ -508,8 +575,10 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
             }
         }
         // this warp is done with the stage: release it to the producer
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
+        if constexpr (!F8) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
     }
 
     // ---- 4. the output, or a partial for the split combine
@@ -580,7 +649,7 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
                 if (r2 < ns) O = fmaf(ov[r2], s_w[r2 * p.Q + qi], O);
             const int r = qi / p.G, gq = qi - r * p.G;
             p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
-                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = O / s_L[qi];
+                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = (O * p.vscale) / s_L[qi];
         }
         cluster.sync();   // keep this CTA's shared memory alive until every reader is done
         return;
@@ -600,8 +669,8 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
                 if (p.n_split == 1) {
                     float *dst = p.out + (static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
                                  static_cast<size_t>(kvh * p.G + gq) * HD + d;
-                    dst[0] = o0 / l_run[mt][h];
-                    dst[1] = o1 / l_run[mt][h];
+                    dst[0] = (o0 * p.vscale) / l_run[mt][h];
+                    dst[1] = (o1 * p.vscale) / l_run[mt][h];
                 } else {
                     __stcg(reinterpret_cast<float2 *>(p.part_o + ((pbase + split) * p.Q + qi) * HD + d),
                            make_float2(o0, o1));
@@ -665,7 +734,8 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
         const float L = s_L[qi];
         float *dst = p.out + (static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
                      static_cast<size_t>(kvh * p.G + gq) * HD + d;
-        *reinterpret_cast<float4 *>(dst) = make_float4(O.x / L, O.y / L, O.z / L, O.w / L);
+        const float vs = p.vscale;
+        *reinterpret_cast<float4 *>(dst) = make_float4((O.x * vs) / L, (O.y * vs) / L, (O.z * vs) / L, (O.w * vs) / L);
     }
     consumers_sync();
     if (tid == 0) *cnt = 0u;
@@ -711,10 +781,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-static bool kv_tensor_map(CUtensorMap *out, void *pool, int n_pages, int nkv, int hd) {
+// fp16 pools: boxes of 16 rows x 64 dims with the 128-byte swizzle; E4M3
+// pools (f8): boxes of 16 rows x hd bytes, unswizzled.
+static bool kv_tensor_map(CUtensorMap *out, void *pool, int n_pages, int nkv, int hd, bool f8) {
     struct Entry {
         void *pool;
         int rows, hd;
+        bool f8;
         CUtensorMap map;
     };
     static Entry cache[512];
@@ -723,33 +796,34 @@ static bool kv_tensor_map(CUtensorMap *out, void *pool, int n_pages, int nkv, in
     std::lock_guard<std::mutex> lk(mu);
     const int rows = n_pages * nkv * 16;
     for (int i = 0; i < n_cache; i++)
-        if (cache[i].pool == pool && cache[i].rows == rows && cache[i].hd == hd) {
+        if (cache[i].pool == pool && cache[i].rows == rows && cache[i].hd == hd && cache[i].f8 == f8) {
             *out = cache[i].map;
             return true;
         }
     PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(hd), static_cast<cuuint64_t>(rows)};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(hd) * 2};
-    const cuuint32_t box[2] = {64, 16};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(hd) * (f8 ? 1 : 2)};
+    const cuuint32_t box[2] = {f8 ? static_cast<cuuint32_t>(hd) : 64u, 16};
     const cuuint32_t estr[2] = {1, 1};
     CUtensorMap m;
-    if (fn(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pool, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-        CUDA_SUCCESS)
+    if (fn(&m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pool, dims, strides, box,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, f8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
     Entry &e = cache[n_cache < 512 ? n_cache++ : (next++ % 512)];
     e.pool = pool;
     e.rows = rows;
     e.hd = hd;
+    e.f8 = f8;
     e.map = m;
     *out = m;
     return true;
 }
 
-template <int HD, int MT, int NST>
+template <int HD, int MT, int NST, int F8>
 static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnParams &p) {
-    const size_t smem = att_smem_fixed<HD, MT, NST>() + static_cast<size_t>(p.max_pages) * 4;
+    const size_t smem = att_smem_fixed<HD, MT, NST, F8>() + static_cast<size_t>(p.max_pages) * 4;
     static size_t attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -762,7 +836,7 @@ static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnPara
         static std::mutex mu;   // host threads may call the library concurrently
         std::lock_guard<std::mutex> lk(mu);
         if (attr_set[dev] < smem) {
-            if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(smem)) != cudaSuccess) {
                 (void)cudaGetLastError();
                 return BW_ERR_CUDA;
@@ -770,7 +844,7 @@ static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnPara
             attr_set[dev] = smem;
         }
         if (q.cluster && !cl_set[dev]) {
-            if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+            if (cudaFuncSetAttribute(attn_kernel<HD, MT, NST, F8>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
                 cudaSuccess) {
                 (void)cudaGetLastError();
                 return BW_ERR_CUDA;
@@ -778,7 +852,7 @@ static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnPara
             cl_set[dev] = true;
         }
     }
-    if (!q.cluster) return launch_pdl(attn_kernel<HD, MT, NST>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
+    if (!q.cluster) return launch_pdl(attn_kernel<HD, MT, NST, F8>, dim3(ns, nkv, B), dim3(ATT_THREADS), smem, st, q);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ns, nkv, B);
     cfg.blockDim = dim3(ATT_THREADS);
@@ -793,18 +867,19 @@ static bw_status attn_go(int ns, int nkv, int B, cudaStream_t st, const AttnPara
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, attn_kernel<HD, MT, NST>, q) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, attn_kernel<HD, MT, NST, F8>, q) != cudaSuccess) {
         (void)cudaGetLastError();
         return BW_ERR_CUDA;
     }
     return BW_OK;
 }
 
-template <int HD, int MT>
+template <int HD, int MT, int F8>
 static bw_status attn_go_st(int ns, int nkv, int B, cudaStream_t st, const AttnParams &p) {
-    // a grid that fits one CTA per SM gets the deep ring
-    return static_cast<long>(ns) * nkv * B <= sm_count() ? attn_go<HD, MT, 4>(ns, nkv, B, st, p)
-                                                         : attn_go<HD, MT, 2>(ns, nkv, B, st, p);
+    // a grid that fits one CTA per SM gets the deep ring, where it fits shared memory
+    const bool fits = att_smem_fixed<HD, MT, 4, F8>() + static_cast<size_t>(p.max_pages) * 4 <= 227 * 1024 - 1024;
+    return static_cast<long>(ns) * nkv * B <= sm_count() && fits ? attn_go<HD, MT, 4, F8>(ns, nkv, B, st, p)
+                                                                 : attn_go<HD, MT, 2, F8>(ns, nkv, B, st, p);
 }
 
 bw_status attn_check(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
@@ -828,7 +903,11 @@ bw_status attn_check(const float *qkv, const float *rope_cos, const float *rope_
 bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
                       void *k_pool, void *v_pool, const int32_t *page_table, int max_pages,
                       int n_pages, const int32_t *pos, int B, int R, int nq, int nkv, int hd,
-                      float *out, const Scratch &sc, cudaStream_t st) {
+                      float *out, const Scratch &sc, cudaStream_t st, int kv_fmt, float kscale, float vscale) {
+    if (kv_fmt != 0 && kv_fmt != 1) return BW_ERR_INVALID_ARG;
+    if (kv_fmt == 1 && !(kscale > 0.0f && vscale > 0.0f && isfinite(kscale) && isfinite(vscale)))
+        return BW_ERR_INVALID_ARG;
+    const bool f8 = kv_fmt == 1;
     const bw_status chk = attn_check(qkv, rope_cos, rope_sin, rope_max_pos, k_pool, v_pool, page_table, max_pages,
                                      n_pages, pos, B, R, nq, nkv, hd, out, sc);
     if (chk != BW_OK) return chk;
@@ -850,17 +929,25 @@ bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope
     p.G = nq / nkv;
     p.Q = p.G * R;
     p.scale = 1.0f / sqrtf(static_cast<float>(hd));
+    p.kscale = f8 ? kscale : 1.0f;
+    p.vscale = f8 ? vscale : 1.0f;
+    if (f8) p.scale = p.scale * kscale;
     p.out = out;
     p.err = sc.err;
     p.cnt = sc.cnt + CNT_ATTN;
-    if (!kv_tensor_map(&p.tmk, k_pool, n_pages, nkv, hd) || !kv_tensor_map(&p.tmv, v_pool, n_pages, nkv, hd))
+    if (!kv_tensor_map(&p.tmk, k_pool, n_pages, nkv, hd, f8) || !kv_tensor_map(&p.tmv, v_pool, n_pages, nkv, hd, f8))
         return BW_ERR_CUDA;
     const int ns = attn_splits(B, nkv, max_pages);
     Carver cv(sc.base);
     p.part_o = ns > 1 ? cv.take<float>(static_cast<size_t>(B) * nkv * ns * p.Q * hd) : nullptr;
     p.part_ml = ns > 1 ? cv.take<float>(static_cast<size_t>(B) * nkv * ns * p.Q * 2) : nullptr;
-    if (hd == 128) return p.Q <= 16 ? attn_go_st<128, 1>(ns, nkv, B, st, p) : attn_go_st<128, 2>(ns, nkv, B, st, p);
-    return p.Q <= 16 ? attn_go_st<64, 1>(ns, nkv, B, st, p) : attn_go_st<64, 2>(ns, nkv, B, st, p);
+    if (f8) {
+        if (hd == 128)
+            return p.Q <= 16 ? attn_go_st<128, 1, 1>(ns, nkv, B, st, p) : attn_go_st<128, 2, 1>(ns, nkv, B, st, p);
+        return p.Q <= 16 ? attn_go_st<64, 1, 1>(ns, nkv, B, st, p) : attn_go_st<64, 2, 1>(ns, nkv, B, st, p);
+    }
+    if (hd == 128) return p.Q <= 16 ? attn_go_st<128, 1, 0>(ns, nkv, B, st, p) : attn_go_st<128, 2, 0>(ns, nkv, B, st, p);
+    return p.Q <= 16 ? attn_go_st<64, 1, 0>(ns, nkv, B, st, p) : attn_go_st<64, 2, 0>(ns, nkv, B, st, p);
 }
 
 }  // namespace bw
@@ -875,7 +962,18 @@ bw_status bw_paged_attn_decode(const float *qkv, const float *rope_cos, const fl
     if (!bw::ws_ok(ws)) return BW_ERR_INVALID_ARG;
     return bw::attn_launch(qkv, rope_cos, rope_sin, rope_max_pos, k_pool, v_pool, page_table,
                            max_pages, n_pages, pos, B, n_rows, nq, nkv, hd, out,
-                           bw::scratch_of(ws, ws_bytes), static_cast<cudaStream_t>(stream));
+                           bw::scratch_of(ws, ws_bytes), static_cast<cudaStream_t>(stream), 0, 1.0f, 1.0f);
+}
+
+bw_status bw_paged_attn_decode_fp8(const float *qkv, const float *rope_cos, const float *rope_sin,
+                                   int rope_max_pos, void *k_pool, void *v_pool, float k_scale, float v_scale,
+                                   const int32_t *page_table, int max_pages, int n_pages,
+                                   const int32_t *pos, int B, int n_rows, int nq, int nkv, int hd,
+                                   float *out, void *ws, size_t ws_bytes, void *stream) {
+    if (!bw::ws_ok(ws)) return BW_ERR_INVALID_ARG;
+    return bw::attn_launch(qkv, rope_cos, rope_sin, rope_max_pos, k_pool, v_pool, page_table,
+                           max_pages, n_pages, pos, B, n_rows, nq, nkv, hd, out,
+                           bw::scratch_of(ws, ws_bytes), static_cast<cudaStream_t>(stream), 1, k_scale, v_scale);
 }
 
 size_t bw_attn_workspace_bytes(int B, int n_rows, int nq, int nkv, int hd, int max_pages) {

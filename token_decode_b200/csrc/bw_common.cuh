@@ -93,7 +93,8 @@ size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages);
 bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
                       void *k_pool, void *v_pool, const int32_t *page_table, int max_pages, int n_pages,
                       const int32_t *pos, int B, int R, int nq, int nkv, int hd, float *out,
-                      const Scratch &sc, cudaStream_t st);
+                      const Scratch &sc, cudaStream_t st, int kv_fmt = 0, float kscale = 1.0f,
+                      float vscale = 1.0f);
 bw_status embed_launch(int fmt, const void *e_q, const void *e_s, float ts, int V, int H,
                        const int32_t *tokens, int M, float *x, uint32_t *err, cudaStream_t st);
 

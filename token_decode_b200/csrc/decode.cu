@@ -160,6 +160,14 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
         !m->final_norm)
         return BW_ERR_INVALID_ARG;
     if ((flags & BW_STEP_ADVANCE) && n_rows != 1) return BW_ERR_INVALID_ARG;
+    if (kv->kv_fmt != 0 && kv->kv_fmt != 1) return BW_ERR_INVALID_ARG;
+    if (kv->kv_fmt == 1) {
+        if (!kv->k_scale || !kv->v_scale) return BW_ERR_INVALID_ARG;
+        for (int l = 0; l < m->L; l++)
+            if (!(kv->k_scale[l] > 0.0f && kv->v_scale[l] > 0.0f && isfinite(kv->k_scale[l]) &&
+                  isfinite(kv->v_scale[l])))
+                return BW_ERR_INVALID_ARG;
+    }
     const int fmt = m->embed.fmt;
     const int nqkv = (m->nq + 2 * m->nkv) * m->hd;
     if (!qw_ok(m->embed, m->V, m->H, fmt) || !qw_ok(m->lm_head, m->V, m->H, fmt))
@@ -179,7 +187,7 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
     if (s != BW_OK || (flags & BW_STEP_VALIDATE_ONLY)) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int R = B * n_rows;
-    if (bf.pk && (flags & BW_STEP_PERSISTENT))
+    if (bf.pk && (flags & BW_STEP_PERSISTENT) && kv->kv_fmt == 0)
         return persistent_step_launch(m, kv, tokens_in, pos, tokens_out, logits, (flags & BW_STEP_ADVANCE) != 0,
                                       bf.x, bf.qkv, bf.attn, bf.act, bf.pk, bf.kern, st);
 
@@ -193,7 +201,8 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
         if (s != BW_OK) return s;
         s = attn_launch(bf.qkv, m->rope_cos, m->rope_sin, m->rope_max_pos, kv->k[l], kv->v[l],
                         kv->page_table, kv->max_pages, kv->n_pages, pos, B, n_rows, m->nq, m->nkv, m->hd,
-                        bf.attn, bf.kern, st);
+                        bf.attn, bf.kern, st, kv->kv_fmt, kv->kv_fmt ? kv->k_scale[l] : 1.0f,
+                        kv->kv_fmt ? kv->v_scale[l] : 1.0f);
         if (s != BW_OK) return s;
         s = gemv_launch(fmt, ly.wo.q, ly.wo.s, ly.wo.ts, ly.wo.ts, m->H, m->nq * m->hd, bf.attn, R,
                         nullptr, m->eps, bf.x, bf.x, nullptr, BW_GEMV_RESIDUAL, bf.kern, st);

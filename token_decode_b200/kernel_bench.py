@@ -71,12 +71,18 @@ class KernelBench:
         out["qkv"] = (lambda l: self._gemv(dm.layers[l].wqkv, self.x, self.qkv, bw.GEMV_RMSNORM,
                                            gamma=self.gamma),
                       lambda l: _wbytes(dm.layers[l].wqkv), L)
-        kv_layer = 2 * cfg.nkv * cfg.hd * 2 * self.B
+        kv_layer = 2 * cfg.nkv * cfg.hd * (1 if dkv.fp8 else 2) * self.B
 
         def attn(l):
-            bw.paged_attn_decode(self.qkv, dm.cos, dm.sin, dm.c.rope_max_pos, dkv.k[l], dkv.v[l],
-                                 dkv.page_table, dkv.c.max_pages, dkv.c.n_pages, self.pos, self.B, 1,
-                                 cfg.nq, cfg.nkv, cfg.hd, self.att, self.ws, stream=self.st)
+            if dkv.fp8:
+                bw.paged_attn_decode_fp8(self.qkv, dm.cos, dm.sin, dm.c.rope_max_pos, dkv.k[l], dkv.v[l],
+                                         dkv._ks[l], dkv._vs[l], dkv.page_table, dkv.c.max_pages, dkv.c.n_pages,
+                                         self.pos, self.B, 1, cfg.nq, cfg.nkv, cfg.hd, self.att, self.ws,
+                                         stream=self.st)
+            else:
+                bw.paged_attn_decode(self.qkv, dm.cos, dm.sin, dm.c.rope_max_pos, dkv.k[l], dkv.v[l],
+                                     dkv.page_table, dkv.c.max_pages, dkv.c.n_pages, self.pos, self.B, 1,
+                                     cfg.nq, cfg.nkv, cfg.hd, self.att, self.ws, stream=self.st)
         out["attn"] = (attn, lambda l: kv_layer * (self.avg_len + 1), L)
         out["o"] = (lambda l: self._gemv(dm.layers[l].wo, self.att, self.x, bw.GEMV_RESIDUAL,
                                          residual=self.x),

@@ -101,7 +101,8 @@ class DeviceModel:
 
 
 class DeviceKV:
-    """The paged fp16 KV pools (one per layer) + page table as a bw_kv."""
+    """The paged KV pools (one per layer) + page table as a bw_kv: fp16 pools, or
+    E4M3 byte pools with per-layer K/V scales when the cache carries k_scale."""
 
     def __init__(self, kv):
         self.k = kv.k
@@ -110,8 +111,15 @@ class DeviceKV:
         L = len(kv.k)
         self._kp = (C.c_void_p * L)(*[bw._ptr(t) for t in kv.k])
         self._vp = (C.c_void_p * L)(*[bw._ptr(t) for t in kv.v])
+        self.fp8 = getattr(kv, "k_scale", None) is not None
+        if self.fp8:
+            self._ks = (C.c_float * L)(*[float(x) for x in kv.k_scale.cpu().tolist()[:L]])
+            self._vs = (C.c_float * L)(*[float(x) for x in kv.v_scale.cpu().tolist()[:L]])
         self.c = bw.KV(C.cast(self._kp, C.c_void_p).value, C.cast(self._vp, C.c_void_p).value,
-                       int(kv.n_pages), int(self.page_table.shape[1]), bw._ptr(self.page_table))
+                       int(kv.n_pages), int(self.page_table.shape[1]), bw._ptr(self.page_table),
+                       bw.KV_E4M3 if self.fp8 else bw.KV_FP16,
+                       C.cast(self._ks, C.c_void_p).value if self.fp8 else None,
+                       C.cast(self._vs, C.c_void_p).value if self.fp8 else None)
 
 
 class Decoder:

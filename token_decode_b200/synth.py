@@ -59,6 +59,7 @@ class Config:
     eps: float = 1.0e-6
     verify_k: int = 0   # draft tokens checked by one speculative-verify pass
     draft_vocab: int = 32768   # output ids of the speculative draft head (the first ids)
+    kv_fp8: bool = False       # the KV cache in E4M3 with per-layer scales (make_kv_fp8)
 
     @property
     def nqkv(self) -> int:
@@ -87,6 +88,8 @@ CONFIGS = {
                      V=151936, fmt=FMT_NVFP4, ctx=4096, steps=256, B=32),
     "27b": Config("27b-dense-nvfp4", L=64, H=5120, nq=64, nkv=8, hd=128, F=25600, V=151936,
                   fmt=FMT_NVFP4, ctx=8192, steps=128, verify_k=3),
+    "9b_b32_fp8": Config("9b-dense-nvfp4-b32-fp8kv", L=36, H=4096, nq=32, nkv=8, hd=128, F=12288,
+                         V=151936, fmt=FMT_NVFP4, ctx=4096, steps=256, B=32, kv_fp8=True),
     "moe": Config("35b-a3b-moe-nvfp4-b32", L=40, H=2048, nq=32, nkv=4, hd=128, F=0,
                   V=151936, fmt=FMT_NVFP4, ctx=2000, steps=128, B=32, n_experts=256,
                   topk=8, F_exp=512),
