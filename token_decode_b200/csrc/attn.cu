@@ -85,7 +85,7 @@ struct AttnParams {
 // with FP8 KV the E4M3 landing ring the copies fill
 template <int HD, int MT, int NST, int F8 = 0>
 __host__ __device__ constexpr size_t att_smem_fixed() {
-    return static_cast<size_t>(NST) * 2 * ATT_ST * HD * 2                // K/V ring (fp16)
+    return static_cast<size_t>(F8 ? 1 : NST) * 2 * ATT_ST * HD * 2       // K/V ring (fp16)
            + static_cast<size_t>(F8) * NST * 2 * ATT_ST * HD              // E4M3 landing ring
            + 2 * static_cast<size_t>(16 * MT) * (HD + 8) * 2              // q hi, lo
            + 2 * 2 * static_cast<size_t>(16 * MT) * ATT_PST * 2           // P hi, lo x 2 buffers
@@ -120,6 +120,25 @@ __device__ __forceinline__ uint32_t kv_off(int T, int d) {
     const int t = T & 15, c = (d & 63) >> 3;
     return static_cast<uint32_t>((((T >> 4) * (HD / 64) + (d >> 6)) << 11) + (t << 7) + ((c ^ (t & 7)) << 4) +
                                  ((d & 7) << 1));
+}
+
+// Byte offset of (token T of a stage, code d) in an E4M3 landing stage: rows
+// of HD bytes, one tensor box of 16 rows per page, with the copy's 128-byte
+// (HD 128) or 64-byte (HD 64) swizzle moving 16-byte chunk c of row T to
+// c ^ (T & 7) or c ^ ((T >> 1) & 3).
+template <int HD>
+__device__ __forceinline__ uint32_t land_off(int T, int d) {
+    const int sw = HD == 128 ? (T & 7) : ((T >> 1) & 3);
+    return static_cast<uint32_t>(T * HD + ((((d >> 4) ^ sw)) << 4) + (d & 15));
+}
+
+// four E4M3 codes (bytes of w, lowest first) -> two fp16x2 words; exact, since
+// every E4M3 value is an fp16 value
+__device__ __forceinline__ void e4m3x4_to_h4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // warp-level tensor-core MMA (m16n8k16, f16 inputs, f32 accumulate) and the
@@ -167,6 +186,9 @@ __device__ __forceinline__ void split_f16(float v, __half &hi, __half &lo) {
 template <int HD, int MT, int NST, int F8>
 __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(const __grid_constant__ AttnParams p) {
     constexpr int ATT_NST = NST;
+    // fp16 ring stages: with FP8 KV one, since each warp converts into it only
+    // what it reads itself (the landing ring is the one the copies run ahead in)
+    constexpr int RS = F8 ? 1 : NST;
     constexpr int QM = 16 * MT;             // query rows of the MMA tiles (padded)
     constexpr int QS = HD + 8;              // padded q row (halves)
     constexpr int NKS = HD / 16;            // k-steps of the score MMA
@@ -176,15 +198,15 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
     constexpr uint32_t PAGE_BYTES = 16 * HD * 2;
     // the cluster merge's partials and weights live in the drained ring
     static_assert(NST != 4 || (static_cast<size_t>(ATT_MAXQ) * HD + 3 * ATT_MAXQ + 2 * ATT_MAXCL * ATT_MAXQ) * 4 <=
-                                  static_cast<size_t>(NST) * 2 * SH * 2,
+                                  static_cast<size_t>(RS) * 2 * SH * 2,
                   "cluster merge scratch exceeds the ring");
     extern __shared__ __align__(1024) unsigned char att_sm_raw[];
     // the swizzle pattern follows address bits, so the ring starts on 1024 bytes
     unsigned char *att_sm = att_sm_raw + ((1024u - (smem_u32(att_sm_raw) & 1023u)) & 1023u);
-    __half *ring = reinterpret_cast<__half *>(att_sm);                                  // [NST][K|V][SH]
+    __half *ring = reinterpret_cast<__half *>(att_sm);                                  // [RS][K|V][SH]
     // E4M3 landing ring [NST][K|V][ATT_ST][HD] (FP8 KV only): 1024-byte aligned,
     // right after the fp16 ring, as tensor copies need
-    unsigned char *land = reinterpret_cast<unsigned char *>(ring + static_cast<size_t>(ATT_NST) * 2 * SH);
+    unsigned char *land = reinterpret_cast<unsigned char *>(ring + static_cast<size_t>(RS) * 2 * SH);
     __half *qh = reinterpret_cast<__half *>(land + static_cast<size_t>(F8) * ATT_NST * 2 * ATT_ST * HD);  // [QM][QS]
     __half *ql = qh + QM * QS;
     __half *Ph = ql + QM * QS;                                                        // [2][QM][PST]
@@ -282,6 +304,7 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
                     const int y = (pages[lp] * p.nkv + kvh) * 16;     // first row of this page
                     if constexpr (F8) {
                         // one box of 16 rows x HD bytes per page, tokens back to back
+                        // (swizzled, see land_off)
                         tma_load_2d(sk + j * PB, &p.tmk, 0, y, &full[st]);
                         tma_load_2d(sk + ATT_ST * HD + j * PB, &p.tmv, 0, y, &full[st]);
                     } else {
@@ -391,31 +414,49 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
     for (int s = 0; s < n_stages; s++) {
         const int st = s % ATT_NST, buf = s & 1;
         mbar_wait(&full[st], static_cast<uint32_t>((s / ATT_NST) & 1), p.err);
-        __half *sk = ring + static_cast<size_t>(st) * 2 * SH;
+        __half *sk = ring + static_cast<size_t>(F8 ? 0 : st) * 2 * SH;
         __half *sv = sk + SH;
         if constexpr (F8) {
-            // E4M3 codes -> fp16 values in the ring's layout (16 codes per item),
-            // then the landing slot goes back to the producer
+            // E4M3 codes -> fp16 values in the ring's layout.  Each warp converts
+            // exactly what it reads below -- K of its 8 tokens (all dims), V of
+            // its WD dims (all tokens) -- so no CTA barrier is needed; the
+            // landing slot goes back to the producer once every warp is done.
             const unsigned char *lk = land + static_cast<size_t>(st) * 2 * ATT_ST * HD;
-            for (int e = tid; e < 2 * ATT_ST * (HD / 16); e += ATT_CT) {
-                const int kv = e / (ATT_ST * (HD / 16)), rem = e - kv * (ATT_ST * (HD / 16));
-                const int T = rem / (HD / 16), d0 = (rem - T * (HD / 16)) * 16;
-                const uint4 c = *reinterpret_cast<const uint4 *>(lk + static_cast<size_t>(kv) * ATT_ST * HD +
-                                                                 static_cast<size_t>(T) * HD + d0);
-                uint32_t h[8];
-                const uint32_t w4[4] = {c.x, c.y, c.z, c.w};
+            const unsigned char *lv = lk + ATT_ST * HD;
+            unsigned char *skb = reinterpret_cast<unsigned char *>(sk), *svb = reinterpret_cast<unsigned char *>(sv);
+            constexpr int KC = HD / 16;                 // 16-code chunks of a token
 #pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    const float2 lo = e4m3x2_to_f2(w4[i] & 0xffffu), hi = e4m3x2_to_f2(w4[i] >> 16);
-                    const __half2 a = __floats2half2_rn(lo.x, lo.y), b2 = __floats2half2_rn(hi.x, hi.y);
-                    h[2 * i] = *reinterpret_cast<const uint32_t *>(&a);
-                    h[2 * i + 1] = *reinterpret_cast<const uint32_t *>(&b2);
-                }
-                unsigned char *dst = reinterpret_cast<unsigned char *>(kv ? sv : sk);
-                *reinterpret_cast<uint4 *>(dst + kv_off<HD>(T, d0)) = make_uint4(h[0], h[1], h[2], h[3]);
-                *reinterpret_cast<uint4 *>(dst + kv_off<HD>(T, d0 + 8)) = make_uint4(h[4], h[5], h[6], h[7]);
+            for (int i = lane; i < 8 * KC; i += 32) {
+                const int T = warp * 8 + i / KC, d0 = (i % KC) * 16;
+                const uint4 c = *reinterpret_cast<const uint4 *>(lk + land_off<HD>(T, d0));
+                uint32_t h[8];
+                e4m3x4_to_h4(c.x, h[0], h[1]);
+                e4m3x4_to_h4(c.y, h[2], h[3]);
+                e4m3x4_to_h4(c.z, h[4], h[5]);
+                e4m3x4_to_h4(c.w, h[6], h[7]);
+                *reinterpret_cast<uint4 *>(skb + kv_off<HD>(T, d0)) = make_uint4(h[0], h[1], h[2], h[3]);
+                *reinterpret_cast<uint4 *>(skb + kv_off<HD>(T, d0 + 8)) = make_uint4(h[4], h[5], h[6], h[7]);
             }
-            consumers_sync();
+            const int vd0 = warp * WD;
+#pragma unroll
+            for (int T = lane; T < ATT_ST; T += 32) {
+                if constexpr (WD == 16) {
+                    const uint4 c = *reinterpret_cast<const uint4 *>(lv + land_off<HD>(T, vd0));
+                    uint32_t h[8];
+                    e4m3x4_to_h4(c.x, h[0], h[1]);
+                    e4m3x4_to_h4(c.y, h[2], h[3]);
+                    e4m3x4_to_h4(c.z, h[4], h[5]);
+                    e4m3x4_to_h4(c.w, h[6], h[7]);
+                    *reinterpret_cast<uint4 *>(svb + kv_off<HD>(T, vd0)) = make_uint4(h[0], h[1], h[2], h[3]);
+                    *reinterpret_cast<uint4 *>(svb + kv_off<HD>(T, vd0 + 8)) = make_uint4(h[4], h[5], h[6], h[7]);
+                } else {
+                    const uint2 c = *reinterpret_cast<const uint2 *>(lv + land_off<HD>(T, vd0));
+                    uint32_t h[4];
+                    e4m3x4_to_h4(c.x, h[0], h[1]);
+                    e4m3x4_to_h4(c.y, h[2], h[3]);
+                    *reinterpret_cast<uint4 *>(svb + kv_off<HD>(T, vd0)) = make_uint4(h[0], h[1], h[2], h[3]);
+                }
+            }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
         }
@@ -430,6 +471,7 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
         if (fix_new || missing || nvalid < ATT_ST) {
             // rows written by this step replace what the copy brought; V rows the
             // copy did not fill are zeroed (their probability is 0, 0 * stale could be NaN)
+            if constexpr (F8) consumers_sync();   // every warp's conversion of the stage is done
             unsigned char *skb = reinterpret_cast<unsigned char *>(sk), *svb = reinterpret_cast<unsigned char *>(sv);
             for (int r = 0; r < p.R; r++) {
                 const int slot = p0 + r - tb;
@@ -585,7 +627,10 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
     if (p.cluster) {
         // the splits form one thread-block cluster: partials stay in shared
         // memory (the drained ring), each CTA merges a slice of the outputs
-        // from every split's shared memory, in split order
+        // from every split's shared memory, in split order.  The partials
+        // overwrite the ring, which slower warps may still be reading (V of
+        // the last stage): all consumers finish first.
+        consumers_sync();
         float *s_o = reinterpret_cast<float *>(att_sm);           // [Q][HD] unnormalized output
         float *s_m = s_o + ATT_MAXQ * HD;                           // [Q]
         float *s_l = s_m + ATT_MAXQ;                                // [Q]
@@ -782,7 +827,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // fp16 pools: boxes of 16 rows x 64 dims with the 128-byte swizzle; E4M3
-// pools (f8): boxes of 16 rows x hd bytes, unswizzled.
+// pools (f8): boxes of 16 rows x hd bytes with the hd-byte swizzle (128 or 64).
 static bool kv_tensor_map(CUtensorMap *out, void *pool, int n_pages, int nkv, int hd, bool f8) {
     struct Entry {
         void *pool;
@@ -808,7 +853,7 @@ static bool kv_tensor_map(CUtensorMap *out, void *pool, int n_pages, int nkv, in
     const cuuint32_t estr[2] = {1, 1};
     CUtensorMap m;
     if (fn(&m, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pool, dims, strides, box,
-           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, f8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, (f8 && hd == 64) ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return false;
     Entry &e = cache[n_cache < 512 ? n_cache++ : (next++ % 512)];

@@ -204,7 +204,7 @@ def main():
     if a.batch:
         cfg = cfg.with_(B=a.batch)
     model = synth.make_model(cfg, "cuda", seed=0, n_layers=cfg.L)
-    kv = synth.make_kv(cfg, "cuda", seed=0, n_layers=cfg.L)
+    kv = (synth.make_kv_fp8 if cfg.kv_fp8 else synth.make_kv)(cfg, "cuda", seed=0, n_layers=cfg.L)
     dm = runtime.DeviceModel(model, cfg.max_pages * synth.PAGE_TOKENS)
     dkv = runtime.DeviceKV(kv)
     del model
