@@ -786,6 +786,676 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
     if (tid == 0) *cnt = 0u;
 }
 
+// ---------------------------------------------------------------------------
+// Grouped-query decode attention with the tokens on the MMA's M side, for up
+// to 8 query rows per (sequence, kv head).
+//
+// The kv head's G * R roped query rows, split into fp16 hi and lo parts, are
+// the N = 8 (up to 4 rows) or 16 (up to 8 rows) columns of the MMA, and 16
+// tokens are its M rows:
+//     S^T [16 tokens x cols]  = K [16 tokens x hd] . Q^T [hd x cols]
+//     O^T [hd x cols]        += V^T [hd x 16 tokens] . P^T [16 tokens x cols]
+// so no MMA row is padding and the hi / lo products cost no second MMA.  Each
+// of the 4 consumer warps owns 16 tokens (one page) of every 64-token stage:
+// its own running max and sum per query row and its own O^T; nothing crosses
+// warps inside the stage loop.  The hi and lo columns are added, and the warps
+// merged, once at the end.
+//
+// With an E4M3 cache the MMA fragments are built straight from the codes in
+// shared memory (cvt.rn.f16x2.e4m3x2, exact): K's dims (the score MMA's k) and
+// V's tokens (the output MMA's k) are taken in an order that puts a lane's
+// codes in whole 32-bit words -- any order of k gives the same sums, as long
+// as Q and P are written in the same order -- and O^T's rows (dims) in an
+// order that lets one word of V feed two m-tiles.
+constexpr int AG_CW = 4;                          // consumer warps
+constexpr int AG_CT = AG_CW * 32;                 // consumer threads
+constexpr int AG_THREADS = AG_CT + 32;            // + the producer warp
+constexpr int AG_PST = 24;                        // padded P^T row (halves): conflict-free ldmatrix
+constexpr int AG_MAXQ = 8;                        // query rows per (sequence, kv head)
+
+__device__ __forceinline__ void ag_sync() { asm volatile("bar.sync 1, %0;" ::"n"(AG_CT) : "memory"); }
+
+__device__ __forceinline__ uint32_t ag_prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// E4M3 K: MMA k-index of dim d.  Lane group t (lane & 3) reads bytes 16t ..
+// 16t + 15 of each 64 dims: word j of them is k-step 4g + j, its bytes the
+// k positions 2t, 2t + 1, 2t + 8, 2t + 9 of that step.
+__device__ __forceinline__ int ag_kidx_f8(int d) {
+    const int g = d >> 6, r = d & 63, t = r >> 4, j = (r >> 2) & 3, e = r & 3;
+    return (4 * g + j) * 16 + 2 * t + (e & 1) + 8 * (e >> 1);
+}
+// E4M3 V: MMA k-index of token tau (0..15) of a warp's page.  Lane group t
+// reads tokens 4t .. 4t + 3: k positions 2t, 2t + 1, 2t + 8, 2t + 9.
+__device__ __forceinline__ int ag_tidx_f8(int tau) {
+    const int t = tau >> 2, e = tau & 3;
+    return 2 * t + (e & 1) + 8 * (e >> 1);
+}
+
+template <int HD, int F8>
+__host__ __device__ constexpr size_t ag_stage_bytes() {
+    return static_cast<size_t>(2) * ATT_ST * HD * (F8 ? 1 : 2);
+}
+
+// byte offset of the per-warp merge scratch in the drained ring: after the
+// split merge's partials, maxima, sums and weights
+template <int HD>
+__host__ __device__ constexpr size_t ag_scratch_off() {
+    return ((static_cast<size_t>(ATT_MAXQ) * HD + 3 * ATT_MAXQ + 2 * ATT_MAXCL * ATT_MAXQ) * 4 + 15) / 16 * 16;
+}
+
+template <int HD, int NQT, int NST, int F8>
+__host__ __device__ constexpr size_t ag_smem_fixed() {
+    return static_cast<size_t>(NST) * ag_stage_bytes<HD, F8>()                 // K/V ring
+           + static_cast<size_t>(8 * NQT) * (HD + 8) * 2                       // Q^T [cols][dims]
+           + static_cast<size_t>(AG_CW) * 8 * NQT * AG_PST * 2                 // P^T per warp [cols][tokens]
+           + 2 * static_cast<size_t>(ATT_MAXR) * HD * (F8 ? 1 : 2)            // new k, v rows
+           + 2 * static_cast<size_t>(AG_CW) * AG_MAXQ * 4                     // warp maxima, sums
+           + 2 * static_cast<size_t>(NST) * 8                                 // mbarriers
+           + 1024;                                                            // ring alignment
+}
+
+template <int HD, int NQT, int NST, int F8>
+__global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_constant__ AttnParams p) {
+    constexpr int NC = 8 * NQT;                 // MMA columns
+    constexpr int QP = 4 * NQT;                 // query rows per part (hi, lo)
+    constexpr int QSS = HD + 8;                 // padded Q^T row (halves)
+    constexpr int NKS = HD / 16;                // k-steps of the score MMA
+    constexpr int NMT = HD / 16;                // m-tiles of O^T
+    constexpr size_t STB = ag_stage_bytes<HD, F8>();
+    constexpr uint32_t PB = 16 * HD * (F8 ? 1 : 2);   // bytes of one page of K (or V)
+    constexpr int EB = F8 ? 1 : 2;              // bytes of a stored element
+    static_assert(ag_scratch_off<HD>() + static_cast<size_t>(AG_CW) * QP * HD * 4 <= NST * STB,
+                  "merge scratch exceeds the ring");
+    extern __shared__ __align__(1024) unsigned char ag_sm_raw[];
+    // the swizzle pattern follows address bits, so the ring starts on 1024 bytes
+    unsigned char *sm = ag_sm_raw + ((1024u - (smem_u32(ag_sm_raw) & 1023u)) & 1023u);
+    unsigned char *ring = sm;                                                   // [NST][K|V]
+    __half *qs = reinterpret_cast<__half *>(ring + NST * STB);                  // [NC][QSS]
+    __half *ps = qs + NC * QSS;                                                 // [CW][NC][PST]
+    unsigned char *newk = reinterpret_cast<unsigned char *>(ps + AG_CW * NC * AG_PST);   // [MAXR][HD]
+    unsigned char *newv = newk + ATT_MAXR * HD * EB;
+    float *s_mw = reinterpret_cast<float *>(newv + ATT_MAXR * HD * EB);        // [CW][MAXQ]
+    float *s_lw = s_mw + AG_CW * AG_MAXQ;
+    uint64_t *full = reinterpret_cast<uint64_t *>(s_lw + AG_CW * AG_MAXQ);     // [NST]
+    uint64_t *empty = full + NST;                                              // [NST]
+    int *pages = reinterpret_cast<int *>(empty + NST);                         // this split's pages
+    __shared__ bool s_last;
+
+    const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int s = 0; s < NST; s++) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], AG_CW);
+        }
+        fence_mbar_init();
+    }
+    pdl_trigger();
+    pdl_wait();
+
+    const int32_t *pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
+    const bool pt_pre = p.max_pages <= ATT_PT_U * AG_THREADS;
+    int pte[ATT_PT_U];
+#pragma unroll
+    for (int u = 0; u < ATT_PT_U; u++) {
+        const int i = tid + u * AG_THREADS;
+        pte[u] = (pt_pre && i < p.max_pages) ? pt[i] : -1;
+    }
+    const int p0 = p.pos[b];
+    int len = p0 + p.R;
+    if (p0 < 0 || len > p.max_pages * 16 || len > p.rope_max_pos) {
+        if (tid == 0) set_error(p.err, BW_DEVERR_BAD_POS);
+        len = max(0, min(len, min(p.max_pages * 16, p.rope_max_pos)));
+    }
+    const int n_pg = (len + 15) / 16;
+    const int pps = (n_pg + p.n_split - 1) / p.n_split;
+    const int pg0 = min(n_pg, split * pps), pg1 = min(n_pg, pg0 + pps);
+    const int npl = pg1 - pg0;                          // pages of this split
+    const int t1 = min(len, pg1 * 16);
+    const int n_stages = (npl + ATT_PPS - 1) / ATT_PPS;
+    const size_t row_stride = static_cast<size_t>(p.nq + 2 * p.nkv) * HD;
+
+    if (pt_pre) {
+#pragma unroll
+        for (int u = 0; u < ATT_PT_U; u++) {
+            const int i = tid + u * AG_THREADS;
+            if (i >= pg0 && i < pg1) {
+                int page = pte[u];
+                if (page < 0 || page >= p.n_pages) {
+                    set_error(p.err, BW_DEVERR_BAD_PAGE);
+                    page = -1;
+                }
+                pages[i - pg0] = page;
+            }
+        }
+    } else {
+        for (int i = tid; i < npl; i += AG_THREADS) {
+            int page = pt[pg0 + i];
+            if (page < 0 || page >= p.n_pages) {
+                set_error(p.err, BW_DEVERR_BAD_PAGE);
+                page = -1;
+            }
+            pages[i] = page;
+        }
+    }
+    __syncthreads();
+
+    if (warp == AG_CW) {
+        // ---- producer: one lane streams the stages
+        if (lane == 0) {
+            for (int s = 0; s < n_stages; s++) {
+                const int st = s % NST;
+                if (s >= NST) mbar_wait(&empty[st], static_cast<uint32_t>((s / NST - 1) & 1), p.err);
+                uint32_t bytes = 0;
+                for (int j = 0; j < ATT_PPS; j++) {
+                    const int lp = s * ATT_PPS + j;
+                    if (lp < npl && pages[lp] >= 0) bytes += 2 * PB;
+                }
+                mbar_arrive_tx(&full[st], bytes);
+                unsigned char *sk = ring + static_cast<size_t>(st) * STB;
+                for (int j = 0; j < ATT_PPS; j++) {
+                    const int lp = s * ATT_PPS + j;
+                    if (lp >= npl || pages[lp] < 0) continue;
+                    const int y = (pages[lp] * p.nkv + kvh) * 16;     // first row of this page
+                    if constexpr (F8) {
+                        // one box of 16 rows x HD bytes per page (swizzled, see land_off)
+                        tma_load_2d(sk + j * PB, &p.tmk, 0, y, &full[st]);
+                        tma_load_2d(sk + STB / 2 + j * PB, &p.tmv, 0, y, &full[st]);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < HD / 64; h++) {
+                            const int box = (j * (HD / 64) + h) << 11;
+                            tma_load_2d(sk + box, &p.tmk, h * 64, y, &full[st]);
+                            tma_load_2d(sk + STB / 2 + box, &p.tmv, h * 64, y, &full[st]);
+                        }
+                    }
+                }
+            }
+        }
+        return;
+    }
+
+    // ---- 1. Q^T: the roped query rows as fp16 hi (columns 0..QP-1) and lo
+    //         (QP..2QP-1) parts, in the MMA's k order; padding rows are zero
+    for (int i = tid; i < QP * (HD / 2); i += AG_CT) {
+        const int qi = i / (HD / 2), d = i - qi * (HD / 2);
+        float ra = 0.0f, rb = 0.0f;
+        if (qi < p.Q) {
+            const int r = qi / p.G, g = qi - r * p.G;
+            const int h = kvh * p.G + g;
+            const int ppos = max(0, min(p0 + r, p.rope_max_pos - 1));
+            const float *src = p.qkv + (static_cast<size_t>(b) * p.R + r) * row_stride + static_cast<size_t>(h) * HD;
+            const float c = p.rope_cos[static_cast<size_t>(ppos) * (HD / 2) + d];
+            const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
+            rope_pair(src[d], src[d + HD / 2], c, s, ra, rb);
+        }
+        __half h0, l0, h1, l1;
+        split_f16(ra, h0, l0);
+        split_f16(rb, h1, l1);
+        const int ka = F8 ? ag_kidx_f8(d) : d, kb = F8 ? ag_kidx_f8(d + HD / 2) : d + HD / 2;
+        qs[qi * QSS + ka] = h0;
+        qs[(QP + qi) * QSS + ka] = l0;
+        qs[qi * QSS + kb] = h1;
+        qs[(QP + qi) * QSS + kb] = l1;
+    }
+
+    // ---- 2. the new rows' k (roped) and v as stored (fp16, or E4M3 codes of
+    //         value / scale): kept for this CTA's stages and written into the pool
+    for (int r = 0; r < p.R; r++) {
+        const int ppos = p0 + r;
+        if (ppos < pg0 * 16 || ppos >= t1) continue;
+        const int page = pages[ppos / 16 - pg0];
+        const bool ok = page >= 0;
+        const size_t off = ((static_cast<size_t>(ok ? page : 0) * p.nkv + kvh) * 16 + (ppos & 15)) * HD;
+        const float *krow = p.qkv + (static_cast<size_t>(b) * p.R + r) * row_stride +
+                            static_cast<size_t>(p.nq + kvh) * HD;
+        const float *vrow = krow + static_cast<size_t>(p.nkv) * HD;
+        for (int d = tid; d < HD / 2; d += AG_CT) {
+            const float c = p.rope_cos[static_cast<size_t>(ppos) * (HD / 2) + d];
+            const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
+            float ra, rb;
+            rope_pair(krow[d], krow[d + HD / 2], c, s, ra, rb);
+            if constexpr (F8) {
+                // E4M3 of value / scale, round to nearest even, saturating to +-448
+                const __nv_fp8_storage_t ca = __nv_cvt_float_to_fp8(__fdiv_rn(ra, p.kscale), __NV_SATFINITE, __NV_E4M3);
+                const __nv_fp8_storage_t cb = __nv_cvt_float_to_fp8(__fdiv_rn(rb, p.kscale), __NV_SATFINITE, __NV_E4M3);
+                newk[r * HD + d] = ca;
+                newk[r * HD + d + HD / 2] = cb;
+                if (ok) {
+                    reinterpret_cast<uint8_t *>(p.k_pool)[off + d] = ca;
+                    reinterpret_cast<uint8_t *>(p.k_pool)[off + d + HD / 2] = cb;
+                }
+            } else {
+                const __half ha = __float2half_rn(ra), hb = __float2half_rn(rb);
+                reinterpret_cast<__half *>(newk)[r * HD + d] = ha;
+                reinterpret_cast<__half *>(newk)[r * HD + d + HD / 2] = hb;
+                if (ok) {
+                    p.k_pool[off + d] = ha;
+                    p.k_pool[off + d + HD / 2] = hb;
+                }
+            }
+        }
+        for (int d = tid; d < HD; d += AG_CT) {
+            if constexpr (F8) {
+                const __nv_fp8_storage_t cv = __nv_cvt_float_to_fp8(__fdiv_rn(vrow[d], p.vscale), __NV_SATFINITE, __NV_E4M3);
+                newv[r * HD + d] = cv;
+                if (ok) reinterpret_cast<uint8_t *>(p.v_pool)[off + d] = cv;
+            } else {
+                const __half hv = __float2half_rn(vrow[d]);
+                reinterpret_cast<__half *>(newv)[r * HD + d] = hv;
+                if (ok) p.v_pool[off + d] = hv;
+            }
+        }
+    }
+    ag_sync();
+
+    // ---- 3. stages of 64 tokens, 16 per warp
+    const int gid = lane >> 2, tig = lane & 3;          // fragment row group / thread in group
+    // this lane's query rows qa, qa + 1 (score and output columns 2 tig, 2 tig + 1)
+    const int qa = NQT == 1 ? 2 * (tig & 1) : 2 * tig;
+    uint32_t qb[NKS][NQT][2];                           // Q^T fragments, held for every stage
+    {
+        const int l8 = lane & 7, kh = ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int kk = 0; kk < NKS; kk++)
+#pragma unroll
+            for (int nt = 0; nt < NQT; nt++)
+                ldsm_x2(qb[kk][nt][0], qb[kk][nt][1], smem_u32(qs + (nt * 8 + l8) * QSS + kk * 16 + kh));
+    }
+    const int tw = warp * 16;                           // this warp's tokens in a stage
+    __half *pw = ps + warp * NC * AG_PST;               // this warp's P^T
+    float m_q[2] = {-INFINITY, -INFINITY}, l_q[2] = {0.0f, 0.0f};
+    float ot[NMT][NQT][4];
+#pragma unroll
+    for (int mt = 0; mt < NMT; mt++)
+#pragma unroll
+        for (int nt = 0; nt < NQT; nt++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) ot[mt][nt][i] = 0.0f;
+
+    for (int s = 0; s < n_stages; s++) {
+        const int st = s % NST;
+        mbar_wait(&full[st], static_cast<uint32_t>((s / NST) & 1), p.err);
+        unsigned char *sk = ring + static_cast<size_t>(st) * STB;
+        unsigned char *sv = sk + STB / 2;
+        const int tb = (pg0 + s * ATT_PPS) * 16;       // position of the stage's first token
+        const int nvalid = min(ATT_ST, t1 - tb);
+        const bool page_ok = s * ATT_PPS + warp < npl && pages[s * ATT_PPS + warp] >= 0;   // this warp's page
+        const bool fix_new = p0 + p.R > tb + tw && p0 < tb + tw + 16;
+        if (fix_new || !page_ok || nvalid < tw + 16) {
+            // this warp's rows written by this step replace what the copy
+            // brought; its V rows the copy did not fill are zeroed (their
+            // probability is 0, and 0 * stale could be NaN)
+            for (int r = 0; r < p.R; r++) {
+                const int slot = p0 + r - tb;
+                if (slot < tw || slot >= tw + 16 || slot >= nvalid || !page_ok) continue;
+                for (int d = lane; d < HD; d += 32) {
+                    if constexpr (F8) {
+                        sk[land_off<HD>(slot, d)] = newk[r * HD + d];
+                        sv[land_off<HD>(slot, d)] = newv[r * HD + d];
+                    } else {
+                        *reinterpret_cast<__half *>(sk + kv_off<HD>(slot, d)) = reinterpret_cast<__half *>(newk)[r * HD + d];
+                        *reinterpret_cast<__half *>(sv + kv_off<HD>(slot, d)) = reinterpret_cast<__half *>(newv)[r * HD + d];
+                    }
+                }
+            }
+            // a token's row is HD / 16 (E4M3) or HD / 8 (fp16) 16-byte chunks: zero them whole
+            constexpr int RC = HD * EB / 16;
+            for (int e = lane; e < 16 * RC; e += 32) {
+                const int T = tw + e / RC, c = e % RC;
+                if (T >= nvalid || !page_ok) {
+                    const uint32_t o16 = F8 ? static_cast<uint32_t>(T * HD + c * 16)
+                                            : static_cast<uint32_t>((((T >> 4) * (HD / 64) + (c >> 3)) << 11) +
+                                                                    ((T & 15) << 7) + ((c & 7) << 4));
+                    *reinterpret_cast<uint4 *>(sv + o16) = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            fence_async_smem();   // a later copy into this stage comes after these writes
+            __syncwarp();
+        }
+        // scores S^T: 16 tokens x NC columns
+        float c[NQT][4];
+#pragma unroll
+        for (int nt = 0; nt < NQT; nt++)
+#pragma unroll
+            for (int i = 0; i < 4; i++) c[nt][i] = 0.0f;
+        if constexpr (F8) {
+#pragma unroll
+            for (int g = 0; g < HD / 64; g++) {
+                const uint4 w0 = *reinterpret_cast<const uint4 *>(sk + land_off<HD>(tw + gid, g * 64 + tig * 16));
+                const uint4 w1 = *reinterpret_cast<const uint4 *>(sk + land_off<HD>(tw + gid + 8, g * 64 + tig * 16));
+                const uint32_t r0[4] = {w0.x, w0.y, w0.z, w0.w}, r1[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    uint32_t a[4];
+                    e4m3x4_to_h4(r0[j], a[0], a[2]);
+                    e4m3x4_to_h4(r1[j], a[1], a[3]);
+#pragma unroll
+                    for (int nt = 0; nt < NQT; nt++) mma16816(c[nt], a, qb[4 * g + j][nt][0], qb[4 * g + j][nt][1]);
+                }
+            }
+        } else {
+            const uint32_t k_a = smem_u32(sk);
+            const int ktok = tw + (lane & 7) + ((lane >> 3) & 1) * 8, kd = (lane >> 4) * 8;
+#pragma unroll
+            for (int kk = 0; kk < NKS; kk++) {
+                uint32_t a[4];
+                ldsm_x4(a, k_a + kv_off<HD>(ktok, kk * 16 + kd));
+#pragma unroll
+                for (int nt = 0; nt < NQT; nt++) mma16816(c[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
+            }
+        }
+        // hi + lo columns: this lane's scores of tokens gid (0, 1) and gid + 8
+        // (2, 3) for query rows qa, qa + 1
+        float sc[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+            sc[i] = NQT == 1 ? c[0][i] + __shfl_xor_sync(0xffffffffu, c[0][i], 2) : c[0][i] + c[NQT - 1][i];
+        const int tokA = tw + gid, tokB = tokA + 8;
+        float corr[2], pr[4];
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+            const int qi = qa + j;
+            const int lim = (qi < p.Q && page_ok) ? min(t1, p0 + qi / p.G + 1) : 0;   // causal limit (exclusive)
+            const float vA = tb + tokA < lim ? sc[j] * p.scale : -INFINITY;
+            const float vB = tb + tokB < lim ? sc[2 + j] * p.scale : -INFINITY;
+            float mx = fmaxf(vA, vB);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float m_new = fmaxf(m_q[j], mx);
+            corr[j] = (m_q[j] == -INFINITY) ? 0.0f : expf(m_q[j] - m_new);
+            m_q[j] = m_new;
+            pr[j] = (vA == -INFINITY) ? 0.0f : expf(vA - m_new);
+            pr[2 + j] = (vB == -INFINITY) ? 0.0f : expf(vB - m_new);
+            l_q[j] = l_q[j] * corr[j] + (pr[j] + pr[2 + j]);
+        }
+        if (__any_sync(0xffffffffu, corr[0] != 1.0f || corr[1] != 1.0f)) {
+#pragma unroll
+            for (int mt = 0; mt < NMT; mt++)
+#pragma unroll
+                for (int nt = 0; nt < NQT; nt++) {
+                    ot[mt][nt][0] *= corr[0];
+                    ot[mt][nt][1] *= corr[1];
+                    ot[mt][nt][2] *= corr[0];
+                    ot[mt][nt][3] *= corr[1];
+                }
+        }
+        // P^T [cols][k] as fp16 hi and lo parts (one part per lane when NQT is
+        // 1: lanes tig and tig ^ 2 hold the same probabilities)
+        {
+            const int kA = F8 ? ag_tidx_f8(gid) : gid, kB = F8 ? ag_tidx_f8(gid + 8) : gid + 8;
+#pragma unroll
+            for (int j = 0; j < 2; j++) {
+                __half hA, lA, hB, lB;
+                split_f16(pr[j], hA, lA);
+                split_f16(pr[2 + j], hB, lB);
+                if constexpr (NQT == 1) {
+                    const bool lo = tig >= 2;
+                    __half *row = pw + ((lo ? QP : 0) + qa + j) * AG_PST;
+                    row[kA] = lo ? lA : hA;
+                    row[kB] = lo ? lB : hB;
+                } else {
+                    pw[(qa + j) * AG_PST + kA] = hA;
+                    pw[(qa + j) * AG_PST + kB] = hB;
+                    pw[(QP + qa + j) * AG_PST + kA] = lA;
+                    pw[(QP + qa + j) * AG_PST + kB] = lB;
+                }
+            }
+        }
+        __syncwarp();
+        uint32_t pb[NQT][2];
+        {
+            const int l8 = lane & 7, i4 = lane >> 3;
+            if constexpr (NQT == 1) {
+                ldsm_x2(pb[0][0], pb[0][1], smem_u32(pw + l8 * AG_PST + (i4 & 1) * 8));
+            } else {
+                uint32_t r4[4];
+                ldsm_x4(r4, smem_u32(pw + ((i4 >> 1) * 8 + l8) * AG_PST + (i4 & 1) * 8));
+                pb[0][0] = r4[0];
+                pb[0][1] = r4[1];
+                pb[NQT - 1][0] = r4[2];
+                pb[NQT - 1][1] = r4[3];
+            }
+        }
+        // O^T += V^T P^T over this warp's 16 tokens
+        if constexpr (F8) {
+#pragma unroll
+            for (int u = 0; u < HD / 32; u++) {
+                uint32_t W[4];
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    W[j] = *reinterpret_cast<const uint32_t *>(sv + land_off<HD>(tw + 4 * tig + j, u * 32 + 4 * gid));
+                // bytes (dim 4 gid + i) of tokens 4 tig + j: m-tile 2u takes dims
+                // i = 0 (row gid) and 1 (row gid + 8), m-tile 2u + 1 dims 2 and 3
+                const uint32_t x01 = ag_prmt(W[0], W[1], 0x5140u), y01 = ag_prmt(W[0], W[1], 0x7362u);
+                const uint32_t x23 = ag_prmt(W[2], W[3], 0x5140u), y23 = ag_prmt(W[2], W[3], 0x7362u);
+                uint32_t a[4];
+                e4m3x4_to_h4(x01, a[0], a[1]);
+                e4m3x4_to_h4(x23, a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NQT; nt++) mma16816(ot[2 * u][nt], a, pb[nt][0], pb[nt][1]);
+                e4m3x4_to_h4(y01, a[0], a[1]);
+                e4m3x4_to_h4(y23, a[2], a[3]);
+#pragma unroll
+                for (int nt = 0; nt < NQT; nt++) mma16816(ot[2 * u + 1][nt], a, pb[nt][0], pb[nt][1]);
+            }
+        } else {
+            const uint32_t v_a = smem_u32(sv);
+            const int vtok = tw + (lane & 7) + ((lane >> 4) & 1) * 8, vd = ((lane >> 3) & 1) * 8;
+#pragma unroll
+            for (int mt = 0; mt < NMT; mt++) {
+                uint32_t a[4];
+                ldsm_x4_t(a, v_a + kv_off<HD>(vtok, mt * 16 + vd));
+#pragma unroll
+                for (int nt = 0; nt < NQT; nt++) mma16816(ot[mt][nt], a, pb[nt][0], pb[nt][1]);
+            }
+        }
+        // this warp is done with the stage: release it to the producer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+    }
+
+    // ---- 4. merge the warps: hi + lo columns, sums over the warp's tokens,
+    //         then every warp's output weighted by exp(m_w - M) into the drained
+    //         ring and summed in warp order into s_o [Q][HD], s_m, s_l
+#pragma unroll
+    for (int j = 0; j < 2; j++) {
+        l_q[j] += __shfl_xor_sync(0xffffffffu, l_q[j], 4);
+        l_q[j] += __shfl_xor_sync(0xffffffffu, l_q[j], 8);
+        l_q[j] += __shfl_xor_sync(0xffffffffu, l_q[j], 16);
+    }
+    float o2[NMT][4];
+#pragma unroll
+    for (int mt = 0; mt < NMT; mt++)
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+            o2[mt][i] = NQT == 1 ? ot[mt][0][i] + __shfl_xor_sync(0xffffffffu, ot[mt][0][i], 2)
+                                 : ot[mt][0][i] + ot[mt][NQT - 1][i];
+    const bool writer = NQT == 2 || tig < 2;            // one lane per (row, query) pair
+    if (writer && gid == 0) {
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+            s_mw[warp * AG_MAXQ + qa + j] = m_q[j];
+            s_lw[warp * AG_MAXQ + qa + j] = l_q[j];
+        }
+    }
+    ag_sync();   // also: every warp is done with the ring
+    float *s_o = reinterpret_cast<float *>(sm);         // [Q][HD] unnormalized output
+    float *s_m = s_o + ATT_MAXQ * HD;                   // [Q]
+    float *s_l = s_m + ATT_MAXQ;                        // [Q]
+    float *scr = reinterpret_cast<float *>(sm + ag_scratch_off<HD>());   // [CW][QP][HD]
+    if (writer) {
+        float wgt[2];
+#pragma unroll
+        for (int j = 0; j < 2; j++) {
+            float M = -INFINITY;
+#pragma unroll
+            for (int w2 = 0; w2 < AG_CW; w2++) M = fmaxf(M, s_mw[w2 * AG_MAXQ + qa + j]);
+            wgt[j] = (m_q[j] == -INFINITY) ? 0.0f : expf(m_q[j] - M);
+        }
+#pragma unroll
+        for (int mt = 0; mt < NMT; mt++)
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                // O^T row gid + 8h of m-tile mt is dim d
+                const int d = F8 ? (mt >> 1) * 32 + 4 * gid + 2 * (mt & 1) + h : mt * 16 + gid + 8 * h;
+#pragma unroll
+                for (int j = 0; j < 2; j++) scr[(warp * QP + qa + j) * HD + d] = o2[mt][2 * h + j] * wgt[j];
+            }
+    }
+    ag_sync();
+    for (int e = tid; e < p.Q * HD; e += AG_CT) {
+        const int qi = e / HD, d = e - qi * HD;
+        float o = 0.0f;
+#pragma unroll
+        for (int w2 = 0; w2 < AG_CW; w2++) o += scr[(w2 * QP + qi) * HD + d];
+        s_o[qi * HD + d] = o;
+    }
+    if (tid < p.Q) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < AG_CW; w2++) M = fmaxf(M, s_mw[w2 * AG_MAXQ + tid]);
+        float L = 0.0f;
+#pragma unroll
+        for (int w2 = 0; w2 < AG_CW; w2++) {
+            const float m2 = s_mw[w2 * AG_MAXQ + tid];
+            L += (m2 == -INFINITY) ? 0.0f : s_lw[w2 * AG_MAXQ + tid] * expf(m2 - M);
+        }
+        s_m[tid] = M;
+        s_l[tid] = L;
+    }
+    ag_sync();
+
+    // ---- 5. the output, or a partial for the split combine
+    if (p.cluster) {
+        // the splits form one thread-block cluster: each CTA merges a slice of
+        // the outputs from every split's shared memory, in split order
+        cg::cluster_group cluster = cg::this_cluster();
+        cluster.sync();
+        const int ns = p.n_split;
+        float *s_w = s_l + ATT_MAXQ;                  // [ns][Q] max, then weight (local only)
+        float *s_sl = s_w + ATT_MAXCL * ATT_MAXQ;     // [ns][Q] sums
+        float *s_L = s_sl + ATT_MAXCL * ATT_MAXQ;     // [Q]
+        for (int e = tid; e < ns * p.Q; e += AG_CT) {
+            const int r2 = e / p.Q, qi = e - r2 * p.Q;
+            s_w[e] = cluster.map_shared_rank(s_m, r2)[qi];
+            s_sl[e] = cluster.map_shared_rank(s_l, r2)[qi];
+        }
+        ag_sync();
+        if (tid < p.Q) {
+            const int qi = tid;
+            float M = -INFINITY;
+            for (int r2 = 0; r2 < ns; r2++) M = fmaxf(M, s_w[r2 * p.Q + qi]);
+            float L = 0.0f;
+            for (int r2 = 0; r2 < ns; r2++) {
+                const float m2 = s_w[r2 * p.Q + qi];
+                const float w = (m2 == -INFINITY) ? 0.0f : expf(m2 - M);
+                s_w[r2 * p.Q + qi] = w;
+                L = fmaf(s_sl[r2 * p.Q + qi], w, L);
+            }
+            s_L[qi] = L;
+        }
+        ag_sync();
+        const int per = (p.Q * HD + ns - 1) / ns;
+        for (int e = split * per + tid; e < min(p.Q * HD, (split + 1) * per); e += AG_CT) {
+            const int qi = e / HD, d = e - qi * HD;
+            float ov[ATT_MAXCL];
+#pragma unroll
+            for (int r2 = 0; r2 < ATT_MAXCL; r2++)
+                ov[r2] = r2 < ns ? cluster.map_shared_rank(s_o, min(r2, ns - 1))[qi * HD + d] : 0.0f;
+            float O = 0.0f;
+#pragma unroll
+            for (int r2 = 0; r2 < ATT_MAXCL; r2++)
+                if (r2 < ns) O = fmaf(ov[r2], s_w[r2 * p.Q + qi], O);
+            const int r = qi / p.G, gq = qi - r * p.G;
+            p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
+                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = (O * p.vscale) / s_L[qi];
+        }
+        cluster.sync();   // keep this CTA's shared memory alive until every reader is done
+        return;
+    }
+    const size_t pbase = (static_cast<size_t>(b) * p.nkv + kvh) * p.n_split;
+    if (p.n_split == 1) {
+        for (int e = tid; e < p.Q * (HD / 4); e += AG_CT) {
+            const int qi = e / (HD / 4), d = (e - qi * (HD / 4)) * 4;
+            const int r = qi / p.G, gq = qi - r * p.G;
+            const float4 o = *reinterpret_cast<const float4 *>(s_o + qi * HD + d);
+            const float L = s_l[qi], vs = p.vscale;
+            *reinterpret_cast<float4 *>(p.out + (static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
+                                        static_cast<size_t>(kvh * p.G + gq) * HD + d) =
+                make_float4((o.x * vs) / L, (o.y * vs) / L, (o.z * vs) / L, (o.w * vs) / L);
+        }
+        return;
+    }
+    for (int e = tid; e < p.Q * (HD / 4); e += AG_CT) {
+        const int qi = e / (HD / 4), d = (e - qi * (HD / 4)) * 4;
+        __stcg(reinterpret_cast<float4 *>(p.part_o + ((pbase + split) * p.Q + qi) * HD + d),
+               *reinterpret_cast<const float4 *>(s_o + qi * HD + d));
+    }
+    if (tid < p.Q)
+        __stcg(reinterpret_cast<float2 *>(p.part_ml + ((pbase + split) * p.Q + tid) * 2), make_float2(s_m[tid], s_l[tid]));
+    // the last split of this (sequence, kv head) to finish combines all of them
+    __threadfence();
+    ag_sync();
+    uint32_t *cnt = p.cnt + static_cast<size_t>(b) * p.nkv + kvh;
+    if (tid == 0) s_last = atomicAdd(cnt, 1u) == static_cast<uint32_t>(p.n_split - 1);
+    ag_sync();
+    if (!s_last) return;
+    __threadfence();
+    const int ns = p.n_split;
+    float *s_w = reinterpret_cast<float *>(sm);            // [ns][Q] max, then weight (the ring is free)
+    float *s_sl = s_w + ATT_MAXNS * ATT_MAXQ;              // [ns][Q] sums
+    float *s_L = s_sl + ATT_MAXNS * ATT_MAXQ;              // [Q]
+    for (int e = tid; e < ns * p.Q; e += AG_CT) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.part_ml + (pbase * p.Q + e) * 2));
+        s_w[e] = ml.x;
+        s_sl[e] = ml.y;
+    }
+    ag_sync();
+    if (tid < p.Q) {
+        const int qi = tid;
+        float M = -INFINITY;
+        for (int r2 = 0; r2 < ns; r2++) M = fmaxf(M, s_w[r2 * p.Q + qi]);
+        float L = 0.0f;
+        for (int r2 = 0; r2 < ns; r2++) {
+            const float m2 = s_w[r2 * p.Q + qi];
+            const float w = (m2 == -INFINITY) ? 0.0f : expf(m2 - M);
+            s_w[r2 * p.Q + qi] = w;
+            L = fmaf(s_sl[r2 * p.Q + qi], w, L);
+        }
+        s_L[qi] = L;
+    }
+    ag_sync();
+    for (int e = tid; e < p.Q * (HD / 4); e += AG_CT) {
+        const int qi = e / (HD / 4), d = (e - qi * (HD / 4)) * 4;
+        const float4 *src = reinterpret_cast<const float4 *>(p.part_o + (pbase * p.Q + qi) * HD + d);
+        const size_t stride = static_cast<size_t>(p.Q) * HD / 4;
+        float4 O = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll 16
+        for (int r2 = 0; r2 < ns; r2++) {
+            const float4 v = __ldcg(src + r2 * stride);
+            const float w = s_w[r2 * p.Q + qi];
+            O.x = fmaf(v.x, w, O.x);
+            O.y = fmaf(v.y, w, O.y);
+            O.z = fmaf(v.z, w, O.z);
+            O.w = fmaf(v.w, w, O.w);
+        }
+        const int r = qi / p.G, gq = qi - r * p.G;
+        const float L = s_L[qi];
+        float *dst = p.out + (static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
+                     static_cast<size_t>(kvh * p.G + gq) * HD + d;
+        const float vs = p.vscale;
+        *reinterpret_cast<float4 *>(dst) = make_float4((O.x * vs) / L, (O.y * vs) / L, (O.z * vs) / L, (O.w * vs) / L);
+    }
+    ag_sync();
+    if (tid == 0) *cnt = 0u;
+}
+
 // Splits per (sequence, kv head).  Many (sequence, kv head) groups: one
 // split, the grid already fills the GPU.  Few: about sqrt(pages) splits --
 // a split streams pages/ns pages, the merge reads ns partials -- bounded so
@@ -927,6 +1597,76 @@ static bw_status attn_go_st(int ns, int nkv, int B, cudaStream_t st, const AttnP
                                                                  : attn_go<HD, MT, 2, F8>(ns, nkv, B, st, p);
 }
 
+template <int HD, int NQT, int NST, int F8>
+static bw_status attn_g_go(int ns, int nkv, int B, bool cl, cudaStream_t st, const AttnParams &p) {
+    const size_t smem = ag_smem_fixed<HD, NQT, NST, F8>() + static_cast<size_t>(p.max_pages) * 4;
+    if (smem > 227 * 1024) return BW_ERR_UNSUPPORTED_SHAPE;
+    static size_t attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return BW_ERR_CUDA;
+    AttnParams q = p;
+    q.n_split = ns;
+    q.cluster = cl ? 1 : 0;
+    {
+        static bool cl_set[64] = {};
+        static std::mutex mu;   // host threads may call the library concurrently
+        std::lock_guard<std::mutex> lk(mu);
+        if (attr_set[dev] < smem) {
+            if (cudaFuncSetAttribute(attn_g_kernel<HD, NQT, NST, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem)) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return BW_ERR_CUDA;
+            }
+            attr_set[dev] = smem;
+        }
+        if (cl && !cl_set[dev]) {
+            if (cudaFuncSetAttribute(attn_g_kernel<HD, NQT, NST, F8>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                     1) != cudaSuccess) {
+                (void)cudaGetLastError();
+                return BW_ERR_CUDA;
+            }
+            cl_set[dev] = true;
+        }
+    }
+    if (!cl) return launch_pdl(attn_g_kernel<HD, NQT, NST, F8>, dim3(ns, nkv, B), dim3(AG_THREADS), smem, st, q);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ns, nkv, B);
+    cfg.blockDim = dim3(AG_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = ns;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    if (cudaLaunchKernelEx(&cfg, attn_g_kernel<HD, NQT, NST, F8>, q) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return BW_ERR_CUDA;
+    }
+    return BW_OK;
+}
+
+// Ring depth and merge of the token-on-M kernel: when every CTA has an SM to
+// itself, a 4-stage ring and (for 2..16 splits) a cluster merge; otherwise
+// two CTAs share an SM: 2 stages of fp16, or 4 of E4M3 (half the bytes).
+template <int HD, int NQT, int F8>
+static bw_status attn_g_st(int ns, int nkv, int B, cudaStream_t st, const AttnParams &p) {
+    const bool deep = static_cast<long>(ns) * nkv * B <= sm_count();
+    const bool cl = deep && ns > 1 && ns <= ATT_MAXCL;
+    if constexpr (F8) {
+        return attn_g_go<HD, NQT, 4, F8>(ns, nkv, B, cl, st, p);
+    } else {
+        const bool fits = ag_smem_fixed<HD, NQT, 4, F8>() + static_cast<size_t>(p.max_pages) * 4 <= 227 * 1024;
+        return deep && fits ? attn_g_go<HD, NQT, 4, F8>(ns, nkv, B, cl, st, p)
+                            : attn_g_go<HD, NQT, 2, F8>(ns, nkv, B, cl, st, p);
+    }
+}
+
 bw_status attn_check(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
                      const void *k_pool, const void *v_pool, const int32_t *page_table, int max_pages, int n_pages,
                      const int32_t *pos, int B, int R, int nq, int nkv, int hd, const float *out, const Scratch &sc) {
@@ -986,6 +1726,17 @@ bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope
     Carver cv(sc.base);
     p.part_o = ns > 1 ? cv.take<float>(static_cast<size_t>(B) * nkv * ns * p.Q * hd) : nullptr;
     p.part_ml = ns > 1 ? cv.take<float>(static_cast<size_t>(B) * nkv * ns * p.Q * 2) : nullptr;
+    if (p.Q <= AG_MAXQ) {
+        // up to 8 query rows: the token-on-M kernel
+        if (f8) {
+            if (hd == 128)
+                return p.Q <= 4 ? attn_g_st<128, 1, 1>(ns, nkv, B, st, p) : attn_g_st<128, 2, 1>(ns, nkv, B, st, p);
+            return p.Q <= 4 ? attn_g_st<64, 1, 1>(ns, nkv, B, st, p) : attn_g_st<64, 2, 1>(ns, nkv, B, st, p);
+        }
+        if (hd == 128)
+            return p.Q <= 4 ? attn_g_st<128, 1, 0>(ns, nkv, B, st, p) : attn_g_st<128, 2, 0>(ns, nkv, B, st, p);
+        return p.Q <= 4 ? attn_g_st<64, 1, 0>(ns, nkv, B, st, p) : attn_g_st<64, 2, 0>(ns, nkv, B, st, p);
+    }
     if (f8) {
         if (hd == 128)
             return p.Q <= 16 ? attn_go_st<128, 1, 1>(ns, nkv, B, st, p) : attn_go_st<128, 2, 1>(ns, nkv, B, st, p);
