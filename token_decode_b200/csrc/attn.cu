@@ -796,7 +796,7 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
 //     S^T [16 tokens x cols]  = K [16 tokens x hd] . Q^T [hd x cols]
 //     O^T [hd x cols]        += V^T [hd x 16 tokens] . P^T [16 tokens x cols]
 // so no MMA row is padding and the hi / lo products cost no second MMA.  Each
-// of the 4 consumer warps owns 16 tokens (one page) of every 64-token stage:
+// consumer warp owns 16 tokens (one page) of every stage:
 // its own running max and sum per query row and its own O^T; nothing crosses
 // warps inside the stage loop.  The hi and lo columns are added, and the warps
 // merged, once at the end.
@@ -807,13 +807,11 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
 // codes in whole 32-bit words -- any order of k gives the same sums, as long
 // as Q and P are written in the same order -- and O^T's rows (dims) in an
 // order that lets one word of V feed two m-tiles.
-constexpr int AG_CW = 4;                          // consumer warps
-constexpr int AG_CT = AG_CW * 32;                 // consumer threads
-constexpr int AG_THREADS = AG_CT + 32;            // + the producer warp
 constexpr int AG_PST = 24;                        // padded P^T row (halves): conflict-free ldmatrix
 constexpr int AG_MAXQ = 8;                        // query rows per (sequence, kv head)
 
-__device__ __forceinline__ void ag_sync() { asm volatile("bar.sync 1, %0;" ::"n"(AG_CT) : "memory"); }
+template <int CT>
+__device__ __forceinline__ void ag_sync() { asm volatile("bar.sync 1, %0;" ::"n"(CT) : "memory"); }
 
 __device__ __forceinline__ uint32_t ag_prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
@@ -835,9 +833,10 @@ __device__ __forceinline__ int ag_tidx_f8(int tau) {
     return 2 * t + (e & 1) + 8 * (e >> 1);
 }
 
-template <int HD, int F8>
+// a stage is one page (16 tokens) per consumer warp, K and V
+template <int HD, int F8, int CW>
 __host__ __device__ constexpr size_t ag_stage_bytes() {
-    return static_cast<size_t>(2) * ATT_ST * HD * (F8 ? 1 : 2);
+    return static_cast<size_t>(2) * 16 * CW * HD * (F8 ? 1 : 2);
 }
 
 // byte offset of the per-warp merge scratch in the drained ring: after the
@@ -847,25 +846,31 @@ __host__ __device__ constexpr size_t ag_scratch_off() {
     return ((static_cast<size_t>(ATT_MAXQ) * HD + 3 * ATT_MAXQ + 2 * ATT_MAXCL * ATT_MAXQ) * 4 + 15) / 16 * 16;
 }
 
-template <int HD, int NQT, int NST, int F8>
+template <int HD, int NQT, int NST, int F8, int CW>
 __host__ __device__ constexpr size_t ag_smem_fixed() {
-    return static_cast<size_t>(NST) * ag_stage_bytes<HD, F8>()                 // K/V ring
+    return static_cast<size_t>(NST) * ag_stage_bytes<HD, F8, CW>()             // K/V ring
            + static_cast<size_t>(8 * NQT) * (HD + 8) * 2                       // Q^T [cols][dims]
-           + static_cast<size_t>(AG_CW) * 8 * NQT * AG_PST * 2                 // P^T per warp [cols][tokens]
+           + static_cast<size_t>(CW) * 8 * NQT * AG_PST * 2                    // P^T per warp [cols][tokens]
            + 2 * static_cast<size_t>(ATT_MAXR) * HD * (F8 ? 1 : 2)            // new k, v rows
-           + 2 * static_cast<size_t>(AG_CW) * AG_MAXQ * 4                     // warp maxima, sums
+           + 2 * static_cast<size_t>(CW) * AG_MAXQ * 4                        // warp maxima, sums
            + 2 * static_cast<size_t>(NST) * 8                                 // mbarriers
            + 1024;                                                            // ring alignment
 }
 
-template <int HD, int NQT, int NST, int F8>
-__global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_constant__ AttnParams p) {
+// CW consumer warps: 4 (two CTAs share an SM) or 8 (a CTA has an SM to itself)
+template <int HD, int NQT, int NST, int F8, int CW>
+__global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(const __grid_constant__ AttnParams p) {
+    constexpr int AG_CW = CW;                   // consumer warps
+    constexpr int AG_CT = CW * 32;              // consumer threads
+    constexpr int AG_THREADS = AG_CT + 32;      // + the producer warp
+    constexpr int AG_ST = 16 * CW;              // tokens per stage: one page per consumer warp
+    constexpr int AG_PPS = CW;
     constexpr int NC = 8 * NQT;                 // MMA columns
     constexpr int QP = 4 * NQT;                 // query rows per part (hi, lo)
     constexpr int QSS = HD + 8;                 // padded Q^T row (halves)
     constexpr int NKS = HD / 16;                // k-steps of the score MMA
     constexpr int NMT = HD / 16;                // m-tiles of O^T
-    constexpr size_t STB = ag_stage_bytes<HD, F8>();
+    constexpr size_t STB = ag_stage_bytes<HD, F8, CW>();
     constexpr uint32_t PB = 16 * HD * (F8 ? 1 : 2);   // bytes of one page of K (or V)
     constexpr int EB = F8 ? 1 : 2;              // bytes of a stored element
     static_assert(ag_scratch_off<HD>() + static_cast<size_t>(AG_CW) * QP * HD * 4 <= NST * STB,
@@ -916,7 +921,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
     const int pg0 = min(n_pg, split * pps), pg1 = min(n_pg, pg0 + pps);
     const int npl = pg1 - pg0;                          // pages of this split
     const int t1 = min(len, pg1 * 16);
-    const int n_stages = (npl + ATT_PPS - 1) / ATT_PPS;
+    const int n_stages = (npl + AG_PPS - 1) / AG_PPS;
     const size_t row_stride = static_cast<size_t>(p.nq + 2 * p.nkv) * HD;
 
     if (pt_pre) {
@@ -951,14 +956,14 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
                 const int st = s % NST;
                 if (s >= NST) mbar_wait(&empty[st], static_cast<uint32_t>((s / NST - 1) & 1), p.err);
                 uint32_t bytes = 0;
-                for (int j = 0; j < ATT_PPS; j++) {
-                    const int lp = s * ATT_PPS + j;
+                for (int j = 0; j < AG_PPS; j++) {
+                    const int lp = s * AG_PPS + j;
                     if (lp < npl && pages[lp] >= 0) bytes += 2 * PB;
                 }
                 mbar_arrive_tx(&full[st], bytes);
                 unsigned char *sk = ring + static_cast<size_t>(st) * STB;
-                for (int j = 0; j < ATT_PPS; j++) {
-                    const int lp = s * ATT_PPS + j;
+                for (int j = 0; j < AG_PPS; j++) {
+                    const int lp = s * AG_PPS + j;
                     if (lp >= npl || pages[lp] < 0) continue;
                     const int y = (pages[lp] * p.nkv + kvh) * 16;     // first row of this page
                     if constexpr (F8) {
@@ -1051,9 +1056,9 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
             }
         }
     }
-    ag_sync();
+    ag_sync<AG_CT>();
 
-    // ---- 3. stages of 64 tokens, 16 per warp
+    // ---- 3. stages of one page per warp
     const int gid = lane >> 2, tig = lane & 3;          // fragment row group / thread in group
     // this lane's query rows qa, qa + 1 (score and output columns 2 tig, 2 tig + 1)
     const int qa = NQT == 1 ? 2 * (tig & 1) : 2 * tig;
@@ -1082,9 +1087,9 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
         mbar_wait(&full[st], static_cast<uint32_t>((s / NST) & 1), p.err);
         unsigned char *sk = ring + static_cast<size_t>(st) * STB;
         unsigned char *sv = sk + STB / 2;
-        const int tb = (pg0 + s * ATT_PPS) * 16;       // position of the stage's first token
-        const int nvalid = min(ATT_ST, t1 - tb);
-        const bool page_ok = s * ATT_PPS + warp < npl && pages[s * ATT_PPS + warp] >= 0;   // this warp's page
+        const int tb = (pg0 + s * AG_PPS) * 16;       // position of the stage's first token
+        const int nvalid = min(AG_ST, t1 - tb);
+        const bool page_ok = s * AG_PPS + warp < npl && pages[s * AG_PPS + warp] >= 0;   // this warp's page
         const bool fix_new = p0 + p.R > tb + tw && p0 < tb + tw + 16;
         if (fix_new || !page_ok || nvalid < tw + 16) {
             // this warp's rows written by this step replace what the copy
@@ -1117,12 +1122,15 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
             fence_async_smem();   // a later copy into this stage comes after these writes
             __syncwarp();
         }
-        // scores S^T: 16 tokens x NC columns
-        float c[NQT][4];
+        // scores S^T: 16 tokens x NC columns, even and odd k-steps in separate
+        // accumulators (two shorter MMA chains)
+        float c[2][NQT][4];
 #pragma unroll
-        for (int nt = 0; nt < NQT; nt++)
+        for (int e = 0; e < 2; e++)
 #pragma unroll
-            for (int i = 0; i < 4; i++) c[nt][i] = 0.0f;
+            for (int nt = 0; nt < NQT; nt++)
+#pragma unroll
+                for (int i = 0; i < 4; i++) c[e][nt][i] = 0.0f;
         if constexpr (F8) {
 #pragma unroll
             for (int g = 0; g < HD / 64; g++) {
@@ -1135,7 +1143,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
                     e4m3x4_to_h4(r0[j], a[0], a[2]);
                     e4m3x4_to_h4(r1[j], a[1], a[3]);
 #pragma unroll
-                    for (int nt = 0; nt < NQT; nt++) mma16816(c[nt], a, qb[4 * g + j][nt][0], qb[4 * g + j][nt][1]);
+                    for (int nt = 0; nt < NQT; nt++) mma16816(c[j & 1][nt], a, qb[4 * g + j][nt][0], qb[4 * g + j][nt][1]);
                 }
             }
         } else {
@@ -1146,15 +1154,17 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
                 uint32_t a[4];
                 ldsm_x4(a, k_a + kv_off<HD>(ktok, kk * 16 + kd));
 #pragma unroll
-                for (int nt = 0; nt < NQT; nt++) mma16816(c[nt], a, qb[kk][nt][0], qb[kk][nt][1]);
+                for (int nt = 0; nt < NQT; nt++) mma16816(c[kk & 1][nt], a, qb[kk][nt][0], qb[kk][nt][1]);
             }
         }
         // hi + lo columns: this lane's scores of tokens gid (0, 1) and gid + 8
         // (2, 3) for query rows qa, qa + 1
         float sc[4];
 #pragma unroll
-        for (int i = 0; i < 4; i++)
-            sc[i] = NQT == 1 ? c[0][i] + __shfl_xor_sync(0xffffffffu, c[0][i], 2) : c[0][i] + c[NQT - 1][i];
+        for (int i = 0; i < 4; i++) {
+            const float c0 = c[0][0][i] + c[1][0][i], c1 = c[0][NQT - 1][i] + c[1][NQT - 1][i];
+            sc[i] = NQT == 1 ? c0 + __shfl_xor_sync(0xffffffffu, c0, 2) : c0 + c1;
+        }
         const int tokA = tw + gid, tokB = tokA + 8;
         float corr[2], pr[4];
 #pragma unroll
@@ -1284,7 +1294,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
             s_lw[warp * AG_MAXQ + qa + j] = l_q[j];
         }
     }
-    ag_sync();   // also: every warp is done with the ring
+    ag_sync<AG_CT>();   // also: every warp is done with the ring
     float *s_o = reinterpret_cast<float *>(sm);         // [Q][HD] unnormalized output
     float *s_m = s_o + ATT_MAXQ * HD;                   // [Q]
     float *s_l = s_m + ATT_MAXQ;                        // [Q]
@@ -1308,7 +1318,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
                 for (int j = 0; j < 2; j++) scr[(warp * QP + qa + j) * HD + d] = o2[mt][2 * h + j] * wgt[j];
             }
     }
-    ag_sync();
+    ag_sync<AG_CT>();
     for (int e = tid; e < p.Q * HD; e += AG_CT) {
         const int qi = e / HD, d = e - qi * HD;
         float o = 0.0f;
@@ -1329,7 +1339,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
         s_m[tid] = M;
         s_l[tid] = L;
     }
-    ag_sync();
+    ag_sync<AG_CT>();
 
     // ---- 5. the output, or a partial for the split combine
     if (p.cluster) {
@@ -1346,7 +1356,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
             s_w[e] = cluster.map_shared_rank(s_m, r2)[qi];
             s_sl[e] = cluster.map_shared_rank(s_l, r2)[qi];
         }
-        ag_sync();
+        ag_sync<AG_CT>();
         if (tid < p.Q) {
             const int qi = tid;
             float M = -INFINITY;
@@ -1360,7 +1370,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
             }
             s_L[qi] = L;
         }
-        ag_sync();
+        ag_sync<AG_CT>();
         const int per = (p.Q * HD + ns - 1) / ns;
         for (int e = split * per + tid; e < min(p.Q * HD, (split + 1) * per); e += AG_CT) {
             const int qi = e / HD, d = e - qi * HD;
@@ -1401,10 +1411,10 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
         __stcg(reinterpret_cast<float2 *>(p.part_ml + ((pbase + split) * p.Q + tid) * 2), make_float2(s_m[tid], s_l[tid]));
     // the last split of this (sequence, kv head) to finish combines all of them
     __threadfence();
-    ag_sync();
+    ag_sync<AG_CT>();
     uint32_t *cnt = p.cnt + static_cast<size_t>(b) * p.nkv + kvh;
     if (tid == 0) s_last = atomicAdd(cnt, 1u) == static_cast<uint32_t>(p.n_split - 1);
-    ag_sync();
+    ag_sync<AG_CT>();
     if (!s_last) return;
     __threadfence();
     const int ns = p.n_split;
@@ -1416,7 +1426,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
         s_w[e] = ml.x;
         s_sl[e] = ml.y;
     }
-    ag_sync();
+    ag_sync<AG_CT>();
     if (tid < p.Q) {
         const int qi = tid;
         float M = -INFINITY;
@@ -1430,7 +1440,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
         }
         s_L[qi] = L;
     }
-    ag_sync();
+    ag_sync<AG_CT>();
     for (int e = tid; e < p.Q * (HD / 4); e += AG_CT) {
         const int qi = e / (HD / 4), d = (e - qi * (HD / 4)) * 4;
         const float4 *src = reinterpret_cast<const float4 *>(p.part_o + (pbase * p.Q + qi) * HD + d);
@@ -1452,7 +1462,7 @@ __global__ void __launch_bounds__(AG_THREADS, 2) attn_g_kernel(const __grid_cons
         const float vs = p.vscale;
         *reinterpret_cast<float4 *>(dst) = make_float4((O.x * vs) / L, (O.y * vs) / L, (O.z * vs) / L, (O.w * vs) / L);
     }
-    ag_sync();
+    ag_sync<AG_CT>();
     if (tid == 0) *cnt = 0u;
 }
 
@@ -1597,9 +1607,9 @@ static bw_status attn_go_st(int ns, int nkv, int B, cudaStream_t st, const AttnP
                                                                  : attn_go<HD, MT, 2, F8>(ns, nkv, B, st, p);
 }
 
-template <int HD, int NQT, int NST, int F8>
+template <int HD, int NQT, int NST, int F8, int CW>
 static bw_status attn_g_go(int ns, int nkv, int B, bool cl, cudaStream_t st, const AttnParams &p) {
-    const size_t smem = ag_smem_fixed<HD, NQT, NST, F8>() + static_cast<size_t>(p.max_pages) * 4;
+    const size_t smem = ag_smem_fixed<HD, NQT, NST, F8, CW>() + static_cast<size_t>(p.max_pages) * 4;
     if (smem > 227 * 1024) return BW_ERR_UNSUPPORTED_SHAPE;
     static size_t attr_set[64] = {};
     int dev = 0;
@@ -1613,7 +1623,7 @@ static bw_status attn_g_go(int ns, int nkv, int B, bool cl, cudaStream_t st, con
         static std::mutex mu;   // host threads may call the library concurrently
         std::lock_guard<std::mutex> lk(mu);
         if (attr_set[dev] < smem) {
-            if (cudaFuncSetAttribute(attn_g_kernel<HD, NQT, NST, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(attn_g_kernel<HD, NQT, NST, F8, CW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(smem)) != cudaSuccess) {
                 (void)cudaGetLastError();
                 return BW_ERR_CUDA;
@@ -1621,7 +1631,7 @@ static bw_status attn_g_go(int ns, int nkv, int B, bool cl, cudaStream_t st, con
             attr_set[dev] = smem;
         }
         if (cl && !cl_set[dev]) {
-            if (cudaFuncSetAttribute(attn_g_kernel<HD, NQT, NST, F8>, cudaFuncAttributeNonPortableClusterSizeAllowed,
+            if (cudaFuncSetAttribute(attn_g_kernel<HD, NQT, NST, F8, CW>, cudaFuncAttributeNonPortableClusterSizeAllowed,
                                      1) != cudaSuccess) {
                 (void)cudaGetLastError();
                 return BW_ERR_CUDA;
@@ -1629,10 +1639,10 @@ static bw_status attn_g_go(int ns, int nkv, int B, bool cl, cudaStream_t st, con
             cl_set[dev] = true;
         }
     }
-    if (!cl) return launch_pdl(attn_g_kernel<HD, NQT, NST, F8>, dim3(ns, nkv, B), dim3(AG_THREADS), smem, st, q);
+    if (!cl) return launch_pdl(attn_g_kernel<HD, NQT, NST, F8, CW>, dim3(ns, nkv, B), dim3((CW + 1) * 32), smem, st, q);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ns, nkv, B);
-    cfg.blockDim = dim3(AG_THREADS);
+    cfg.blockDim = dim3((CW + 1) * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -1644,27 +1654,24 @@ static bw_status attn_g_go(int ns, int nkv, int B, bool cl, cudaStream_t st, con
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, attn_g_kernel<HD, NQT, NST, F8>, q) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, attn_g_kernel<HD, NQT, NST, F8, CW>, q) != cudaSuccess) {
         (void)cudaGetLastError();
         return BW_ERR_CUDA;
     }
     return BW_OK;
 }
 
-// Ring depth and merge of the token-on-M kernel: when every CTA has an SM to
-// itself, a 4-stage ring and (for 2..16 splits) a cluster merge; otherwise
-// two CTAs share an SM: 2 stages of fp16, or 4 of E4M3 (half the bytes).
+// Shape of the token-on-M kernel.  When every CTA has an SM to itself: 8
+// consumer warps (stages of 8 pages) and, for 2..16 splits, a cluster merge;
+// otherwise 4 consumer warps and two CTAs per SM.  Ring: 2 stages of fp16,
+// or 4 of E4M3 (half the bytes).
 template <int HD, int NQT, int F8>
 static bw_status attn_g_st(int ns, int nkv, int B, cudaStream_t st, const AttnParams &p) {
     const bool deep = static_cast<long>(ns) * nkv * B <= sm_count();
     const bool cl = deep && ns > 1 && ns <= ATT_MAXCL;
-    if constexpr (F8) {
-        return attn_g_go<HD, NQT, 4, F8>(ns, nkv, B, cl, st, p);
-    } else {
-        const bool fits = ag_smem_fixed<HD, NQT, 4, F8>() + static_cast<size_t>(p.max_pages) * 4 <= 227 * 1024;
-        return deep && fits ? attn_g_go<HD, NQT, 4, F8>(ns, nkv, B, cl, st, p)
-                            : attn_g_go<HD, NQT, 2, F8>(ns, nkv, B, cl, st, p);
-    }
+    constexpr int NST = F8 ? 4 : 2;
+    return deep ? attn_g_go<HD, NQT, NST, F8, 8>(ns, nkv, B, cl, st, p)
+                : attn_g_go<HD, NQT, NST, F8, 4>(ns, nkv, B, cl, st, p);
 }
 
 bw_status attn_check(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
