@@ -368,6 +368,30 @@ const float *bw_decode_hidden(const bw_model *m, const bw_kv *kv, int B, int n_r
 bw_status bw_decode_moe_route(const bw_model *m, const bw_kv *kv, int B, int n_rows, const void *ws,
                               const int32_t **idx, const float **w);
 
+/* Chunked prefill of one sequence: the prompt tokens[0..n-1] at positions
+ * pos0 .. pos0 + n - 1.  "bw24" deep-dive page (10100.com), section 5, stage 3:
+ * the prompt goes through in chunks, one after another; each chunk updates
+ * the KV cache and only the last one returns logits.  Each chunk of up to
+ * `chunk` tokens runs as one bw_decode_step with n_rows = the chunk's tokens
+ * (rows causal within the chunk, each row's K/V written at its position), so
+ * the cache and the result equal decoding the prompt one token at a time, up
+ * to fp32 summation order.
+ *   kv: its page table's FIRST row is the sequence (for sequence b of a
+ *       batched cache, pass a bw_kv whose page_table points at row b);
+ *   tokens: device int32 [n]; next_token: device int32 [1], the greedy token
+ *   after the last prompt token; logits: device fp32 [V] of that last row, or
+ *   NULL.
+ * 1 <= chunk <= BW_MAX_VERIFY_ROWS, and the decode step's limits for n_rows =
+ * chunk (nq / nkv * chunk <= 32) -- else BW_ERR_UNSUPPORTED_SHAPE;
+ * pos0 + n <= min(16 * max_pages, rope_max_pos) -- else BW_ERR_INVALID_ARG.
+ * Every chunk's checks run before the first launch.  Launches: one position
+ * fill, then ceil(n / chunk) decode steps, then two device copies; graph
+ * capturable.  ws must hold bw_prefill_workspace_bytes(m, kv, chunk) (the
+ * decode step's workspace for n_rows = chunk comes first). */
+bw_status bw_prefill(const bw_model *m, const bw_kv *kv, const int32_t *tokens, int n, int pos0, int chunk,
+                     int32_t *next_token, float *logits, void *ws, size_t ws_bytes, void *stream);
+size_t bw_prefill_workspace_bytes(const bw_model *m, const bw_kv *kv, int chunk);
+
 /* Speculative draft head: K draft tokens for the next verify pass.  "bw24"
  * deep-dive page (10100.com), section 7 (a light MTP draft head sharing the
  * main model's embedding, its output vocabulary pruned to the first ids) and

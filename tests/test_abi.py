@@ -132,3 +132,54 @@ def test_noalloc_gemv_refuses_shapes_beyond_its_fixed_scratch(lib):
     assert lib.bw_gemv_q4_0_noalloc(fake, fake, 0, 512, fake, 1, None, C.c_float(1e-6), None, fake,
                                     None, 0, None) == 1
     assert lib.bw_read_error(fake, None, None) == 1
+
+
+def test_prefill_host_checks_reject_before_any_launch():
+    """bw_prefill refuses, on the host, a chunk the attention cannot hold (7
+    query heads per kv head x 5 rows > 32), a chunk above the verify-row limit,
+    a prompt running past the cache, and a workspace sized for fewer rows.
+    Only calls that must fail before launching are made (descriptors point at
+    host memory)."""
+    import ctypes as C
+    import numpy as np
+    from token_decode_b200 import bw, synth
+    L = bw.lib()
+    keep = []
+
+    def buf(n):
+        a = np.zeros(n + 256, np.uint8)
+        keep.append(a)
+        return a.ctypes.data + (-a.ctypes.data % 256)
+
+    cfg = synth.CONFIGS["7b"].with_(L=1)
+
+    def qw(N, K):
+        q, s = bw.repack_bytes(N, K)
+        return bw.QWeight(cfg.fmt, N, K, buf(q), buf(s), 1.0, 1.0)
+
+    layers = (bw.Layer * 1)()
+    ly = layers[0]
+    ly.attn_norm, ly.ffn_norm = buf(4 * cfg.H), buf(4 * cfg.H)
+    ly.wqkv, ly.wo = qw(cfg.nqkv, cfg.H), qw(cfg.H, cfg.nq * cfg.hd)
+    ly.wgu, ly.wd = qw(2 * cfg.F, cfg.H), qw(cfg.H, cfg.F)
+    maxpos = cfg.max_pages * 16
+    m = bw.Model(1, cfg.H, cfg.nq, cfg.nkv, cfg.hd, cfg.F, cfg.V, 0, 0, 0, cfg.eps, qw(cfg.V, cfg.H),
+                 qw(cfg.V, cfg.H), buf(4 * cfg.H), buf(2 * maxpos * cfg.hd), buf(2 * maxpos * cfg.hd), maxpos,
+                 C.cast(layers, C.c_void_p).value)
+    pool = 16 * 2 * cfg.nkv * cfg.hd
+    kp = (C.c_void_p * 1)(buf(pool))   # never read: every call below fails first
+    vp = (C.c_void_p * 1)(buf(pool))
+    kv = bw.KV(C.cast(kp, C.c_void_p).value, C.cast(vp, C.c_void_p).value, cfg.n_pages, cfg.max_pages,
+               buf(4 * cfg.max_pages), 0, None, None)
+    n8 = L.bw_prefill_workspace_bytes(C.byref(m), C.byref(kv), 8)
+    assert n8 > L.bw_decode_workspace_bytes(C.byref(m), C.byref(kv), 1, 8)
+    ws, tok, nxt = buf(n8), buf(4 * 64), buf(4)
+
+    def run(n, pos0, chunk, ws_bytes=n8):
+        return L.bw_prefill(C.byref(m), C.byref(kv), tok, n, pos0, chunk, nxt, None, ws, ws_bytes, None)
+
+    assert run(8, cfg.ctx, 5) == bw.ERR_UNSUPPORTED_SHAPE     # 7 x 5 query rows
+    assert run(8, cfg.ctx, 9) == bw.ERR_UNSUPPORTED_SHAPE     # above BW_MAX_VERIFY_ROWS
+    assert run(8, maxpos - 4, 4) == bw.ERR_INVALID_ARG        # past the cache
+    assert run(0, cfg.ctx, 4) == bw.ERR_INVALID_ARG
+    assert run(8, cfg.ctx, 4, L.bw_prefill_workspace_bytes(C.byref(m), C.byref(kv), 4) - 1) == bw.ERR_INVALID_ARG

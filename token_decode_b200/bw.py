@@ -32,7 +32,7 @@ EXPORTS = (
     "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
     "bw_paged_attn_decode", "bw_paged_attn_decode_fp8", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
     "bw_moe_workspace_bytes", "bw_decode_step", "bw_decode_workspace_bytes", "bw_decode_hidden", "bw_spec_accept",
-    "bw_decode_moe_route", "bw_mtp_draft", "bw_mtp_workspace_bytes",
+    "bw_decode_moe_route", "bw_mtp_draft", "bw_mtp_workspace_bytes", "bw_prefill", "bw_prefill_workspace_bytes",
 )
 
 
@@ -110,6 +110,8 @@ def lib() -> C.CDLL:
             "bw_decode_moe_route": (i, [p, p, i, i, p, p, p]),
             "bw_mtp_draft": (i, [p, p, p, i, p, p, i, p, z, p]),
             "bw_mtp_workspace_bytes": (z, [p, p]),
+            "bw_prefill": (i, [p, p, p, i, i, i, p, p, p, z, p]),
+            "bw_prefill_workspace_bytes": (z, [p, p, i]),
             "bw_spec_accept": (i, [p, p, i, i, p, p, i, p, p]),
         }
         for name, (res, args) in sig.items():
@@ -296,6 +298,16 @@ def decode_step(model: Model, kv: KV, tokens_in, pos, B, n_rows, tokens_out, ws,
     _check(lib().bw_decode_step(C.byref(model), C.byref(kv), _ptr(tokens_in), _ptr(pos), B, n_rows,
                                 _ptr(tokens_out), _ptr(logits), flags, _ptr(ws), ws.numel(),
                                 _stream(stream)), "bw_decode_step")
+
+
+def prefill_workspace_bytes(model: Model, kv: KV, chunk: int) -> int:
+    return lib().bw_prefill_workspace_bytes(C.byref(model), C.byref(kv), chunk)
+
+
+def prefill(model: Model, kv: KV, tokens, n, pos0, chunk, next_token, ws, logits=None, stream=None):
+    """Chunked prefill of the sequence in kv's first page-table row (see bw.h)."""
+    _check(lib().bw_prefill(C.byref(model), C.byref(kv), _ptr(tokens), n, pos0, chunk, _ptr(next_token),
+                            _ptr(logits), _ptr(ws), ws.numel(), _stream(stream)), "bw_prefill")
 
 
 def mtp_workspace_bytes(model: Model, dh: DraftHead) -> int:

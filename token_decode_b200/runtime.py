@@ -147,6 +147,23 @@ class DeviceDraftHead:
         self._keep = keep + [head.norm]
 
 
+class Prefiller:
+    """Chunked prefill (bw_prefill) of the sequence in the cache's first page-table
+    row: owns the workspace for `chunk` rows per step."""
+
+    def __init__(self, dm: DeviceModel, dkv: DeviceKV, chunk: int):
+        self.dm, self.dkv, self.chunk = dm, dkv, chunk
+        self.ws = bw.workspace(bw.prefill_workspace_bytes(dm.c, dkv.c, chunk))
+        self.next_token = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def run(self, tokens, pos0: int, logits=None, stream=None):
+        """tokens: device int32 [n]; afterwards next_token holds the greedy token
+        after the last prompt token."""
+        bw.prefill(self.dm.c, self.dkv.c, tokens, int(tokens.numel()), int(pos0), self.chunk, self.next_token,
+                   self.ws, logits=logits, stream=stream)
+        return self.next_token
+
+
 class SpecDecoder:
     """Speculative decoding of one sequence with K drafts per pass: a plain step
     gives the first token and the hidden state the draft head starts from; each

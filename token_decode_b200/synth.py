@@ -381,5 +381,10 @@ def start_tokens(cfg: Config, seed: int = 0, n: Optional[int] = None) -> torch.T
     return torch.randint(0, cfg.V, (n,), generator=_gen("cpu", seed, "tokens"), dtype=torch.int32)
 
 
+def prompt_tokens(cfg: Config, n: int, seed: int = 0) -> torch.Tensor:
+    """A synthetic prompt: n token ids uniform over the vocabulary."""
+    return torch.randint(0, cfg.V, (n,), generator=_gen("cpu", seed, "prompt"), dtype=torch.int32)
+
+
 def draft_tokens(cfg: Config, k: int, seed: int = 0) -> torch.Tensor:
     return torch.randint(0, cfg.V, (cfg.B, k), generator=_gen("cpu", seed, "drafts"), dtype=torch.int32)
