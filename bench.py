@@ -375,6 +375,8 @@ def measure(cfg, model, kv, dm, rank, world, local, steps, warmup, cpu_budget, s
     if cfg.verify_k:
         entry["verify_pass"] = verify_pass(cfg, dm, kv, stream, ms_step)
         entry["speculative"] = speculative(cfg, dm, kv, stream, ms_step)
+    if cfg.prefill_prompt and cfg.B == 1:
+        entry["prefill"] = prefill(cfg, dm, kv, stream)
     if rank == 0 and world == 1 and cpu_budget > 0:
         entry["cpu_baseline"] = cpu_baseline(cfg, model, kv, toks, budget_s=cpu_budget)
     del dec, dkv
@@ -411,6 +413,29 @@ def verify_pass(cfg, dm, kv, stream, ms_plain):
     return {"rows": R, "drafts": cfg.verify_k, "ms_per_pass": round(ms, 4),
             "vs_plain_step": round(ms / ms_plain, 3), "device_error_word": err,
             "path": "kernel chain, %d rows per projection" % R}
+
+
+def prefill(cfg, dm, kv, stream):
+    """Chunked prefill (bw_prefill) of a synthetic prompt of cfg.prefill_prompt
+    tokens at positions 0.. into a copy of the cache: device time of one whole
+    prefill after one untimed run (the time to the first token, less the host)."""
+    from token_decode_b200 import bw, runtime, synth
+    chunk = max(1, min(bw.MAX_VERIFY_ROWS, 32 // (cfg.nq // cfg.nkv)))
+    pf = runtime.Prefiller(dm, runtime.DeviceKV(kv.clone()), chunk)
+    tok = synth.prompt_tokens(cfg, cfg.prefill_prompt, 0).to("cuda")
+    with torch.cuda.stream(stream):
+        pf.run(tok, 0, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        pf.run(tok, 0, stream=stream)
+        e1.record(stream)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1)
+    err = bw.read_error(pf.ws, stream)
+    n = cfg.prefill_prompt
+    return {"prompt_tokens": n, "chunk": chunk, "steps": -(-n // chunk), "ms": round(ms, 2),
+            "tok_s": round(n / ms * 1000.0, 1), "device_error_word": err,
+            "path": "bw_prefill: chunks of %d rows through bw_decode_step, logits for the last row only" % chunk}
 
 
 def speculative(cfg, dm, kv, stream, ms_plain, passes=8):
@@ -516,7 +541,7 @@ def run_ours(args):
     }
     for k in ("path", "hbm_gbs_step", "roofline_step_frac_of_8tbs", "roofline_step_frac_of_measured",
               "bytes_per_step", "roofline", "kernels", "e2e", "gpu_launches", "device_error_word", "clocks",
-              "cpu_baseline", "verify_pass", "speculative"):
+              "cpu_baseline", "verify_pass", "speculative", "prefill"):
         if k in h:
             line[k] = h[k]
     line["configs"] = {n: e for n, e in entries.items() if n != names[0]}

@@ -5,7 +5,8 @@ launching stream, reported as microseconds per launch and algorithmic GB/s
 (the bytes of weights and KV that launch must touch, divided by its time).
 
 "step" (batch 1, dense models) is the whole decode step run as one persistent
-kernel (bw_decode_step with BW_STEP_PERSISTENT).
+kernel (bw_decode_step with BW_STEP_PERSISTENT); "chain" is the whole step as
+its usual chain of launches (for launch lists under ncu).
 
 Also the small, self-contained target for `ncu` captures:
 
@@ -120,6 +121,16 @@ class KernelBench:
                 bw.decode_step(dm.c, dkv.c, tin, self.pos, 1, 1, tout, self._sws, flags=bw.STEP_PERSISTENT,
                                stream=self.st)
             out["step"] = (step, lambda l: step_b, 1)
+        if self.with_chain:
+            # the whole step as the usual chain of launches (bw_decode_step): the
+            # target of launch-list captures; bytes as for "step"
+            tin = torch.zeros(self.B, dtype=torch.int32, device="cuda")
+            tout = torch.zeros(self.B, dtype=torch.int32, device="cuda")
+            self._cws = bw.workspace(bw.decode_workspace_bytes(dm.c, dkv.c, self.B, 1))
+
+            def chain(l):
+                bw.decode_step(dm.c, dkv.c, tin, self.pos, self.B, 1, tout, self._cws, stream=self.st)
+            out["chain"] = (chain, lambda l: 0, 1)
         lm = dm.c.lm_head
         out["lm_head"] = (lambda l: self._gemv(lm, self.x, self.logits, bw.GEMV_RMSNORM | bw.GEMV_ARGMAX,
                                                gamma=self.gamma, argmax_out=self.am),
@@ -128,6 +139,7 @@ class KernelBench:
 
     moe_expert_bytes = 0
     with_step = False   # also the persistent whole-step kernel (only when asked for by name)
+    with_chain = False  # also the whole step as its chain of launches (only when asked for by name)
 
     def time(self, name, reps=10):
         """Graph of the kind over all its layers, replayed `reps` times."""
@@ -175,6 +187,7 @@ def moe_touched_bytes(dm, B, kb: KernelBench) -> int:
 def run_all(dm, dkv, B, stream, pos, reps=10, only=None):
     kb = KernelBench(dm, dkv, B, stream, pos)
     kb.with_step = only == "step"
+    kb.with_chain = only == "chain"
     if dm.cfg.n_experts:
         kb.moe_expert_bytes = moe_touched_bytes(dm, B, kb)
     res = {}
@@ -213,6 +226,7 @@ def main():
     if a.eager:
         kb = KernelBench(dm, dkv, cfg.B, st, pos)
         kb.with_step = a.only == "step"
+        kb.with_chain = a.only == "chain"
         if cfg.n_experts:
             kb.moe_expert_bytes = moe_touched_bytes(dm, cfg.B, kb)
         for name, (fn, _, n) in kb.kinds().items():

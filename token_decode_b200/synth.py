@@ -60,6 +60,7 @@ class Config:
     verify_k: int = 0   # draft tokens checked by one speculative-verify pass
     draft_vocab: int = 32768   # output ids of the speculative draft head (the first ids)
     kv_fp8: bool = False       # the KV cache in E4M3 with per-layer scales (make_kv_fp8)
+    prefill_prompt: int = 0    # prompt tokens of a timed chunked prefill (0: none)
 
     @property
     def nqkv(self) -> int:
@@ -81,7 +82,7 @@ CONFIGS = {
     "tiny": Config("tiny-1L-h256-q4_0", L=1, H=256, nq=4, nkv=2, hd=64, F=704, V=1024,
                    fmt=FMT_Q4_0, ctx=128, steps=8, draft_vocab=256),
     "7b": Config("7b-dense-q4_0", L=28, H=3584, nq=28, nkv=4, hd=128, F=18944, V=152064,
-                 fmt=FMT_Q4_0, ctx=2000, steps=512),
+                 fmt=FMT_Q4_0, ctx=2000, steps=512, prefill_prompt=2000),
     "9b": Config("9b-dense-nvfp4", L=36, H=4096, nq=32, nkv=8, hd=128, F=12288, V=151936,
                  fmt=FMT_NVFP4, ctx=4096, steps=256),
     "9b_b32": Config("9b-dense-nvfp4-b32", L=36, H=4096, nq=32, nkv=8, hd=128, F=12288,
