@@ -148,18 +148,25 @@ def step_bytes(cfg, model, avg_ctx, moe_layer_bytes=0):
     return model.weight_bytes_dense() + kv_read + kv_write + moe
 
 
-# ncu summaries of the dominant kernel: DRAM traffic per launch, valid while the
-# kernel's sources hash to the recorded value
+# ncu summaries of the dominant kernels: DRAM traffic per launch, valid while the
+# kernel sources a summary lists still hash to the value it records
 _PROFILE_FILES = {("gu", "7b-dense-q4_0"): "gemv_gate_up_7b.md",
-                  ("step", "7b-dense-q4_0"): "step_persistent_7b.md"}
-_KERNEL_SOURCES = {"gu": ("gemv.cu", "gemv_core.cuh", "bw_common.cuh"),
-                   "step": ("step_persistent.cu", "gemv_core.cuh", "bw_common.cuh")}
+                  ("down", "7b-dense-q4_0"): "gemv_down_7b.md",
+                  ("qkv", "7b-dense-q4_0"): "gemv_qkv_7b.md",
+                  ("o", "7b-dense-q4_0"): "gemv_o_7b.md",
+                  ("lm_head", "7b-dense-q4_0"): "gemv_lm_head_7b.md",
+                  ("attn", "7b-dense-q4_0"): "attn_7b_b1.md",
+                  ("attn", "27b-dense-nvfp4"): "attn_27b_b1.md",
+                  ("attn", "9b-dense-nvfp4-b32"): "attn_9b_b32.md",
+                  ("attn", "9b-dense-nvfp4-b32-fp8kv"): "attn_9b_b32_fp8.md",
+                  ("gu", "9b-dense-nvfp4-b32"): "mma_gemm_gate_up_9b_b32.md",
+                  ("moe", "35b-a3b-moe-nvfp4-b32"): "moe_grouped_gemv_b32.md"}
 
 
-def kernel_sources_sha(kind):
+def kernel_sources_sha(files):
     import hashlib
     h = hashlib.sha256()
-    for f in _KERNEL_SOURCES[kind]:
+    for f in files:
         with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "token_decode_b200",
                                "csrc", f), "rb") as fh:
             h.update(fh.read())
@@ -168,8 +175,6 @@ def kernel_sources_sha(kind):
 
 def _ncu_traffic(kind, cfg_name):
     name = _PROFILE_FILES.get((kind, cfg_name))
-    if kind not in _KERNEL_SOURCES:
-        return None
     if name is None:
         return None
     path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles", name)
@@ -180,11 +185,12 @@ def _ncu_traffic(kind, cfg_name):
         if ln.startswith("- ") and ":" in ln:
             k, v = ln[2:].split(":", 1)
             vals[k.strip().strip("`")] = v.strip().strip("`")
-    if vals.get("kernel_sources_sha") != kernel_sources_sha(kind):
-        return None
+    files = vals.get("kernel_sources", "").split()
     try:
+        if not files or vals.get("kernel_sources_sha") != kernel_sources_sha(files):
+            return None
         return int(vals["traffic_bytes_per_launch"])
-    except (KeyError, ValueError):
+    except (KeyError, ValueError, OSError):
         return None
 
 
@@ -275,7 +281,10 @@ def measure(cfg, model, kv, dm, rank, world, local, steps, warmup, cpu_budget, s
     for op in warm_ops + timed_ops:
         if op != "reset":
             graph_for(op)
-    # graph capture ran extra steps: rebuild the exact start, then warm up
+    # a graph's first replay also uploads it to the device: replay every graph
+    # the timed region uses once, untimed
+    run(timed_ops)
+    # capture and upload ran extra steps: rebuild the exact start, then warm up
     with torch.cuda.stream(stream):
         reset()
     run(warm_ops)
