@@ -15,14 +15,21 @@
 // to fp16 (RNE) for the B operand -- the only rounding beyond fp32
 // reordering, graded by tolerance.
 //
-// One CTA per SM, 6 warps:
+// One CTA per SM, 10 warps:
 //   warp 0     producer: streams weight tiles (32 KB codes + 4 KB scales, the
 //              tiled layout of bw.h) into a ring of shared-memory stages with
 //              plain bulk copies (no multicast);
 //   warp 1     owns the tensor memory (alloc/dealloc); lane 0 issues the MMAs;
 //   warps 2..5 dequantize (one weight row per thread: TMEM lane = row) into
-//              A slots in tensor memory with tcgen05.st, then run the
-//              epilogue from the accumulator (tcgen05.ld).
+//              A slots in tensor memory with tcgen05.st;
+//   warps 6..9 run each row block's epilogue from its accumulator (tcgen05.ld):
+//              once it is in registers the next row block's MMAs start, and the
+//              rest of the epilogue (split-K partial sums, residual, SiLU gate,
+//              argmax) overlaps them.
+// A tcgen05.mma of M = 128, K = 16 costs the issuing thread about 150-200
+// cycles whatever N (16..256) and wherever A lives (measured on a B200), so at
+// N = 32 the MMA issue sets the pace (one 64-column A slot = 4 MMAs); the
+// dequant of a slot takes less, and the epilogue must not stall it.
 // MMA: kind::f16, M = 128 weight rows, N = the activation rows padded to 16
 // or 32, K = 16 per instruction; A from tensor memory, B from shared memory
 // in the canonical K-major layout without swizzle.  The activations are
@@ -37,7 +44,7 @@
 
 namespace bw {
 
-constexpr int MM_THREADS = 192;
+constexpr int MM_THREADS = 320;
 constexpr int MM_DW = 4;                 // dequant / epilogue warps (warps 2..5)
 constexpr int MM_NA = 4;                 // A slots in tensor memory, 64 columns of K each
 constexpr int MM_SLOT_COLS = 32;         // 64 fp16 per row = 32 x 32-bit columns
@@ -142,7 +149,16 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
         :
         : "memory");
 }
-__device__ __forceinline__ void dq_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// atomic add with acquire-release semantics at GPU scope (the split-K
+// arrival counter: it publishes this CTA's partial sums and, for the last
+// arriver, acquires everyone else's)
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *addr, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+    return old;
+}
+// the four epilogue warps' barrier
+__device__ __forceinline__ void ep_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // Shared-memory matrix descriptor, K-major canonical layout without swizzle:
 // 8-row x 16-byte core matrices, `lbo` bytes between the two core matrices
@@ -200,8 +216,8 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
     uint64_t *bars = reinterpret_cast<uint64_t *>(bsm + b_bytes);
     uint64_t *full = bars, *empty = bars + MM_NST;
     uint64_t *afull = empty + MM_NST, *aempty = afull + MM_NA;
-    uint64_t *dfull = aempty + MM_NA, *dempty = dfull + 2;
-    uint64_t *bfull = dempty + 2;
+    uint64_t *dfull = aempty + MM_NA, *dread = dfull + 2;
+    uint64_t *bfull = dread + 1;
     __shared__ uint32_t s_tmem;
     __shared__ float s_bv[MM_DW][MM_MAXM];
     __shared__ int s_bi[MM_DW][MM_MAXM];
@@ -224,10 +240,8 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
             mbar_init(&afull[i], MM_DW);
             mbar_init(&aempty[i], 1);
         }
-        for (int i = 0; i < 2; i++) {
-            mbar_init(&dfull[i], 1);
-            mbar_init(&dempty[i], MM_DW);
-        }
+        for (int i = 0; i < 2; i++) mbar_init(&dfull[i], 1);
+        mbar_init(dread, MM_DW);
         mbar_init(bfull, 1);
         fence_mbar_init();
     }
@@ -279,7 +293,11 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
             int g = 0;   // A-slot step
             for (int item = 0; item < n_items; item++) {
                 const int db = item & 1;
-                if (item >= 2) mbar_wait(&dempty[db], static_cast<uint32_t>(((item - 2) / 2) & 1), p.err);
+                // the previous row block's accumulator is in the epilogue warps'
+                // registers: MMAs running while another warp reads tensor memory
+                // with tcgen05.ld corrupted lanes of that read on a B200 (even
+                // with the two accumulators 64 columns apart), so they never overlap
+                if (item >= 1) mbar_wait(dread, static_cast<uint32_t>((item - 1) & 1), p.err);
                 tc_fence_after();
                 const uint32_t d_t = tmem + MM_ACC_COL + static_cast<uint32_t>(db * p.Mp);
                 for (int kt = 0; kt < T; kt++) {
@@ -302,24 +320,13 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
             }
         }
         __syncwarp();
-    } else {
-        // ---- dequant + epilogue warps: quarter qd of the tile rows
-        const int dw = warp - 2;                  // 0..3 (arrival bookkeeping)
+    } else if (warp < 2 + MM_DW) {
+        // ---- dequant warps: quarter qd of the tile rows into the A slots
         const int qd = warp & 3;                  // tensor-memory lane quarter this warp may access
         const int r = qd * 32 + lane;             // tile row = tensor-memory lane
-        const int dtid = dw * 32 + lane;          // 0..127
         const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16);
-        const float tsc = ((p.flags & BW_GEMV_SILU_GATE) && (r & 7) >= 4) ? p.ts_up : p.ts;
-        float bestv[MM_MAXM];
-        int besti[MM_MAXM];
-#pragma unroll
-        for (int m = 0; m < MM_MAXM; m++) {
-            bestv[m] = -INFINITY;
-            besti[m] = 0x7fffffff;
-        }
         int g = 0, t = 0;
         for (int item = 0; item < n_items; item++) {
-            const int rb = j0 + item * p.per_slice;
             for (int kt = 0; kt < T; kt++, t++) {
                 const int s = t % MM_NST;
                 mbar_wait(&full[s], static_cast<uint32_t>((t / MM_NST) & 1), p.err);
@@ -351,6 +358,25 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
                     if (lane == 0) mbar_arrive(&afull[a]);
                 }
             }
+        }
+    } else {
+        // ---- epilogue warps: each row block's accumulator (quarter qd of its
+        //      rows) while the next row block's MMAs run
+        const int ew = warp - 2 - MM_DW;          // 0..3 (arrival bookkeeping)
+        const int qd = warp & 3;                  // tensor-memory lane quarter this warp may access
+        const int r = qd * 32 + lane;             // tile row = tensor-memory lane
+        const int dtid = ew * 32 + lane;          // 0..127
+        const uint32_t t_row = tmem + (static_cast<uint32_t>(qd * 32) << 16);
+        const float tsc = ((p.flags & BW_GEMV_SILU_GATE) && (r & 7) >= 4) ? p.ts_up : p.ts;
+        float bestv[MM_MAXM];
+        int besti[MM_MAXM];
+#pragma unroll
+        for (int m = 0; m < MM_MAXM; m++) {
+            bestv[m] = -INFINITY;
+            besti[m] = 0x7fffffff;
+        }
+        for (int item = 0; item < n_items; item++) {
+            const int rb = j0 + item * p.per_slice;
             // ---- accumulator of this row block (the epilogue reads what earlier
             //      kernels wrote: wait for them once)
             if (item == 0) pdl_wait();
@@ -365,7 +391,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
             tmem_ld_wait(acc_u);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&dempty[db]);
+            if (lane == 0) mbar_arrive(dread);
             float v[MM_MAXM];
 #pragma unroll
             for (int m = 0; m < MM_MAXM; m++) v[m] = __uint_as_float(acc_u[m]);
@@ -378,10 +404,14 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
                 for (int m = 0; m < MM_MAXM; m += 4)
                     if (m < p.Mp)
                         __stcg(reinterpret_cast<float4 *>(dst + m), make_float4(v[m], v[m + 1], v[m + 2], v[m + 3]));
+                // release every lane's partial sums, then count this slice's arrival
                 __threadfence();
-                dq_sync();
-                if (dtid == 0) s_last = atomicAdd(p.rb_cnt + rb, 1u) == static_cast<uint32_t>(p.S - 1);
-                dq_sync();
+                ep_sync();
+                if (dtid == 0) {
+                    __threadfence();
+                    s_last = atom_add_acq_rel(p.rb_cnt + rb, 1u) == static_cast<uint32_t>(p.S - 1);
+                }
+                ep_sync();
                 act = s_last;
                 if (act) {
                     __threadfence();
@@ -447,11 +477,11 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
                     }
                 }
                 if (lane == 0) {
-                    s_bv[dw][m] = bv;
-                    s_bi[dw][m] = bi;
+                    s_bv[ew][m] = bv;
+                    s_bi[ew][m] = bi;
                 }
             }
-            dq_sync();
+            ep_sync();
             if (dtid < p.M) {
                 const int m = dtid;
                 float bv = s_bv[0][m];
@@ -465,12 +495,12 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
                 __stcg(p.am_idx + blockIdx.x * p.Mp + m, bi);
             }
             __threadfence();
-            dq_sync();
+            ep_sync();
             if (dtid == 0) s_last = atomicAdd(p.am_cnt, 1u) == gridDim.x - 1;
-            dq_sync();
+            ep_sync();
             if (s_last) {
                 __threadfence();
-                for (int m = dw; m < p.M; m += MM_DW) {
+                for (int m = ew; m < p.M; m += MM_DW) {
                     float bv = -INFINITY;
                     int bi = 0x7fffffff;
                     for (int b = lane; b < static_cast<int>(gridDim.x); b += 32) {
@@ -587,9 +617,11 @@ static MmaPlan plan_mma(int N, int K, int Mp) {
         if (fixed + mma_b_bytes(Mp, CT) > MM_SMEM_LIMIT) continue;
         const int per_slice = max(1, min(RB, G / S));
         const int rounds = (RB + per_slice - 1) / per_slice;
-        // an item costs its tiles; the activation staging costs about a tile per
-        // slice; split K adds a partial-sum pass
-        const double cost = static_cast<double>(rounds) * (CT + (S > 1 ? 1.0 : 0.5)) + 0.5 * CT;
+        // the MMAs of a CTA's tiles are the critical path (the epilogue warps
+        // overlap them); split K adds an item's fp32 partial sums, 128 x Mp x 4
+        // bytes against a tile's 36 KB, that go back to memory
+        const double part = S > 1 ? 128.0 * Mp * 4 / GV_STAGE_BYTES : 0.0;
+        const double cost = static_cast<double>(rounds) * (CT + part) + 0.01 * S;
         if (cost < best - 1e-9) {
             best = cost;
             bestS = S;
