@@ -546,6 +546,8 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
 // * 16 bytes; the column tiles of K are therefore contiguous blocks.  Rows
 // M..Mp-1 and columns K..KT*512-1 are zero.  With gamma, the row is
 // normalized first: (x * r) * gamma, r = 1 / sqrt(mean(x^2) + eps).
+// Grid (Mp, KT): each CTA packs one 512-column tile of one row (and sums the
+// squares of the whole row for its norm -- a few KB from L2).
 __global__ void act_pack_kernel(const float *x, int M, int Mp, int K, int KT, const float *gamma, float eps,
                                 uint8_t *out) {
     pdl_trigger();
@@ -569,8 +571,9 @@ __global__ void act_pack_kernel(const float *x, int M, int Mp, int K, int KT, co
         __syncthreads();
     }
     const float rn = (gamma && real) ? s_rn : 1.0f;
-    const int KC = KT * 64;
-    for (int kc = threadIdx.x; kc < KC; kc += blockDim.x) {
+    // this CTA's column tile: 64 core columns of 8
+    const int kc1 = (blockIdx.y + 1) * 64;
+    for (int kc = blockIdx.y * 64 + threadIdx.x; kc < kc1; kc += blockDim.x) {
         const int k = kc * 8;
         uint32_t h[4] = {0u, 0u, 0u, 0u};
         if (real && k < K) {
@@ -711,7 +714,7 @@ bw_status mma_gemm_launch(const void *wq, const void *ws_scales, float ts, float
         p.adv_tokens = adv_tokens ? adv_tokens + m0 : nullptr;
         p.adv_pos = adv_pos ? adv_pos + m0 : nullptr;
         p.err = sc.err;
-        const bw_status s0 = launch_pdl(act_pack_kernel, dim3(Mp), dim3(256), 0, st, x + static_cast<size_t>(m0) * K,
+        const bw_status s0 = launch_pdl(act_pack_kernel, dim3(Mp, p.KT), dim3(256), 0, st, x + static_cast<size_t>(m0) * K,
                                         Mr, Mp, K, p.KT, (flags & BW_GEMV_RMSNORM) ? gamma : nullptr, eps, bpk);
         if (s0 != BW_OK) return s0;
         {
