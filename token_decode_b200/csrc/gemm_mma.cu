@@ -397,6 +397,15 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
             for (int m = 0; m < MM_MAXM; m++) v[m] = __uint_as_float(acc_u[m]);
 
             const int n = rb * GV_TR + r;
+            // the residual rows of this output row, all loads issued at once
+            // (y may be the residual itself, so they cannot wait for the
+            // stores), before the split-K hand-off whose round trip they overlap
+            float res[MM_MAXM];
+            if ((p.flags & BW_GEMV_RESIDUAL) && n < p.N) {
+#pragma unroll
+                for (int m = 0; m < MM_MAXM; m++)
+                    res[m] = m < p.M ? __ldcg(p.residual + static_cast<size_t>(m) * p.N + n) : 0.0f;
+            }
             bool act = true;
             if (p.S > 1) {
                 float *dst = p.partial + (static_cast<size_t>(slice) * p.RB * GV_TR + n) * p.Mp;
@@ -404,17 +413,18 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
                 for (int m = 0; m < MM_MAXM; m += 4)
                     if (m < p.Mp)
                         __stcg(reinterpret_cast<float4 *>(dst + m), make_float4(v[m], v[m + 1], v[m + 2], v[m + 3]));
-                // release every lane's partial sums, then count this slice's arrival
-                __threadfence();
+                // every lane's partial sums are written (barrier), then one thread
+                // publishes them and counts this slice's arrival: a GPU-scope
+                // fence after the barrier covers the other lanes' stores
                 ep_sync();
                 if (dtid == 0) {
                     __threadfence();
                     s_last = atom_add_acq_rel(p.rb_cnt + rb, 1u) == static_cast<uint32_t>(p.S - 1);
+                    if (s_last) __threadfence();
                 }
                 ep_sync();
                 act = s_last;
                 if (act) {
-                    __threadfence();
 #pragma unroll
                     for (int m = 0; m < MM_MAXM; m++) v[m] = 0.0f;
                     for (int s2 = 0; s2 < p.S; s2++) {
@@ -450,7 +460,7 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
                     if (m >= p.M) break;
                     float val = v[m];
                     const size_t o = static_cast<size_t>(m) * p.N + n;
-                    if (p.flags & BW_GEMV_RESIDUAL) val = p.residual[o] + val;
+                    if (p.flags & BW_GEMV_RESIDUAL) val = res[m] + val;
                     if (p.y) p.y[o] = val;
                     if (better(val, n, bestv[m], besti[m])) {
                         bestv[m] = val;
