@@ -490,7 +490,7 @@ def speculative(cfg, dm, kv, stream, ms_plain, passes=8):
 
 
 KERNEL_NAMES = {"gu": "gemv_kernel (fused RMSNorm + gate/up + SiLU gate)", "down": "gemv_kernel (down + residual)",
-                "attn": "attn_kernel (paged GQA decode attention)", "qkv": "gemv_kernel (RMSNorm + QKV)",
+                "attn": "attn_g_kernel (paged GQA decode attention; attn_kernel above 8 query rows per kv head)", "qkv": "gemv_kernel (RMSNorm + QKV)",
                 "o": "gemv_kernel (O + residual)", "lm_head": "gemv_kernel (LM head + argmax)",
                 "moe": "MoE FFN (route + grouped expert GEMVs + combine)"}
 
