@@ -144,6 +144,38 @@ def test_launch_count_claim_matches_the_committed_launch_lists():
     assert bench.step_launches(moe) - bench.step_launches(dense) == moe.L * (6 - 2 * 2)
     text = open(os.path.join(ROOT, "profiles", "launches_moe_layer_b32.md")).read()
     assert re.search(r"^12 launches", text, flags=re.M)
+    # at 32 rows every NVFP4 projection is an activation pack plus a tensor-core GEMM
+    text = open(os.path.join(ROOT, "profiles", "launches_decode_step_9b_b32.md")).read()
+    n_listed = int(re.search(r"^(\d+) launches", text, flags=re.M).group(1))
+    assert bench.step_launches(synth.CONFIGS["9b_b32"]) == n_listed == 1 + 36 * 9 + 2
+
+
+def test_roofline_traffic_only_from_a_summary_of_the_current_sources(tmp_path, monkeypatch):
+    """roofline.traffic comes from a committed ncu summary only while the
+    kernel sources it lists still hash to the value it records."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    srcs = ["gemv.cu", "bw_common.cuh"]
+    sha = bench.kernel_sources_sha(srcs)
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    good = "- kernel_sources: `%s`\n- kernel_sources_sha: `%s`\n- traffic_bytes_per_launch: `1234`\n" % (
+        " ".join(srcs), sha)
+    (prof / "good.md").write_text(good)
+    (prof / "stale.md").write_text(good.replace(sha, "0" * 16))
+    (prof / "nosrc.md").write_text("- traffic_bytes_per_launch: `99`\n")
+    monkeypatch.setattr(bench, "_PROFILE_FILES", {("a", "c"): "good.md", ("b", "c"): "stale.md",
+                                                  ("d", "c"): "nosrc.md", ("e", "c"): "missing.md"})
+    # summaries looked up under tmp_path; the hash of the real sources as computed above
+    monkeypatch.setattr(bench, "__file__", str(tmp_path / "bench.py"))
+    monkeypatch.setattr(bench, "kernel_sources_sha", lambda files: sha if files == srcs else "-")
+    assert bench._ncu_traffic("a", "c") == 1234
+    assert bench._ncu_traffic("b", "c") is None
+    assert bench._ncu_traffic("d", "c") is None
+    assert bench._ncu_traffic("e", "c") is None
+    assert bench._ncu_traffic("zz", "c") is None
 
 
 def test_step_bytes_counts_weights_kv_and_routed_experts():
