@@ -68,7 +68,9 @@ struct AttnParams {
     const int32_t *pos;
     int B, R, nq, nkv, G, Q, n_split;
     int cluster;          // 1: the splits of a (sequence, kv head) are one cluster and merge through DSMEM
+    int early;            // 1: pos and the page table are complete before this launch (see attn_launch)
     float scale;          // 1/sqrt(hd), times the K scale with FP8 KV
+    float scale2;         // scale * log2(e) (base-2 softmax)
     float kscale, vscale; // FP8 KV: a stored code c stands for e4m3(c) * scale (1 for fp16)
     float *out;
     float *part_o;        // [B][nkv][n_split][Q][HD]
@@ -853,8 +855,41 @@ __host__ __device__ constexpr size_t ag_smem_fixed() {
            + static_cast<size_t>(CW) * 8 * NQT * AG_PST * 2                    // P^T per warp [cols][tokens]
            + 2 * static_cast<size_t>(ATT_MAXR) * HD * (F8 ? 1 : 2)            // new k, v rows
            + 2 * static_cast<size_t>(CW) * AG_MAXQ * 4                        // warp maxima, sums
-           + 2 * static_cast<size_t>(NST) * 8                                 // mbarriers
+           + (2 * static_cast<size_t>(NST) + 2) * 8                           // mbarriers
            + 1024;                                                            // ring alignment
+}
+
+// Cluster merge: each non-leader split writes its partial -- O [Q][HD]
+// (unnormalized), then (max, sum) per query row -- into slot rank - 1 of the
+// leader's receive area, which follows the page list.
+__host__ __device__ constexpr int ag_slot_floats(int Q, int HD) { return (Q * HD + 2 * Q + 3) / 4 * 4; }
+__host__ __device__ constexpr uint32_t ag_push_bytes(int Q, int HD) { return static_cast<uint32_t>(Q * HD + 2 * Q) * 4; }
+__host__ __device__ constexpr size_t ag_recv_bytes(int ns, int Q, int HD) {
+    return ns > 1 ? 16 + static_cast<size_t>(ns - 1) * ag_slot_floats(Q, HD) * 4 : 0;
+}
+
+__device__ __forceinline__ void cluster_arrive_rel() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait_acq() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+// this CTA's shared address `a` as seen in cluster rank `rank`'s shared memory
+__device__ __forceinline__ uint32_t ag_mapa(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+// stores into another CTA's shared memory that complete_tx on its mbarrier
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float4 v, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+                 "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ void st_async_v2(uint32_t addr, float a, float b, uint32_t mbar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr), "f"(a),
+                 "f"(b), "r"(mbar)
+                 : "memory");
+}
+// arrive on an mbarrier in another CTA of the cluster
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(mbar) : "memory");
 }
 
 // CW consumer warps: 4 (two CTAs share an SM) or 8 (a CTA has an SM to itself)
@@ -887,7 +922,11 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
     float *s_lw = s_mw + AG_CW * AG_MAXQ;
     uint64_t *full = reinterpret_cast<uint64_t *>(s_lw + AG_CW * AG_MAXQ);     // [NST]
     uint64_t *empty = full + NST;                                              // [NST]
-    int *pages = reinterpret_cast<int *>(empty + NST);                         // this split's pages
+    uint64_t *mrecv = empty + NST;             // leader: the other splits' partials have landed
+    uint64_t *mack = mrecv + 1;                // non-leader: the leader has all of this split's partial
+    int *pages = reinterpret_cast<int *>(mack + 1);                            // this split's pages
+    float *rcv = reinterpret_cast<float *>(sm + (reinterpret_cast<uintptr_t>(pages + p.max_pages) -
+                                                 reinterpret_cast<uintptr_t>(sm) + 15) / 16 * 16);   // [ns-1][slot]
     __shared__ bool s_last;
 
     const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -897,10 +936,21 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], AG_CW);
         }
+        if (p.cluster) {
+            mbar_init(mrecv, 1);
+            mbar_init(mack, 1);
+        }
         fence_mbar_init();
+        // the leader expects every other split's partial before any can arrive
+        if (p.cluster && split == 0) mbar_arrive_tx(mrecv, (p.n_split - 1) * ag_push_bytes(p.Q, HD));
     }
-    pdl_trigger();
-    pdl_wait();
+    // every thread: this CTA's barriers exist (released to the cluster)
+    if (p.cluster) cluster_arrive_rel();
+    // With p.early the launch that precedes this one signalled its dependents
+    // only after its own dependency wait, so every launch before that one --
+    // and with them pos and the page table -- is complete: the page list and
+    // the first K/V copies need not wait for the previous kernel (L2 loads).
+    if (!p.early) pdl_wait();
 
     const int32_t *pt = p.page_table + static_cast<size_t>(b) * p.max_pages;
     const bool pt_pre = p.max_pages <= ATT_PT_U * AG_THREADS;
@@ -908,9 +958,9 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
 #pragma unroll
     for (int u = 0; u < ATT_PT_U; u++) {
         const int i = tid + u * AG_THREADS;
-        pte[u] = (pt_pre && i < p.max_pages) ? pt[i] : -1;
+        pte[u] = (pt_pre && i < p.max_pages) ? __ldcg(pt + i) : -1;
     }
-    const int p0 = p.pos[b];
+    const int p0 = __ldcg(p.pos + b);
     int len = p0 + p.R;
     if (p0 < 0 || len > p.max_pages * 16 || len > p.rope_max_pos) {
         if (tid == 0) set_error(p.err, BW_DEVERR_BAD_POS);
@@ -939,7 +989,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
         }
     } else {
         for (int i = tid; i < npl; i += AG_THREADS) {
-            int page = pt[pg0 + i];
+            int page = __ldcg(pt + pg0 + i);
             if (page < 0 || page >= p.n_pages) {
                 set_error(p.err, BW_DEVERR_BAD_PAGE);
                 page = -1;
@@ -981,8 +1031,11 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
                 }
             }
         }
+        if (p.cluster) cluster_wait_acq();   // pairs this warp's arrive
         return;
     }
+
+    if (p.early) pdl_wait();   // the query rows and new k/v come from the previous kernel
 
     // ---- 1. Q^T: the roped query rows as fp16 hi (columns 0..QP-1) and lo
     //         (QP..2QP-1) parts, in the MMA's k order; padding rows are zero
@@ -1085,6 +1138,10 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
     for (int s = 0; s < n_stages; s++) {
         const int st = s % NST;
         mbar_wait(&full[st], static_cast<uint32_t>((s / NST) & 1), p.err);
+        // the next kernel (it streams only its weights before its wait) starts
+        // once this CTA's first K/V stage has landed, so that its copies do not
+        // compete with the first stage
+        if (s == 0) pdl_trigger();
         unsigned char *sk = ring + static_cast<size_t>(st) * STB;
         unsigned char *sv = sk + STB / 2;
         const int tb = (pg0 + s * AG_PPS) * 16;       // position of the stage's first token
@@ -1171,17 +1228,17 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
         for (int j = 0; j < 2; j++) {
             const int qi = qa + j;
             const int lim = (qi < p.Q && page_ok) ? min(t1, p0 + qi / p.G + 1) : 0;   // causal limit (exclusive)
-            const float vA = tb + tokA < lim ? sc[j] * p.scale : -INFINITY;
-            const float vB = tb + tokB < lim ? sc[2 + j] * p.scale : -INFINITY;
+            const float vA = tb + tokA < lim ? sc[j] * p.scale2 : -INFINITY;
+            const float vB = tb + tokB < lim ? sc[2 + j] * p.scale2 : -INFINITY;
             float mx = fmaxf(vA, vB);
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             const float m_new = fmaxf(m_q[j], mx);
-            corr[j] = (m_q[j] == -INFINITY) ? 0.0f : expf(m_q[j] - m_new);
+            corr[j] = (m_q[j] == -INFINITY) ? 0.0f : exp2f(m_q[j] - m_new);
             m_q[j] = m_new;
-            pr[j] = (vA == -INFINITY) ? 0.0f : expf(vA - m_new);
-            pr[2 + j] = (vB == -INFINITY) ? 0.0f : expf(vB - m_new);
+            pr[j] = (vA == -INFINITY) ? 0.0f : exp2f(vA - m_new);
+            pr[2 + j] = (vB == -INFINITY) ? 0.0f : exp2f(vB - m_new);
             l_q[j] = l_q[j] * corr[j] + (pr[j] + pr[2 + j]);
         }
         if (__any_sync(0xffffffffu, corr[0] != 1.0f || corr[1] != 1.0f)) {
@@ -1306,7 +1363,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
             float M = -INFINITY;
 #pragma unroll
             for (int w2 = 0; w2 < AG_CW; w2++) M = fmaxf(M, s_mw[w2 * AG_MAXQ + qa + j]);
-            wgt[j] = (m_q[j] == -INFINITY) ? 0.0f : expf(m_q[j] - M);
+            wgt[j] = (m_q[j] == -INFINITY) ? 0.0f : exp2f(m_q[j] - M);
         }
 #pragma unroll
         for (int mt = 0; mt < NMT; mt++)
@@ -1319,12 +1376,30 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
             }
     }
     ag_sync<AG_CT>();
-    for (int e = tid; e < p.Q * HD; e += AG_CT) {
-        const int qi = e / HD, d = e - qi * HD;
-        float o = 0.0f;
+    // a non-leader split of a cluster writes its partial straight into the
+    // leader's receive slot (stores that count down the leader's barrier)
+    const bool pusher = p.cluster && split != 0;
+    uint32_t slot_a = 0, mrecv_a = 0;
+    if (p.cluster) cluster_wait_acq();   // every CTA of the cluster has its barriers
+    if (pusher) {
+        slot_a = ag_mapa(smem_u32(rcv + (split - 1) * ag_slot_floats(p.Q, HD)), 0);
+        mrecv_a = ag_mapa(smem_u32(mrecv), 0);
+    }
+    for (int e4 = tid; e4 < p.Q * (HD / 4); e4 += AG_CT) {
+        const int qi = e4 / (HD / 4), d = (e4 - qi * (HD / 4)) * 4;
+        float4 o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-        for (int w2 = 0; w2 < AG_CW; w2++) o += scr[(w2 * QP + qi) * HD + d];
-        s_o[qi * HD + d] = o;
+        for (int w2 = 0; w2 < AG_CW; w2++) {
+            const float4 v = *reinterpret_cast<const float4 *>(scr + (w2 * QP + qi) * HD + d);
+            o.x += v.x;
+            o.y += v.y;
+            o.z += v.z;
+            o.w += v.w;
+        }
+        if (pusher)
+            st_async_v4(slot_a + static_cast<uint32_t>(e4) * 16, o, mrecv_a);
+        else
+            *reinterpret_cast<float4 *>(s_o + qi * HD + d) = o;
     }
     if (tid < p.Q) {
         float M = -INFINITY;
@@ -1334,59 +1409,85 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
 #pragma unroll
         for (int w2 = 0; w2 < AG_CW; w2++) {
             const float m2 = s_mw[w2 * AG_MAXQ + tid];
-            L += (m2 == -INFINITY) ? 0.0f : s_lw[w2 * AG_MAXQ + tid] * expf(m2 - M);
+            L += (m2 == -INFINITY) ? 0.0f : s_lw[w2 * AG_MAXQ + tid] * exp2f(m2 - M);
         }
-        s_m[tid] = M;
-        s_l[tid] = L;
+        if (pusher) {
+            st_async_v2(slot_a + static_cast<uint32_t>(p.Q * HD + 2 * tid) * 4, M, L, mrecv_a);
+        } else {
+            s_m[tid] = M;
+            s_l[tid] = L;
+        }
+    }
+    if (pusher) {
+        // stay (with the stores in flight) until the leader holds all of them
+        mbar_wait(mack, 0, p.err);
+        return;
     }
     ag_sync<AG_CT>();
 
     // ---- 5. the output, or a partial for the split combine
     if (p.cluster) {
-        // the splits form one thread-block cluster: each CTA merges a slice of
-        // the outputs from every split's shared memory, in split order
-        cg::cluster_group cluster = cg::this_cluster();
-        cluster.sync();
-        const int ns = p.n_split;
-        float *s_w = s_l + ATT_MAXQ;                  // [ns][Q] max, then weight (local only)
-        float *s_sl = s_w + ATT_MAXCL * ATT_MAXQ;     // [ns][Q] sums
-        float *s_L = s_sl + ATT_MAXCL * ATT_MAXQ;     // [Q]
-        for (int e = tid; e < ns * p.Q; e += AG_CT) {
-            const int r2 = e / p.Q, qi = e - r2 * p.Q;
-            s_w[e] = cluster.map_shared_rank(s_m, r2)[qi];
-            s_sl[e] = cluster.map_shared_rank(s_l, r2)[qi];
+        // the cluster's leader: every split's partial is in shared memory
+        // (its own in s_o, s_m, s_l; the others in the receive slots); the
+        // splits are combined in split order
+        const int ns = p.n_split, SF = ag_slot_floats(p.Q, HD);
+        mbar_wait(mrecv, 0, p.err);
+        {
+            // the other splits may leave: their partials are all here
+            const int r = tid - (AG_CT - 32);
+            if (r >= 1 && r < ns) mbar_arrive_remote(ag_mapa(smem_u32(mack), static_cast<uint32_t>(r)));
         }
-        ag_sync<AG_CT>();
-        if (tid < p.Q) {
-            const int qi = tid;
+        // split r's (max, sum) of query row qi
+        auto m_of = [&](int r, int qi) { return r == 0 ? s_m[qi] : rcv[(r - 1) * SF + p.Q * HD + 2 * qi]; };
+        auto l_of = [&](int r, int qi) { return r == 0 ? s_l[qi] : rcv[(r - 1) * SF + p.Q * HD + 2 * qi + 1]; };
+        float *s_w = s_l + ATT_MAXQ;                  // [ns][Q] weights 2^(m_r - M)
+        if (tid < ns * p.Q) {
+            const int r = tid / p.Q, qi = tid - r * p.Q;
             float M = -INFINITY;
-            for (int r2 = 0; r2 < ns; r2++) M = fmaxf(M, s_w[r2 * p.Q + qi]);
-            float L = 0.0f;
-            for (int r2 = 0; r2 < ns; r2++) {
-                const float m2 = s_w[r2 * p.Q + qi];
-                const float w = (m2 == -INFINITY) ? 0.0f : expf(m2 - M);
-                s_w[r2 * p.Q + qi] = w;
-                L = fmaf(s_sl[r2 * p.Q + qi], w, L);
-            }
-            s_L[qi] = L;
+#pragma unroll
+            for (int r2 = 0; r2 < ATT_MAXCL; r2++)
+                if (r2 < ns) M = fmaxf(M, m_of(r2, qi));
+            const float m = m_of(r, qi);
+            s_w[tid] = (m == -INFINITY) ? 0.0f : exp2f(m - M);
         }
         ag_sync<AG_CT>();
-        const int per = (p.Q * HD + ns - 1) / ns;
-        for (int e = split * per + tid; e < min(p.Q * HD, (split + 1) * per); e += AG_CT) {
-            const int qi = e / HD, d = e - qi * HD;
-            float ov[ATT_MAXCL];
+        // four dims of one query row per thread; sums in split order
+        const float4 *rcv4 = reinterpret_cast<const float4 *>(rcv);
+        for (int e4 = tid; e4 < p.Q * (HD / 4); e4 += AG_CT) {
+            const int qi = e4 / (HD / 4), d = (e4 - qi * (HD / 4)) * 4;
+            float L = 0.0f;
+            float4 O = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int r0 = 0; r0 < ns; r0 += 4) {
+                // four splits' loads in flight, then their terms in order
+                float wv[4], lv[4];
+                float4 ov[4];
 #pragma unroll
-            for (int r2 = 0; r2 < ATT_MAXCL; r2++)
-                ov[r2] = r2 < ns ? cluster.map_shared_rank(s_o, min(r2, ns - 1))[qi * HD + d] : 0.0f;
-            float O = 0.0f;
+                for (int u = 0; u < 4; u++) {
+                    const int r2 = r0 + u;
+                    if (r2 < ns) {
+                        wv[u] = s_w[r2 * p.Q + qi];
+                        lv[u] = l_of(r2, qi);
+                        ov[u] = r2 == 0 ? *reinterpret_cast<const float4 *>(s_o + qi * HD + d)
+                                        : rcv4[((r2 - 1) * SF) / 4 + e4];
+                    }
+                }
 #pragma unroll
-            for (int r2 = 0; r2 < ATT_MAXCL; r2++)
-                if (r2 < ns) O = fmaf(ov[r2], s_w[r2 * p.Q + qi], O);
+                for (int u = 0; u < 4; u++) {
+                    if (r0 + u < ns) {
+                        L = fmaf(lv[u], wv[u], L);
+                        O.x = fmaf(ov[u].x, wv[u], O.x);
+                        O.y = fmaf(ov[u].y, wv[u], O.y);
+                        O.z = fmaf(ov[u].z, wv[u], O.z);
+                        O.w = fmaf(ov[u].w, wv[u], O.w);
+                    }
+                }
+            }
             const int r = qi / p.G, gq = qi - r * p.G;
-            p.out[(static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
-                  static_cast<size_t>(kvh * p.G + gq) * HD + d] = (O * p.vscale) / s_L[qi];
+            const float vs = p.vscale;
+            *reinterpret_cast<float4 *>(p.out + (static_cast<size_t>(b) * p.R + r) * (static_cast<size_t>(p.nq) * HD) +
+                                        static_cast<size_t>(kvh * p.G + gq) * HD + d) =
+                make_float4((O.x * vs) / L, (O.y * vs) / L, (O.z * vs) / L, (O.w * vs) / L);
         }
-        cluster.sync();   // keep this CTA's shared memory alive until every reader is done
         return;
     }
     const size_t pbase = (static_cast<size_t>(b) * p.nkv + kvh) * p.n_split;
@@ -1434,7 +1535,7 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
         float L = 0.0f;
         for (int r2 = 0; r2 < ns; r2++) {
             const float m2 = s_w[r2 * p.Q + qi];
-            const float w = (m2 == -INFINITY) ? 0.0f : expf(m2 - M);
+            const float w = (m2 == -INFINITY) ? 0.0f : exp2f(m2 - M);
             s_w[r2 * p.Q + qi] = w;
             L = fmaf(s_sl[r2 * p.Q + qi], w, L);
         }
@@ -1609,7 +1710,11 @@ static bw_status attn_go_st(int ns, int nkv, int B, cudaStream_t st, const AttnP
 
 template <int HD, int NQT, int NST, int F8, int CW>
 static bw_status attn_g_go(int ns, int nkv, int B, bool cl, cudaStream_t st, const AttnParams &p) {
-    const size_t smem = ag_smem_fixed<HD, NQT, NST, F8, CW>() + static_cast<size_t>(p.max_pages) * 4;
+    const size_t base = ag_smem_fixed<HD, NQT, NST, F8, CW>() + static_cast<size_t>(p.max_pages) * 4;
+    // the cluster leader's receive area must fit next to the ring; otherwise
+    // the splits combine through the workspace
+    if (cl && base + ag_recv_bytes(ns, p.Q, HD) > 227 * 1024) cl = false;
+    const size_t smem = base + (cl ? ag_recv_bytes(ns, p.Q, HD) : 0);
     if (smem > 227 * 1024) return BW_ERR_UNSUPPORTED_SHAPE;
     static size_t attr_set[64] = {};
     int dev = 0;
@@ -1695,7 +1800,8 @@ bw_status attn_check(const float *qkv, const float *rope_cos, const float *rope_
 bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
                       void *k_pool, void *v_pool, const int32_t *page_table, int max_pages,
                       int n_pages, const int32_t *pos, int B, int R, int nq, int nkv, int hd,
-                      float *out, const Scratch &sc, cudaStream_t st, int kv_fmt, float kscale, float vscale) {
+                      float *out, const Scratch &sc, cudaStream_t st, int kv_fmt, float kscale, float vscale,
+                      bool early) {
     if (kv_fmt != 0 && kv_fmt != 1) return BW_ERR_INVALID_ARG;
     if (kv_fmt == 1 && !(kscale > 0.0f && vscale > 0.0f && isfinite(kscale) && isfinite(vscale)))
         return BW_ERR_INVALID_ARG;
@@ -1724,9 +1830,13 @@ bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope
     p.kscale = f8 ? kscale : 1.0f;
     p.vscale = f8 ? vscale : 1.0f;
     if (f8) p.scale = p.scale * kscale;
+    // the token-on-M kernel's softmax runs in base 2: scores times log2(e)
+    p.scale2 = static_cast<float>(static_cast<double>(p.scale) * 1.4426950408889634);
     p.out = out;
     p.err = sc.err;
     p.cnt = sc.cnt + CNT_ATTN;
+    p.cluster = 0;
+    p.early = early ? 1 : 0;
     if (!kv_tensor_map(&p.tmk, k_pool, n_pages, nkv, hd, f8) || !kv_tensor_map(&p.tmv, v_pool, n_pages, nkv, hd, f8))
         return BW_ERR_CUDA;
     const int ns = attn_splits(B, nkv, max_pages);

@@ -90,11 +90,15 @@ bw_status mma_gemm_launch(const void *wq, const void *wscales, float ts, float t
                           float *y, int32_t *argmax_out, unsigned flags, const Scratch &sc, cudaStream_t st,
                           int32_t *adv_tokens, int32_t *adv_pos);
 size_t attn_scratch_bytes(int B, int R, int nq, int nkv, int hd, int max_pages);
+// early: pos and page_table were written before the launch that precedes
+// this one, and that launch (one of this library's projection kernels)
+// signals its dependents only after its own dependency wait; the kernel then
+// reads them, and starts the K/V copies, before its own wait.
 bw_status attn_launch(const float *qkv, const float *rope_cos, const float *rope_sin, int rope_max_pos,
                       void *k_pool, void *v_pool, const int32_t *page_table, int max_pages, int n_pages,
                       const int32_t *pos, int B, int R, int nq, int nkv, int hd, float *out,
                       const Scratch &sc, cudaStream_t st, int kv_fmt = 0, float kscale = 1.0f,
-                      float vscale = 1.0f);
+                      float vscale = 1.0f, bool early = false);
 bw_status embed_launch(int fmt, const void *e_q, const void *e_s, float ts, int V, int H,
                        const int32_t *tokens, int M, float *x, uint32_t *err, cudaStream_t st);
 

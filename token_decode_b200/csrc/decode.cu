@@ -202,7 +202,7 @@ bw_status bw_decode_step(const bw_model *m, const bw_kv *kv, int32_t *tokens_in,
         s = attn_launch(bf.qkv, m->rope_cos, m->rope_sin, m->rope_max_pos, kv->k[l], kv->v[l],
                         kv->page_table, kv->max_pages, kv->n_pages, pos, B, n_rows, m->nq, m->nkv, m->hd,
                         bf.attn, bf.kern, st, kv->kv_fmt, kv->kv_fmt ? kv->k_scale[l] : 1.0f,
-                        kv->kv_fmt ? kv->v_scale[l] : 1.0f);
+                        kv->kv_fmt ? kv->v_scale[l] : 1.0f, /*early=*/true);
         if (s != BW_OK) return s;
         s = gemv_launch(fmt, ly.wo.q, ly.wo.s, ly.wo.ts, ly.wo.ts, m->H, m->nq * m->hd, bf.attn, R,
                         nullptr, m->eps, bf.x, bf.x, nullptr, BW_GEMV_RESIDUAL, bf.kern, st);

@@ -253,7 +253,6 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = s_tmem;
-    pdl_trigger();
 
     if (warp == 0) {
         // ---- producer: the first stages of constant weights before the
@@ -274,6 +273,10 @@ __global__ void __launch_bounds__(MM_THREADS, 1) mma_gemm_kernel(const MmaParams
             const int pre = min(MM_NST, n_tiles);
             for (int t = 0; t < pre; t++) issue(t);
             pdl_wait();
+            // dependents launch only once this kernel's dependency is met:
+            // a kernel after this one may read, before its own wait, what
+            // the launches before this one wrote
+            pdl_trigger();
             if (n_tiles > 0) {
                 const uint32_t col_bytes = static_cast<uint32_t>(GV_TC * 4 * (p.Mp / 8) * 128);   // one column tile
                 mbar_arrive_tx(bfull, static_cast<uint32_t>(T) * col_bytes);

@@ -90,12 +90,14 @@ __device__ __forceinline__ void load_residual(const GemvParams &p, int rg, int l
 }
 
 // Final values of row group rg (lanes with (lane & 1) == 0 hold row
-// (lane >> 1) & 7): scale, epilogue (res: the residual to add), outputs,
+// (lane >> 1) & 7): scale (rs: the RMSNorm factor of each activation row, or
+// 1), epilogue (res: the residual to add), outputs,
 // argmax tracking.  All lanes must call it (it shuffles); `act` gates the
 // stores.
 template <int FMT, int M>
 __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, const float (&tot)[M],
-                                         const float (&res)[M], float (&bestv)[M], int (&besti)[M], bool act) {
+                                         const float (&rs)[M], const float (&res)[M], float (&bestv)[M],
+                                         int (&besti)[M], bool act) {
     const int r = (lane >> 1) & 7;
     const bool gu = p.flags & BW_GEMV_SILU_GATE;
     float val[M];
@@ -107,7 +109,7 @@ __device__ __forceinline__ void epilogue(const GemvParams &p, int rg, int lane, 
         } else {
             v = v * ((gu && r >= 4) ? p.ts_up : p.ts);
         }
-        val[m] = v;
+        val[m] = v * rs[m];
     }
     if (gu) {
         // gate row r (< 4) pairs with up row r + 4, held by lane + 8
@@ -174,7 +176,6 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
         fence_mbar_init();
     }
     __syncthreads();
-    pdl_trigger();
 
     if (warp == GV_CW) {
         // ---- producer: constant weights only, so no dependency wait
@@ -201,27 +202,39 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
     const int ne = nc * 32;
     // the slice's RMSNorm gains are model data like the weights: staged
     // before the dependency wait
-    if (norm)
+    if (norm) {
         (void)stage_row4(reinterpret_cast<const float4 *>(p.gamma + c0 * 32), ne / 4, reinterpret_cast<float4 *>(gt),
                          0, ne / 4, ctid);
+        consumer_sync();
+    }
     pdl_wait();
-    // pass 1: the slice's activations in natural order, one batch of
-    // independent 16-byte loads per thread; with RMSNorm over a K slice the
-    // whole row is read in the same batch, for the sum of squares
+    // dependents launch only once this kernel's own dependency is met (the
+    // producer warp never signals): a kernel that starts after this one may
+    // read, before its own wait, whatever the launches before this one wrote
+    pdl_trigger();
+    // the slice's activations, one batch of independent 16-byte loads per
+    // thread, stored straight in the staged form (times the gains); with
+    // RMSNorm over a K slice the whole row is read in the same batch, for the
+    // sum of squares.  The norm's 1/rms factor is a scalar per row: the
+    // epilogue applies it to the dot products.
     float ss[M];
 #pragma unroll
     for (int m = 0; m < M; m++) {
-        float4 *xs4 = reinterpret_cast<float4 *>(xs + static_cast<size_t>(m) * CS * 32);
+        float *xm = xs + static_cast<size_t>(m) * CS * 32;
+        float *ctm = ct + static_cast<size_t>(m) * CS;
         if (m >= p.M) {
-            for (int e = ctid; e < ne / 4; e += GV_CW * 32) xs4[e] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            float4 *xm4 = reinterpret_cast<float4 *>(xm);
+            for (int e = ctid; e < ne / 4; e += GV_CW * 32) xm4[e] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int e = ctid; e < nc; e += GV_CW * 32) ctm[e] = 0.0f;
             ss[m] = 0.0f;
             continue;
         }
         const float4 *xr4 = reinterpret_cast<const float4 *>(p.x + static_cast<size_t>(m) * p.K);
+        const float4 *gt4 = norm ? reinterpret_cast<const float4 *>(gt) : nullptr;
         if (norm && p.S > 1)
-            ss[m] = stage_row4(xr4, p.K / 4, xs4, c0 * 8, ne / 4, ctid);
+            ss[m] = stage_row_t<FMT>(xr4, p.K / 4, xm, ctm, gt4, c0 * 8, ne / 4, ctid);
         else
-            ss[m] = stage_row4(xr4 + c0 * 8, ne / 4, xs4, 0, ne / 4, ctid);
+            ss[m] = stage_row_t<FMT>(xr4 + c0 * 8, ne / 4, xm, ctm, gt4, 0, ne / 4, ctid);
     }
     if (norm) {
 #pragma unroll
@@ -237,9 +250,9 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
         }
     }
     consumer_sync();
-    // pass 2: swizzle and pre-scale in place
-    stage_pass2<FMT, M>(xs, ct, norm ? gt : nullptr, s_rnorm, CS, nc, warp, lane);
-    consumer_sync();
+    float rs[M];   // per-row output factor: 1/rms with RMSNorm
+#pragma unroll
+    for (int m = 0; m < M; m++) rs[m] = norm ? s_rnorm[m] : 1.0f;
 
     float acc[8][M];
 #pragma unroll
@@ -277,7 +290,7 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
 #pragma unroll
             for (int m = 0; m < M; m++) acc[r][m] = 0.0f;
         if (p.S == 1) {
-            epilogue<FMT, M>(p, rg, lane, tot, res, bestv, besti, true);
+            epilogue<FMT, M>(p, rg, lane, tot, rs, res, bestv, besti, true);
         } else {
             // split K: leave the partial sums; the last slice to finish a row
             // group (per half-warp) adds them in slice order and runs the epilogue
@@ -316,7 +329,7 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
                                 for (int m = 0; m < M; m++) sum[m] += v[u][m];
                     }
             }
-            epilogue<FMT, M>(p, rg, lane, sum, res, bestv, besti, last);
+            epilogue<FMT, M>(p, rg, lane, sum, rs, res, bestv, besti, last);
             if (last && (lane & 15) == 0) p.rg_cnt[rg] = 0u;
         }
     }

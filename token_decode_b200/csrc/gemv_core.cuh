@@ -115,6 +115,72 @@ __device__ __forceinline__ float stage_row4(const float4 *src, int n4, float4 *d
     return ss;
 }
 
+// One-pass staging: loads the 16-byte elements [0, n4) of a row (a batch of
+// 8 independent loads per thread in flight) and stores elements
+// [lo, lo + n_keep) -- times the gains gt4[e - lo] when gt4 is given -- in the
+// staged form of stage_x below: chunk c (8 elements of 16 bytes) at
+// xs + 32 c, granules XOR-swizzled by c, Q4_0 values pre-scaled per nibble
+// slot and the chunk's -8 term in ct[c].  The 8 elements of a chunk are
+// loaded by 8 consecutive lanes (lo is a multiple of 8), which exchange
+// halves with the lane 4 apart to form the Q4_0 granules and add up the
+// chunk sum.  Returns this thread's sum of squares over every element it
+// loaded (before the gains).
+template <int FMT>
+__device__ __forceinline__ float stage_row_t(const float4 *src, int n4, float *xs, float *ct, const float4 *gt4, int lo,
+                                             int n_keep, int tid) {
+    constexpr int U = 8, STEP = GV_CW * 32;
+    const int j = tid & 7;
+    float ss = 0.0f;
+    for (int b = 0; b < n4; b += U * STEP) {
+        float4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int e = b + u * STEP + tid;
+            v[u] = e < n4 ? src[e] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            ss = fma_rn(v[u].x, v[u].x, ss);
+            ss = fma_rn(v[u].y, v[u].y, ss);
+            ss = fma_rn(v[u].z, v[u].z, ss);
+            ss = fma_rn(v[u].w, v[u].w, ss);
+            const int d = b + u * STEP + tid - lo;
+            const bool keep = d >= 0 && d < n_keep;
+            float4 w = keep ? v[u] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (gt4 && keep) {
+                const float4 g = gt4[d];
+                w = make_float4(w.x * g.x, w.y * g.y, w.z * g.z, w.w * g.w);
+            }
+            const int c = keep ? d >> 3 : 0;
+            if constexpr (FMT == BW_FMT_Q4_0) {
+                // lanes j < 4 hold elements 4j .. 4j+3 of the chunk, lanes j >= 4
+                // elements 16 + 4(j-4) ..: granule 2j takes (A.x, B.x, A.y, B.y),
+                // granule 2j+1 (A.z, B.z, A.w, B.w), A from lane j, B from lane j+4
+                const float4 o = make_float4(__shfl_xor_sync(0xffffffffu, w.x, 4), __shfl_xor_sync(0xffffffffu, w.y, 4),
+                                             __shfl_xor_sync(0xffffffffu, w.z, 4), __shfl_xor_sync(0xffffffffu, w.w, 4));
+                const bool low = j < 4;
+                const float4 A = low ? w : o, B = low ? o : w;
+                const int G = low ? 2 * j : 2 * (j - 4) + 1;
+                const float4 gr = low ? make_float4(A.x, B.x, A.y, B.y) : make_float4(A.z, B.z, A.w, B.w);
+                float cs = (w.x + w.y) + (w.z + w.w);
+                cs += __shfl_xor_sync(0xffffffffu, cs, 1);
+                cs += __shfl_xor_sync(0xffffffffu, cs, 2);
+                cs += __shfl_xor_sync(0xffffffffu, cs, 4);
+                if (keep) {
+                    // 2^(101 - 4p) for granule slot p
+                    *reinterpret_cast<float4 *>(xs + c * 32 + 4 * (G ^ (c & 7))) =
+                        make_float4(gr.x * __int_as_float((127 + 101) << 23), gr.y * __int_as_float((127 + 97) << 23),
+                                    gr.z * __int_as_float((127 + 93) << 23), gr.w * __int_as_float((127 + 89) << 23));
+                    if (j == 0) ct[c] = cs * -2.8421709430404007e-14f;   // -8 * 2^-48
+                }
+            } else {
+                if (keep) *reinterpret_cast<float4 *>(xs + c * 32 + 4 * (j ^ (c & 7))) = w;
+            }
+        }
+    }
+    return ss;
+}
+
 // Staged activations: chunk c of row m at (m*chunk_stride + c)*128 bytes; its
 // 16-byte granule g is stored at granule (g ^ (c & 7)), so 8 lanes reading
 // granule g of 8 consecutive chunks hit 8 different bank groups.
