@@ -1038,27 +1038,29 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
     if (p.early) pdl_wait();   // the query rows and new k/v come from the previous kernel
 
     // ---- 1. Q^T: the roped query rows as fp16 hi (columns 0..QP-1) and lo
-    //         (QP..2QP-1) parts, in the MMA's k order; padding rows are zero
-    for (int i = tid; i < QP * (HD / 2); i += AG_CT) {
+    //         (QP..2QP-1) parts, in the MMA's k order; padding rows are zero.
+    //         Their loads are issued first, so that they are in flight with
+    //         the new rows' loads (one round trip for both).
+    constexpr int NQI = (QP * (HD / 2) + AG_CT - 1) / AG_CT;
+    float qx[NQI], qy[NQI], qc[NQI], qn[NQI];
+#pragma unroll
+    for (int u = 0; u < NQI; u++) {
+        const int i = tid + u * AG_CT;
         const int qi = i / (HD / 2), d = i - qi * (HD / 2);
-        float ra = 0.0f, rb = 0.0f;
-        if (qi < p.Q) {
+        qx[u] = 0.0f;
+        qy[u] = 0.0f;
+        qc[u] = 0.0f;
+        qn[u] = 0.0f;
+        if (i < QP * (HD / 2) && qi < p.Q) {
             const int r = qi / p.G, g = qi - r * p.G;
             const int h = kvh * p.G + g;
             const int ppos = max(0, min(p0 + r, p.rope_max_pos - 1));
             const float *src = p.qkv + (static_cast<size_t>(b) * p.R + r) * row_stride + static_cast<size_t>(h) * HD;
-            const float c = p.rope_cos[static_cast<size_t>(ppos) * (HD / 2) + d];
-            const float s = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
-            rope_pair(src[d], src[d + HD / 2], c, s, ra, rb);
+            qx[u] = src[d];
+            qy[u] = src[d + HD / 2];
+            qc[u] = p.rope_cos[static_cast<size_t>(ppos) * (HD / 2) + d];
+            qn[u] = p.rope_sin[static_cast<size_t>(ppos) * (HD / 2) + d];
         }
-        __half h0, l0, h1, l1;
-        split_f16(ra, h0, l0);
-        split_f16(rb, h1, l1);
-        const int ka = F8 ? ag_kidx_f8(d) : d, kb = F8 ? ag_kidx_f8(d + HD / 2) : d + HD / 2;
-        qs[qi * QSS + ka] = h0;
-        qs[(QP + qi) * QSS + ka] = l0;
-        qs[qi * QSS + kb] = h1;
-        qs[(QP + qi) * QSS + kb] = l1;
     }
 
     // ---- 2. the new rows' k (roped) and v as stored (fp16, or E4M3 codes of
@@ -1107,6 +1109,23 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
                 reinterpret_cast<__half *>(newv)[r * HD + d] = hv;
                 if (ok) p.v_pool[off + d] = hv;
             }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < NQI; u++) {
+        const int i = tid + u * AG_CT;
+        if (i < QP * (HD / 2)) {
+            const int qi = i / (HD / 2), d = i - qi * (HD / 2);
+            float ra = 0.0f, rb = 0.0f;
+            if (qi < p.Q) rope_pair(qx[u], qy[u], qc[u], qn[u], ra, rb);
+            __half h0, l0, h1, l1;
+            split_f16(ra, h0, l0);
+            split_f16(rb, h1, l1);
+            const int ka = F8 ? ag_kidx_f8(d) : d, kb = F8 ? ag_kidx_f8(d + HD / 2) : d + HD / 2;
+            qs[qi * QSS + ka] = h0;
+            qs[(QP + qi) * QSS + ka] = l0;
+            qs[qi * QSS + kb] = h1;
+            qs[(QP + qi) * QSS + kb] = l1;
         }
     }
     ag_sync<AG_CT>();
@@ -1511,13 +1530,13 @@ __global__ void __launch_bounds__((CW + 1) * 32, CW == 4 ? 2 : 1) attn_g_kernel(
     if (tid < p.Q)
         __stcg(reinterpret_cast<float2 *>(p.part_ml + ((pbase + split) * p.Q + tid) * 2), make_float2(s_m[tid], s_l[tid]));
     // the last split of this (sequence, kv head) to finish combines all of them
-    __threadfence();
+    fence_acq_rel_gpu();
     ag_sync<AG_CT>();
     uint32_t *cnt = p.cnt + static_cast<size_t>(b) * p.nkv + kvh;
     if (tid == 0) s_last = atomicAdd(cnt, 1u) == static_cast<uint32_t>(p.n_split - 1);
     ag_sync<AG_CT>();
     if (!s_last) return;
-    __threadfence();
+    fence_acq_rel_gpu();
     const int ns = p.n_split;
     float *s_w = reinterpret_cast<float *>(sm);            // [ns][Q] max, then weight (the ring is free)
     float *s_sl = s_w + ATT_MAXNS * ATT_MAXQ;              // [ns][Q] sums

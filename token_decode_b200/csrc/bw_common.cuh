@@ -197,6 +197,11 @@ __device__ __forceinline__ float half_bits_to_f(uint32_t h) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
 }
 
+// Release/acquire fence at GPU scope: with a relaxed atomic after it (writer)
+// or before it (reader), orders plain global accesses across CTAs (lighter
+// than the sequentially consistent __threadfence).
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
 __device__ __forceinline__ void set_error(uint32_t *err, uint32_t bit) {
     if (err) atomicOr(err, bit);
 }

@@ -301,7 +301,7 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
 #pragma unroll
                 for (int m = 0; m < M; m++) __stcg(dst + m, tot[m]);
             }
-            __threadfence();
+            fence_acq_rel_gpu();
             __syncwarp();
             uint32_t old = 0;
             if ((lane & 15) == 0 && real) old = atomicAdd(p.rg_cnt + rg, 1u);
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
 #pragma unroll
             for (int m = 0; m < M; m++) sum[m] = 0.0f;
             if (last) {
-                __threadfence();
+                fence_acq_rel_gpu();
                 if ((lane & 1) == 0)
                     // batches of 8 slices' loads in flight, added in slice order
                     for (int s0 = 0; s0 < p.S; s0 += 8) {
