@@ -155,6 +155,8 @@ _PROFILE_FILES = {("gu", "7b-dense-q4_0"): "gemv_gate_up_7b.md",
                   ("qkv", "7b-dense-q4_0"): "gemv_qkv_7b.md",
                   ("o", "7b-dense-q4_0"): "gemv_o_7b.md",
                   ("lm_head", "7b-dense-q4_0"): "gemv_lm_head_7b.md",
+                  ("gu", "9b-dense-nvfp4"): "gemv_gate_up_9b.md",
+                  ("gu", "27b-dense-nvfp4"): "gemv_gate_up_27b.md",
                   ("attn", "7b-dense-q4_0"): "attn_7b_b1.md",
                   ("attn", "27b-dense-nvfp4"): "attn_27b_b1.md",
                   ("attn", "9b-dense-nvfp4-b32"): "attn_9b_b32.md",

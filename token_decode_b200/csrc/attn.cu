@@ -809,6 +809,24 @@ __global__ void __launch_bounds__(ATT_THREADS, NST == 2 ? 2 : 1) attn_kernel(con
 // codes in whole 32-bit words -- any order of k gives the same sums, as long
 // as Q and P are written in the same order -- and O^T's rows (dims) in an
 // order that lets one word of V feed two m-tiles.
+//
+// Softmax in base 2: the scores are scaled by log2(e) / sqrt(hd) and
+// exponentiated with exp2f; the merges use the same units.
+//
+// Splits of a (sequence, kv head) that fit one thread-block cluster (2..16)
+// combine in the leader (rank 0): every other split writes its partial --
+// unnormalized O, then (max, sum) per query row -- straight from registers
+// into a receive slot in the leader's shared memory with st.async, whose
+// bytes count down a transaction barrier the leader armed for all of them at
+// start; the leader adds the partials in split order and releases the others
+// (a remote arrive on a barrier of theirs, so that none exits while its
+// stores are in flight).  One cluster barrier, split into an arrive at start
+// and a wait before the first remote access, orders the barriers'
+// initialisation.  More splits combine through the workspace (last arriver).
+//
+// Inside a decode step (AttnParams::early) the page list, the position and the
+// first K/V copies do not wait for the previous kernel (the projection), only
+// the query rows and the new k/v row do.
 constexpr int AG_PST = 24;                        // padded P^T row (halves): conflict-free ldmatrix
 constexpr int AG_MAXQ = 8;                        // query rows per (sequence, kv head)
 

@@ -21,7 +21,10 @@
 // sums in the workspace and the last warp to finish a row group (atomic
 // counter, no waiting) adds them in slice order, so results are
 // deterministic.  The activation slice of a CTA is staged once in shared
-// memory (16-byte granules XOR-swizzled by chunk, conflict-free per warp).
+// memory (16-byte granules XOR-swizzled by chunk, conflict-free per warp),
+// transformed as it is loaded; with the RMSNorm prologue the staged values
+// are x * gamma and the scalar 1/rms of each row multiplies the dot products
+// in the epilogue.
 //
 // Q4_0 arithmetic without integer->float conversions: a nibble q masked in
 // place into the low bits of an fp32 word is the denormal q * 2^(4p-149)
@@ -153,7 +156,6 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
     uint64_t *empty = full + nst;
     const uint32_t stages_a = smem_u32(stages), xs_a = smem_u32(xs), ct_a = smem_u32(ct);
     __shared__ float s_red[GV_CW][M];
-    __shared__ float s_rnorm[M];
     __shared__ float s_bv[GV_CW][M];
     __shared__ int s_bi[GV_CW][M];
     __shared__ bool s_last;
@@ -242,17 +244,21 @@ __global__ void __launch_bounds__(GV_THREADS, gv_ctas_per_sm<M>()) gemv_kernel(c
             ss[m] = warp_sum(ss[m]);
             if (lane == 0) s_red[warp][m] = ss[m];
         }
-        consumer_sync();
-        if (ctid < M) {
-            float t = 0.0f;
-            for (int w2 = 0; w2 < GV_CW; w2++) t += s_red[w2][ctid];
-            s_rnorm[ctid] = 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps);
-        }
     }
     consumer_sync();
-    float rs[M];   // per-row output factor: 1/rms with RMSNorm
+    // per-row output factor: 1/rms with RMSNorm (every thread adds the warps'
+    // sums in the same order)
+    float rs[M];
 #pragma unroll
-    for (int m = 0; m < M; m++) rs[m] = norm ? s_rnorm[m] : 1.0f;
+    for (int m = 0; m < M; m++) {
+        rs[m] = 1.0f;
+        if (norm) {
+            float t = 0.0f;
+#pragma unroll
+            for (int w2 = 0; w2 < GV_CW; w2++) t += s_red[w2][m];
+            rs[m] = 1.0f / sqrtf(t / static_cast<float>(p.K) + p.eps);
+        }
+    }
 
     float acc[8][M];
 #pragma unroll

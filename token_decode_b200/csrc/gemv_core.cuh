@@ -140,6 +140,7 @@ __device__ __forceinline__ float stage_row_t(const float4 *src, int n4, float *x
         }
 #pragma unroll
         for (int u = 0; u < U; u++) {
+            if (b + u * STEP >= n4) break;   // no lane of the CTA has this element (uniform)
             ss = fma_rn(v[u].x, v[u].x, ss);
             ss = fma_rn(v[u].y, v[u].y, ss);
             ss = fma_rn(v[u].z, v[u].z, ss);
