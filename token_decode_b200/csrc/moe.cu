@@ -88,8 +88,12 @@ struct Routing {
 // argmax (value descending, lower expert index on ties) over the experts not
 // yet chosen; softmax over the chosen logits in selection order.  Then the
 // assignments are bucketed by expert (index order) and, within an expert, by
-// row (row order) -- deterministic.
+// row (row order) -- deterministic: per-expert counts (shared-memory atomics,
+// order-free), one block-wide exclusive scan over the experts for the bucket
+// offsets, group indices and work items, then for each selected expert a warp
+// walks the rows 32 at a time and places them with a ballot prefix.
 constexpr int MOE_NRC = 4;   // row-block chunks per expert matrix (work items per pass)
+constexpr int MOE_SLB = 4;   // router slices loaded per batch (up to 256 experts)
 
 template <int LV>   // logits per lane: ceil(E / 32) <= LV
 __global__ void __launch_bounds__(1024) moe_topk_kernel(const float *part, int n_slices, int R, int E, int K,
@@ -99,31 +103,44 @@ __global__ void __launch_bounds__(1024) moe_topk_kernel(const float *part, int n
     __shared__ int s_sel[MOE_RMAX][MOE_KMAX];
     __shared__ int s_cnt[MOE_EMAX];
     __shared__ int s_off[MOE_EMAX];
-    __shared__ int s_sh_off;
-    __shared__ int s_gexp[MOE_EMAX + 1];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ int s_wsum[3][32];
+    __shared__ int s_tot[3];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int per_lane = (E + 31) / 32;
-    for (int i = threadIdx.x; i < R * K; i += blockDim.x) rt.inv[i] = -1;
+    for (int e = tid; e < MOE_EMAX; e += blockDim.x) s_cnt[e] = 0;
+    for (int i = tid; i < R * K; i += blockDim.x) rt.inv[i] = -1;
+    __syncthreads();
     for (int r = warp; r < R; r += 32) {
         // this row's logits in registers: lane holds experts lane + 32 j, the
-        // router slices summed in slice order
+        // router slices added in slice order, a batch of slices' loads in flight
+        constexpr int SB = LV <= 8 ? MOE_SLB : 1;
         float lv[LV];
 #pragma unroll
-        for (int j = 0; j < LV; j++) {
-            const int e = lane + 32 * j;
-            lv[j] = (j < per_lane && e < E) ? part[static_cast<size_t>(r) * E + e] : -INFINITY;
-        }
-        // slice by slice (in slice order), each slice's loads issued together
-        for (int sl = 1; sl < n_slices; sl++) {
-            float t[LV];
+        for (int j = 0; j < LV; j++) lv[j] = 0.0f;
+        for (int sl0 = 0; sl0 < n_slices; sl0 += SB) {
+            float t[SB][LV];
 #pragma unroll
-            for (int j = 0; j < LV; j++) {
-                const int e = lane + 32 * j;
-                t[j] = (j < per_lane && e < E) ? part[(static_cast<size_t>(sl) * R + r) * E + e] : 0.0f;
-            }
+            for (int b = 0; b < SB; b++)
 #pragma unroll
-            for (int j = 0; j < LV; j++) lv[j] += t[j];
+                for (int j = 0; j < LV; j++) {
+                    const int e = lane + 32 * j;
+                    t[b][j] = (sl0 + b < n_slices && j < per_lane && e < E)
+                                  ? part[(static_cast<size_t>(sl0 + b) * R + r) * E + e]
+                                  : 0.0f;
+                }
+#pragma unroll
+            for (int b = 0; b < SB; b++)
+#pragma unroll
+                for (int j = 0; j < LV; j++) {
+                    if (sl0 + b == 0)
+                        lv[j] = t[b][j];
+                    else if (sl0 + b < n_slices)
+                        lv[j] += t[b][j];
+                }
         }
+#pragma unroll
+        for (int j = 0; j < LV; j++)
+            if (!(j < per_lane && lane + 32 * j < E)) lv[j] = -INFINITY;
         uint32_t used = 0;
         float sv[MOE_KMAX];
         for (int t = 0; t < K; t++) {
@@ -150,7 +167,10 @@ __global__ void __launch_bounds__(1024) moe_topk_kernel(const float *part, int n
                 }
             }
             if (be != 0x7fffffff && (be & 31) == lane) used |= 1u << (be >> 5);
-            if (lane == 0) s_sel[r][t] = be;
+            if (lane == 0) {
+                s_sel[r][t] = be;
+                if (be != 0x7fffffff) atomicAdd(&s_cnt[be], 1);
+            }
             sv[t] = bv;
         }
         if (lane == 0) {
@@ -168,53 +188,83 @@ __global__ void __launch_bounds__(1024) moe_topk_kernel(const float *part, int n
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int c = 0;
-        for (int r = 0; r < R; r++)
-            for (int t = 0; t < K; t++) c += (s_sel[r][t] == e);
-        s_cnt[e] = c;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int off = 0, g = 0;
-        for (int e = 0; e < E; e++) {
-            s_off[e] = off;
-            if (s_cnt[e] > 0) {
-                rt.grp_expert[g] = e;
-                s_gexp[g] = e;
-                rt.grp_off[g] = off;
-                off += s_cnt[e];
-                g++;
+    // exclusive scan over the experts (thread = expert) of: assignments,
+    // "selected" (the group index) and work items
+    {
+        const int e = tid;
+        const int c = e < E ? s_cnt[e] : 0;
+        int v[3] = {c, c > 0 ? 1 : 0, c > 0 ? MOE_NRC * ((c + MOE_M - 1) / MOE_M) : 0};
+        int inc[3] = {v[0], v[1], v[2]};
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1)
+#pragma unroll
+            for (int q = 0; q < 3; q++) {
+                const int u = __shfl_up_sync(0xffffffffu, inc[q], o);
+                if (lane >= o) inc[q] += u;
+            }
+        if (lane == 31)
+#pragma unroll
+            for (int q = 0; q < 3; q++) s_wsum[q][warp] = inc[q];
+        __syncthreads();
+        if (warp == 0) {
+            const int nw = blockDim.x >> 5;
+#pragma unroll
+            for (int q = 0; q < 3; q++) {
+                const int x = lane < nw ? s_wsum[q][lane] : 0;
+                int y = x;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int u = __shfl_up_sync(0xffffffffu, y, o);
+                    if (lane >= o) y += u;
+                }
+                if (lane < nw) s_wsum[q][lane] = y - x;   // exclusive warp prefix
+                if (lane == 31) s_tot[q] = y;
             }
         }
-        rt.grp_expert[g] = -1;           // shared expert: every row
-        rt.grp_off[g] = off;
-        rt.grp_off[g + 1] = off + R;
-        *rt.grp_n = g + 1;
-        s_sh_off = off;
-        // work items: MOE_NRC row-block chunks x passes of MOE_M rows per group
-        int it = 0;
-        for (int gg = 0; gg <= g; gg++) {
-            rt.grp_item[gg] = it;
-            const int cnt = (gg < g) ? s_cnt[s_gexp[gg]] : R;
-            it += MOE_NRC * ((cnt + MOE_M - 1) / MOE_M);
+        __syncthreads();
+        int ex[3];
+#pragma unroll
+        for (int q = 0; q < 3; q++) ex[q] = inc[q] - v[q] + s_wsum[q][warp];
+        if (e < MOE_EMAX) s_off[e] = ex[0];
+        if (c > 0) {
+            rt.grp_expert[ex[1]] = e;
+            rt.grp_off[ex[1]] = ex[0];
+            rt.grp_item[ex[1]] = ex[2];
         }
-        rt.grp_item[g + 1] = it;
-        *rt.n_items = it;
+        if (tid == 0) {
+            const int g = s_tot[1], sh = s_tot[0], it = s_tot[2];
+            rt.grp_expert[g] = -1;   // shared expert: every row
+            rt.grp_off[g] = sh;
+            rt.grp_off[g + 1] = sh + R;
+            *rt.grp_n = g + 1;
+            rt.grp_item[g] = it;
+            const int it2 = it + MOE_NRC * ((R + MOE_M - 1) / MOE_M);
+            rt.grp_item[g + 1] = it2;
+            *rt.n_items = it2;
+        }
     }
-    __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    __syncthreads();   // s_off
+    // each selected expert's assignments, rows in order: a warp walks the rows
+    // 32 at a time (lane = row) and places the ones that chose the expert
+    for (int e = warp; e < E; e += blockDim.x >> 5) {
         if (s_cnt[e] == 0) continue;
-        int j = s_off[e];
-        for (int r = 0; r < R; r++)
-            for (int t = 0; t < K; t++)
-                if (s_sel[r][t] == e) {
-                    rt.asg_row[j] = r;
-                    rt.inv[r * K + t] = j;
-                    j++;
-                }
+        int j0 = s_off[e];
+        for (int r0 = 0; r0 < R; r0 += 32) {
+            const int r = r0 + lane;
+            int slot = -1;
+            if (r < R)
+                for (int t = 0; t < K; t++)
+                    if (s_sel[r][t] == e) slot = t;
+            const uint32_t m = __ballot_sync(0xffffffffu, slot >= 0);
+            if (slot >= 0) {
+                const int j = j0 + __popc(m & ((1u << lane) - 1u));
+                rt.asg_row[j] = r;
+                rt.inv[r * K + slot] = j;
+            }
+            j0 += __popc(m);
+        }
     }
-    for (int r = threadIdx.x; r < R; r += blockDim.x) rt.asg_row[s_sh_off + r] = r;
+    for (int r = tid; r < R; r += blockDim.x) rt.asg_row[s_tot[0] + r] = r;
 }
 
 // ------------------------------------------------------- grouped GEMV
