@@ -50,14 +50,41 @@ __global__ void __launch_bounds__(256) moe_router_kernel(const float *y, const f
     const int e0 = blockIdx.x * 8, k0 = blockIdx.y * MOE_KS, r0 = blockIdx.z * 32;
     const int kn = min(MOE_KS, H - k0), nr = min(32, R - r0);
     // the router weights are constant: stage them before the dependency wait
-    for (int i = threadIdx.x; i < 8 * MOE_KS; i += 256) {
-        const int w = i / MOE_KS, k = i - w * MOE_KS;
-        wsm[i] = (e0 + w < E && k < kn) ? wr[static_cast<size_t>(e0 + w) * H + k0 + k] : 0.0f;
+    // (16-byte loads; H is a multiple of 32, so kn and every row start are too)
+    constexpr int K4 = MOE_KS / 4;
+    {
+        constexpr int NW = 8 * K4 / 256;
+        float4 v[NW];
+#pragma unroll
+        for (int u = 0; u < NW; u++) {
+            const int i = threadIdx.x + u * 256, w = i / K4, k4 = i - w * K4;
+            v[u] = (e0 + w < E && 4 * k4 < kn)
+                       ? *reinterpret_cast<const float4 *>(wr + static_cast<size_t>(e0 + w) * H + k0 + 4 * k4)
+                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int u = 0; u < NW; u++) reinterpret_cast<float4 *>(wsm)[threadIdx.x + u * 256] = v[u];
     }
     pdl_wait();
-    for (int i = threadIdx.x; i < 32 * MOE_KS; i += 256) {
-        const int r = i / MOE_KS, k = i - r * MOE_KS;
-        ys[k * 33 + r] = (r < nr && k < kn) ? y[static_cast<size_t>(r0 + r) * H + k0 + k] : 0.0f;
+    {
+        // the rows' slice: every load in flight at once, then stored transposed
+        constexpr int NY = 32 * K4 / 256;
+        float4 v[NY];
+#pragma unroll
+        for (int u = 0; u < NY; u++) {
+            const int i = threadIdx.x + u * 256, r = i / K4, k4 = i - r * K4;
+            v[u] = (r < nr && 4 * k4 < kn)
+                       ? *reinterpret_cast<const float4 *>(y + static_cast<size_t>(r0 + r) * H + k0 + 4 * k4)
+                       : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int u = 0; u < NY; u++) {
+            const int i = threadIdx.x + u * 256, r = i / K4, k = 4 * (i - r * K4);
+            ys[k * 33 + r] = v[u].x;
+            ys[(k + 1) * 33 + r] = v[u].y;
+            ys[(k + 2) * 33 + r] = v[u].z;
+            ys[(k + 3) * 33 + r] = v[u].w;
+        }
     }
     __syncthreads();
     const int e = e0 + warp;
