@@ -146,6 +146,13 @@ def test_tiny_moe_decode_and_router_topk():
                      [r["moe_logits"][l] for r in ress], cfg.topk)
 
 
+def test_tiny_moe_q4_0_decode():
+    """The MoE block with Q4_0 experts (the grouped GEMV's Q4_0 staging and
+    chunk sums) against the oracle: logits, tokens and each layer's experts."""
+    cfg = _tiny_moe(fmt=synth.FMT_Q4_0, name="tiny-moe-q4")
+    _run_steps(cfg, 2, seed=5, check_route=True)
+
+
 @pytest.mark.parametrize("E,k", [(16, 4), (256, 8)])
 def test_router_topk_bit_exact_on_identical_logits(E, k):
     """bw_moe_route_gemv's selection fed logits the oracle computes identically

@@ -344,16 +344,74 @@ __device__ __forceinline__ MoeItem moe_item(const GroupedParams &p, int i) {
     return it;
 }
 
-// One item's row blocks with MR activation rows: the staged activations are
-// pre-scaled and swizzled, then each row block's KT tiles are consumed and
-// its outputs written.  `step` counts the ring stages (shared with the producer).
+// One-pass staging of up to MR activation rows (rows mcnt..MR-1 staged as
+// zeros) in the staged form of stage_x: every row's 16-byte loads of a batch
+// in flight together, the 8 lanes that loaded a chunk exchanging halves with
+// the lane 4 apart (Q4_0 granules) and adding up its sum; chunks never
+// straddle rows (a row is a multiple of 8 elements).  Row m lands at xs + m * CS * 32, its chunk terms at ct + m * CS.
 template <int FMT, int MR>
-__device__ __forceinline__ void moe_item_rows(const GroupedParams &p, const MoeItem &it, float *xs, float *ct, int CS,
-                                              int nc, int warp, int lane, uint32_t stages_a, uint32_t xs_a,
-                                              uint32_t ct_a, uint64_t *full, uint64_t *empty, int &step, float ts,
-                                              float ts_up) {
+__device__ __forceinline__ void stage_rows_t(const float4 *const (&src)[MR], int mcnt, int n4, float *xs, float *ct,
+                                             int CS, int tid) {
+    constexpr int U = 8, STEP = GV_CW * 32;
+    const int j = tid & 7, tot = MR * n4;
+    for (int b = 0; b < tot; b += U * STEP) {
+        float4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int i = b + u * STEP + tid;
+            const int m = i / n4, e = i - m * n4;
+            const float4 *row = src[0];
+#pragma unroll
+            for (int mm = 1; mm < MR; mm++)
+                if (m == mm) row = src[mm];
+            v[u] = (i < tot && m < mcnt) ? row[e] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            if (b + u * STEP >= tot) break;   // uniform
+            const int i = b + u * STEP + tid;
+            const bool keep = i < tot;
+            const int m = keep ? i / n4 : 0, d = keep ? i - m * n4 : 0;
+            const float4 w = v[u];
+            const int c = d >> 3;
+            float *xm = xs + static_cast<size_t>(m) * CS * 32;
+            if constexpr (FMT == BW_FMT_Q4_0) {
+                const float4 o = make_float4(__shfl_xor_sync(0xffffffffu, w.x, 4), __shfl_xor_sync(0xffffffffu, w.y, 4),
+                                             __shfl_xor_sync(0xffffffffu, w.z, 4), __shfl_xor_sync(0xffffffffu, w.w, 4));
+                const bool low = j < 4;
+                const float4 A = low ? w : o, B = low ? o : w;
+                const int G = low ? 2 * j : 2 * (j - 4) + 1;
+                const float4 gr = low ? make_float4(A.x, B.x, A.y, B.y) : make_float4(A.z, B.z, A.w, B.w);
+                float cs = (w.x + w.y) + (w.z + w.w);
+                cs += __shfl_xor_sync(0xffffffffu, cs, 1);
+                cs += __shfl_xor_sync(0xffffffffu, cs, 2);
+                cs += __shfl_xor_sync(0xffffffffu, cs, 4);
+                if (keep) {
+                    *reinterpret_cast<float4 *>(xm + c * 32 + 4 * (G ^ (c & 7))) =
+                        make_float4(gr.x * __int_as_float((127 + 101) << 23), gr.y * __int_as_float((127 + 97) << 23),
+                                    gr.z * __int_as_float((127 + 93) << 23), gr.w * __int_as_float((127 + 89) << 23));
+                    if (j == 0) ct[static_cast<size_t>(m) * CS + c] = cs * -2.8421709430404007e-14f;   // -8 * 2^-48
+                }
+            } else {
+                if (keep) *reinterpret_cast<float4 *>(xm + c * 32 + 4 * (j ^ (c & 7))) = w;
+            }
+        }
+    }
+}
+
+// One item's row blocks with MR activation rows: the item's rows are staged
+// (pre-scaled and swizzled as they are loaded), then each row block's KT
+// tiles are consumed and its outputs written.  `step` counts the ring stages (shared with the producer).
+template <int FMT, int MR>
+__device__ __forceinline__ void moe_item_rows(const GroupedParams &p, const MoeItem &it, const float4 *const (&xr)[MOE_M],
+                                              float *xs, float *ct, int CS, int nc, int warp, int lane,
+                                              uint32_t stages_a, uint32_t xs_a, uint32_t ct_a, uint64_t *full,
+                                              uint64_t *empty, int &step, float ts, float ts_up) {
     const int nst = p.nst, T = p.KT;
-    stage_pass2<FMT, MR>(xs, ct, nullptr, nullptr, CS, nc, warp, lane);
+    const float4 *rows[MR];
+#pragma unroll
+    for (int m = 0; m < MR; m++) rows[m] = xr[m];
+    stage_rows_t<FMT, MR>(rows, it.mcnt, nc * 8, xs, ct, CS, static_cast<int>(threadIdx.x));
     consumer_sync();
     for (int rb = it.rb0; rb < it.rb1; rb++) {
         const int rg = rb * (GV_TR / 8) + 2 * warp + (lane >> 4);
@@ -470,47 +528,22 @@ __global__ void __launch_bounds__(GV_THREADS, 1) moe_grouped_gemv_kernel(const G
             }
         }
         consumer_sync();   // the previous item is done with the staged activations
-        // the item's activation rows in natural order: the 16-byte loads of
-        // all its rows in flight together (rows past its count are zeros)
-        {
-            const float *xr[M];
+        const float4 *xr[M];
 #pragma unroll
-            for (int m = 0; m < M; m++) {
-                xr[m] = p.x;
-                if (m < it.mcnt) {
-                    const int j = it.off + m;
-                    xr[m] = p.x + static_cast<size_t>(p.gather ? p.asg_row[j] : j) * p.K;
-                }
-            }
-            const int n4 = nc * 8, tot = M * n4;
-            for (int b = 0; b < tot; b += 8 * GV_CW * 32) {
-                float4 v[8];
-                int at[8];
-#pragma unroll
-                for (int u = 0; u < 8; u++) {
-                    const int i = b + u * GV_CW * 32 + static_cast<int>(threadIdx.x);
-                    const int m = i / n4, e = i - m * n4;
-                    const float *row = xr[0];
-#pragma unroll
-                    for (int mm = 1; mm < M; mm++)
-                        if (m == mm) row = xr[mm];
-                    v[u] = (i < tot && m < it.mcnt) ? reinterpret_cast<const float4 *>(row)[e]
-                                                    : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    at[u] = i < tot ? m * CS * 8 + e : -1;
-                }
-#pragma unroll
-                for (int u = 0; u < 8; u++)
-                    if (at[u] >= 0) reinterpret_cast<float4 *>(xs)[at[u]] = v[u];
+        for (int m = 0; m < M; m++) {
+            xr[m] = reinterpret_cast<const float4 *>(p.x);
+            if (m < it.mcnt) {
+                const int j = it.off + m;
+                xr[m] = reinterpret_cast<const float4 *>(p.x + static_cast<size_t>(p.gather ? p.asg_row[j] : j) * p.K);
             }
         }
-        consumer_sync();
         // the inner loop for the item's actual row count (1, 2 or up to 4)
         if (it.mcnt == 1)
-            moe_item_rows<FMT, 1>(p, it, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
+            moe_item_rows<FMT, 1>(p, it, xr, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
         else if (it.mcnt == 2)
-            moe_item_rows<FMT, 2>(p, it, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
+            moe_item_rows<FMT, 2>(p, it, xr, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
         else
-            moe_item_rows<FMT, M>(p, it, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
+            moe_item_rows<FMT, M>(p, it, xr, xs, ct, CS, nc, warp, lane, stages_a, xs_a, ct_a, full, empty, step, ts, ts_up);
     }
 }
 
