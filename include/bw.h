@@ -130,6 +130,15 @@ bw_status bw_workspace_init(void *ws, size_t bytes, void *stream);
  * *err_out (host) and clear it on the device.  ws == NULL reads the error word
  * of bw_gemv_q4_0_noalloc's fixed scratch on the current device instead. */
 bw_status bw_read_error(void *ws, uint32_t *err_out, void *stream);
+/* Asynchronous form of bw_read_error: enqueue on `stream`, after everything
+ * already queued there, one tiny kernel that ORs the device error word of `ws`
+ * (NULL: bw_gemv_q4_0_noalloc's fixed scratch on the current device) into
+ * *dst and clears the word.  dst is DEVICE memory (4-byte aligned) owned by
+ * the caller; nothing synchronizes, so the call can be captured in a CUDA
+ * graph -- e.g. after every step of a multi-step graph, with one copy of
+ * *dst to the host at the end.  Returns BW_ERR_INVALID_ARG (nothing queued)
+ * for a NULL or misaligned dst or a misaligned ws. */
+bw_status bw_drain_error(void *ws, uint32_t *dst, void *stream);
 
 /* ---------------------------------------------------------------- layout */
 

@@ -98,6 +98,10 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.bw_spec_accept(fake, fake, 1, 9, fake, None, 1, None, None) == 1
     assert lib.bw_spec_accept(fake, fake, 0, 4, fake, None, 1, None, None) == 1
     assert lib.bw_spec_accept(fake, fake, 1, 4, fake, fake, 0, None, None) == 1
+    # error drain: no destination, a misaligned destination or workspace
+    assert lib.bw_drain_error(fake, None, None) == 1
+    assert lib.bw_drain_error(fake, p(4098), None) == 1
+    assert lib.bw_drain_error(p(4096 + 16), fake, None) == 1
 
 
 def test_workspace_queries_are_host_only(lib):

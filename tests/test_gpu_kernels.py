@@ -492,3 +492,34 @@ def test_paged_attention_fp8_rejects_bad_scales():
         with pytest.raises(bw.BWError):
             bw.paged_attn_decode_fp8(qkv, cos, cos, max_pages * 16, kp8, kp8.clone(), ks, 0.05, table, max_pages,
                                      n_pages, pos, 1, 1, 4, 2, 64, out, ws)
+
+
+def test_drain_error_moves_the_word_without_a_sync_and_in_a_graph():
+    """bw_drain_error ORs a workspace's device error word into a device
+    accumulator and clears it, queued on the stream (eagerly and inside a
+    captured graph)."""
+    ws = bw.workspace(1 << 18)
+    word = ws[:4].view(torch.int32)
+    dst = torch.full((1,), 2, dtype=torch.int32, device="cuda")
+    word.fill_(5)                      # a planted error word: bits 0 and 2
+    bw.drain_error(ws, dst)
+    torch.cuda.synchronize()
+    assert int(dst.item()) == 7 and int(word.item()) == 0
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            bw.drain_error(ws, dst, stream=s)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    dst.zero_()
+    word.fill_(8)
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    assert int(dst.item()) == 8 and int(word.item()) == 0
+    g.replay()                         # nothing planted: the accumulator keeps its bits
+    torch.cuda.synchronize()
+    assert int(dst.item()) == 8
+    assert bw.read_error(ws) == 0

@@ -27,7 +27,7 @@ MAX_VERIFY_ROWS = 8
 
 # every symbol include/bw.h declares (checked by the CPU test-suite)
 EXPORTS = (
-    "bw_status_string", "bw_abi_version", "bw_workspace_init", "bw_read_error",
+    "bw_status_string", "bw_abi_version", "bw_workspace_init", "bw_read_error", "bw_drain_error",
     "bw_repack_bytes", "bw_repack_q4_0", "bw_repack_nvfp4", "bw_gemv_q4_0", "bw_gemv_nvfp4",
     "bw_gemv_workspace_bytes", "bw_gemv_q4_0_noalloc", "bw_rmsnorm_fused", "bw_embed", "bw_rope_table", "bw_argmax",
     "bw_paged_attn_decode", "bw_paged_attn_decode_fp8", "bw_attn_workspace_bytes", "bw_moe_route_gemv",
@@ -88,6 +88,7 @@ def lib() -> C.CDLL:
             "bw_abi_version": (i, []),
             "bw_workspace_init": (i, [p, z, p]),
             "bw_read_error": (i, [p, p, p]),
+            "bw_drain_error": (i, [p, p, p]),
             "bw_repack_bytes": (i, [i, i, p, p]),
             "bw_repack_q4_0": (i, [p, p, i, i, p, p, p]),
             "bw_repack_nvfp4": (i, [p, p, p, p, i, i, p, p, p]),
@@ -167,6 +168,12 @@ def read_error(ws: torch.Tensor, stream=None) -> int:
     out = C.c_uint32(0)
     _check(lib().bw_read_error(_ptr(ws), C.byref(out), _stream(stream)), "bw_read_error")
     return out.value
+
+
+def drain_error(ws, dst: torch.Tensor, stream=None) -> None:
+    """Enqueue: OR ws's device error word (ws None: the no-alloc scratch's)
+    into dst[0] (a device int32/uint32 tensor) and clear it; no synchronization."""
+    _check(lib().bw_drain_error(_ptr(ws), _ptr(dst), _stream(stream)), "bw_drain_error")
 
 
 def repack_bytes(rows, K):

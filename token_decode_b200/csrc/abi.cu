@@ -22,6 +22,14 @@ int sm_count() {
     return cached[dev];
 }
 
+// one thread: the error word moves into the caller's accumulator
+__global__ void drain_error_kernel(uint32_t *err, uint32_t *dst) {
+    if (threadIdx.x == 0) {
+        const uint32_t v = atomicExch(err, 0u);
+        if (v) atomicOr(dst, v);
+    }
+}
+
 bw_status launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? BW_OK : BW_ERR_CUDA;
@@ -74,6 +82,18 @@ bw_status bw_read_error(void *ws, uint32_t *err_out, void *stream) {
     }
     *err_out = v;
     return BW_OK;
+}
+
+bw_status bw_drain_error(void *ws, uint32_t *dst, void *stream) {
+    if (!dst || (reinterpret_cast<uintptr_t>(dst) & 3u)) return BW_ERR_INVALID_ARG;
+    if (ws && !bw::ws_ok(ws)) return BW_ERR_INVALID_ARG;
+    if (!ws) {
+        const bw_status s = bw::noalloc_scratch(&ws);
+        if (s != BW_OK) return s;
+    }
+    // a plain launch: ordered after all the stream's earlier work
+    bw::drain_error_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t *>(ws), dst);
+    return bw::launch_status();
 }
 
 }  // extern "C"
